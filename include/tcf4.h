@@ -1,0 +1,133 @@
+/*
+ * tcf4.h -- C ABI of the trellis-coded FP4 (XOR-Trellis / HEPH) decode library for B200.
+ *
+ * The library decodes weights stored as an XOR-Trellis bitstream ("XOR-Trellis: Hadamard-free
+ * FP4 LLM quantization" news page, bullet "XOR-Trellis FP4 decoder": 16-bit sliding state, four
+ * masked parities 0x1089/0x2112/0x0A24/0x2441 giving p0,p1,q0,q1, palettes P0..P3) under HEPH's
+ * grid-aligned convention ("HEPH: 3-Bit Grid-Aligned Trellis Quantization of MXFP4
+ * Mixture-of-Experts ...", abstract): each decoded weight is an E2M1 value times its 32-weight
+ * block's UE8M0 scale 2^(E-127), i.e. a valid MXFP4 element. HEPH serves such weights in two
+ * modes, both exported here: the stream stays resident and is decoded inside the product kernels
+ * (trellis_gemv, trellis_grouped_moe), or it is expanded once into a resident packed MXFP4 tensor
+ * (trellis_decode_to_mxfp4).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout. A matrix W is [rows][cols] row-major, cols % 32 == 0, scales run along cols.
+ *   stream: uint32 [rows][cols/32][2]; for 32-weight block j of row n, word 0 holds the low bit
+ *           and word 1 the high bit of the 2-bit branch symbols (bit i = symbol 32j+i).
+ *   scales: uint8 [rows][cols/32], UE8M0 (value 2^(E-127); 0xFF is NaN and propagates).
+ *   seg_len: the trellis state is 0 at the start of every seg_len-weight segment of a row;
+ *           seg_len is a positive multiple of 32 that divides cols (32 = one MXFP4 block).
+ *   Decoder reading: the new symbol b enters the state at bits 14-15 (s = s>>2 | b<<14);
+ *   p = p0 + 2*p1 picks the palette, q = q0 + 2*q1, entry = b XOR q; P3's zero is -0.
+ *   Activations and outputs are bf16 passed as their uint16 bit patterns.
+ * Memory. Every data pointer is DEVICE memory owned by the caller. The library never allocates,
+ *   frees or synchronizes; every call is asynchronous on `stream` (a cudaStream_t, NULL = the
+ *   legacy default stream). Inputs must stay valid until the work on `stream` completes.
+ * Alignment. stream, x and y pointers must be 16-byte aligned; MXFP4 outputs too.
+ * Errors. Arguments are checked on the host before anything is launched: a bad argument returns
+ *   TCF4_ERR_INVALID_ARG / TCF4_ERR_MISALIGNED / TCF4_ERR_UNSUPPORTED / TCF4_ERR_WORKSPACE and
+ *   launches nothing. A failed launch returns TCF4_ERR_CUDA (the CUDA error is left set for the
+ *   caller to read). Empty problems (rows == 0, T == 0) return TCF4_OK and launch nothing.
+ * Threads. Calls are reentrant; no global state is written.
+ */
+#ifndef TCF4_H
+#define TCF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TCF4_API __attribute__((visibility("default")))
+#else
+#define TCF4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TCF4_OK = 0,
+  TCF4_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, cols % 32, bad seg_len, bad k/E/T */
+  TCF4_ERR_MISALIGNED = 2,   /* a pointer that must be 16-byte aligned is not */
+  TCF4_ERR_UNSUPPORTED = 3,  /* a size beyond the limits stated below */
+  TCF4_ERR_WORKSPACE = 4,    /* workspace missing or smaller than trellis_grouped_moe_workspace */
+  TCF4_ERR_CUDA = 5          /* a kernel launch failed */
+} tcf4_status;
+
+/* One trellis-coded matrix (all pointers device memory). */
+typedef struct {
+  const uint32_t *stream; /* [rows][cols/32][2] planar trellis words */
+  const uint8_t *scales;  /* [rows][cols/32] UE8M0 block scales */
+  int64_t rows;
+  int64_t cols;           /* multiple of 32 */
+  int32_t seg_len;        /* multiple of 32 dividing cols */
+} tcf4_matrix;
+
+/* HEPH abstract, second serving mode: expand the stream into a resident packed MXFP4 tensor.
+ *   out_nibbles: uint8 [rows][cols/2]; byte u of a row holds element 2u in its low nibble and
+ *                element 2u+1 in its high nibble (OCP E2M1 codes, sign in bit 3).
+ *   out_scales:  uint8 [rows][cols/32], a byte-for-byte copy of w.scales.
+ * Bit-exact with the decoder definition. out_nibbles must be 16-byte aligned. */
+TCF4_API tcf4_status trellis_decode_to_mxfp4(tcf4_matrix w, uint8_t *out_nibbles, uint8_t *out_scales,
+                                    void *stream);
+
+/* HEPH abstract, first serving mode: fused decode + product.
+ *   y[t][n] = bf16( sum_k w[n][k] * x[t][k] ), fp32 accumulation, round to nearest even.
+ *   x: bf16 bits [T][cols]; y: bf16 bits [T][rows]; 1 <= T <= 32 (T == 0 is a no-op).
+ * Accuracy: |y - exact| <= 2e-3 * ||w_row||_2 * ||x_t||_2 per output plus the bf16 rounding.
+ * Limits: cols <= 16384. */
+TCF4_API tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream);
+
+/* Router for the MoE layer: for each token, the k experts with the largest logits (ties to the
+ * lower expert index) and softmax weights over those k logits (fp32).
+ *   logits: fp32 [T][E]; topk_ids: int32 [T][k]; topk_w: fp32 [T][k].
+ * Limits: 1 <= k <= 8, k <= E <= 256, T <= 32. */
+TCF4_API tcf4_status trellis_moe_route(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *topk_ids,
+                              float *topk_w, void *stream);
+
+/* One MoE layer: E experts, hidden size H, intermediate size I.
+ *   gate_up: HOST array of E descriptors, each [2I][H] (gate rows 0..I-1, up rows I..2I-1);
+ *   down:    HOST array of E descriptors, each [H][I].
+ * All gate_up matrices share one seg_len, and all down matrices share one seg_len. The host
+ * arrays are read during the call only. */
+typedef struct {
+  const tcf4_matrix *gate_up;
+  const tcf4_matrix *down;
+  int32_t E;
+  int32_t H;
+  int32_t I;
+} tcf4_moe;
+
+/* Bytes of device workspace trellis_grouped_moe needs for T tokens and top-k routing
+ * (0 when the arguments are invalid). */
+TCF4_API size_t trellis_grouped_moe_workspace(const tcf4_moe *m, int32_t T, int32_t k);
+
+/* HEPH abstract, first serving mode for a routed MoE layer: for every token t and every selected
+ * expert j = topk_ids[t][*]: g,u = gate_up_j . x_t, h = bf16(silu(g) * u), y_j = down_j . h, and
+ *   out[t] = bf16( sum_j topk_w[t][j] * y_j )   (fp32 accumulation and combine).
+ * Tokens routed to the same expert share one decode of its weights.
+ *   x: bf16 bits [T][H]; topk_ids: int32 [T][k] (device); topk_w: fp32 [T][k] (device);
+ *   out: bf16 bits [T][H]; workspace: device scratch of at least
+ *   trellis_grouped_moe_workspace(m, T, k) bytes, 256-byte aligned, owned by the caller.
+ * After the call the workspace holds, among other things, h as bf16 [T*k][I] in (t, j) order at
+ * offset trellis_grouped_moe_hidden_offset(m, T, k).
+ * Limits: 1 <= T <= 32, 1 <= k <= 8, E <= 256, H and I <= 16384. Expert ids outside [0, E) in
+ * topk_ids make the affected (t, j) contribute nothing. */
+TCF4_API tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, int32_t T, const int32_t *topk_ids,
+                                const float *topk_w, int32_t k, uint16_t *out, void *workspace,
+                                size_t ws_bytes, void *stream);
+
+/* Byte offset of h (bf16 [T*k][I]) inside the workspace of trellis_grouped_moe. */
+TCF4_API size_t trellis_grouped_moe_hidden_offset(const tcf4_moe *m, int32_t T, int32_t k);
+
+/* A static, human-readable description of a status code. */
+TCF4_API const char *tcf4_status_string(tcf4_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TCF4_H */

@@ -1,0 +1,90 @@
+"""Shared helpers for the GPU parity tests: upload synthetic inputs, compare with the oracle.
+
+Tolerance for products (fp32 accumulation, bf16 out): |y_gpu - y_exact| <= 2e-3 ||w_row|| ||x_t||
+per output, against the unrounded exact product.
+"""
+import numpy as np
+import torch
+
+import oracle
+import trellis_coded_fp4_b200 as tc
+from trellis_coded_fp4_b200 import synth
+
+TOL = 2e-3
+
+
+def upload_matrix(rows, cols, seed, seg_len=32, lo=120, hi=126):
+    st = synth.stream(rows, cols, seed)
+    sc = synth.scales(rows, cols, seed, lo, hi)
+    return st, sc, tc.TrellisMatrix.from_numpy(st, sc, rows, cols, seg_len)
+
+
+def bf16_to_f64(t):
+    return oracle.bf16_bits_to_f64(synth.bf16_bits(t.cpu()))
+
+
+def assert_products_close(y_gpu, y_exact, wnorm, xnorm, what=""):
+    """y_gpu: bf16 tensor [T][n]; y_exact [T][n] fp64; wnorm [n]; xnorm [T]."""
+    got = bf16_to_f64(y_gpu)
+    bound = TOL * np.outer(xnorm, wnorm)
+    err = np.abs(got - y_exact)
+    bad = err > bound
+    if bad.any():
+        i = np.argwhere(bad)[0]
+        raise AssertionError(f"{what}: {bad.sum()} outputs out of tolerance; first {tuple(i)}: gpu {got[tuple(i)]!r} "
+                             f"exact {y_exact[tuple(i)]!r} bound {bound[tuple(i)]!r}")
+
+
+def xnorms(x_bits):
+    return np.linalg.norm(oracle.bf16_bits_to_f64(x_bits), axis=1)
+
+
+def check_moe(layer, W, x, ids, wts, out, ws, k, seg_gu, seg_dn=None, rows_h=None, rows_out=None):
+    """Two-stage check of a grouped-MoE call.
+
+    (i) h (read back from the workspace) against h_exact = silu(g) u from exact g, u, within the
+        bound propagated from the product tolerance on g and u plus one bf16 rounding;
+    (ii) out against sum_j w_j (down_j . h_gpu_j) computed exactly from the GPU's own h, within
+        2e-3 sum_j |w_j| ||down_row|| ||h_j||.
+    rows_h / rows_out: optional subsets of intermediate / output rows (sampled checks)."""
+    T = x.shape[0]
+    H, I = layer.H, layer.I
+    seg_dn = seg_gu if seg_dn is None else seg_dn
+    x_bits = synth.bf16_bits(x.cpu())
+    ids_np = ids.cpu().numpy()
+    w_np = wts.cpu().numpy().astype(np.float64)
+    off = W.hidden_offset(T, k)
+    h_gpu = ws[off:off + T * k * I * 2].view(torch.int16).cpu().numpy().view(np.uint16).reshape(T, k, I)
+    ri = np.arange(I) if rows_h is None else np.asarray(rows_h)
+    rn = np.arange(H) if rows_out is None else np.asarray(rows_out)
+    xn = xnorms(x_bits)
+    for t in range(T):
+        for j in range(k):
+            e = int(ids_np[t, j])
+            if not 0 <= e < layer.E:
+                continue
+            gu_rows = np.concatenate([ri, I + ri])
+            y, wn = oracle.gemv(layer.gu_stream[e], layer.gu_scales[e], 2 * I, H, seg_gu, x_bits[t:t + 1],
+                                row_ids=gu_rows)
+            g, u = y[0, :len(ri)], y[0, len(ri):]
+            dg, du = TOL * wn[:len(ri)] * xn[t], TOL * wn[len(ri):] * xn[t]
+            sg = oracle.silu(g)
+            h_exact = sg * u
+            bound = 1.1 * np.abs(u) * dg + (np.abs(sg) + 1.1 * dg) * du + 2.0 ** -8 * np.abs(h_exact) + 1e-30
+            h_got = oracle.bf16_bits_to_f64(h_gpu[t, j, ri])
+            bad = np.abs(h_got - h_exact) > bound
+            assert not bad.any(), f"h out of bound at t={t} j={j} rows {ri[bad][:5]}"
+    out_got = bf16_to_f64(out)
+    for t in range(T):
+        acc = np.zeros(len(rn))
+        bnd = np.zeros(len(rn))
+        for j in range(k):
+            e = int(ids_np[t, j])
+            if not 0 <= e < layer.E:
+                continue
+            hb = h_gpu[t, j][None, :]
+            y, wn = oracle.gemv(layer.dn_stream[e], layer.dn_scales[e], H, I, seg_dn, hb, row_ids=rn)
+            acc += w_np[t, j] * y[0]
+            bnd += abs(w_np[t, j]) * wn * np.linalg.norm(oracle.bf16_bits_to_f64(hb))
+        bad = np.abs(out_got[t, rn] - acc) > TOL * bnd + 1e-30
+        assert not bad.any(), f"out out of bound at t={t} rows {rn[bad][:5]}"

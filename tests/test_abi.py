@@ -1,0 +1,95 @@
+"""The C-ABI library loads, exports every symbol include/tcf4.h declares, and rejects bad arguments
+on the host before launching anything (these calls make no CUDA call, so they run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from trellis_coded_fp4_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def _declared():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"TCF4_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert set(declared) == set(_abi.EXPORTED)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.tcf4_status_string(s)
+    assert lib.tcf4_status_string(99) == b"unknown status"
+
+
+def _mat(stream=16, scales=16, rows=4, cols=64, seg=32):
+    return _abi.Matrix(stream, scales, rows, cols, seg)
+
+
+def test_gemv_argument_checks(lib):
+    ok_x, ok_y = ctypes.c_void_p(4096), ctypes.c_void_p(8192)
+    s0 = ctypes.c_void_p(0)
+    assert lib.trellis_gemv(_mat(cols=48), ok_x, 1, ok_y, s0) == 1          # cols % 32
+    assert lib.trellis_gemv(_mat(seg=48), ok_x, 1, ok_y, s0) == 1           # seg_len % 32
+    assert lib.trellis_gemv(_mat(seg=96), ok_x, 1, ok_y, s0) == 1           # seg_len does not divide cols
+    assert lib.trellis_gemv(_mat(stream=0), ok_x, 1, ok_y, s0) == 1         # null stream
+    assert lib.trellis_gemv(_mat(stream=8), ok_x, 1, ok_y, s0) == 2         # misaligned stream
+    assert lib.trellis_gemv(_mat(), ctypes.c_void_p(4098), 1, ok_y, s0) == 2
+    assert lib.trellis_gemv(_mat(), ok_x, 33, ok_y, s0) == 3                # T > 32
+    assert lib.trellis_gemv(_mat(), ok_x, -1, ok_y, s0) == 1
+    assert lib.trellis_gemv(_mat(), ok_x, 0, ok_y, s0) == 0                 # empty: no launch
+    assert lib.trellis_gemv(_mat(rows=0), ok_x, 1, ok_y, s0) == 0
+    assert lib.trellis_gemv(_mat(cols=32768, seg=32), ok_x, 1, ok_y, s0) == 3
+    assert lib.trellis_gemv(_mat(), ctypes.c_void_p(0), 1, ok_y, s0) == 1
+
+
+def test_expand_and_route_argument_checks(lib):
+    s0 = ctypes.c_void_p(0)
+    assert lib.trellis_decode_to_mxfp4(_mat(), ctypes.c_void_p(0), ctypes.c_void_p(64), s0) == 1
+    assert lib.trellis_decode_to_mxfp4(_mat(), ctypes.c_void_p(72), ctypes.c_void_p(64), s0) == 2
+    assert lib.trellis_decode_to_mxfp4(_mat(rows=0), ctypes.c_void_p(0), ctypes.c_void_p(0), s0) == 0
+    p = ctypes.c_void_p(256)
+    assert lib.trellis_moe_route(p, 4, 8, 9, p, p, s0) == 1                  # k > E
+    assert lib.trellis_moe_route(p, 4, 300, 4, p, p, s0) == 3                # E > 256
+    assert lib.trellis_moe_route(p, 4, 32, 9, p, p, s0) == 3                 # k > 8
+    assert lib.trellis_moe_route(p, 0, 32, 4, p, p, s0) == 0
+
+
+def test_moe_workspace_and_checks(lib):
+    E, H, I = 4, 64, 96
+    gu = (_abi.Matrix * E)(*[_abi.Matrix(256, 256, 2 * I, H, 32) for _ in range(E)])
+    dn = (_abi.Matrix * E)(*[_abi.Matrix(256, 256, H, I, 32) for _ in range(E)])
+    m = _abi.Moe(gu, dn, E, H, I)
+    ws = lib.trellis_grouped_moe_workspace(ctypes.byref(m), 3, 2)
+    off = lib.trellis_grouped_moe_hidden_offset(ctypes.byref(m), 3, 2)
+    assert ws > 0 and ws % 256 == 0 and 0 < off < ws
+    assert ws - off >= 3 * 2 * I * 2 + 3 * 2 * H * 4
+    p = ctypes.c_void_p(256)
+    s0 = ctypes.c_void_p(0)
+    assert lib.trellis_grouped_moe(ctypes.byref(m), p, 3, p, p, 2, p, p, ws - 1, s0) == 4
+    assert lib.trellis_grouped_moe(ctypes.byref(m), p, 3, p, p, 2, p, ctypes.c_void_p(0), ws, s0) == 4
+    assert lib.trellis_grouped_moe(ctypes.byref(m), p, 3, p, p, 2, p, ctypes.c_void_p(512 + 16), ws, s0) == 2
+    assert lib.trellis_grouped_moe(ctypes.byref(m), p, 33, p, p, 2, p, p, ws, s0) == 3
+    bad = _abi.Moe(gu, dn, E, H, I + 32)                                      # shapes disagree
+    assert lib.trellis_grouped_moe_workspace(ctypes.byref(bad), 3, 2) == 0
+    dn2 = (_abi.Matrix * E)(*[_abi.Matrix(256, 256, H, I, 32 if e else 96) for e in range(E)])
+    mixed = _abi.Moe(gu, dn2, E, H, I)                                        # mixed seg_len
+    assert lib.trellis_grouped_moe(ctypes.byref(mixed), p, 3, p, p, 2, p, p, ws, s0) == 3
+    assert lib.trellis_grouped_moe(ctypes.byref(m), p, 0, p, p, 2, p, p, ws, s0) == 0

@@ -1,0 +1,68 @@
+"""The word-wide XOR identities the CUDA decoder uses, checked against the oracle on the CPU.
+
+The kernels decode a 32-weight block with shifted XORs of its two bit planes instead of walking
+the state weight by weight. This test restates those identities in numpy (test-only code; the
+kernels are CUDA) and compares them with the oracle's step-by-step decoder for every 16-bit state
+and for random multi-block rows, with and without a carry from the previous block. The GPU
+parity tests then check the kernels themselves bit for bit.
+"""
+import numpy as np
+
+import oracle
+from trellis_coded_fp4_b200 import synth
+
+M32 = np.uint64(0xFFFFFFFF)
+
+
+def _dly(x, px, d):
+    return ((x << np.uint64(d)) | (px >> np.uint64(32 - d))) & M32
+
+
+def _planes(L, H, pL, pH):
+    L, H, pL, pH = (np.asarray(v, np.uint64) for v in (L, H, pL, pH))
+    Ld = {d: _dly(L, pL, d) for d in range(1, 8)}
+    Hd = {d: _dly(H, pH, d) for d in range(1, 8)}
+    neg = ~(H ^ Ld[7] ^ Ld[4] ^ Ld[2] ^ Hd[1]) & M32
+    n0 = neg ^ Ld[7] ^ Hd[6] ^ Hd[4] ^ Ld[1]
+    n1 = neg ^ Hd[7] ^ Ld[5] ^ Ld[3] ^ Hd[1]
+    n2 = neg ^ L ^ Ld[6] ^ Hd[5] ^ Hd[3] ^ Hd[2]
+    return n0, n1, n2, neg
+
+
+def _codes_from_planes(n):
+    i = np.arange(32, dtype=np.uint64)
+    return sum(((n[c][..., None] >> i) & np.uint64(1)) << np.uint64(c) for c in range(4)).astype(np.uint8)
+
+
+def test_identity_for_every_state():
+    # The last weight of a block decoded after a 7-symbol history covers every 16-bit state.
+    s = np.arange(1 << 16, dtype=np.uint64)
+    # state bits 2m / 2m+1 hold symbol i-7+m; place history in the previous block's top bits and
+    # the current symbol at bit 0 of this block, then read weight 0's code.
+    pL = np.zeros_like(s)
+    pH = np.zeros_like(s)
+    for m in range(7):
+        pL |= ((s >> np.uint64(2 * m)) & np.uint64(1)) << np.uint64(25 + m)
+        pH |= ((s >> np.uint64(2 * m + 1)) & np.uint64(1)) << np.uint64(25 + m)
+    L = (s >> np.uint64(14)) & np.uint64(1)
+    H = (s >> np.uint64(15)) & np.uint64(1)
+    codes = _codes_from_planes(_planes(L, H, pL, pH))[:, 0]
+    ref = np.array([oracle.state_code(int(v)) for v in s], np.uint8)
+    assert (codes == ref).all()
+
+
+def test_identity_on_rows_with_and_without_carry():
+    rows, cols = 8, 256
+    st = synth.stream(rows, cols, seed=51).astype(np.uint64)
+    for seg_len in (32, 128, 256):
+        ref = oracle.decode_codes(st.astype(np.uint32), rows, cols, seg_len)
+        sb = seg_len // 32
+        got = np.zeros((rows, cols), np.uint8)
+        for j in range(cols // 32):
+            L, H = st[:, j, 0], st[:, j, 1]
+            if j % sb == 0:
+                pL = pH = np.zeros(rows, np.uint64)
+            else:
+                pL, pH = st[:, j - 1, 0], st[:, j - 1, 1]
+            got[:, 32 * j:32 * j + 32] = _codes_from_planes(_planes(L, H, pL, pH))
+        assert (got == ref).all(), seg_len

@@ -1,0 +1,114 @@
+// k_expand.cu -- HEPH's second serving mode: expand a trellis stream into packed MXFP4.
+//
+// "HEPH: 3-Bit Grid-Aligned Trellis Quantization of MXFP4 Mixture-of-Experts ..." (abstract):
+// the ~3-bpw stream can be expanded into a resident 4.25-bpw MXFP4 tensor. Each decoded weight is
+// already an E2M1 code under its block's UE8M0 scale, so expansion = decode + nibble packing, and
+// the scales are copied unchanged.
+//
+// HBM-bound streaming kernel: per 32-weight block it reads 8 bytes of stream and writes 16 bytes
+// of nibbles (plus one scale byte read and written): 0.8125 B/weight. One thread handles a pair
+// of consecutive blocks: one 16-byte load, two 16-byte stores, coalesced across the warp.
+#include "tcf4_device.cuh"
+#include "tcf4_internal.h"
+
+namespace tcf4 {
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_stream(uint4 *p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// SEG32: every block starts a segment (state 0), so no carry between blocks.
+template <bool SEG32>
+__global__ void __launch_bounds__(256) k_expand(const uint2 *__restrict__ stream, uint32_t nblocks,
+                                                uint32_t blocks_per_row, uint32_t seg_blocks,
+                                                uint4 *__restrict__ out, const uint8_t *__restrict__ scales,
+                                                uint8_t *__restrict__ out_scales, int scales_aligned16) {
+  const uint32_t pair = blockIdx.x * blockDim.x + threadIdx.x;
+  const uint32_t npairs = (nblocks + 1u) >> 1;
+  const uint32_t g0 = 2u * pair;
+  const bool valid = pair < npairs;
+  const bool has2 = g0 + 1u < nblocks;
+
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (valid) {
+    if (has2) {
+      v = ld_stream(reinterpret_cast<const uint4 *>(stream + g0));
+    } else {
+      const uint2 t = stream[g0];
+      v.x = t.x;
+      v.y = t.y;
+    }
+  }
+
+  uint32_t pL0 = 0u, pH0 = 0u, pL1 = 0u, pH1 = 0u;  // carries into blocks g0 and g0+1
+  if (!SEG32) {
+    // The predecessor of block g0 is the previous thread's second block.
+    uint32_t uL = __shfl_up_sync(0xffffffffu, v.z, 1), uH = __shfl_up_sync(0xffffffffu, v.w, 1);
+    if (valid && (g0 % blocks_per_row) % seg_blocks != 0u) {
+      if ((threadIdx.x & 31u) == 0u) {
+        const uint2 t = stream[g0 - 1u];
+        uL = t.x;
+        uH = t.y;
+      }
+      pL0 = uL;
+      pH0 = uH;
+    }
+    if (has2 && ((g0 + 1u) % blocks_per_row) % seg_blocks != 0u) {
+      pL1 = v.x;
+      pH1 = v.y;
+    }
+  }
+
+  if (valid) {
+    uint4 o;
+    planes_to_nibbles_natural(decode_block(v.x, v.y, pL0, pH0), o.x, o.y, o.z, o.w);
+    st_stream(out + g0, o);
+    if (has2) {
+      planes_to_nibbles_natural(decode_block(v.z, v.w, pL1, pH1), o.x, o.y, o.z, o.w);
+      st_stream(out + g0 + 1u, o);
+    }
+  }
+
+  // Scale bytes are copied verbatim: 16-byte chunks, then the tail byte by byte.
+  const uint32_t nchunk = scales_aligned16 ? nblocks >> 4 : 0u;
+  if (pair < nchunk) {
+    reinterpret_cast<uint4 *>(out_scales)[pair] = reinterpret_cast<const uint4 *>(scales)[pair];
+  } else {
+    const uint32_t b = (nchunk << 4) + (pair - nchunk);
+    if (b < nblocks && (scales_aligned16 ? (pair - nchunk) < 16u : true)) out_scales[b] = scales[b];
+  }
+}
+
+cudaError_t launch_expand(const MatView &w, uint8_t *out_nibbles, uint8_t *out_scales, cudaStream_t s) {
+  const uint32_t nblocks = (uint32_t)((int64_t)w.rows * w.nbr);
+  const bool aligned = ((reinterpret_cast<uintptr_t>(w.scales) | reinterpret_cast<uintptr_t>(out_scales)) & 15u) == 0;
+  const uint32_t npairs = (nblocks + 1u) / 2u;
+  // enough threads for the pairs and for every scale byte that is not in a 16-byte chunk
+  uint32_t nthreads = npairs;
+  if (aligned) {
+    nthreads = npairs > (nblocks >> 4) + 16u ? npairs : (nblocks >> 4) + 16u;
+  } else {
+    nthreads = nblocks;
+  }
+  const uint32_t grid = (nthreads + 255u) / 256u;
+  auto *out = reinterpret_cast<uint4 *>(out_nibbles);
+  if (w.seg_blocks == 1) {
+    k_expand<true><<<grid, 256, 0, s>>>(w.stream, nblocks, (uint32_t)w.nbr, 1u, out, w.scales, out_scales,
+                                        aligned ? 1 : 0);
+  } else {
+    k_expand<false><<<grid, 256, 0, s>>>(w.stream, nblocks, (uint32_t)w.nbr, (uint32_t)w.seg_blocks, out,
+                                         w.scales, out_scales, aligned ? 1 : 0);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace tcf4

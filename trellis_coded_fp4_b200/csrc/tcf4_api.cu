@@ -1,0 +1,137 @@
+// tcf4_api.cu -- the extern "C" entry points declared in include/tcf4.h.
+//
+// Validates every argument on the host before any launch, converts the public descriptors into
+// device views, and dispatches to the kernels. No allocation, no synchronisation.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tcf4.h"
+#include "tcf4_internal.h"
+
+using namespace tcf4;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tcf4_status check_matrix(const tcf4_matrix &w) {
+  if (w.rows < 0 || w.cols < 0) return TCF4_ERR_INVALID_ARG;
+  if (w.cols % 32 != 0) return TCF4_ERR_INVALID_ARG;
+  if (w.rows == 0 || w.cols == 0) return TCF4_OK;
+  if (w.stream == nullptr || w.scales == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (w.seg_len <= 0 || w.seg_len % 32 != 0 || w.cols % w.seg_len != 0) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(w.stream)) return TCF4_ERR_MISALIGNED;
+  if (w.rows > INT32_MAX || w.cols / 32 > INT32_MAX) return TCF4_ERR_UNSUPPORTED;
+  return TCF4_OK;
+}
+
+MatView view(const tcf4_matrix &w) {
+  MatView v;
+  v.stream = reinterpret_cast<const uint2 *>(w.stream);
+  v.scales = w.scales;
+  v.rows = (int32_t)w.rows;
+  v.nbr = (int32_t)(w.cols / 32);
+  v.seg_blocks = w.seg_len / 32;
+  return v;
+}
+
+tcf4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TCF4_OK : TCF4_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *tcf4_status_string(tcf4_status s) {
+  switch (s) {
+    case TCF4_OK: return "ok";
+    case TCF4_ERR_INVALID_ARG: return "invalid argument";
+    case TCF4_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case TCF4_ERR_UNSUPPORTED: return "size beyond the supported limits";
+    case TCF4_ERR_WORKSPACE: return "workspace missing or too small";
+    case TCF4_ERR_CUDA: return "CUDA launch failed";
+  }
+  return "unknown status";
+}
+
+tcf4_status trellis_decode_to_mxfp4(tcf4_matrix w, uint8_t *out_nibbles, uint8_t *out_scales, void *stream) {
+  tcf4_status st = check_matrix(w);
+  if (st != TCF4_OK) return st;
+  if (w.rows == 0 || w.cols == 0) return TCF4_OK;
+  if (out_nibbles == nullptr || out_scales == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(out_nibbles)) return TCF4_ERR_MISALIGNED;
+  if (w.rows * (w.cols / 32) >= ((int64_t)1 << 31)) return TCF4_ERR_UNSUPPORTED;
+  return from_cuda(launch_expand(view(w), out_nibbles, out_scales, static_cast<cudaStream_t>(stream)));
+}
+
+tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream) {
+  tcf4_status st = check_matrix(w);
+  if (st != TCF4_OK) return st;
+  if (T < 0) return TCF4_ERR_INVALID_ARG;
+  if (T == 0 || w.rows == 0) return TCF4_OK;
+  if (T > kMaxTokens) return TCF4_ERR_UNSUPPORTED;
+  if (w.cols == 0) return TCF4_ERR_INVALID_ARG;
+  if (w.cols > kMaxCols) return TCF4_ERR_UNSUPPORTED;
+  if (x == nullptr || y == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return TCF4_ERR_MISALIGNED;
+  return from_cuda(launch_gemv(view(w), x, T, y, static_cast<cudaStream_t>(stream)));
+}
+
+tcf4_status trellis_moe_route(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *topk_ids,
+                              float *topk_w, void *stream) {
+  if (T < 0 || k < 1 || E < k) return TCF4_ERR_INVALID_ARG;
+  if (T == 0) return TCF4_OK;
+  if (k > kMaxTopK || E > kMaxExperts || T > kMaxTokens) return TCF4_ERR_UNSUPPORTED;
+  if (logits == nullptr || topk_ids == nullptr || topk_w == nullptr) return TCF4_ERR_INVALID_ARG;
+  return from_cuda(launch_route(logits, T, E, k, topk_ids, topk_w, static_cast<cudaStream_t>(stream)));
+}
+
+static tcf4_status check_moe(const tcf4_moe *m, int32_t T, int32_t k, int *gu_seg, int *dn_seg) {
+  if (m == nullptr || m->gate_up == nullptr || m->down == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (m->E < 1 || m->H < 32 || m->I < 32 || m->H % 32 != 0 || m->I % 32 != 0) return TCF4_ERR_INVALID_ARG;
+  if (T < 0 || k < 1 || k > m->E) return TCF4_ERR_INVALID_ARG;
+  if (m->E > kMaxExperts || k > kMaxTopK || T > kMaxTokens || m->H > kMaxCols || m->I > kMaxCols)
+    return TCF4_ERR_UNSUPPORTED;
+  *gu_seg = m->gate_up[0].seg_len / 32;
+  *dn_seg = m->down[0].seg_len / 32;
+  for (int e = 0; e < m->E; e++) {
+    const tcf4_matrix &g = m->gate_up[e], &d = m->down[e];
+    if (g.rows != 2 * (int64_t)m->I || g.cols != m->H) return TCF4_ERR_INVALID_ARG;
+    if (d.rows != m->H || d.cols != m->I) return TCF4_ERR_INVALID_ARG;
+    tcf4_status s1 = check_matrix(g), s2 = check_matrix(d);
+    if (s1 != TCF4_OK) return s1;
+    if (s2 != TCF4_OK) return s2;
+    if (g.seg_len / 32 != *gu_seg || d.seg_len / 32 != *dn_seg) return TCF4_ERR_UNSUPPORTED;
+  }
+  return TCF4_OK;
+}
+
+size_t trellis_grouped_moe_workspace(const tcf4_moe *m, int32_t T, int32_t k) {
+  int a, b;
+  if (check_moe(m, T, k, &a, &b) != TCF4_OK) return 0;
+  return moe_workspace_layout(m->E, T, k, m->H, m->I).total;
+}
+
+size_t trellis_grouped_moe_hidden_offset(const tcf4_moe *m, int32_t T, int32_t k) {
+  int a, b;
+  if (check_moe(m, T, k, &a, &b) != TCF4_OK) return 0;
+  return moe_workspace_layout(m->E, T, k, m->H, m->I).hidden;
+}
+
+tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, int32_t T, const int32_t *topk_ids,
+                                const float *topk_w, int32_t k, uint16_t *out, void *workspace, size_t ws_bytes,
+                                void *stream) {
+  int gu_seg = 1, dn_seg = 1;
+  tcf4_status st = check_moe(m, T, k, &gu_seg, &dn_seg);
+  if (st != TCF4_OK) return st;
+  if (T == 0) return TCF4_OK;
+  if (x == nullptr || topk_ids == nullptr || topk_w == nullptr || out == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return TCF4_ERR_MISALIGNED;
+  const size_t need = moe_workspace_layout(m->E, T, k, m->H, m->I).total;
+  if (workspace == nullptr || ws_bytes < need) return TCF4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
+  return from_cuda(launch_moe(*m, gu_seg, dn_seg, x, T, topk_ids, topk_w, k, out, workspace,
+                              static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

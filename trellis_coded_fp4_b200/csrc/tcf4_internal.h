@@ -1,0 +1,46 @@
+// tcf4_internal.h -- launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "tcf4.h"
+
+namespace tcf4 {
+
+constexpr int kMaxExperts = 256;
+constexpr int kMaxTokens = 32;
+constexpr int kMaxTopK = 8;
+constexpr int kMaxCols = 16384;
+
+// Device-side view of one trellis-coded matrix.
+struct MatView {
+  const uint2 *stream;    // [rows][nbr] block words (lo plane, hi plane)
+  const uint8_t *scales;  // [rows][nbr]
+  int32_t rows;
+  int32_t nbr;            // blocks per row = cols / 32
+  int32_t seg_blocks;     // seg_len / 32
+};
+
+// Per-expert pointer table passed by value to the MoE kernels.
+template <int MAXE>
+struct MoeTable {
+  const uint2 *gu[MAXE];
+  const uint8_t *gus[MAXE];
+  const uint2 *dn[MAXE];
+  const uint8_t *dns[MAXE];
+};
+
+// Offsets of the MoE workspace regions (bytes, 256-aligned).
+struct MoeWorkspace {
+  size_t counts, offsets, active, list, n_active, hidden, y, total;
+};
+MoeWorkspace moe_workspace_layout(int E, int T, int k, int H, int I);
+
+cudaError_t launch_expand(const MatView &w, uint8_t *out_nibbles, uint8_t *out_scales, cudaStream_t s);
+cudaError_t launch_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s);
+cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *wts, cudaStream_t s);
+cudaError_t launch_moe(const tcf4_moe &m, int gu_seg, int dn_seg, const uint16_t *x, int T, const int32_t *ids,
+                       const float *wts, int k, uint16_t *out, void *ws, cudaStream_t s);
+
+}  // namespace tcf4
