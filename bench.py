@@ -169,9 +169,20 @@ class Step:
         self.moe_weights = K_TOP * (2 * I * H + H * I)  # distinct experts at T = 1: exactly k
         self.weights_per_step = self.nG + self.nD + self.moe_weights + self.nG + self.nD
 
-    def run(self, i, ev=None):
+    def run(self, i, ev=None, only=None):
         tc = self.tc
         v = i % len(self.x)
+        if only is not None:
+            calls = {"expand_gate_up": lambda: tc.decode_to_mxfp4(self.G, self.nibG, self.scG),
+                     "expand_down": lambda: tc.decode_to_mxfp4(self.D, self.nibD, self.scD),
+                     "route": lambda: tc.moe_route(self.logits[v], K_TOP, self.ids, self.wts),
+                     "grouped_moe": lambda: tc.grouped_moe(self.M, self.x[v], self.ids, self.wts, self.out, self.ws),
+                     "gemv_gate_up": lambda: tc.gemv(self.G, self.x[v], self.yG),
+                     "gemv_down": lambda: tc.gemv(self.D, self.xd[v], self.yD)}
+            if only == "grouped_moe":
+                calls["route"]()
+            calls[only]()
+            return
         def mark(name):
             if ev is not None:
                 e = torch.cuda.Event(enable_timing=True)
@@ -335,6 +346,8 @@ def main():
     ap.add_argument("--impl", default="tcf4", choices=["tcf4", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default=None,
+                    help="run only this call of the step (e.g. gemv_gate_up), for profiling one kernel")
     args = ap.parse_args()
     if args.impl == "reference":
         return reference_arm(args)
@@ -354,6 +367,13 @@ def main():
     build.build()
     seed = synth.SEED_BASE + 1 + rank
     step = Step(seed, device)
+    if args.only is not None:  # profiling mode: a few launches of one call, no timing line
+        for i in range(args.warmup + args.steps):
+            step.run(i, only=args.only)
+        torch.cuda.synchronize()
+        print(json.dumps({"only": args.only, "launches": args.warmup + args.steps,
+                          "timeouts": step.tc.device_timeouts()}))
+        return 0
 
     for i in range(max(args.warmup, 3)):
         step.run(i)

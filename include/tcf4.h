@@ -28,9 +28,12 @@
  * Alignment. stream, x and y pointers must be 16-byte aligned; MXFP4 outputs too.
  * Errors. Arguments are checked on the host before anything is launched: a bad argument returns
  *   TCF4_ERR_INVALID_ARG / TCF4_ERR_MISALIGNED / TCF4_ERR_UNSUPPORTED / TCF4_ERR_WORKSPACE and
- *   launches nothing. A failed launch returns TCF4_ERR_CUDA (the CUDA error is left set for the
- *   caller to read). Empty problems (rows == 0, T == 0) return TCF4_OK and launch nothing.
- * Threads. Calls are reentrant; no global state is written.
+ *   launches nothing. A valid call first clears a pending non-sticky CUDA error left by earlier
+ *   calls (cudaGetLastError), so that it is not mistaken for its own; a failed launch then returns
+ *   TCF4_ERR_CUDA with the CUDA error left set for the caller to read. Empty problems (rows == 0,
+ *   T == 0) return TCF4_OK and launch nothing.
+ * Threads. Calls are reentrant. The only process state the library writes is a one-time
+ *   per-device kernel attribute (the dynamic shared-memory limit of its kernels).
  */
 #ifndef TCF4_H
 #define TCF4_H
@@ -122,6 +125,12 @@ TCF4_API tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, i
 
 /* Byte offset of h (bf16 [T*k][I]) inside the workspace of trellis_grouped_moe. */
 TCF4_API size_t trellis_grouped_moe_hidden_offset(const tcf4_moe *m, int32_t T, int32_t k);
+
+/* Bounded waits that gave up inside the library's kernels since the last call, then resets the
+ * count. Kernels that stage weights with bulk copies wait on shared-memory barriers with an
+ * iteration limit; a wait that runs out is counted and the affected outputs are invalid. Never
+ * expected in a correct run. Synchronous: it waits for the current device's work to finish. */
+TCF4_API unsigned int tcf4_device_timeouts(void);
 
 /* A static, human-readable description of a status code. */
 TCF4_API const char *tcf4_status_string(tcf4_status s);

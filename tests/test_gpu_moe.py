@@ -77,3 +77,8 @@ def test_moe_256_experts_hidden_7168_sampled(T):
     r = np.random.default_rng(100 + T)
     check_moe(layer, W, x, ids, wts, out, ws, k, 32, rows_h=r.choice(I, 24, replace=False),
               rows_out=r.choice(H, 24, replace=False))
+
+
+def test_no_bounded_wait_gave_up():
+    # Every bulk-copy wait in the kernels above completed within its iteration limit.
+    assert tc.device_timeouts() == 0

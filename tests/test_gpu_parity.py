@@ -42,7 +42,7 @@ def test_expand_unaligned_scale_pointers():
     rows, cols = 7, 160
     st, sc, W = upload_matrix(rows, cols, seed=77)
     big = torch.zeros(rows * cols // 32 + 1, dtype=torch.uint8, device="cuda")
-    W.scales = torch.from_numpy(np.concatenate([[0], sc.ravel()])).cuda()[1:]   # odd address
+    W.scales = torch.from_numpy(np.concatenate([np.zeros(1, np.uint8), sc.ravel()])).cuda()[1:]  # odd address
     out_sc = big[1:]
     nib, _ = tc.decode_to_mxfp4(W, out_scales=out_sc)
     torch.cuda.synchronize()

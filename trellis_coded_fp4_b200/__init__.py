@@ -17,7 +17,7 @@ import torch
 from . import _abi
 
 __all__ = ["TrellisMatrix", "MoEWeights", "decode_to_mxfp4", "gemv", "moe_route", "grouped_moe",
-           "moe_workspace_bytes", "moe_hidden_offset", "Tcf4Error"]
+           "moe_workspace_bytes", "moe_hidden_offset", "device_timeouts", "Tcf4Error"]
 
 Tcf4Error = _abi.Tcf4Error
 
@@ -135,3 +135,8 @@ def grouped_moe(m: MoEWeights, x: torch.Tensor, ids: torch.Tensor, wts: torch.Te
                                                _ptr(workspace), workspace.numel(), _stream_handle()),
                "trellis_grouped_moe")
     return out, workspace
+
+
+def device_timeouts() -> int:
+    """Bounded waits that gave up in the library's kernels since the last query (synchronizes)."""
+    return int(_abi.load().tcf4_device_timeouts())

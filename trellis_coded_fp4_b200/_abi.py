@@ -11,7 +11,8 @@ STATUS_NAMES = {0: "TCF4_OK", 1: "TCF4_ERR_INVALID_ARG", 2: "TCF4_ERR_MISALIGNED
 
 # Every symbol include/tcf4.h declares.
 EXPORTED = ("trellis_decode_to_mxfp4", "trellis_gemv", "trellis_moe_route", "trellis_grouped_moe_workspace",
-            "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "tcf4_status_string")
+            "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "tcf4_device_timeouts",
+            "tcf4_status_string")
 
 
 class Matrix(ctypes.Structure):
@@ -51,6 +52,8 @@ def load(path: str = LIB_PATH):
     L.trellis_grouped_moe_hidden_offset.restype = sz
     L.trellis_grouped_moe.argtypes = [ctypes.POINTER(Moe), vp, i32, vp, vp, i32, vp, vp, sz, vp]
     L.trellis_grouped_moe.restype = ctypes.c_int
+    L.tcf4_device_timeouts.argtypes = []
+    L.tcf4_device_timeouts.restype = ctypes.c_uint
     L.tcf4_status_string.argtypes = [ctypes.c_int]
     L.tcf4_status_string.restype = ctypes.c_char_p
     _lib = L

@@ -38,6 +38,10 @@ MatView view(const tcf4_matrix &w) {
 
 tcf4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TCF4_OK : TCF4_ERR_CUDA; }
 
+// A non-sticky error left pending by earlier, unrelated CUDA calls would otherwise be reported
+// as this call's launch failure; clear it before launching (documented in tcf4.h).
+void clear_pending_error() { (void)cudaGetLastError(); }
+
 }  // namespace
 
 extern "C" {
@@ -61,6 +65,7 @@ tcf4_status trellis_decode_to_mxfp4(tcf4_matrix w, uint8_t *out_nibbles, uint8_t
   if (out_nibbles == nullptr || out_scales == nullptr) return TCF4_ERR_INVALID_ARG;
   if (!aligned16(out_nibbles)) return TCF4_ERR_MISALIGNED;
   if (w.rows * (w.cols / 32) >= ((int64_t)1 << 31)) return TCF4_ERR_UNSUPPORTED;
+  clear_pending_error();
   return from_cuda(launch_expand(view(w), out_nibbles, out_scales, static_cast<cudaStream_t>(stream)));
 }
 
@@ -74,6 +79,7 @@ tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *
   if (w.cols > kMaxCols) return TCF4_ERR_UNSUPPORTED;
   if (x == nullptr || y == nullptr) return TCF4_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return TCF4_ERR_MISALIGNED;
+  clear_pending_error();
   return from_cuda(launch_gemv(view(w), x, T, y, static_cast<cudaStream_t>(stream)));
 }
 
@@ -83,6 +89,7 @@ tcf4_status trellis_moe_route(const float *logits, int32_t T, int32_t E, int32_t
   if (T == 0) return TCF4_OK;
   if (k > kMaxTopK || E > kMaxExperts || T > kMaxTokens) return TCF4_ERR_UNSUPPORTED;
   if (logits == nullptr || topk_ids == nullptr || topk_w == nullptr) return TCF4_ERR_INVALID_ARG;
+  clear_pending_error();
   return from_cuda(launch_route(logits, T, E, k, topk_ids, topk_w, static_cast<cudaStream_t>(stream)));
 }
 
@@ -130,8 +137,14 @@ tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, int32_t T,
   const size_t need = moe_workspace_layout(m->E, T, k, m->H, m->I).total;
   if (workspace == nullptr || ws_bytes < need) return TCF4_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
+  clear_pending_error();
   return from_cuda(launch_moe(*m, gu_seg, dn_seg, x, T, topk_ids, topk_w, k, out, workspace,
                               static_cast<cudaStream_t>(stream)));
+}
+
+unsigned int tcf4_device_timeouts(void) {
+  cudaDeviceSynchronize();
+  return take_timeouts_gemv() + take_timeouts_moe();
 }
 
 }  // extern "C"

@@ -31,16 +31,41 @@ struct MoeTable {
   const uint8_t *dns[MAXE];
 };
 
-// Offsets of the MoE workspace regions (bytes, 256-aligned).
+// Offsets of the MoE workspace regions (bytes, 256-aligned): per-row-chunk counters of the down
+// kernel, h (bf16 [T*k][I]) and y (fp32 [T*k][H]).
 struct MoeWorkspace {
-  size_t counts, offsets, active, list, n_active, hidden, y, total;
+  size_t counters, hidden, y, total;
 };
 MoeWorkspace moe_workspace_layout(int E, int T, int k, int H, int I);
+
+// Allow a kernel the largest dynamic shared memory the device offers beyond its static shared
+// memory, once per device (a bit per device ordinal in `done`).
+template <class F>
+cudaError_t ensure_max_dynamic_smem(F *func, unsigned long long &done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done & bit) return cudaSuccess;
+  cudaFuncAttributes a;
+  e = cudaFuncGetAttributes(&a, func);
+  if (e != cudaSuccess) return e;
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)a.sharedSizeBytes);
+  if (e == cudaSuccess) done |= bit;
+  return e;
+}
 
 cudaError_t launch_expand(const MatView &w, uint8_t *out_nibbles, uint8_t *out_scales, cudaStream_t s);
 cudaError_t launch_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s);
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *wts, cudaStream_t s);
 cudaError_t launch_moe(const tcf4_moe &m, int gu_seg, int dn_seg, const uint16_t *x, int T, const int32_t *ids,
                        const float *wts, int k, uint16_t *out, void *ws, cudaStream_t s);
+
+// Read and clear the bounded-wait timeout counters of the kernel files.
+unsigned int take_timeouts_gemv();
+unsigned int take_timeouts_moe();
 
 }  // namespace tcf4
