@@ -164,6 +164,8 @@ class Step:
         self.ids = torch.empty((T, K_TOP), dtype=torch.int32, device=device)
         self.wts = torch.empty((T, K_TOP), dtype=torch.float32, device=device)
         self.ws = torch.empty(self.M.workspace_bytes(T, K_TOP), dtype=torch.uint8, device=device)
+        self.wsG = torch.empty(max(1, tc.gemv_workspace_bytes(self.G, T)), dtype=torch.uint8, device=device)
+        self.wsD = torch.empty(max(1, tc.gemv_workspace_bytes(self.D, T)), dtype=torch.uint8, device=device)
         self.launches_per_step = 2 + 1 + 4 + 2
         self.nG, self.nD = E * 2 * I * H, E * H * I
         self.moe_weights = K_TOP * (2 * I * H + H * I)  # distinct experts at T = 1: exactly k
@@ -177,8 +179,8 @@ class Step:
                      "expand_down": lambda: tc.decode_to_mxfp4(self.D, self.nibD, self.scD),
                      "route": lambda: tc.moe_route(self.logits[v], K_TOP, self.ids, self.wts),
                      "grouped_moe": lambda: tc.grouped_moe(self.M, self.x[v], self.ids, self.wts, self.out, self.ws),
-                     "gemv_gate_up": lambda: tc.gemv(self.G, self.x[v], self.yG),
-                     "gemv_down": lambda: tc.gemv(self.D, self.xd[v], self.yD)}
+                     "gemv_gate_up": lambda: tc.gemv(self.G, self.x[v], self.yG, self.wsG),
+                     "gemv_down": lambda: tc.gemv(self.D, self.xd[v], self.yD, self.wsD)}
             if only == "grouped_moe":
                 calls["route"]()
             calls[only]()
@@ -197,9 +199,9 @@ class Step:
         mark("grouped_moe")
         tc.grouped_moe(self.M, self.x[v], self.ids, self.wts, self.out, self.ws)
         mark("gemv_gate_up")
-        tc.gemv(self.G, self.x[v], self.yG)
+        tc.gemv(self.G, self.x[v], self.yG, self.wsG)
         mark("gemv_down")
-        tc.gemv(self.D, self.xd[v], self.yD)
+        tc.gemv(self.D, self.xd[v], self.yD, self.wsD)
         mark("end")
 
     # algorithmic bytes per call (what the method must move)

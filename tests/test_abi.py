@@ -46,18 +46,23 @@ def _mat(stream=16, scales=16, rows=4, cols=64, seg=32):
 def test_gemv_argument_checks(lib):
     ok_x, ok_y = ctypes.c_void_p(4096), ctypes.c_void_p(8192)
     s0 = ctypes.c_void_p(0)
-    assert lib.trellis_gemv(_mat(cols=48), ok_x, 1, ok_y, s0) == 1          # cols % 32
-    assert lib.trellis_gemv(_mat(seg=48), ok_x, 1, ok_y, s0) == 1           # seg_len % 32
-    assert lib.trellis_gemv(_mat(seg=96), ok_x, 1, ok_y, s0) == 1           # seg_len does not divide cols
-    assert lib.trellis_gemv(_mat(stream=0), ok_x, 1, ok_y, s0) == 1         # null stream
-    assert lib.trellis_gemv(_mat(stream=8), ok_x, 1, ok_y, s0) == 2         # misaligned stream
-    assert lib.trellis_gemv(_mat(), ctypes.c_void_p(4098), 1, ok_y, s0) == 2
-    assert lib.trellis_gemv(_mat(), ok_x, 33, ok_y, s0) == 3                # T > 32
-    assert lib.trellis_gemv(_mat(), ok_x, -1, ok_y, s0) == 1
-    assert lib.trellis_gemv(_mat(), ok_x, 0, ok_y, s0) == 0                 # empty: no launch
-    assert lib.trellis_gemv(_mat(rows=0), ok_x, 1, ok_y, s0) == 0
-    assert lib.trellis_gemv(_mat(cols=32768, seg=32), ok_x, 1, ok_y, s0) == 3
-    assert lib.trellis_gemv(_mat(), ctypes.c_void_p(0), 1, ok_y, s0) == 1
+    ws0 = ctypes.c_void_p(0)
+
+    def gemv(w, x, T, y):  # these checks never reach a launch, so no workspace is involved
+        return lib.trellis_gemv(w, x, T, y, ws0, 0, s0)
+
+    assert gemv(_mat(cols=48), ok_x, 1, ok_y) == 1          # cols % 32
+    assert gemv(_mat(seg=48), ok_x, 1, ok_y) == 1           # seg_len % 32
+    assert gemv(_mat(seg=96), ok_x, 1, ok_y) == 1           # seg_len does not divide cols
+    assert gemv(_mat(stream=0), ok_x, 1, ok_y) == 1         # null stream
+    assert gemv(_mat(stream=8), ok_x, 1, ok_y) == 2         # misaligned stream
+    assert gemv(_mat(), ctypes.c_void_p(4098), 1, ok_y) == 2
+    assert gemv(_mat(), ok_x, 33, ok_y) == 3                # T > 32
+    assert gemv(_mat(), ok_x, -1, ok_y) == 1
+    assert gemv(_mat(), ok_x, 0, ok_y) == 0                 # empty: no launch
+    assert gemv(_mat(rows=0), ok_x, 1, ok_y) == 0
+    assert gemv(_mat(cols=32768, seg=32), ok_x, 1, ok_y) == 3
+    assert gemv(_mat(), ctypes.c_void_p(0), 1, ok_y) == 1
 
 
 def test_expand_and_route_argument_checks(lib):

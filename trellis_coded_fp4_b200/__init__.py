@@ -16,7 +16,8 @@ import torch
 
 from . import _abi
 
-__all__ = ["TrellisMatrix", "MoEWeights", "decode_to_mxfp4", "gemv", "moe_route", "grouped_moe",
+__all__ = ["TrellisMatrix", "MoEWeights", "decode_to_mxfp4", "gemv", "gemv_workspace_bytes", "moe_route",
+           "grouped_moe",
            "moe_workspace_bytes", "moe_hidden_offset", "device_timeouts", "Tcf4Error"]
 
 Tcf4Error = _abi.Tcf4Error
@@ -60,13 +61,23 @@ def decode_to_mxfp4(w: TrellisMatrix, out_nibbles=None, out_scales=None):
     return out_nibbles, out_scales
 
 
-def gemv(w: TrellisMatrix, x: torch.Tensor, out=None):
+def gemv_workspace_bytes(w: TrellisMatrix, T: int) -> int:
+    """Scratch bytes trellis_gemv needs for T tokens (0: the call needs none)."""
+    return int(_abi.load().trellis_gemv_workspace(w.abi(), T))
+
+
+def gemv(w: TrellisMatrix, x: torch.Tensor, out=None, workspace=None):
     """y = bf16(W x) for bf16 activations x [T][cols] (T <= 32): returns bf16 [T][rows]."""
     x = x if x.dim() == 2 else x.view(1, -1)
     T = x.shape[0]
     if out is None:
         out = torch.empty((T, w.rows), dtype=torch.bfloat16, device=x.device)
-    _abi.check(_abi.load().trellis_gemv(w.abi(), _ptr(x), T, _ptr(out), _stream_handle()), "trellis_gemv")
+    need = gemv_workspace_bytes(w, T)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    nbytes = workspace.numel() if workspace is not None else 0
+    _abi.check(_abi.load().trellis_gemv(w.abi(), _ptr(x), T, _ptr(out), _ptr(workspace), nbytes, _stream_handle()),
+               "trellis_gemv")
     return out
 
 

@@ -69,7 +69,7 @@ tcf4_status trellis_decode_to_mxfp4(tcf4_matrix w, uint8_t *out_nibbles, uint8_t
   return from_cuda(launch_expand(view(w), out_nibbles, out_scales, static_cast<cudaStream_t>(stream)));
 }
 
-tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream) {
+static tcf4_status check_gemv(const tcf4_matrix &w, int32_t T) {
   tcf4_status st = check_matrix(w);
   if (st != TCF4_OK) return st;
   if (T < 0) return TCF4_ERR_INVALID_ARG;
@@ -77,10 +77,36 @@ tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *
   if (T > kMaxTokens) return TCF4_ERR_UNSUPPORTED;
   if (w.cols == 0) return TCF4_ERR_INVALID_ARG;
   if (w.cols > kMaxCols) return TCF4_ERR_UNSUPPORTED;
+  return TCF4_OK;
+}
+
+// The tensor-core path runs whenever it applies (seg_len 32, see gemv_mma_supported); it needs
+// the workspace for the activation split. Other shapes run the CUDA-core kernel without one.
+static bool gemv_uses_mma(const tcf4_matrix &w, int32_t T) {
+  return w.seg_len == 32 && w.rows > 0 && T > 0 && gemv_mma_supported(view(w), T);
+}
+
+size_t trellis_gemv_workspace(tcf4_matrix w, int32_t T) {
+  if (check_gemv(w, T) != TCF4_OK || T == 0 || w.rows == 0) return 0;
+  return gemv_uses_mma(w, T) ? gemv_mma_workspace(view(w), T) : 0;
+}
+
+tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *workspace,
+                         size_t ws_bytes, void *stream) {
+  tcf4_status st = check_gemv(w, T);
+  if (st != TCF4_OK) return st;
+  if (T == 0 || w.rows == 0) return TCF4_OK;
   if (x == nullptr || y == nullptr) return TCF4_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return TCF4_ERR_MISALIGNED;
+  const MatView v = view(w);
+  if (gemv_uses_mma(w, T)) {
+    if (workspace == nullptr || ws_bytes < gemv_mma_workspace(v, T)) return TCF4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
+    clear_pending_error();
+    return from_cuda(launch_gemv_mma(v, x, T, y, workspace, static_cast<cudaStream_t>(stream)));
+  }
   clear_pending_error();
-  return from_cuda(launch_gemv(view(w), x, T, y, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_gemv(v, x, T, y, static_cast<cudaStream_t>(stream)));
 }
 
 tcf4_status trellis_moe_route(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *topk_ids,
@@ -144,7 +170,7 @@ tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, int32_t T,
 
 unsigned int tcf4_device_timeouts(void) {
   cudaDeviceSynchronize();
-  return take_timeouts_gemv() + take_timeouts_moe();
+  return take_timeouts_gemv() + take_timeouts_moe() + take_timeouts_mma();
 }
 
 }  // extern "C"

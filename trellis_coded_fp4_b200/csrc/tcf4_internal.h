@@ -64,8 +64,14 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids,
 cudaError_t launch_moe(const tcf4_moe &m, int gu_seg, int dn_seg, const uint16_t *x, int T, const int32_t *ids,
                        const float *wts, int k, uint16_t *out, void *ws, cudaStream_t s);
 
+// Tensor-core fused decode GEMV (k_mma.cu): whether it applies, its workspace, its launch.
+bool gemv_mma_supported(const MatView &w, int T);
+size_t gemv_mma_workspace(const MatView &w, int T);
+cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s);
+
 // Read and clear the bounded-wait timeout counters of the kernel files.
 unsigned int take_timeouts_gemv();
 unsigned int take_timeouts_moe();
+unsigned int take_timeouts_mma();
 
 }  // namespace tcf4

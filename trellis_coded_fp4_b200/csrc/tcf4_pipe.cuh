@@ -11,7 +11,10 @@
 
 namespace tcf4 {
 
-constexpr uint32_t kSpinLimit = 1u << 24;  // try_wait rounds before a wait is declared stuck
+// A wait gives up after kSpinLimit rounds of try_wait, each suspending for at most ~kSuspendNs:
+// about two seconds, far beyond any real wait (microseconds).
+constexpr uint32_t kSpinLimit = 1u << 20;
+constexpr uint32_t kSuspendNs = 2000u;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -34,10 +37,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
