@@ -79,6 +79,19 @@ def test_moe_256_experts_hidden_7168_sampled(T):
               rows_out=r.choice(H, 24, replace=False))
 
 
+def test_moe_tensor_core_path_many_tokens_per_expert():
+    # K = 1024 takes the tensor-core path; 20 tokens on each of two experts split into groups of 16
+    # and 4 columns pairs of the MMA.
+    E, H, I, k, T = 8, 1024, 1024, 2, 20
+    layer = synth.moe_layer(E, H, I, seed=4300)
+    ids = torch.tensor([[1, 5]] * T, dtype=torch.int32).cuda()
+    wts = torch.rand(T, k, generator=torch.Generator().manual_seed(4300)).cuda()
+    W, x, ids, wts, out, ws = _run(layer, T, k, 4300, ids=ids, wts=wts)
+    r = np.random.default_rng(4300)
+    check_moe(layer, W, x, ids, wts, out, ws, k, 32, rows_h=r.choice(I, 64, replace=False),
+              rows_out=r.choice(H, 64, replace=False))
+
+
 def test_no_bounded_wait_gave_up():
     # Every bulk-copy wait in the kernels above completed within its iteration limit.
     assert tc.device_timeouts() == 0

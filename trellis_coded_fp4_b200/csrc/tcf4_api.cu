@@ -139,15 +139,23 @@ static tcf4_status check_moe(const tcf4_moe *m, int32_t T, int32_t k, int *gu_se
   return TCF4_OK;
 }
 
+// The tensor-core MoE runs whenever it applies (see moe_mma_supported); otherwise the CUDA-core
+// kernels do. The workspace layout follows the path.
+static bool moe_uses_mma(const tcf4_moe *m, int gu_seg, int dn_seg, int32_t T) {
+  return T > 0 && moe_mma_supported(*m, gu_seg, dn_seg, T);
+}
+
 size_t trellis_grouped_moe_workspace(const tcf4_moe *m, int32_t T, int32_t k) {
   int a, b;
   if (check_moe(m, T, k, &a, &b) != TCF4_OK) return 0;
+  if (moe_uses_mma(m, a, b, T)) return moe_mma_workspace_layout(*m, T, k).total;
   return moe_workspace_layout(m->E, T, k, m->H, m->I).total;
 }
 
 size_t trellis_grouped_moe_hidden_offset(const tcf4_moe *m, int32_t T, int32_t k) {
   int a, b;
   if (check_moe(m, T, k, &a, &b) != TCF4_OK) return 0;
+  if (moe_uses_mma(m, a, b, T)) return moe_mma_workspace_layout(*m, T, k).hidden;
   return moe_workspace_layout(m->E, T, k, m->H, m->I).hidden;
 }
 
@@ -160,10 +168,13 @@ tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, int32_t T,
   if (T == 0) return TCF4_OK;
   if (x == nullptr || topk_ids == nullptr || topk_w == nullptr || out == nullptr) return TCF4_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out)) return TCF4_ERR_MISALIGNED;
-  const size_t need = moe_workspace_layout(m->E, T, k, m->H, m->I).total;
+  const bool mma = moe_uses_mma(m, gu_seg, dn_seg, T);
+  const size_t need = mma ? moe_mma_workspace_layout(*m, T, k).total : moe_workspace_layout(m->E, T, k, m->H, m->I).total;
   if (workspace == nullptr || ws_bytes < need) return TCF4_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
   clear_pending_error();
+  if (mma)
+    return from_cuda(launch_moe_mma(*m, x, T, topk_ids, topk_w, k, out, workspace, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_moe(*m, gu_seg, dn_seg, x, T, topk_ids, topk_w, k, out, workspace,
                               static_cast<cudaStream_t>(stream)));
 }

@@ -59,12 +59,15 @@ __device__ __forceinline__ Planes decode_block0(uint32_t L, uint32_t H) {
   return decode_block(L, H, 0u, 0u);
 }
 
-// Exchange the bits of a selected by (m << s) with the bits of b selected by m.
+// Exchange the bits of a selected by (M << S) with the bits of b selected by M, as two bit selects
+// (two shifts and two three-input logic ops).
 template <int S, uint32_t M>
 __device__ __forceinline__ void delta_swap(uint32_t &a, uint32_t &b) {
-  const uint32_t t = ((a >> S) ^ b) & M;
-  b ^= t;
-  a ^= t << S;
+  const uint32_t a_sh = a >> S, b_sh = b << S;
+  const uint32_t nb = (b & ~M) | (a_sh & M);
+  const uint32_t na = (a & ~(M << S)) | (b_sh & (M << S));
+  a = na;
+  b = nb;
 }
 
 // Planes -> four nibble words in "interleaved" order: word j, nibble v holds the code of weight
