@@ -217,7 +217,7 @@ __host__ __device__ inline MmaGeom mma_geom(int nbr, int NMAX, int mode) {
   g.off_U = g.off_X + kNA * 1024u;
   g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)(NMAX / 2) * 4u : 0u);
   g.off_S = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
-  g.slab = round_up(128u * (uint32_t)nbr, 16u);
+  g.slab = round_up(128u * (uint32_t)nbr + 16u, 16u);  // +16: tail reads of a row's 4 scale bytes
   g.smem = g.off_S + 2u * g.slab;
   return g;
 }
@@ -230,6 +230,12 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
 
 __device__ __forceinline__ void sts_u2(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 __device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t a) {
@@ -380,29 +386,37 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_mma(const __grid_constant__ 
   if (warp < 8) {
     // ---------------------------------------------------------------- decode warps
     const int sp = warp & 3, h = warp >> 2, m = 32 * sp + lane;
-    const uint32_t cbase = smem_u32(smem + geo.off_C), fbase = smem_u32(smem + geo.off_F);
+    const uint32_t cbase = smem_u32(smem + geo.off_C) + (uint32_t)tid * 32u;
+    const uint32_t fbase = smem_u32(smem + geo.off_F) + (uint32_t)tid * 16u;
     const uint32_t xbase = smem_u32(smem + geo.off_X);
-    // the prefetch front: job jl_i, stage s_i
+    const uint32_t sbase = smem_u32(smem + geo.off_S);
+    const int tail_blocks = nbr - 8 * (S - 1) - 4 * h;  // this thread's blocks in the last stage
+    const uint32_t tail = tail_blocks <= 0 ? 0u : (tail_blocks >= 4 ? 32u : 8u * (uint32_t)tail_blocks);
+
+    // Prefetch front: job jl_i, stage s_i; src walks this thread's row 64 bytes per stage.
     int jl_i = 0, s_i = 0;
-    JobRows ji = my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)) : JobRows{};
-    auto issue_next = [&](int q) {
-      if (q < nq) {
-        const int kb0 = 8 * s_i + 4 * h;
-        int nbv = nbr - kb0;
-        nbv = nbv < 0 ? 0 : (nbv > 4 ? 4 : nbv);
-        const bool valid = row_valid(ji, m);
-        const uint32_t bytes = valid ? (uint32_t)nbv * 8u : 0u;
-        const uint2 *src = a.w.stream;
-        if (bytes) src = (ji.split && m >= 64 ? ji.st1 + (size_t)(m - 64) * nbr : ji.st0 + (size_t)m * nbr) + kb0;
-        if (src == nullptr) src = reinterpret_cast<const uint2 *>(a.Bg);  // never read: 0 bytes
-        const uint32_t dst = cbase + (uint32_t)((q % kPref) * kDec + tid) * 32u;
-        cp_async16(dst, src, bytes > 16u ? 16u : bytes);
-        cp_async16(dst + 16u, bytes > 16u ? src + 2 : src, bytes > 16u ? bytes - 16u : 0u);
-        if (warp < 4)
-          cp_async16(fbase + (uint32_t)((q % kPref) * 128 + tid) * 16u,
-                     a.Bsf + (size_t)ji.group * bsf_group_words(S) + ((size_t)s_i * 32 + lane) * 4, 16u);
+    const uint2 *src_i = a.w.stream;
+    bool rv_i = false;
+    const uint32_t *bsf_i = a.Bsf;
+    JobRows ji{};
+    auto start_job_front = [&]() {
+      ji = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_i));
+      rv_i = row_valid(ji, m);
+      src_i = rv_i ? (ji.split && m >= 64 ? ji.st1 + (size_t)(m - 64) * nbr : ji.st0 + (size_t)m * nbr) + 4 * h
+                   : a.w.stream;
+      bsf_i = a.Bsf + (size_t)ji.group * bsf_group_words(S) + (size_t)lane * 4;
+    };
+    if (my_jobs) start_job_front();
+    uint32_t slot_i = 0;  // ring slot of the front (q % kPref)
+    auto issue_next = [&](bool live) {
+      if (live) {
+        const uint32_t bytes = rv_i ? (s_i == S - 1 ? tail : 32u) : 0u;
+        const uint32_t dst = cbase + slot_i * (uint32_t)(kDec * 32);
+        cp_async16(dst, src_i, bytes > 16u ? 16u : bytes);
+        cp_async16(dst + 16u, bytes > 16u ? src_i + 2 : src_i, bytes > 16u ? bytes - 16u : 0u);
+        if (warp < 4) cp_async16(fbase + slot_i * (128u * 16u), bsf_i, 16u);
         if (s_i == 0) {  // the job's scale bytes, into slab buffer jl_i % 2
-          const uint32_t sdst = smem_u32(smem + geo.off_S + (uint32_t)(jl_i & 1) * geo.slab);
+          const uint32_t sdst = sbase + (uint32_t)(jl_i & 1) * geo.slab;
           const uint32_t t0 = (uint32_t)ji.na * (uint32_t)nbr;
           for (uint32_t c = tid; c * 16u < t0; c += kDec)
             cp_async16(sdst + c * 16u, ji.sc0 + c * 16u, t0 - c * 16u < 16u ? t0 - c * 16u : 16u);
@@ -412,20 +426,22 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_mma(const __grid_constant__ 
               cp_async16(sdst + o1 + c * 16u, ji.sc1 + c * 16u, t1 - c * 16u < 16u ? t1 - c * 16u : 16u);
           }
         }
+        src_i += 8;
+        bsf_i += 32 * 4;
         if (++s_i == S) {
           s_i = 0;
-          if (++jl_i < my_jobs) ji = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_i));
+          if (++jl_i < my_jobs) start_job_front();
         }
+        slot_i = (slot_i + 1) & (kPref - 1);
       }
       cp_async_commit();
     };
 
-    // scale factors of stage qp into TMEM (warps 0-3), then release the stage to the MMA
-    auto publish_scales = [&](int qp, const uint4 &sfb) {
-      const int bp = qp % kNA;
+    // scale factors of the stage in A buffer bp into TMEM (warps 0-3), then release it to the MMA
+    auto publish_scales = [&](uint32_t bp, const uint4 &sfb) {
       const uint32_t lane_addr = tbase + ((uint32_t)(32 * warp) << 16);
-      const uint4 x0 = lds_u4(xbase + (uint32_t)bp * 1024u + (uint32_t)lane * 32u);
-      const uint4 x1 = lds_u4(xbase + (uint32_t)bp * 1024u + (uint32_t)lane * 32u + 16u);
+      const uint4 x0 = lds_u4(xbase + bp * 1024u + (uint32_t)lane * 32u);
+      const uint4 x1 = lds_u4(xbase + bp * 1024u + (uint32_t)lane * 32u + 16u);
       const uint32_t w8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
       tmem_st_x8(lane_addr + kSfaCol + 8u * bp, w8);
       tmem_st_x4(lane_addr + kSfbCol + 4u * bp, sfb.x, sfb.y, sfb.z, sfb.w);
@@ -501,67 +517,59 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_mma(const __grid_constant__ 
       }
     };
 
-    for (int q = 0; q < kPref; q++) issue_next(q);
+    for (int q = 0; q < kPref; q++) issue_next(q < nq);
     uint4 sfb_prev = make_uint4(0u, 0u, 0u, 0u);
     int jl = 0, s = 0, q = 0;
-    JobRows jc = my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)) : JobRows{};
+    uint32_t b = 0, bprev = kNA - 1, empty_phase = 0u, slot = 0;  // A buffer, previous, a_empty parities
+    uint32_t srow = sbase + (uint32_t)m * (uint32_t)nbr + 4u * (uint32_t)h;  // this row's scale bytes, job 0
     for (; q < nq; q++) {
-      const int b = q % kNA;
       cp_async_wait<kPref - 1>();
       named_bar(1, kDec);
       if (*abort_flag) break;
-      if (warp < 4 && q >= 1) publish_scales(q - 1, sfb_prev);
-      const uint32_t cslot = cbase + (uint32_t)((q % kPref) * kDec + tid) * 32u;
-      const uint4 c0 = lds_u4(cslot), c1 = lds_u4(cslot + 16u);
-      if (warp < 4) sfb_prev = lds_u4(fbase + (uint32_t)((q % kPref) * 128 + tid) * 16u);
-      // this row's 4 scale bytes of the stage, from the job's slab
-      uint32_t sfw = 0u;
-      {
-        const uint32_t sb = smem_u32(smem + geo.off_S + (uint32_t)(jl & 1) * geo.slab);
-        const bool valid = row_valid(jc, m);
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-          const int jb = 8 * s + 4 * h + i;
-          const uint32_t byte = (valid && jb < nbr) ? lds_u8(sb + (uint32_t)(m * nbr + jb)) : 127u;
-          sfw |= byte << (8 * i);
-        }
-      }
-      issue_next(q + kPref);
+      if (warp < 4 && q >= 1) publish_scales(bprev, sfb_prev);
+      const uint4 c0 = lds_u4(cbase + slot * (uint32_t)(kDec * 32)), c1 = lds_u4(cbase + slot * (uint32_t)(kDec * 32) + 16u);
+      if (warp < 4) sfb_prev = lds_u4(fbase + slot * (128u * 16u));
+      // this row's 4 scale bytes of the stage (two 16-bit reads of the job's slab)
+      const uint32_t sa = srow + (uint32_t)(jl & 1) * geo.slab + 8u * (uint32_t)s;
+      const uint32_t sfw = lds_u16(sa) | (lds_u16(sa + 2u) << 16);
+      issue_next(q + kPref < nq);
       uint32_t W[4][4];
       planes_to_nibbles_interleaved(decode_block0(c0.x, c0.y), W[0][0], W[0][1], W[0][2], W[0][3]);
       planes_to_nibbles_interleaved(decode_block0(c0.z, c0.w), W[1][0], W[1][1], W[1][2], W[1][3]);
       planes_to_nibbles_interleaved(decode_block0(c1.x, c1.y), W[2][0], W[2][1], W[2][2], W[2][3]);
       planes_to_nibbles_interleaved(decode_block0(c1.z, c1.w), W[3][0], W[3][1], W[3][2], W[3][3]);
-      const uint32_t u = (uint32_t)(q / kNA);
-      if (u >= 1) {
-        if (lane == 0 && !mbar_wait(&a_empty[b], (u - 1u) & 1u, tmo)) *abort_flag = 1;
+      if (q >= kNA) {
+        if (lane == 0 && !mbar_wait(&a_empty[b], (empty_phase >> b) & 1u, tmo)) *abort_flag = 1;
+        empty_phase ^= 1u << b;
         __syncwarp();
       }
-      const uint32_t abase = smem_u32(smem + geo.off_A + (uint32_t)b * 128u * kKS) + (uint32_t)(m >> 3) * kSboA +
-                             (uint32_t)(m & 7) * 16u;
+      const uint32_t abase = smem_u32(smem + geo.off_A) + b * (128u * kKS) + (uint32_t)(m >> 3) * kSboA +
+                             (uint32_t)(m & 7) * 16u + (uint32_t)h * 1024u;
 #pragma unroll
       for (int i = 0; i < 4; i++) {
-        const uint32_t chunk = 2u * (uint32_t)(4 * h + i);
-        sts_u2(abase + chunk * 128u, W[i][0], W[i][1]);
-        sts_u2(abase + (chunk + 1u) * 128u, W[i][2], W[i][3]);
+        sts_u2(abase + (uint32_t)(2 * i) * 128u, W[i][0], W[i][1]);
+        sts_u2(abase + (uint32_t)(2 * i + 1) * 128u, W[i][2], W[i][3]);
       }
       // scale word of row m (row group sp), K-blocks 4h..4h+3 -> staging word 4h+sp of this lane
-      sts_u32(xbase + (uint32_t)b * 1024u + (uint32_t)lane * 32u + (uint32_t)(4 * h + sp) * 4u, sfw);
+      sts_u32(xbase + b * 1024u + (uint32_t)lane * 32u + (uint32_t)(4 * h + sp) * 4u, sfw);
       fence_proxy_async_smem();
       if (warp >= 4) {  // warps 4-7 release the stage now; warps 0-3 after its scales are in TMEM
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[b]);
       }
       if (warp < 4 && jl >= 1 && s == 1) epilogue(jl - 1);
+      bprev = b;
+      b = b + 1 == kNA ? 0u : b + 1;
+      slot = (slot + 1) & (kPref - 1);
       if (++s == S) {
         s = 0;
-        if (++jl < my_jobs) jc = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl));
+        ++jl;
       }
     }
     if (q == nq && nq > 0) {
       named_bar(1, kDec);  // the last stage's scale staging is complete
       if (warp < 4) {
-        publish_scales(nq - 1, sfb_prev);
+        publish_scales(bprev, sfb_prev);
         epilogue(my_jobs - 1);
       }
     }
@@ -571,57 +579,82 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_mma(const __grid_constant__ 
     if (lane == 0) {
       const uint32_t bstage = (uint32_t)NMAX * kKS;
       int jl_b = 0, s_b = 0;
-      int grp_b = my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).group : 0;
-      auto issue_b = [&](int qb) {  // B stage of the prefetch front (jl_b, s_b)
-        if (qb < nq) {
-          const int bb = qb % kNB;
-          mbar_arrive_expect_tx(&b_full[bb], bstage);
-          bulk_g2s(smem + geo.off_B + (uint32_t)bb * bstage,
-                   a.Bg + (size_t)grp_b * bsplit_group_bytes(S, NMAX) + (size_t)s_b * bstage, bstage, &b_full[bb]);
-          if (++s_b == S) {
-            s_b = 0;
-            if (++jl_b < my_jobs) grp_b = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_b)).group;
-          }
-        }
+      const uint8_t *bsrc = a.Bg;
+      auto front_group = [&]() {
+        bsrc = a.Bg + (size_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_b)).group * bsplit_group_bytes(S, NMAX);
       };
-      for (int qb = 0; qb < kNB; qb++) issue_b(qb);
+      if (my_jobs) front_group();
+      uint32_t bb_i = 0;
+      auto issue_b = [&]() {  // B stage of the prefetch front (jl_b, s_b) into ring slot bb_i
+        mbar_arrive_expect_tx(&b_full[bb_i], bstage);
+        bulk_g2s(smem + geo.off_B + bb_i * bstage, bsrc, bstage, &b_full[bb_i]);
+        bsrc += bstage;
+        if (++s_b == S) {
+          s_b = 0;
+          if (++jl_b < my_jobs) front_group();
+        }
+        bb_i = bb_i + 1 == kNB ? 0u : bb_i + 1;
+      };
+      int issued_b = 0;
+      for (; issued_b < kNB && issued_b < nq; issued_b++) issue_b();
+      // instruction descriptors for the four scale-factor byte positions
       int jl = 0, s = 0;
-      JobRows jc = my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)) : JobRows{};
+      uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : NMAX);
+      uint32_t idesc[4];
+      for (int i = 0; i < 4; i++) idesc[i] = idesc_mxf8f6f4_e2m1_e4m3(ncols, (uint32_t)i, (uint32_t)i);
+      uint32_t b = 0, bb = 0, full_phase = 0u, bfull_phase = 0u, bempty_phase = 0u, acc_phase = 0u;
+      const uint32_t a0 = smem_u32(smem + geo.off_A), b0 = smem_u32(smem + geo.off_B);
       for (int q = 0; q < nq; q++) {
-        const int b = q % kNA, bb = q % kNB;
-        bool ok = mbar_wait(&a_full[b], (uint32_t)(q / kNA) & 1u, tmo);
-        ok = ok && mbar_wait(&b_full[bb], (uint32_t)(q / kNB) & 1u, tmo);
-        if (ok && s == 0 && jl >= 2) ok = mbar_wait(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo);
+        bool ok = mbar_wait(&a_full[b], (full_phase >> b) & 1u, tmo);
+        full_phase ^= 1u << b;
+        ok = ok && mbar_wait(&b_full[bb], (bfull_phase >> bb) & 1u, tmo);
+        bfull_phase ^= 1u << bb;
+        if (ok && s == 0 && jl >= 2) {
+          ok = mbar_wait(&acc_empty[jl & 1], (acc_phase >> (jl & 1)) & 1u, tmo);
+          acc_phase ^= 1u << (jl & 1);
+        }
         if (!ok) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
         const int nkb = nbr - 8 * s < 8 ? nbr - 8 * s : 8;
-        const uint32_t a_s = smem_u32(smem + geo.off_A + (uint32_t)b * 128u * kKS);
-        const uint32_t b_s = smem_u32(smem + geo.off_B + (uint32_t)bb * bstage);
+        uint64_t ad = smem_desc(a0 + b * (128u * kKS), 128u, kSboA);
+        uint64_t bd = smem_desc(b0 + bb * (uint32_t)NMAX * kKS, 128u, kSboA);
         const uint32_t d_t = tbase + (uint32_t)((jl & 1) * NMAX);
+        const uint32_t sfa0 = tbase + kSfaCol + 8u * b, sfb0 = tbase + kSfbCol + 4u * b;
         for (int kb = 0; kb < nkb; kb++) {
-          const uint64_t ad = smem_desc(a_s + 256u * kb, 128u, kSboA);
-          const uint64_t bd = smem_desc(b_s + 256u * kb, 128u, kSboA);
-          const uint32_t id = idesc_mxf8f6f4_e2m1_e4m3((uint32_t)jc.ncols, (uint32_t)(kb & 3), (uint32_t)(kb & 3));
-          const uint32_t sfa_t = (tbase + kSfaCol + 8u * b + 4u * (uint32_t)(kb >> 2)) | ((uint32_t)(kb & 3) << 30);
-          const uint32_t sfb_t = (tbase + kSfbCol + 4u * b + 2u * (uint32_t)(kb >> 2)) | ((uint32_t)(kb & 3) << 30);
-          mma_mxf8f6f4(d_t, ad, bd, id, sfa_t, sfb_t, !(s == 0 && kb == 0));
+          const uint32_t byte = (uint32_t)(kb & 3) << 30;
+          mma_mxf8f6f4(d_t, ad, bd, idesc[kb & 3], (sfa0 + 4u * (uint32_t)(kb >> 2)) | byte,
+                       (sfb0 + 2u * (uint32_t)(kb >> 2)) | byte, !(s == 0 && kb == 0));
+          ad += 16u;  // +256 bytes (descriptor start address counts 16-byte units)
+          bd += 16u;
         }
         tc_commit(&a_empty[b]);
         tc_commit(&b_empty[bb]);
         if (s == S - 1) tc_commit(&acc_full[jl & 1]);
-        if (q >= 1 && q - 1 + kNB < nq) {
-          if (!mbar_wait(&b_empty[(q - 1) % kNB], (uint32_t)((q - 1) / kNB) & 1u, tmo)) {
+        // refill the B slot of stage q-1 once its MMAs are done (stage q-1+kNB)
+        if (q >= 1 && issued_b < nq) {
+          const uint32_t pb = bb == 0 ? kNB - 1 : bb - 1;
+          if (!mbar_wait(&b_empty[pb], (bempty_phase >> pb) & 1u, tmo)) {
             *abort_flag = 1;
             break;
           }
-          issue_b(q - 1 + kNB);
+          bempty_phase ^= 1u << pb;
+          issue_b();
+          issued_b++;
         }
+        b = b + 1 == kNA ? 0u : b + 1;
+        bb = bb + 1 == kNB ? 0u : bb + 1;
         if (++s == S) {
           s = 0;
-          if (++jl < my_jobs) jc = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl));
+          if (++jl < my_jobs) {
+            const uint32_t nc = (uint32_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl)).ncols;
+            if (nc != ncols) {
+              ncols = nc;
+              for (int i = 0; i < 4; i++) idesc[i] = idesc_mxf8f6f4_e2m1_e4m3(ncols, (uint32_t)i, (uint32_t)i);
+            }
+          }
         }
       }
     }
