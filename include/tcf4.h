@@ -80,10 +80,11 @@ TCF4_API tcf4_status trellis_decode_to_mxfp4(tcf4_matrix w, uint8_t *out_nibbles
 /* HEPH abstract, first serving mode: fused decode + product.
  *   y[t][n] = bf16( sum_k w[n][k] * x[t][k] ), fp32 accumulation, round to nearest even.
  *   x: bf16 bits [T][cols]; y: bf16 bits [T][rows]; 1 <= T <= 32 (T == 0 is a no-op).
- * Two kernels behind one call: when seg_len == 32, cols is a multiple of 64 with 1024 <= cols and
- * the scales are 16-byte aligned, the product runs on the tensor cores (block-scaled MXFP4 x E4M3
- * MMA, the activations split exactly into two E4M3 terms) and needs `workspace`; otherwise it runs
- * on CUDA cores and needs none. trellis_gemv_workspace tells which (0 bytes = none needed).
+ * Two kernels behind one call: when seg_len == 32 and cols is a multiple of 64, the product runs on
+ * the tensor cores (block-scaled MXFP4 x MXFP4 MMA: each 32-block of x is written as a sum of six
+ * E2M1 terms with their own UE8M0 scales, which leaves at most 5^-6 of the block's largest |x|
+ * unrepresented) and needs `workspace`; otherwise it runs on CUDA cores and needs none.
+ * trellis_gemv_workspace tells which (0 bytes = none needed).
  *   workspace: device scratch of at least trellis_gemv_workspace(w, T) bytes, 256-byte aligned,
  *   owned by the caller (may be NULL when that size is 0).
  * Accuracy: |y - exact| <= 2e-3 * ||w_row||_2 * ||x_t||_2 per output plus the bf16 rounding.

@@ -6,6 +6,9 @@ kernels are CUDA) and compares them with the oracle's step-by-step decoder for e
 and for random multi-block rows, with and without a carry from the previous block. The GPU
 parity tests then check the kernels themselves bit for bit.
 """
+import os
+import re
+
 import numpy as np
 
 import oracle
@@ -66,3 +69,54 @@ def test_identity_on_rows_with_and_without_carry():
                 pL, pH = st[:, j - 1, 0], st[:, j - 1, 1]
             got[:, 32 * j:32 * j + 32] = _codes_from_planes(_planes(L, H, pL, pH))
         assert (got == ref).all(), seg_len
+
+
+# ----------------------------------------------------------------------------- nibble transposes
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "trellis_coded_fp4_b200", "csrc", "tcf4_device.cuh")
+
+
+def _lop3(a, b, c, lut):
+    """Bitwise three-input function by truth table: bit (a<<2 | b<<1 | c) of lut."""
+    out = np.zeros_like(a)
+    for i in range(8):
+        if (lut >> i) & 1:
+            ma = a if i & 4 else ~a
+            mb = b if i & 2 else ~b
+            mc = c if i & 1 else ~c
+            out |= ma & mb & mc
+    return out & M32
+
+
+def test_delta_swap_select_table():
+    # Each three-input op in delta_swap takes operands (mask, x, y) and must compute mask ? x : y.
+    text = open(HEADER).read()
+    body = text[text.index("void delta_swap"):text.index("void planes_to_nibbles_interleaved")]
+    luts = [int(v, 16) for v in re.findall(r"lop3\.b32 %0, %1, %2, %3, (0x[0-9A-Fa-f]+);", body)]
+    assert len(luts) == 2
+    rng = np.random.default_rng(7)
+    m, x, y = (rng.integers(0, 1 << 32, 64, dtype=np.uint64) for _ in range(3))
+    for lut in luts:
+        assert (_lop3(m, x, y, lut) == ((m & x) | (~m & y & M32))).all(), hex(lut)
+
+
+def _delta_swap(a, b, s, mask):
+    mask = np.uint64(mask)
+    nb = (mask & (a >> np.uint64(s))) | (~mask & b & M32)
+    ms = (mask << np.uint64(s)) & M32
+    na = (ms & (b << np.uint64(s)) & M32) | (~ms & a & M32)
+    return na, nb
+
+
+def test_interleaved_nibble_order():
+    # planes -> four words with weight 4v+j in nibble v of word j (the order the MMA operands use)
+    rng = np.random.default_rng(8)
+    codes = rng.integers(0, 16, (16, 32)).astype(np.uint64)
+    n = [sum(((codes[:, i] >> np.uint64(c)) & np.uint64(1)) << np.uint64(i) for i in range(32)) for c in range(4)]
+    a, b = _delta_swap(n[0], n[1], 1, 0x55555555)
+    c, d = _delta_swap(n[2], n[3], 1, 0x55555555)
+    a, c = _delta_swap(a, c, 2, 0x33333333)
+    b, d = _delta_swap(b, d, 2, 0x33333333)
+    for j, w in enumerate((a, b, c, d)):
+        for v in range(8):
+            assert ((w >> np.uint64(4 * v)) & np.uint64(15) == codes[:, 4 * v + j]).all()

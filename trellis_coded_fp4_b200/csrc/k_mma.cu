@@ -1,28 +1,31 @@
 // k_mma.cu -- fused trellis decode + block-scaled tensor-core product (tcgen05, sm_100a).
 //
 // HEPH abstract, first serving mode: the compressed stream stays resident and is decoded inside the
-// product. The product runs on the 5th-generation tensor cores: the decoded weights are already
-// MXFP4 elements (E2M1 codes with a UE8M0 scale per 32 weights), so they feed a block-scaled
-// kind::mxf8f6f4 MMA directly as the A operand (E2M1, scale factors = the weights' own UE8M0
-// bytes). The bf16 activations are the B operand, split exactly into two E4M3 terms per element
-// (hi + lo, each 32-block with its own UE8M0 scale): B column 2t holds token t's hi term and column
-// 2t+1 its lo term, so y[t] = D[:, 2t] + D[:, 2t+1] in fp32.
+// product. The decoded weights are MXFP4 elements (E2M1 codes, one UE8M0 scale per 32 weights), so
+// they feed a block-scaled kind::mxf4 MMA (K = 64 per instruction) directly as the A operand, the
+// scale factors being the weights' own UE8M0 bytes. The bf16 activations are the B operand,
+// written as a sum of kTerms E2M1 terms per 32-block, each term with its own UE8M0 scale (a greedy
+// residual expansion, see split_terms): B column kTerms*t + j holds term j of token t, and
+// y[t] = sum_j D[:, kTerms*t + j] in fp32.
 //
-// One persistent CTA per SM: 8 decode warps + 1 control warp, over 128-row tiles ("jobs"):
-//  * decode thread (warp w, lane l) owns tile row 32(w%4)+l and K-blocks 4(w/4)..4(w/4)+3 of each
-//    256-wide K stage. It keeps kPref stages of its 32 bytes of trellis words in flight with
-//    cp.async, decodes them in registers (bit-sliced) into E2M1 codes in the shared A stage, and
-//    stages its row's 4 scale bytes; one stage later warps 0-3 move the stage's A and B scale
-//    factors into TMEM (tcgen05.st) and release it.
-//  * the control thread streams the pre-split activations (B) with bulk copies kNB stages ahead
-//    and issues the stage's 8 MMAs (K = 32 each) into a double-buffered TMEM accumulator.
+// One persistent CTA per SM, over 128-row tiles ("jobs") of K stages of 256 (8 blocks of 32):
+//  * loader warp: lane 0 streams each stage's trellis words (128 rows x 64 bytes) into a ring of
+//    shared-memory slots with 2-D TMA tile loads (64-byte swizzle); all lanes stage the stage's
+//    weight scale bytes in the layout tcgen05.cp copies into TMEM.
+//  * 8 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and K-blocks 4(w/4)..4(w/4)+3
+//    of a stage. It reads its 32 bytes of trellis words, decodes them in registers (bit-sliced) and
+//    stores the four 16-byte E2M1 chunks into the stage's A tile.
+//  * MMA warp: lane 0 streams the activation terms (B) with bulk copies, copies the stage's scale
+//    factors into TMEM (tcgen05.cp) and issues the stage's 4 MMAs into a double-buffered TMEM
+//    accumulator.
 //  * the epilogue of job i (tcgen05.ld, then the GEMV output, the SwiGLU of gate/up rows, or the MoE
-//    down rows and their combine) runs in warps 0-3 during job i+1.
-// Every mbarrier wait is bounded; a wait that gives up raises a shared abort flag that all decode
-// threads read after the per-stage named barrier, so the CTA leaves together and frees its TMEM.
+//    down rows and their combine) runs in decode warps 0-3 early in job i+1.
+// Every wait is a bounded mbarrier wait; a wait that gives up raises a shared abort flag that every
+// role polls once per stage, and each role drains its own asynchronous copies and MMAs before the
+// CTA frees its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include "tcf4_device.cuh"
 #include "tcf4_internal.h"
@@ -33,28 +36,40 @@ namespace tcf4 {
 
 __device__ unsigned int g_tcf4_timeouts_mma = 0;
 
-constexpr int kKS = 256;              // K elements per stage (8 blocks of 32)
-constexpr int kNA = 3;                // A stages (E2M1 tile + scale-factor TMEM slot)
-constexpr int kNB = 4;                // B stages (activation split)
-constexpr int kPref = 4;              // trellis-word stages in flight per decode thread
-constexpr int kDec = 256;             // decode threads
-constexpr int kMmaThreads = kDec + 32;
-constexpr uint32_t kTmemCols = 128;
-constexpr uint32_t kSfaCol = 64, kSfbCol = 88;  // scale-factor slots: 8 and 4 TMEM columns per stage
-constexpr uint32_t kSboA = 2048;      // 16 K chunks x 128 B per 8-row group of a stage
-constexpr int kMaxGroups = kMaxTokens * kMaxTopK + kMaxExperts / 2;
+constexpr int kNW = 6;               // trellis-word stages in flight (TMA ring)
+constexpr int kNA = 4;               // A stages (E2M1 tile + scale staging + TMEM scale slots)
+constexpr int kNB = 3;               // B stages (activation terms + their scales)
+constexpr int kTerms = 6;            // E2M1 terms per activation block
+constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> kNW jobs in flight)
+constexpr int kLoadWarp = 8, kMmaWarp = 9, kThreads = 320;
+constexpr uint32_t kWStage = 8192;   // 128 rows x 64 bytes of trellis words (two 64-row TMA boxes)
+constexpr uint32_t kAStage = 16384;  // 128 rows x 256 E2M1 elements, packed
+constexpr uint32_t kSbo = 1024;      // 8 rows x 8 chunks x 16 bytes: one 8-row group of a stage
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
 
-// K position (0..31) inside a 32-block of the MMA that holds weight i of the block: the decoder's
-// interleaved nibble words put weight 4v+j in nibble v of word j, and word j fills bytes 4j..4j+3
-// of the block's 16 data bytes (16-element chunk j/2, elements 8(j%2)..8(j%2)+7).
-__host__ __device__ constexpr int kpos_of_weight(int i) { return 16 * ((i & 3) >> 1) + 8 * (i & 1) + (i >> 2); }
+template <int NMAX>
+struct Cfg {
+  static constexpr int kTok = NMAX / kTerms;                   // tokens per group
+  static constexpr int kSlots = (NMAX + kTerms - 1) / kTerms;  // token slots the split writes
+  static_assert(NMAX <= 128, "B scale factors of a 4-block group fit one 4-column TMEM slot");
+  static constexpr uint32_t kBTile = NMAX * 128u;              // NMAX rows x 256 E2M1
+  static constexpr uint32_t kBSlot = kBTile + 2u * 512u;       // + scales: one 32x128b copy per group
+  static constexpr uint32_t kSfaCol = 2u * NMAX;               // TMEM: accumulators first
+  static constexpr uint32_t kSfbCol = kSfaCol + 8u * kNA;
+  static constexpr uint32_t kUsed = kSfbCol + 8u * kNA;
+  static constexpr uint32_t kTmemCols = kUsed <= 128 ? 128 : (kUsed <= 256 ? 256 : 512);
+};
 
-// Byte offset of element (n, k), k < 256, in a K-major no-swizzle stage of 8-bit containers:
-// core matrices of 8 rows x 16 bytes, LBO = 128 (K chunks), SBO = 2048 (8-row groups).
-__host__ __device__ constexpr uint32_t kmajor_off(uint32_t n, uint32_t k) {
-  return (n >> 3) * kSboA + (k >> 4) * 128u + (n & 7u) * 16u + (k & 15u);
+// Position (0..31) inside a 32-element chunk of the MMA operand of weight i of the block: the
+// decoder's interleaved nibble words put weight 4v+j in nibble v of word j, and word j fills bytes
+// 4j..4j+3 of the chunk (element 2b in the low nibble of byte b).
+__host__ __device__ constexpr int kpos_of_weight(int i) { return 8 * (i & 3) + (i >> 2); }
+
+// Byte offset of chunk c (0..7) of row n in a K-major, no-swizzle stage: core matrices of 8 rows
+// x 16 bytes, LBO = 128 (adjacent chunks), SBO = 1024 (adjacent 8-row groups).
+__host__ __device__ constexpr uint32_t chunk_off(uint32_t n, uint32_t c) {
+  return (n >> 3) * kSbo + c * 128u + (n & 7u) * 16u;
 }
 
 // ------------------------------------------------------------------------------- routing groups
@@ -64,9 +79,9 @@ struct GroupPlan {
   int off[kMaxExperts];
   int list[kMaxTokens * kMaxTopK];  // pairs p = t*k + j per expert, in p order
   int ids[kMaxTokens * kMaxTopK];
-  int g_e[kMaxGroups];              // expert of group g
-  int g_first[kMaxGroups];          // first index into list[] of group g
-  int g_cnt[kMaxGroups];            // pairs in group g (<= gmax)
+  int g_e[kMaxTokens * kMaxTopK];   // expert of group g
+  int g_first[kMaxTokens * kMaxTopK];
+  int g_cnt[kMaxTokens * kMaxTopK];
   int n_groups;
 };
 
@@ -106,155 +121,202 @@ __device__ void build_groups(GroupPlan &pl, const int32_t *__restrict__ ids, int
   __syncthreads();
 }
 
-// ------------------------------------------------------------------------------- activation split
-// One 32-element block of one source row -> hi/lo E4M3 terms. hi = E4M3(x / 2^Eh) with
-// Eh = floor(log2 max|x|) - 7 over the block (so max|x|/2^Eh lies in [128, 256)); lo the same for
-// the residual x - hi*2^Eh, exact in fp32. hi*2^Eh + lo*2^El reproduces every bf16 x of the block
-// except elements more than ~17 binades below the block maximum.
-__device__ __forceinline__ void split_e4m3(float v, float mx, uint8_t &q, uint32_t &sf, float &back) {
-  if (!(mx > 0.f)) {
-    q = 0;
-    sf = 127u;
-    back = 0.f;
-    return;
-  }
-  int e = ilogbf(mx) - 7;
-  e = e < -126 ? -126 : (e > 127 ? 127 : e);
-  q = (uint8_t)__nv_cvt_float_to_fp8(scalbnf(v, -e), __NV_SATFINITE, __NV_E4M3);
-  const __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)q, __NV_E4M3);
-  back = scalbnf(__half2float(__half(hr)), e);
-  sf = (uint32_t)(e + 127);
-}
-
+// ------------------------------------------------------------------------------- activation terms
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
 
-// Per group: Bg [S stages][NMAX*256 bytes] (one K-major B stage each) and Bsf [S][32 lanes][4
-// words], word 2g+c of a lane = UE8M0 bytes of B column 32c+lane for K-blocks 4g..4g+3.
-__host__ __device__ inline size_t bsplit_group_bytes(int S, int NMAX) { return (size_t)S * NMAX * 256; }
-__host__ __device__ inline size_t bsf_group_words(int S) { return (size_t)S * 32 * 4; }
+// fp32 -> E2M1 code (round to nearest even, saturating at +-6).
+__device__ __forceinline__ uint32_t to_e2m1(float v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(0.f), "f"(v));
+  return r & 15u;
+}
 
-// Write the split of one block (p = token slot, kb = 32-block) into one group's B stages.
+// E2M1 code -> value (exact).
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  const uint32_t mag = c & 7u;
+  const float v = mag < 2u ? 0.5f * (float)mag : ldexpf(1.f + 0.5f * (float)(mag & 1u), (int)(mag >> 1) - 1);
+  return (c & 8u) ? -v : v;
+}
+
+// One 32-element block of one activation row (lane = element) -> kTerms E2M1 terms with UE8M0
+// scales, written as B rows kTerms*t .. kTerms*t+kTerms-1 of chunk kb of the group's B stages.
+// Term j: with m the largest |residual| of the block, scale 2^S with S = ceil(log2(m / 6)) puts the
+// block in (3, 6]; each residual is rounded to the E2M1 grid (nearest even) and the rounded value
+// removed (exactly: Sterbenz). The largest residual shrinks by at least 5x per term, so after
+// kTerms terms |x - sum| <= 5^-6 max|x| over the block.
 template <int NMAX>
-__device__ __forceinline__ void bsplit_block(float v, int p, int kb, uint8_t *Bg_g, uint32_t *Bsf_g) {
+__device__ __forceinline__ void split_terms(float v, int t, int kb, uint8_t *Bg) {
+  using C = Cfg<NMAX>;
   const int lane = threadIdx.x & 31;
-  uint8_t qh, ql;
-  uint32_t sfh, sfl;
-  float bh, bl;
-  split_e4m3(v, warp_max(fabsf(v)), qh, sfh, bh);
-  const float res = v - bh;
-  split_e4m3(res, warp_max(fabsf(res)), ql, sfl, bl);
-  const int s = kb >> 3, kin = (kb & 7) * 32 + kpos_of_weight(lane);
-  uint8_t *stage = Bg_g + (size_t)s * NMAX * 256;
-  stage[kmajor_off(2 * p, kin)] = qh;
-  stage[kmajor_off(2 * p + 1, kin)] = ql;
-  if (lane < 2) {
-    const int n = 2 * p + lane, g = (kb & 7) >> 2;
-    uint8_t *sfb = reinterpret_cast<uint8_t *>(Bsf_g + ((size_t)s * 32 + (n & 31)) * 4 + 2 * g + (n >> 5));
-    sfb[kb & 3] = (uint8_t)(lane == 0 ? sfh : sfl);
+  const int s = kb >> 3, c = kb & 7, g = c >> 2;
+  uint8_t *slot = Bg + (size_t)s * C::kBSlot;
+  const int kp = kpos_of_weight(lane);
+  float r = v;
+#pragma unroll
+  for (int j = 0; j < kTerms; j++) {
+    const int n = kTerms * t + j;
+    const float m = warp_max(fabsf(r));
+    int S = -127;
+    if (m > 0.f) {
+      const int e = ilogbf(m);
+      S = scalbnf(m, -e) <= 1.5f ? e - 2 : e - 1;
+      S = S < -127 ? -127 : (S > 127 ? 127 : S);
+    }
+    const uint32_t code = to_e2m1(scalbnf(r, -S));
+    r -= scalbnf(e2m1_value(code), S);
+    const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 4);
+    if (n < NMAX) {
+      if (((lane >> 2) & 1) == 0)
+        slot[chunk_off((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code | (partner << 4));
+      if (lane == 0)  // group g's copy: lane n%32, word n/32 (TMEM column 4g + n/32), byte = block in group
+        slot[C::kBTile + g * 512 + (n & 31) * 16 + (n >> 5) * 4 + (c & 3)] = (uint8_t)(S + 127);
+    }
   }
 }
 
-// Plain GEMV: one group, token slots 0..T-1 (the other slots up to NMAX/2 are zero columns).
+// Plain GEMV: one group, token slots 0..T-1 (slots up to kSlots are zero rows).
 template <int NMAX>
 __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
-                                                     uint8_t *__restrict__ Bg, uint32_t *__restrict__ Bsf) {
+                                                     uint8_t *__restrict__ Bg) {
   const int nb = K >> 5, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < (NMAX / 2) * nb; wi += nwarps) {
-    const int p = wi / nb, kb = wi - p * nb;
-    const float v = p < T ? __uint_as_float((uint32_t)x[(size_t)p * K + kb * 32 + lane] << 16) : 0.f;
-    bsplit_block<NMAX>(v, p, kb, Bg, Bsf);
+  for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < Cfg<NMAX>::kSlots * nb; wi += nwarps) {
+    const int t = wi / nb, kb = wi - t * nb;
+    const float v = t < T ? __uint_as_float((uint32_t)x[(size_t)t * K + kb * 32 + lane] << 16) : 0.f;
+    split_terms<NMAX>(v, t, kb, Bg);
   }
 }
 
 // MoE: group g's token slot i is pair list[g_first + i]; its activation row is src[pair / div]
 // (gate_up reads x rows of tokens: div = k; down reads h rows of pairs: div = 1). Block 0 also
-// clears the down kernel's chunk counters when `counters` is given.
+// clears the down kernel's counters when `counters` is given.
 template <int NMAX>
 __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ ids, int P, int E, int div,
                                                     const uint16_t *__restrict__ src, int K, uint8_t *__restrict__ Bg,
-                                                    uint32_t *__restrict__ Bsf, int *__restrict__ counters,
-                                                    int n_counters) {
+                                                    int *__restrict__ counters, int n_counters) {
   __shared__ GroupPlan pl;
   if (counters != nullptr && blockIdx.x == 0)
     for (int c = threadIdx.x; c < n_counters; c += blockDim.x) counters[c] = 0;
-  build_groups(pl, ids, P, E, NMAX / 2);
+  build_groups(pl, ids, P, E, Cfg<NMAX>::kTok);
   const int nb = K >> 5, S = (nb + 7) >> 3;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int per_group = (NMAX / 2) * nb;
+  const int per_group = Cfg<NMAX>::kSlots * nb;
   for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < pl.n_groups * per_group; wi += nwarps) {
     const int g = wi / per_group, r = wi - g * per_group;
-    const int p = r / nb, kb = r - p * nb;
+    const int t = r / nb, kb = r - t * nb;
     float v = 0.f;
-    if (p < pl.g_cnt[g]) {
-      const int row = pl.list[pl.g_first[g] + p] / div;
+    if (t < pl.g_cnt[g]) {
+      const int row = pl.list[pl.g_first[g] + t] / div;
       v = __uint_as_float((uint32_t)src[(size_t)row * K + kb * 32 + lane] << 16);
     }
-    bsplit_block<NMAX>(v, p, kb, Bg + (size_t)g * bsplit_group_bytes(S, NMAX), Bsf + (size_t)g * bsf_group_words(S));
+    split_terms<NMAX>(v, t, kb, Bg + (size_t)g * S * Cfg<NMAX>::kBSlot);
   }
 }
 
 // ------------------------------------------------------------------------------- geometry
 
-// Shared memory: barriers | A ring | B ring | trellis-word ring | B-scale ring | scale staging
-// | gate/up exchange | group plan | two scale slabs.
+// Shared memory: barriers + tensor-map copy | word ring | A ring | scale staging | B ring
+// | gate/up exchange | group plan.
 struct MmaGeom {
-  uint32_t off_A, off_B, off_C, off_F, off_X, off_U, off_P, off_S, slab, smem;
+  uint32_t off_W, off_A, off_X, off_B, off_U, off_P, smem;
 };
 
-__host__ __device__ inline MmaGeom mma_geom(int nbr, int NMAX, int mode) {
+template <int NMAX>
+__host__ __device__ inline MmaGeom mma_geom(int mode) {
   MmaGeom g;
-  g.off_A = 1024u;
-  g.off_B = g.off_A + kNA * 128u * kKS;
-  g.off_C = g.off_B + kNB * (uint32_t)NMAX * kKS;
-  g.off_F = g.off_C + kPref * kDec * 32u;
-  g.off_X = g.off_F + kPref * 128u * 16u;
-  g.off_U = g.off_X + kNA * 1024u;
-  g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)(NMAX / 2) * 4u : 0u);
-  g.off_S = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
-  g.slab = round_up(128u * (uint32_t)nbr + 16u, 16u);  // +16: tail reads of a row's 4 scale bytes
-  g.smem = g.off_S + 2u * g.slab;
+  g.off_W = 1024u;
+  g.off_A = g.off_W + kNW * kWStage;
+  g.off_X = g.off_A + kNA * kAStage;
+  g.off_B = g.off_X + kNA * 1024u;
+  g.off_U = g.off_B + kNB * Cfg<NMAX>::kBSlot;
+  g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)Cfg<NMAX>::kTok * 4u : 0u);
+  g.smem = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
   return g;
 }
+
+// ------------------------------------------------------------------------------- instructions
 
 __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
-
-__device__ __forceinline__ void sts_u2(uint32_t addr, uint32_t a, uint32_t b) {
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+__device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
+// 2-D TMA tile load (no multicast; the tensor map covers this GPU's memory only).
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
 }
 
-__device__ __forceinline__ void sts_u32(uint32_t addr, uint32_t a) {
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(a) : "memory");
+// Shared memory (32 rows x 16 bytes) -> 4 TMEM columns of 32 lanes, replicated into all four lane
+// quarters.
+__device__ __forceinline__ void tmem_cp_32x128_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+// Instruction descriptor of a block-scaled kind::mxf4 MMA: A = B = E2M1, K-major, UE8M0 scales per
+// 32, fp32 accumulation, M = 128, N columns; sf = scale-factor byte pair (0 or 2) of both operands.
+__device__ __forceinline__ uint32_t idesc_mxf4(uint32_t N, uint32_t sf) {
+  uint32_t d = 0;
+  d |= (sf & 3u) << 4;     // B scale-factor id
+  d |= 1u << 7;            // A format: E2M1
+  d |= 1u << 10;           // B format: E2M1
+  d |= (N >> 3) << 17;     // N / 8
+  d |= 1u << 23;           // scale format: UE8M0
+  d |= (128u >> 4) << 24;  // M / 16
+  d |= (sf & 3u) << 29;    // A scale-factor id
+  return d;                // bit 31 = 0: K = 64
+}
+
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Per-job tensor maps of the grouped MoE: lane 0 rewrites the global address of the shared-memory
+// copy, then the whole warp publishes it to the CTA's global slot for the TMA unit.
+__device__ __forceinline__ void tmap_set_address(uint32_t smap, const void *addr) {
+  asm volatile("tensormap.replace.tile.global_address.shared::cta.b1024.b64 [%0], %1;" ::"r"(smap), "l"(addr)
                : "memory");
 }
+__device__ __forceinline__ void tmap_publish(void *gmap, uint32_t smap) {
+  asm volatile(
+      "tensormap.cp_fenceproxy.global.shared::cta.tensormap::generic.release.gpu.sync.aligned [%0], [%1], "
+      "128;" ::"l"(gmap),
+      "r"(smap)
+      : "memory");
+}
+__device__ __forceinline__ void tmap_acquire(const void *gmap) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmap) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
 // ------------------------------------------------------------------------------- kernel arguments
 
 struct MmaArgs {
-  MatView w;              // GEMV: the matrix (MoE: rows/stream unused; experts come from the table)
+  const uint8_t *scales;  // GEMV: the matrix's scales (MoE: from the table)
+  int rows;               // GEMV rows
   int nbr;                // 32-blocks per row (K / 32)
-  const uint8_t *Bg;      // activation split, per group
-  const uint32_t *Bsf;
+  const uint8_t *Bg;      // activation terms, per group [S][kBSlot]
   int T;                  // GEMV tokens
   uint16_t *y;            // GEMV out [T][rows]
   const int32_t *ids;     // MoE routing [T][k]
@@ -262,117 +324,131 @@ struct MmaArgs {
   int P, E, k, Tm, H, I;
   uint16_t *hidden;       // [P][I] bf16
   float *yws;             // [P][H] fp32
-  int *counters;          // per 128-row chunk of H
+  int *counters;          // 4 per 128-row chunk of H
   uint16_t *out;          // [T][H] bf16
+  unsigned char *maps;    // MoE: per-CTA tensor-map slots [gridDim][kMapSlots][128]
 };
 
-// A job is one 128-row tile: rows [0, na) from (st0, sc0) and, when split, rows [64, 64 + nb) from
-// (st1, sc1); B group `group`, MMA width ncols; `cnt` tokens starting at list index `first`.
+// A job is one 128-row tile: tile rows [0, 64) are matrix rows y0.., tile rows [64, 128) matrix
+// rows y1..; na / nb of them valid. B group `group`, MMA width ncols; `cnt` tokens starting at
+// list index `first`.
 struct JobRows {
-  const uint2 *st0, *st1;
-  const uint8_t *sc0, *sc1;
-  int na, nb, split, group, ncols, row0, chunk, cnt, first;
+  const void *st;     // the matrix stream (MoE: the tensor map's address)
+  const uint8_t *sc;  // its scales
+  int y0, y1, na, nb, group, ncols, row0, chunk, cnt, first;
 };
 
 template <int MAXE, int MODE, int NMAX>
 __device__ __forceinline__ JobRows job_rows(const MmaArgs &a, const MoeTable<MAXE> &tab, const GroupPlan *pl,
                                             int job) {
   JobRows j;
-  j.split = 0;
-  j.st1 = nullptr;
-  j.sc1 = nullptr;
-  j.nb = 0;
   if (MODE == kModeGemv) {
     const int r0 = job * 128;
-    j.st0 = a.w.stream + (size_t)r0 * a.nbr;
-    j.sc0 = a.w.scales + (size_t)r0 * a.nbr;
-    j.na = a.w.rows - r0 < 128 ? a.w.rows - r0 : 128;
+    j.st = nullptr;
+    j.sc = a.scales;
+    j.y0 = r0;
+    j.y1 = r0 + 64;
+    j.na = a.rows - r0 < 64 ? a.rows - r0 : 64;
+    j.nb = a.rows - r0 - 64 < 0 ? 0 : (a.rows - r0 - 64 < 64 ? a.rows - r0 - 64 : 64);
     j.group = 0;
-    j.ncols = NMAX;
-    j.row0 = r0;
-    j.chunk = job;
     j.cnt = a.T;
     j.first = 0;
+    j.row0 = r0;
+    j.chunk = job;
   } else if (MODE == kModeGateUp) {
     const int nch = (a.I + 63) / 64;
     const int g = job / nch, c = job - g * nch, e = pl->g_e[g];
     const int i0 = 64 * c;
-    j.split = 1;
-    j.st0 = tab.gu[e] + (size_t)i0 * a.nbr;
-    j.sc0 = tab.gus[e] + (size_t)i0 * a.nbr;
-    j.st1 = tab.gu[e] + (size_t)(a.I + i0) * a.nbr;
-    j.sc1 = tab.gus[e] + (size_t)(a.I + i0) * a.nbr;
+    j.st = tab.gu[e];
+    j.sc = tab.gus[e];
+    j.y0 = i0;
+    j.y1 = a.I + i0;
     j.na = j.nb = a.I - i0 < 64 ? a.I - i0 : 64;
     j.group = g;
     j.cnt = pl->g_cnt[g];
     j.first = pl->g_first[g];
-    j.ncols = (2 * j.cnt + 15) / 16 * 16;
     j.row0 = i0;
     j.chunk = c;
   } else {
     const int nch = (a.H + 127) / 128;
     const int g = job / nch, c = job - g * nch, e = pl->g_e[g];
     const int n0 = 128 * c;
-    j.st0 = tab.dn[e] + (size_t)n0 * a.nbr;
-    j.sc0 = tab.dns[e] + (size_t)n0 * a.nbr;
-    j.na = a.H - n0 < 128 ? a.H - n0 : 128;
+    j.st = tab.dn[e];
+    j.sc = tab.dns[e];
+    j.y0 = n0;
+    j.y1 = n0 + 64;
+    j.na = a.H - n0 < 64 ? a.H - n0 : 64;
+    j.nb = a.H - n0 - 64 < 0 ? 0 : (a.H - n0 - 64 < 64 ? a.H - n0 - 64 : 64);
     j.group = g;
     j.cnt = pl->g_cnt[g];
     j.first = pl->g_first[g];
-    j.ncols = (2 * j.cnt + 15) / 16 * 16;
     j.row0 = n0;
     j.chunk = c;
   }
+  j.ncols = (kTerms * j.cnt + 15) / 16 * 16;
   return j;
 }
 
-__device__ __forceinline__ bool row_valid(const JobRows &j, int m) {
-  return j.split ? (m < 64 ? m < j.na : m - 64 < j.nb) : m < j.na;
+// Matrix row of tile row m (0..127), or -1 when the row is outside the tile's valid rows.
+__device__ __forceinline__ int tile_row(const JobRows &j, int m) {
+  return m < 64 ? (m < j.na ? j.y0 + m : -1) : (m - 64 < j.nb ? j.y1 + m - 64 : -1);
 }
 
 // ------------------------------------------------------------------------------- the kernel
 
 template <int MAXE, int MODE, int NMAX>
-__global__ void __launch_bounds__(kMmaThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
-                                                        const __grid_constant__ MoeTable<MAXE> tab) {
+__global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
+                                                     const __grid_constant__ MoeTable<MAXE> tab,
+                                                     const __grid_constant__ CUtensorMap wmap) {
+  using C = Cfg<NMAX>;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = a.nbr, S = (nbr + 7) >> 3;
-  const MmaGeom geo = mma_geom(nbr, NMAX, MODE);
-  uint64_t *a_full = reinterpret_cast<uint64_t *>(smem);
-  uint64_t *a_empty = a_full + 4, *b_full = a_full + 8, *b_empty = a_full + 16, *acc_full = a_full + 24,
-           *acc_empty = a_full + 26;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 256);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 260);
-  volatile int *s_last = reinterpret_cast<volatile int *>(smem + 264);
+  const MmaGeom geo = mma_geom<NMAX>(MODE);
+  uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *w_empty = w_full + 8, *a_full = w_full + 16, *a_empty = w_full + 20, *b_full = w_full + 24,
+           *b_empty = w_full + 28, *acc_full = w_full + 32, *acc_empty = w_full + 34, *u_full = w_full + 36,
+           *u_empty = w_full + 38, *drain = w_full + 40;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 384);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 388);
+  unsigned char *smap = smem + 512;  // shared-memory copy of the tensor map (grouped MoE)
   unsigned int *tmo = &g_tcf4_timeouts_mma;
   GroupPlan *pl = reinterpret_cast<GroupPlan *>(smem + geo.off_P);
 
   if (tid == 0) {
-    for (int b = 0; b < kNA; b++) {
-      mbar_init(&a_full[b], 8);
-      mbar_init(&a_empty[b], 1);
+    for (int i = 0; i < kNW; i++) {
+      mbar_init(&w_full[i], 1);
+      mbar_init(&w_empty[i], 8);
     }
-    for (int b = 0; b < kNB; b++) {
-      mbar_init(&b_full[b], 1);
-      mbar_init(&b_empty[b], 1);
+    for (int i = 0; i < kNA; i++) {
+      mbar_init(&a_full[i], 9);
+      mbar_init(&a_empty[i], 1);
+    }
+    for (int i = 0; i < kNB; i++) {
+      mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], 1);
     }
     for (int i = 0; i < 2; i++) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);
+      mbar_init(&u_full[i], 2);
+      mbar_init(&u_empty[i], 2);
     }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 8) {
-    tmem_alloc(tmem_slot, kTmemCols);
+  if (MODE != kModeGemv && tid < 32)
+    reinterpret_cast<uint32_t *>(smap)[tid] = reinterpret_cast<const uint32_t *>(&wmap)[tid];
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   int njobs;
   if (MODE == kModeGemv) {
-    njobs = (a.w.rows + 127) >> 7;
+    njobs = (a.rows + 127) >> 7;
   } else {
-    build_groups(*pl, a.ids, a.P, a.E, NMAX / 2);  // synchronizes the CTA
+    build_groups(*pl, a.ids, a.P, a.E, C::kTok);  // synchronizes the CTA
     njobs = pl->n_groups * (MODE == kModeGateUp ? (a.I + 63) / 64 : (a.H + 127) / 128);
   }
   tc_fence_before();
@@ -382,267 +458,324 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_mma(const __grid_constant__ 
   const int my_jobs = (int)blockIdx.x < njobs ? (njobs - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int nq = my_jobs * S;
   auto job_of = [&](int jl) { return (int)blockIdx.x + jl * (int)gridDim.x; };
+  const int s_epi = S > 1 ? 1 : 0;  // the epilogue of job jl-1 runs after the A stage (jl, s_epi)
 
   if (warp < 8) {
     // ---------------------------------------------------------------- decode warps
     const int sp = warp & 3, h = warp >> 2, m = 32 * sp + lane;
-    const uint32_t cbase = smem_u32(smem + geo.off_C) + (uint32_t)tid * 32u;
-    const uint32_t fbase = smem_u32(smem + geo.off_F) + (uint32_t)tid * 16u;
-    const uint32_t xbase = smem_u32(smem + geo.off_X);
-    const uint32_t sbase = smem_u32(smem + geo.off_S);
+    const uint32_t rb = (uint32_t)(m & 63), sw = (rb >> 1) & 3u;  // row in its TMA box, 64-byte swizzle
+    const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * 4096u + rb * 64u;
+    const uint32_t woff0 = ((2u * h) ^ sw) * 16u, woff1 = ((2u * h + 1u) ^ sw) * 16u;
+    const uint32_t abase = smem_u32(smem + geo.off_A) + chunk_off((uint32_t)m, 4u * (uint32_t)h);
     const int tail_blocks = nbr - 8 * (S - 1) - 4 * h;  // this thread's blocks in the last stage
-    const uint32_t tail = tail_blocks <= 0 ? 0u : (tail_blocks >= 4 ? 32u : 8u * (uint32_t)tail_blocks);
 
-    // Prefetch front: job jl_i, stage s_i; src walks this thread's row 64 bytes per stage.
-    int jl_i = 0, s_i = 0;
-    const uint2 *src_i = a.w.stream;
-    bool rv_i = false;
-    const uint32_t *bsf_i = a.Bsf;
-    JobRows ji{};
-    auto start_job_front = [&]() {
-      ji = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_i));
-      rv_i = row_valid(ji, m);
-      src_i = rv_i ? (ji.split && m >= 64 ? ji.st1 + (size_t)(m - 64) * nbr : ji.st0 + (size_t)m * nbr) + 4 * h
-                   : a.w.stream;
-      bsf_i = a.Bsf + (size_t)ji.group * bsf_group_words(S) + (size_t)lane * 4;
-    };
-    if (my_jobs) start_job_front();
-    uint32_t slot_i = 0;  // ring slot of the front (q % kPref)
-    auto issue_next = [&](bool live) {
-      if (live) {
-        const uint32_t bytes = rv_i ? (s_i == S - 1 ? tail : 32u) : 0u;
-        const uint32_t dst = cbase + slot_i * (uint32_t)(kDec * 32);
-        cp_async16(dst, src_i, bytes > 16u ? 16u : bytes);
-        cp_async16(dst + 16u, bytes > 16u ? src_i + 2 : src_i, bytes > 16u ? bytes - 16u : 0u);
-        if (warp < 4) cp_async16(fbase + slot_i * (128u * 16u), bsf_i, 16u);
-        if (s_i == 0) {  // the job's scale bytes, into slab buffer jl_i % 2
-          const uint32_t sdst = sbase + (uint32_t)(jl_i & 1) * geo.slab;
-          const uint32_t t0 = (uint32_t)ji.na * (uint32_t)nbr;
-          for (uint32_t c = tid; c * 16u < t0; c += kDec)
-            cp_async16(sdst + c * 16u, ji.sc0 + c * 16u, t0 - c * 16u < 16u ? t0 - c * 16u : 16u);
-          if (ji.split) {
-            const uint32_t t1 = (uint32_t)ji.nb * (uint32_t)nbr, o1 = 64u * (uint32_t)nbr;
-            for (uint32_t c = tid; c * 16u < t1; c += kDec)
-              cp_async16(sdst + o1 + c * 16u, ji.sc1 + c * 16u, t1 - c * 16u < 16u ? t1 - c * 16u : 16u);
-          }
-        }
-        src_i += 8;
-        bsf_i += 32 * 4;
-        if (++s_i == S) {
-          s_i = 0;
-          if (++jl_i < my_jobs) start_job_front();
-        }
-        slot_i = (slot_i + 1) & (kPref - 1);
+    auto epilogue = [&](int jl_e) {
+      const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
+      const int buf = jl_e & 1;
+      if (!mbar_wait(&acc_full[buf], (uint32_t)(jl_e >> 1) & 1u, tmo)) {
+        *abort_flag = 1;
+        return;
       }
-      cp_async_commit();
-    };
-
-    // scale factors of the stage in A buffer bp into TMEM (warps 0-3), then release it to the MMA
-    auto publish_scales = [&](uint32_t bp, const uint4 &sfb) {
-      const uint32_t lane_addr = tbase + ((uint32_t)(32 * warp) << 16);
-      const uint4 x0 = lds_u4(xbase + bp * 1024u + (uint32_t)lane * 32u);
-      const uint4 x1 = lds_u4(xbase + bp * 1024u + (uint32_t)lane * 32u + 16u);
-      const uint32_t w8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-      tmem_st_x8(lane_addr + kSfaCol + 8u * bp, w8);
-      tmem_st_x4(lane_addr + kSfbCol + 4u * bp, sfb.x, sfb.y, sfb.z, sfb.w);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[bp]);
-    };
-
-    // epilogue of local job jl (warps 0-3)
-    auto epilogue = [&](int jl) {
-      const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl));
-      const int buf = jl & 1;
-      if (!mbar_wait(&acc_full[buf], (uint32_t)(jl >> 1) & 1u, tmo)) *abort_flag = 1;
       tc_fence_after();
-      float v[NMAX / 2];
+      float v[C::kTok];
 #pragma unroll
-      for (int c0 = 0; c0 < NMAX; c0 += 16) {
+      for (int t = 0; t < C::kTok; t++) v[t] = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < C::kTok * kTerms; c0 += 16) {
         uint32_t r[16];
         tmem_ld_x16(tbase + ((uint32_t)(32 * warp) << 16) + (uint32_t)(buf * NMAX + c0), r);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 8; j++) v[c0 / 2 + j] = __uint_as_float(r[2 * j]) + __uint_as_float(r[2 * j + 1]);
+        for (int i = 0; i < 16; i++)
+          if (c0 + i < C::kTok * kTerms) v[(c0 + i) / kTerms] += __uint_as_float(r[i]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);
       const int mrow = 32 * warp + lane;
       if (MODE == kModeGemv) {
-        if (mrow < jr.na)
+        const int row = tile_row(jr, mrow);
+        if (row >= 0)
 #pragma unroll
-          for (int t = 0; t < NMAX / 2; t++)
-            if (t < a.T)
-              a.y[(size_t)t * a.w.rows + jr.row0 + mrow] = __bfloat16_as_ushort(__float2bfloat16_rn(v[t]));
+          for (int t = 0; t < C::kTok; t++)
+            if (t < a.T) a.y[(size_t)t * a.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v[t]));
       } else if (MODE == kModeGateUp) {
-        float *U = reinterpret_cast<float *>(smem + geo.off_U) + (size_t)buf * 64 * (NMAX / 2);
-        if (mrow >= 64)
-#pragma unroll
-          for (int t = 0; t < NMAX / 2; t++) U[(mrow - 64) * (NMAX / 2) + t] = v[t];
-        named_bar(3, 128);
-        if (mrow < 64 && mrow < jr.na)
-#pragma unroll
-          for (int t = 0; t < NMAX / 2; t++)
-            if (t < jr.cnt) {
-              const float g = v[t], u = U[mrow * (NMAX / 2) + t];
-              const int p = pl->list[jr.first + t];
-              a.hidden[(size_t)p * a.I + jr.row0 + mrow] =
-                  __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.0f + expf(-g)) * u));
-            }
-      } else {
-        if (mrow < jr.na)
-#pragma unroll
-          for (int t = 0; t < NMAX / 2; t++)
-            if (t < jr.cnt) a.yws[(size_t)pl->list[jr.first + t] * a.H + jr.row0 + mrow] = v[t];
-        __threadfence();
-        named_bar(3, 128);
-        // the last group to finish this 128-row chunk combines it: out = sum_j w_j y_j (fixed j order)
-        if (tid == 0) *s_last = atomicAdd(&a.counters[jr.chunk], 1) == pl->n_groups - 1;
-        named_bar(3, 128);
-        if (*s_last) {
-          __threadfence();
-          for (int i = tid; i < a.Tm * jr.na; i += 128) {
-            const int t = i / jr.na, n = jr.row0 + (i - t * jr.na);
-            float acc = 0.f;
-            for (int jj = 0; jj < a.k; jj++) {
-              const int p = t * a.k + jj, ee = pl->ids[p];
-              if (ee < 0 || ee >= a.E) continue;
-              acc = fmaf(__ldg(a.wts + p), __ldcg(a.yws + (size_t)p * a.H + n), acc);
-            }
-            a.out[(size_t)t * a.H + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+        float *U = reinterpret_cast<float *>(smem + geo.off_U) + (size_t)buf * 64 * C::kTok;
+        const uint32_t use = (uint32_t)(jl_e >> 1);
+        if (warp >= 2) {  // up rows: hand them to the gate rows' warps
+          if (use >= 1 && !mbar_wait(&u_empty[buf], (use - 1u) & 1u, tmo)) {
+            *abort_flag = 1;
+            return;
           }
+#pragma unroll
+          for (int t = 0; t < C::kTok; t++) U[(mrow - 64) * C::kTok + t] = v[t];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&u_full[buf]);
+        } else {
+          if (!mbar_wait(&u_full[buf], use & 1u, tmo)) {
+            *abort_flag = 1;
+            return;
+          }
+          if (mrow < jr.na)
+#pragma unroll
+            for (int t = 0; t < C::kTok; t++)
+              if (t < jr.cnt) {
+                const float g = v[t], u = U[mrow * C::kTok + t];
+                const int p = pl->list[jr.first + t];
+                a.hidden[(size_t)p * a.I + jr.row0 + mrow] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.0f + expf(-g)) * u));
+              }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&u_empty[buf]);
+        }
+      } else {
+        const int row = tile_row(jr, mrow);
+        if (row >= 0)
+#pragma unroll
+          for (int t = 0; t < C::kTok; t++)
+            if (t < jr.cnt) a.yws[(size_t)pl->list[jr.first + t] * a.H + row] = v[t];
+        __threadfence();
+        __syncwarp();
+        // the last group to finish this warp's 32 rows of the chunk combines them:
+        // out = sum_j w_j y_j over the token's routed pairs, in fixed j order
+        int last = 0;
+        if (lane == 0) last = atomicAdd(&a.counters[jr.chunk * 4 + warp], 1) == pl->n_groups - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          const int n = jr.row0 + mrow;
+          if (n < a.H)
+            for (int t = 0; t < a.Tm; t++) {
+              float acc = 0.f;
+              for (int jj = 0; jj < a.k; jj++) {
+                const int p = t * a.k + jj, ee = pl->ids[p];
+                if (ee < 0 || ee >= a.E) continue;
+                acc = fmaf(__ldg(a.wts + p), __ldcg(a.yws + (size_t)p * a.H + n), acc);
+              }
+              a.out[(size_t)t * a.H + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+            }
         }
       }
     };
 
-    for (int q = 0; q < kPref; q++) issue_next(q < nq);
-    uint4 sfb_prev = make_uint4(0u, 0u, 0u, 0u);
     int jl = 0, s = 0, q = 0;
-    uint32_t b = 0, bprev = kNA - 1, empty_phase = 0u, slot = 0;  // A buffer, previous, a_empty parities
-    uint32_t srow = sbase + (uint32_t)m * (uint32_t)nbr + 4u * (uint32_t)h;  // this row's scale bytes, job 0
+    uint32_t ws = 0, wph = 0, b = 0, eph = 0;  // word slot + phase bits, A slot + a_empty phase bits
     for (; q < nq; q++) {
-      cp_async_wait<kPref - 1>();
-      named_bar(1, kDec);
       if (*abort_flag) break;
-      if (warp < 4 && q >= 1) publish_scales(bprev, sfb_prev);
-      const uint4 c0 = lds_u4(cbase + slot * (uint32_t)(kDec * 32)), c1 = lds_u4(cbase + slot * (uint32_t)(kDec * 32) + 16u);
-      if (warp < 4) sfb_prev = lds_u4(fbase + slot * (128u * 16u));
-      // this row's 4 scale bytes of the stage (two 16-bit reads of the job's slab)
-      const uint32_t sa = srow + (uint32_t)(jl & 1) * geo.slab + 8u * (uint32_t)s;
-      const uint32_t sfw = lds_u16(sa) | (lds_u16(sa + 2u) << 16);
-      issue_next(q + kPref < nq);
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&w_full[ws], (wph >> ws) & 1u, tmo);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+      wph ^= 1u << ws;
+      const uint32_t wa = wrow + ws * kWStage;
+      const uint4 c0 = lds_u4(wa + woff0), c1 = lds_u4(wa + woff1);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&w_empty[ws]);
+      ws = ws + 1 == kNW ? 0u : ws + 1;
       uint32_t W[4][4];
       planes_to_nibbles_interleaved(decode_block0(c0.x, c0.y), W[0][0], W[0][1], W[0][2], W[0][3]);
       planes_to_nibbles_interleaved(decode_block0(c0.z, c0.w), W[1][0], W[1][1], W[1][2], W[1][3]);
       planes_to_nibbles_interleaved(decode_block0(c1.x, c1.y), W[2][0], W[2][1], W[2][2], W[2][3]);
       planes_to_nibbles_interleaved(decode_block0(c1.z, c1.w), W[3][0], W[3][1], W[3][2], W[3][3]);
       if (q >= kNA) {
-        if (lane == 0 && !mbar_wait(&a_empty[b], (empty_phase >> b) & 1u, tmo)) *abort_flag = 1;
-        empty_phase ^= 1u << b;
-        __syncwarp();
+        if (lane == 0) ok = mbar_wait(&a_empty[b], (eph >> b) & 1u, tmo);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        eph ^= 1u << b;
+        if (!ok) {
+          *abort_flag = 1;
+          break;
+        }
       }
-      const uint32_t abase = smem_u32(smem + geo.off_A) + b * (128u * kKS) + (uint32_t)(m >> 3) * kSboA +
-                             (uint32_t)(m & 7) * 16u + (uint32_t)h * 1024u;
+      const uint32_t ab = abase + b * kAStage;
+      const int nblk = s == S - 1 ? tail_blocks : 4;
 #pragma unroll
-      for (int i = 0; i < 4; i++) {
-        sts_u2(abase + (uint32_t)(2 * i) * 128u, W[i][0], W[i][1]);
-        sts_u2(abase + (uint32_t)(2 * i + 1) * 128u, W[i][2], W[i][3]);
-      }
-      // scale word of row m (row group sp), K-blocks 4h..4h+3 -> staging word 4h+sp of this lane
-      sts_u32(xbase + b * 1024u + (uint32_t)lane * 32u + (uint32_t)(4 * h + sp) * 4u, sfw);
+      for (int i = 0; i < 4; i++)
+        if (i < nblk) sts_u4(ab + (uint32_t)i * 128u, W[i][0], W[i][1], W[i][2], W[i][3]);
       fence_proxy_async_smem();
-      if (warp >= 4) {  // warps 4-7 release the stage now; warps 0-3 after its scales are in TMEM
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[b]);
-      }
-      if (warp < 4 && jl >= 1 && s == 1) epilogue(jl - 1);
-      bprev = b;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[b]);
       b = b + 1 == kNA ? 0u : b + 1;
-      slot = (slot + 1) & (kPref - 1);
+      if (warp < 4 && jl >= 1 && s == s_epi) epilogue(jl - 1);
       if (++s == S) {
         s = 0;
         ++jl;
       }
     }
-    if (q == nq && nq > 0) {
-      named_bar(1, kDec);  // the last stage's scale staging is complete
-      if (warp < 4) {
-        publish_scales(bprev, sfb_prev);
-        epilogue(my_jobs - 1);
+    if (q == nq && nq > 0 && warp < 4 && !*abort_flag) epilogue(my_jobs - 1);
+  } else if (warp == kLoadWarp) {
+    // ---------------------------------------------------------------- loader warp
+    // TMA front: stage qi of job jl_i; scale staging: stage q of job jl.
+    const uint32_t wbase = smem_u32(smem + geo.off_W), xbase = smem_u32(smem + geo.off_X);
+    unsigned char *my_maps = MODE == kModeGemv ? nullptr : a.maps + (size_t)blockIdx.x * kMapSlots * 128;
+    int qi = 0, jl_i = 0, s_i = 0;
+    uint32_t wi = 0, weph = 0;
+    const void *map_i = &wmap;
+    JobRows ji{};
+    auto start_front_job = [&]() {  // whole warp
+      ji = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_i));
+      if (MODE != kModeGemv) {
+        unsigned char *gm = my_maps + (size_t)(jl_i % kMapSlots) * 128;
+        if (lane == 0) tmap_set_address(smem_u32(smap), ji.st);
+        __syncwarp();
+        tmap_publish(gm, smem_u32(smap));
+        if (lane == 0) tmap_acquire(gm);
+        map_i = gm;
+      }
+    };
+    auto issue_front = [&]() -> bool {  // whole warp; lane 0 issues the two boxes of stage qi
+      if (s_i == 0) start_front_job();
+      bool ok = true;
+      if (lane == 0) {
+        if (qi >= kNW) ok = mbar_wait(&w_empty[wi], (weph >> wi) & 1u, tmo);
+        if (ok) {
+          mbar_arrive_expect_tx(&w_full[wi], kWStage);
+          const uint32_t dst = wbase + wi * kWStage;
+          tma_load_2d(dst, map_i, 64 * s_i, ji.y0, &w_full[wi]);
+          tma_load_2d(dst + 4096u, map_i, 64 * s_i, ji.y1, &w_full[wi]);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) return false;
+      if (qi >= kNW) weph ^= 1u << wi;
+      wi = wi + 1 == kNW ? 0u : wi + 1;
+      qi++;
+      if (++s_i == S) {
+        s_i = 0;
+        jl_i++;
+      }
+      return true;
+    };
+    bool ok = true;
+    while (ok && qi < nq && qi < kNW - 1) ok = issue_front();
+    int jl = 0, s = 0, q = 0;
+    uint32_t b = 0, eph = 0;
+    const uint8_t *rs[4] = {nullptr, nullptr, nullptr, nullptr};  // scale rows of this lane
+    for (; q < nq && ok; q++) {
+      if (*abort_flag) break;
+      if (qi < nq && !(ok = issue_front())) break;
+      if (s == 0) {
+        const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl));
+#pragma unroll
+        for (int r = 0; r < 4; r++) {
+          const int row = tile_row(jr, 32 * r + lane);
+          rs[r] = row >= 0 ? jr.sc + (size_t)row * nbr : nullptr;
+          if (rs[r] != nullptr)
+            for (int o = 0; o < nbr; o += 64) prefetch_l1(rs[r] + o);
+        }
+      }
+      if (q >= kNA) {
+        if (lane == 0) ok = mbar_wait(&a_empty[b], (eph >> b) & 1u, tmo);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        eph ^= 1u << b;
+        if (!ok) break;
+      }
+      // scale bytes of blocks 8s..8s+7 of rows lane, 32+lane, 64+lane, 96+lane (in pairs: nbr is
+      // even, so a pair of blocks is either whole or beyond the row)
+      uint32_t w0[4], w1[4];
+#pragma unroll
+      for (int r = 0; r < 4; r++) {
+        uint32_t p[4] = {0u, 0u, 0u, 0u};
+        if (rs[r] != nullptr) {
+          const unsigned short *src = reinterpret_cast<const unsigned short *>(rs[r] + 8 * s);
+#pragma unroll
+          for (int i = 0; i < 4; i++)
+            if (8 * s + 2 * i < nbr) p[i] = __ldg(src + i);
+        }
+        w0[r] = p[0] | (p[1] << 16);
+        w1[r] = p[2] | (p[3] << 16);
+      }
+      const uint32_t xb = xbase + b * 1024u + (uint32_t)lane * 16u;
+      sts_u4(xb, w0[0], w0[1], w0[2], w0[3]);
+      sts_u4(xb + 512u, w1[0], w1[1], w1[2], w1[3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[b]);
+      b = b + 1 == kNA ? 0u : b + 1;
+      if (++s == S) {
+        s = 0;
+        ++jl;
       }
     }
-    cp_async_wait_all();
+    if (!ok) *abort_flag = 1;
+    // drain: the last min(kNW, qi) issued stages may still be in flight
+    if (lane == 0)
+      for (int d = qi - 1; d >= 0 && d >= qi - kNW; d--)
+        if (!mbar_wait(&w_full[d % kNW], (uint32_t)(d / kNW) & 1u, tmo)) break;
+    __syncwarp();
   } else {
-    // ---------------------------------------------------------------- control warp
+    // ---------------------------------------------------------------- MMA warp
     if (lane == 0) {
-      const uint32_t bstage = (uint32_t)NMAX * kKS;
-      int jl_b = 0, s_b = 0;
+      const uint32_t bslot = C::kBSlot;
+      int issued_b = 0, jl_b = 0, s_b = 0;
       const uint8_t *bsrc = a.Bg;
       auto front_group = [&]() {
-        bsrc = a.Bg + (size_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_b)).group * bsplit_group_bytes(S, NMAX);
+        bsrc = a.Bg + (size_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_b)).group * S * bslot;
       };
       if (my_jobs) front_group();
       uint32_t bb_i = 0;
-      auto issue_b = [&]() {  // B stage of the prefetch front (jl_b, s_b) into ring slot bb_i
-        mbar_arrive_expect_tx(&b_full[bb_i], bstage);
-        bulk_g2s(smem + geo.off_B + bb_i * bstage, bsrc, bstage, &b_full[bb_i]);
-        bsrc += bstage;
+      auto issue_b = [&]() {
+        mbar_arrive_expect_tx(&b_full[bb_i], bslot);
+        bulk_g2s(smem + geo.off_B + bb_i * bslot, bsrc, bslot, &b_full[bb_i]);
+        bsrc += bslot;
         if (++s_b == S) {
           s_b = 0;
           if (++jl_b < my_jobs) front_group();
         }
         bb_i = bb_i + 1 == kNB ? 0u : bb_i + 1;
+        issued_b++;
       };
-      int issued_b = 0;
-      for (; issued_b < kNB && issued_b < nq; issued_b++) issue_b();
-      // instruction descriptors for the four scale-factor byte positions
+      while (issued_b < kNB && issued_b < nq) issue_b();
       int jl = 0, s = 0;
-      uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : NMAX);
-      uint32_t idesc[4];
-      for (int i = 0; i < 4; i++) idesc[i] = idesc_mxf8f6f4_e2m1_e4m3(ncols, (uint32_t)i, (uint32_t)i);
-      uint32_t b = 0, bb = 0, full_phase = 0u, bfull_phase = 0u, bempty_phase = 0u, acc_phase = 0u;
-      const uint32_t a0 = smem_u32(smem + geo.off_A), b0 = smem_u32(smem + geo.off_B);
+      uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : 16);
+      uint32_t idesc0 = idesc_mxf4(ncols, 0u), idesc2 = idesc_mxf4(ncols, 2u);
+      uint32_t b = 0, bb = 0, aph = 0u, bph = 0u, beph = 0u, cph = 0u;
+      const uint32_t a0 = smem_u32(smem + geo.off_A), b0 = smem_u32(smem + geo.off_B), x0 = smem_u32(smem + geo.off_X);
+      bool ok = true;
       for (int q = 0; q < nq; q++) {
-        bool ok = mbar_wait(&a_full[b], (full_phase >> b) & 1u, tmo);
-        full_phase ^= 1u << b;
-        ok = ok && mbar_wait(&b_full[bb], (bfull_phase >> bb) & 1u, tmo);
-        bfull_phase ^= 1u << bb;
+        if (*abort_flag) break;
+        ok = mbar_wait(&a_full[b], (aph >> b) & 1u, tmo);
+        aph ^= 1u << b;
+        ok = ok && mbar_wait(&b_full[bb], (bph >> bb) & 1u, tmo);
+        bph ^= 1u << bb;
         if (ok && s == 0 && jl >= 2) {
-          ok = mbar_wait(&acc_empty[jl & 1], (acc_phase >> (jl & 1)) & 1u, tmo);
-          acc_phase ^= 1u << (jl & 1);
+          ok = mbar_wait(&acc_empty[jl & 1], (cph >> (jl & 1)) & 1u, tmo);
+          cph ^= 1u << (jl & 1);
         }
-        if (!ok) {
-          *abort_flag = 1;
-          break;
-        }
+        if (!ok) break;
         tc_fence_after();
-        const int nkb = nbr - 8 * s < 8 ? nbr - 8 * s : 8;
-        uint64_t ad = smem_desc(a0 + b * (128u * kKS), 128u, kSboA);
-        uint64_t bd = smem_desc(b0 + bb * (uint32_t)NMAX * kKS, 128u, kSboA);
+        // the stage's scale factors into TMEM: A (2 groups x 4 lane quarters), then B
+        const uint32_t sfa = tbase + C::kSfaCol + 8u * b, sfb = tbase + C::kSfbCol + 8u * b;
+        const uint32_t xs = x0 + b * 1024u, bs = b0 + bb * bslot;
+        tmem_cp_32x128_x4(sfa, smem_desc(xs, 128u, 128u));
+        tmem_cp_32x128_x4(sfa + 4u, smem_desc(xs + 512u, 128u, 128u));
+        tmem_cp_32x128_x4(sfb, smem_desc(bs + C::kBTile, 128u, 128u));
+        tmem_cp_32x128_x4(sfb + 4u, smem_desc(bs + C::kBTile + 512u, 128u, 128u));
+        const int nmma = (nbr - 8 * s < 8 ? nbr - 8 * s : 8) >> 1;
+        uint64_t ad = smem_desc(a0 + b * kAStage, 128u, kSbo);
+        uint64_t bd = smem_desc(bs, 128u, kSbo);
         const uint32_t d_t = tbase + (uint32_t)((jl & 1) * NMAX);
-        const uint32_t sfa0 = tbase + kSfaCol + 8u * b, sfb0 = tbase + kSfbCol + 4u * b;
-        for (int kb = 0; kb < nkb; kb++) {
-          const uint32_t byte = (uint32_t)(kb & 3) << 30;
-          mma_mxf8f6f4(d_t, ad, bd, idesc[kb & 3], (sfa0 + 4u * (uint32_t)(kb >> 2)) | byte,
-                       (sfb0 + 2u * (uint32_t)(kb >> 2)) | byte, !(s == 0 && kb == 0));
-          ad += 16u;  // +256 bytes (descriptor start address counts 16-byte units)
+        for (int j = 0; j < nmma; j++) {
+          const uint32_t g = (uint32_t)(j >> 1), sf = (uint32_t)(j & 1) * 2u;
+          mma_mxf4(d_t, ad, bd, sf ? idesc2 : idesc0, (sfa + 4u * g) | (sf << 30), (sfb + 4u * g) | (sf << 30),
+                   !(s == 0 && j == 0));
+          ad += 16u;  // +256 bytes: two chunks (the descriptor's start address counts 16-byte units)
           bd += 16u;
         }
         tc_commit(&a_empty[b]);
         tc_commit(&b_empty[bb]);
         if (s == S - 1) tc_commit(&acc_full[jl & 1]);
-        // refill the B slot of stage q-1 once its MMAs are done (stage q-1+kNB)
+        // refill the B slot of stage q-1 once its MMAs are done (with stage q-1+kNB)
         if (q >= 1 && issued_b < nq) {
           const uint32_t pb = bb == 0 ? kNB - 1 : bb - 1;
-          if (!mbar_wait(&b_empty[pb], (bempty_phase >> pb) & 1u, tmo)) {
-            *abort_flag = 1;
+          if (!mbar_wait(&b_empty[pb], (beph >> pb) & 1u, tmo)) {
+            ok = false;
             break;
           }
-          bempty_phase ^= 1u << pb;
+          beph ^= 1u << pb;
           issue_b();
-          issued_b++;
         }
         b = b + 1 == kNA ? 0u : b + 1;
         bb = bb + 1 == kNB ? 0u : bb + 1;
@@ -652,81 +785,126 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_mma(const __grid_constant__ 
             const uint32_t nc = (uint32_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl)).ncols;
             if (nc != ncols) {
               ncols = nc;
-              for (int i = 0; i < 4; i++) idesc[i] = idesc_mxf8f6f4_e2m1_e4m3(ncols, (uint32_t)i, (uint32_t)i);
+              idesc0 = idesc_mxf4(ncols, 0u);
+              idesc2 = idesc_mxf4(ncols, 2u);
             }
           }
         }
       }
+      if (!ok) *abort_flag = 1;
+      // drain: every tcgen05 operation issued so far, then the B copies that may be in flight
+      tc_commit(drain);
+      mbar_wait(drain, 0u, tmo);
+      for (int d = issued_b - 1; d >= 0 && d >= issued_b - kNB; d--)
+        if (!mbar_wait(&b_full[d % kNB], (uint32_t)(d / kNB) & 1u, tmo)) break;
     }
     __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 8) tmem_dealloc(tbase, kTmemCols);
+  if (warp == kMmaWarp) tmem_dealloc(tbase, C::kTmemCols);
 }
 
 // ------------------------------------------------------------------------------- host side
 
-static int nmax_for(int tokens_per_group) { return tokens_per_group <= 8 ? 16 : 32; }
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
 
-static bool mma_fits(int nbr, int NMAX, int mode) {
+// Tensor map of a trellis stream seen as a [rows][nbr*8] byte matrix, boxes of 64 rows x 64 bytes
+// with the 64-byte swizzle (the decode threads' 16-byte reads of consecutive rows then fall in
+// distinct banks); rows and columns beyond the matrix read as zero.
+static bool make_word_map(CUtensorMap *map, const void *stream, int rows, int nbr) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)nbr * 8u, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)nbr * 8u};
+  cuuint32_t box[2] = {64u, 64u};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(stream), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// GEMV tokens per pass; B width (template NMAX) for a pass or group of T tokens.
+constexpr int kGemvTok = Cfg<96>::kTok;
+static int nmax_for(int tokens_per_group) { return tokens_per_group <= Cfg<32>::kTok ? 32 : 96; }
+
+static bool mma_fits(int NMAX, int mode) {
   int dev = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
-  return mma_geom(nbr, NMAX, mode).smem <= (uint32_t)optin;
+  const uint32_t need = NMAX == 32 ? mma_geom<32>(mode).smem : mma_geom<96>(mode).smem;
+  return need <= (uint32_t)optin;
 }
 
-// The tensor-core path needs at least kPref K stages (K >= 1024), an even number of 32-blocks per
-// row (16-byte aligned row starts), 16-byte aligned scales, and its buffers within shared memory.
-static bool k_ok(int nbr) { return nbr >= 8 * kPref && nbr % 2 == 0; }
+// The tensor-core path needs an even number of 32-blocks per row (whole K = 64 MMAs, and a row
+// pitch that is a multiple of 16 bytes for the tensor map) and a 16-byte aligned stream.
+static bool k_ok(int nbr) { return nbr >= 2 && nbr % 2 == 0; }
 
 bool gemv_mma_supported(const MatView &w, int T) {
-  return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.scales) & 15u) == 0 &&
-         mma_fits(w.nbr, nmax_for(T < 16 ? T : 16), kModeGemv);
+  return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.stream) & 15u) == 0 && tensor_map_encoder() != nullptr &&
+         mma_fits(nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv);
 }
 
-// Tokens beyond 16 run as further passes of at most 16, each with its own split of x.
+// Tokens beyond kGemvTok run as further passes, each with its own split of x.
 size_t gemv_mma_workspace(const MatView &w, int T) {
-  const int S = (w.nbr + 7) / 8, NMAX = nmax_for(T < 16 ? T : 16);
-  return bsplit_group_bytes(S, NMAX) + bsf_group_words(S) * 4;
+  const int S = (w.nbr + 7) / 8;
+  return nmax_for(T < kGemvTok ? T : kGemvTok) == 32 ? (size_t)S * Cfg<32>::kBSlot : (size_t)S * Cfg<96>::kBSlot;
 }
 
-template <int NMAX>
-static cudaError_t launch_gemv_pass(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws,
-                                    cudaStream_t s) {
-  const int S = (w.nbr + 7) / 8;
-  uint8_t *Bg = static_cast<uint8_t *>(ws);
-  uint32_t *Bsf = reinterpret_cast<uint32_t *>(Bg + bsplit_group_bytes(S, NMAX));
-  const int warps = (NMAX / 2) * w.nbr;
-  k_bsplit_gemv<NMAX><<<(warps + 7) / 8, 256, 0, s>>>(x, T, w.nbr * 32, Bg, Bsf);
-  static unsigned long long attr = 0;
-  cudaError_t e = ensure_max_dynamic_smem(k_mma<32, kModeGemv, NMAX>, attr);
-  if (e != cudaSuccess) return e;
+static int sm_count() {
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int ntiles = (w.rows + 127) / 128;
+  return nsm;
+}
+
+template <int NMAX>
+static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, const uint16_t *x, int T, uint16_t *y,
+                                    void *ws, cudaStream_t s) {
+  uint8_t *Bg = static_cast<uint8_t *>(ws);
+  const int warps = Cfg<NMAX>::kSlots * w.nbr;
+  k_bsplit_gemv<NMAX><<<(warps + 7) / 8, 256, 0, s>>>(x, T, w.nbr * 32, Bg);
+  static unsigned long long attr = 0;
+  cudaError_t e = ensure_max_dynamic_smem(k_mma<32, kModeGemv, NMAX>, attr);
+  if (e != cudaSuccess) return e;
+  const int ntiles = (w.rows + 127) / 128, nsm = sm_count();
   MmaArgs args{};
-  args.w = w;
+  args.scales = w.scales;
+  args.rows = w.rows;
   args.nbr = w.nbr;
   args.Bg = Bg;
-  args.Bsf = Bsf;
   args.T = T;
   args.y = y;
   MoeTable<32> none{};
-  k_mma<32, kModeGemv, NMAX><<<ntiles < nsm ? ntiles : nsm, kMmaThreads, mma_geom(w.nbr, NMAX, kModeGemv).smem, s>>>(
-      args, none);
+  k_mma<32, kModeGemv, NMAX><<<ntiles < nsm ? ntiles : nsm, kThreads, mma_geom<NMAX>(kModeGemv).smem, s>>>(args, none,
+                                                                                                          map);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
-  for (int t0 = 0; t0 < T; t0 += 16) {
-    const int n = T - t0 < 16 ? T - t0 : 16;
+  CUtensorMap map;
+  if (!make_word_map(&map, w.stream, w.rows, w.nbr)) return cudaErrorInvalidValue;
+  const bool n32 = nmax_for(T < kGemvTok ? T : kGemvTok) == 32;
+  for (int t0 = 0; t0 < T; t0 += kGemvTok) {
+    const int n = T - t0 < kGemvTok ? T - t0 : kGemvTok;
     const uint16_t *xp = x + (size_t)t0 * w.nbr * 32;
     uint16_t *yp = y + (size_t)t0 * w.rows;
-    cudaError_t e = nmax_for(T < 16 ? T : 16) == 16 ? launch_gemv_pass<16>(w, xp, n, yp, ws, s)
-                                                    : launch_gemv_pass<32>(w, xp, n, yp, ws, s);
+    cudaError_t e =
+        n32 ? launch_gemv_pass<32>(w, map, xp, n, yp, ws, s) : launch_gemv_pass<96>(w, map, xp, n, yp, ws, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -738,28 +916,28 @@ static int moe_groups_max(int E, int P, int gmax) { return (E < P ? E : P) + P /
 
 bool moe_mma_supported(const tcf4_moe &m, int gu_seg, int dn_seg, int T) {
   if (gu_seg != 1 || dn_seg != 1) return false;
-  const int nbr_gu = m.H / 32, nbr_dn = m.I / 32, NMAX = nmax_for(T);
-  if (!k_ok(nbr_gu) || !k_ok(nbr_dn)) return false;
-  if (((size_t)m.I * nbr_gu) % 16 != 0) return false;
+  if (!k_ok(m.H / 32) || !k_ok(m.I / 32) || tensor_map_encoder() == nullptr) return false;
   for (int e = 0; e < m.E; e++)
-    if ((reinterpret_cast<uintptr_t>(m.gate_up[e].scales) | reinterpret_cast<uintptr_t>(m.down[e].scales)) & 15u)
+    if ((reinterpret_cast<uintptr_t>(m.gate_up[e].stream) | reinterpret_cast<uintptr_t>(m.down[e].stream)) & 15u)
       return false;
-  return mma_fits(nbr_gu, NMAX, kModeGateUp) && mma_fits(nbr_dn, NMAX, kModeDown);
+  const int NMAX = nmax_for(T);
+  return mma_fits(NMAX, kModeGateUp) && mma_fits(NMAX, kModeDown);
 }
 
 MoeMmaWorkspace moe_mma_workspace_layout(const tcf4_moe &m, int T, int k) {
   auto a256 = [](size_t v) { return (v + 255) & ~(size_t)255; };
-  const int P = T * k, NMAX = nmax_for(T), G = moe_groups_max(m.E, P, NMAX / 2);
+  const int P = T * k, NMAX = nmax_for(T);
+  const int G = moe_groups_max(m.E, P, NMAX == 32 ? Cfg<32>::kTok : Cfg<96>::kTok);
+  const size_t bslot = NMAX == 32 ? Cfg<32>::kBSlot : Cfg<96>::kBSlot;
   const int S_gu = (m.H / 32 + 7) / 8, S_dn = (m.I / 32 + 7) / 8;
   MoeMmaWorkspace L;
   size_t off = 0;
-  L.counters = off; off = a256(off + sizeof(int) * ((m.H + 127) / 128));
+  L.counters = off; off = a256(off + sizeof(int) * 4 * ((m.H + 127) / 128));
   L.hidden = off;   off = a256(off + sizeof(uint16_t) * (size_t)P * m.I);
   L.y = off;        off = a256(off + sizeof(float) * (size_t)P * m.H);
-  L.bg_gu = off;    off = a256(off + (size_t)G * bsplit_group_bytes(S_gu, NMAX));
-  L.bsf_gu = off;   off = a256(off + (size_t)G * bsf_group_words(S_gu) * 4);
-  L.bg_dn = off;    off = a256(off + (size_t)G * bsplit_group_bytes(S_dn, NMAX));
-  L.bsf_dn = off;   off = a256(off + (size_t)G * bsf_group_words(S_dn) * 4);
+  L.bg_gu = off;    off = a256(off + (size_t)G * S_gu * bslot);
+  L.bg_dn = off;    off = a256(off + (size_t)G * S_dn * bslot);
+  L.maps = off;     off = a256(off + (size_t)sm_count() * kMapSlots * 128);
   L.total = off;
   return L;
 }
@@ -775,6 +953,10 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
     tab.dn[e] = ok ? reinterpret_cast<const uint2 *>(m.down[e].stream) : nullptr;
     tab.dns[e] = ok ? m.down[e].scales : nullptr;
   }
+  CUtensorMap map_gu, map_dn;  // templates from expert 0 (every expert's matrices have the same shape)
+  if (!make_word_map(&map_gu, m.gate_up[0].stream, 2 * m.I, m.H / 32) ||
+      !make_word_map(&map_dn, m.down[0].stream, m.H, m.I / 32))
+    return cudaErrorInvalidValue;
   const MoeMmaWorkspace L = moe_mma_workspace_layout(m, T, k);
   char *base = static_cast<char *>(ws);
   MmaArgs args{};
@@ -790,59 +972,53 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
   args.yws = reinterpret_cast<float *>(base + L.y);
   args.counters = reinterpret_cast<int *>(base + L.counters);
   args.out = out;
-  args.w.stream = reinterpret_cast<const uint2 *>(base);  // a valid address for zero-byte copies
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  const int P = T * k, G = moe_groups_max(m.E, P, NMAX / 2);
+  args.maps = reinterpret_cast<unsigned char *>(base + L.maps);
+  const int nsm = sm_count();
+  const int P = T * k, G = moe_groups_max(m.E, P, Cfg<NMAX>::kTok);
 
   // gate_up: split x per group (and clear the down counters), then decode + MMA + SwiGLU
   {
     uint8_t *Bg = reinterpret_cast<uint8_t *>(base + L.bg_gu);
-    uint32_t *Bsf = reinterpret_cast<uint32_t *>(base + L.bsf_gu);
     const int nbr = m.H / 32;
-    const int warps = G * (NMAX / 2) * nbr;
+    const int warps = G * Cfg<NMAX>::kSlots * nbr;
     k_bsplit_moe<NMAX><<<(warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm, 256, 0, s>>>(
-        ids, P, m.E, k, x, m.H, Bg, Bsf, args.counters, (m.H + 127) / 128);
+        ids, P, m.E, k, x, m.H, Bg, args.counters, 4 * ((m.H + 127) / 128));
     static unsigned long long attr = 0;
     cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, kModeGateUp, NMAX>, attr);
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.Bg = Bg;
-    args.Bsf = Bsf;
     const int jobs = G * ((m.I + 63) / 64);
-    k_mma<MAXE, kModeGateUp, NMAX><<<jobs < nsm ? jobs : nsm, kMmaThreads, mma_geom(nbr, NMAX, kModeGateUp).smem, s>>>(
-        args, tab);
+    k_mma<MAXE, kModeGateUp, NMAX><<<jobs < nsm ? jobs : nsm, kThreads, mma_geom<NMAX>(kModeGateUp).smem, s>>>(
+        args, tab, map_gu);
   }
   // down: split h per group, then decode + MMA, y to the workspace, last arriver per chunk combines
   {
     uint8_t *Bg = reinterpret_cast<uint8_t *>(base + L.bg_dn);
-    uint32_t *Bsf = reinterpret_cast<uint32_t *>(base + L.bsf_dn);
     const int nbr = m.I / 32;
-    const int warps = G * (NMAX / 2) * nbr;
+    const int warps = G * Cfg<NMAX>::kSlots * nbr;
     k_bsplit_moe<NMAX><<<(warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm, 256, 0, s>>>(
-        ids, P, m.E, 1, args.hidden, m.I, Bg, Bsf, nullptr, 0);
+        ids, P, m.E, 1, args.hidden, m.I, Bg, nullptr, 0);
     static unsigned long long attr = 0;
     cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, kModeDown, NMAX>, attr);
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.Bg = Bg;
-    args.Bsf = Bsf;
     const int jobs = G * ((m.H + 127) / 128);
-    k_mma<MAXE, kModeDown, NMAX><<<jobs < nsm ? jobs : nsm, kMmaThreads, mma_geom(nbr, NMAX, kModeDown).smem, s>>>(
-        args, tab);
+    k_mma<MAXE, kModeDown, NMAX><<<jobs < nsm ? jobs : nsm, kThreads, mma_geom<NMAX>(kModeDown).smem, s>>>(args, tab,
+                                                                                                         map_dn);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_moe_mma(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts, int k,
                            uint16_t *out, void *ws, cudaStream_t s) {
-  const bool n16 = nmax_for(T) == 16;
+  const bool n32 = nmax_for(T) == 32;
   if (m.E <= 32)
-    return n16 ? launch_moe_mma_t<32, 16>(m, x, T, ids, wts, k, out, ws, s)
-               : launch_moe_mma_t<32, 32>(m, x, T, ids, wts, k, out, ws, s);
-  return n16 ? launch_moe_mma_t<256, 16>(m, x, T, ids, wts, k, out, ws, s)
-             : launch_moe_mma_t<256, 32>(m, x, T, ids, wts, k, out, ws, s);
+    return n32 ? launch_moe_mma_t<32, 32>(m, x, T, ids, wts, k, out, ws, s)
+               : launch_moe_mma_t<32, 96>(m, x, T, ids, wts, k, out, ws, s);
+  return n32 ? launch_moe_mma_t<256, 32>(m, x, T, ids, wts, k, out, ws, s)
+             : launch_moe_mma_t<256, 96>(m, x, T, ids, wts, k, out, ws, s);
 }
 
 unsigned int take_timeouts_mma() {

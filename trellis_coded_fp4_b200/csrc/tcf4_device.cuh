@@ -60,13 +60,14 @@ __device__ __forceinline__ Planes decode_block0(uint32_t L, uint32_t H) {
 }
 
 // Exchange the bits of a selected by (M << S) with the bits of b selected by M, as two bit selects
-// (two shifts and two three-input logic ops; lop3 LUT 0xE4 = "mask ? x : y").
+// (two shifts and two three-input logic ops; with operands (mask, x, y), lop3 LUT 0xCA is
+// "mask ? x : y").
 template <int S, uint32_t M>
 __device__ __forceinline__ void delta_swap(uint32_t &a, uint32_t &b) {
   uint32_t na, nb;
   const uint32_t a_sh = a >> S, b_sh = b << S;
-  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(nb) : "r"(M), "r"(a_sh), "r"(b));
-  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(na) : "r"(M << S), "r"(b_sh), "r"(a));
+  asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(nb) : "r"(M), "r"(a_sh), "r"(b));
+  asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(na) : "r"(M << S), "r"(b_sh), "r"(a));
   a = na;
   b = nb;
 }

@@ -70,10 +70,10 @@ size_t gemv_mma_workspace(const MatView &w, int T);
 cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s);
 
 // Tensor-core grouped MoE (k_mma.cu): workspace regions (bytes, 256-aligned): the down kernel's
-// per-128-row counters, h (bf16 [T*k][I]), y (fp32 [T*k][H]), and the activation splits of the
-// gate_up and down passes.
+// counters (4 per 128-row chunk of H), h (bf16 [T*k][I]), y (fp32 [T*k][H]), the activation terms
+// of the gate_up and down passes, and per-CTA tensor-map slots.
 struct MoeMmaWorkspace {
-  size_t counters, hidden, y, bg_gu, bsf_gu, bg_dn, bsf_dn, total;
+  size_t counters, hidden, y, bg_gu, bg_dn, maps, total;
 };
 bool moe_mma_supported(const tcf4_moe &m, int gu_seg, int dn_seg, int T);
 MoeMmaWorkspace moe_mma_workspace_layout(const tcf4_moe &m, int T, int k);
