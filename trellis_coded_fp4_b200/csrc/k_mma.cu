@@ -10,11 +10,11 @@
 //
 // One persistent CTA per SM, over 128-row tiles ("jobs") of K stages of 256 (8 blocks of 32):
 //  * loader warp: lane 0 streams each stage's trellis words (128 rows x 64 bytes) into a ring of
-//    shared-memory slots with 2-D TMA tile loads (64-byte swizzle); all lanes stage the stage's
-//    weight scale bytes in the layout tcgen05.cp copies into TMEM.
-//  * 8 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and K-blocks 4(w/4)..4(w/4)+3
-//    of a stage. It reads its 32 bytes of trellis words, decodes them in registers (bit-sliced) and
-//    stores the four 16-byte E2M1 chunks into the stage's A tile.
+//    shared-memory slots with 2-D TMA tile loads (64-byte swizzle).
+//  * 16 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and K-blocks 2(w/4), 2(w/4)+1
+//    of a stage. It reads its 16 bytes of trellis words, decodes them in registers (bit-sliced),
+//    stores the two 16-byte E2M1 chunks into the stage's A tile, and stages the two blocks' scale
+//    bytes (loaded a few stages ahead) in the layout tcgen05.cp copies into TMEM.
 //  * MMA warp: lane 0 streams the activation terms (B) with bulk copies, copies the stage's scale
 //    factors into TMEM (tcgen05.cp) and issues the stage's 4 MMAs into a double-buffered TMEM
 //    accumulator.
@@ -38,10 +38,12 @@ __device__ unsigned int g_tcf4_timeouts_mma = 0;
 
 constexpr int kNW = 6;               // trellis-word stages in flight (TMA ring)
 constexpr int kNA = 4;               // A stages (E2M1 tile + scale staging + TMEM scale slots)
-constexpr int kNB = 3;               // B stages (activation terms + their scales)
+constexpr int kNB = 6;               // B stages (activation terms + their scales)
+constexpr int kBLag = 2;             // a B slot is refilled kBLag stages after its MMAs were issued
+constexpr int kPF = 4;               // stages of weight scale bytes a decode thread keeps in flight
 constexpr int kTerms = 6;            // E2M1 terms per activation block
 constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> kNW jobs in flight)
-constexpr int kLoadWarp = 8, kMmaWarp = 9, kThreads = 320;
+constexpr int kDecWarps = 16, kLoadWarp = 16, kMmaWarp = 17, kThreads = 576;
 constexpr uint32_t kWStage = 8192;   // 128 rows x 64 bytes of trellis words (two 64-row TMA boxes)
 constexpr uint32_t kAStage = 16384;  // 128 rows x 256 E2M1 elements, packed
 constexpr uint32_t kSbo = 1024;      // 8 rows x 8 chunks x 16 bytes: one 8-row group of a stage
@@ -252,6 +254,10 @@ __device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+__device__ __forceinline__ void sts_u16(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"((unsigned short)v) : "memory");
+}
+
 // 2-D TMA tile load (no multicast; the tensor map covers this GPU's memory only).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, int x, int y, uint64_t *bar) {
   asm volatile(
@@ -407,10 +413,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   const MmaGeom geo = mma_geom<NMAX>(MODE);
   uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *w_empty = w_full + 8, *a_full = w_full + 16, *a_empty = w_full + 20, *b_full = w_full + 24,
-           *b_empty = w_full + 28, *acc_full = w_full + 32, *acc_empty = w_full + 34, *u_full = w_full + 36,
-           *u_empty = w_full + 38, *drain = w_full + 40;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 384);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 388);
+           *b_empty = w_full + 32, *acc_full = w_full + 40, *acc_empty = w_full + 42, *u_full = w_full + 44,
+           *u_empty = w_full + 46, *drain = w_full + 48;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 448);  // barriers use bytes [0, 392)
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 452);
   unsigned char *smap = smem + 512;  // shared-memory copy of the tensor map (grouped MoE)
   unsigned int *tmo = &g_tcf4_timeouts_mma;
   GroupPlan *pl = reinterpret_cast<GroupPlan *>(smem + geo.off_P);
@@ -418,10 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   if (tid == 0) {
     for (int i = 0; i < kNW; i++) {
       mbar_init(&w_full[i], 1);
-      mbar_init(&w_empty[i], 8);
+      mbar_init(&w_empty[i], kDecWarps);
     }
     for (int i = 0; i < kNA; i++) {
-      mbar_init(&a_full[i], 9);
+      mbar_init(&a_full[i], kDecWarps);
       mbar_init(&a_empty[i], 1);
     }
     for (int i = 0; i < kNB; i++) {
@@ -460,14 +466,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   auto job_of = [&](int jl) { return (int)blockIdx.x + jl * (int)gridDim.x; };
   const int s_epi = S > 1 ? 1 : 0;  // the epilogue of job jl-1 runs after the A stage (jl, s_epi)
 
-  if (warp < 8) {
+  if (warp < kDecWarps) {
     // ---------------------------------------------------------------- decode warps
     const int sp = warp & 3, h = warp >> 2, m = 32 * sp + lane;
     const uint32_t rb = (uint32_t)(m & 63), sw = (rb >> 1) & 3u;  // row in its TMA box, 64-byte swizzle
-    const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * 4096u + rb * 64u;
-    const uint32_t woff0 = ((2u * h) ^ sw) * 16u, woff1 = ((2u * h + 1u) ^ sw) * 16u;
-    const uint32_t abase = smem_u32(smem + geo.off_A) + chunk_off((uint32_t)m, 4u * (uint32_t)h);
-    const int tail_blocks = nbr - 8 * (S - 1) - 4 * h;  // this thread's blocks in the last stage
+    const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * 4096u + rb * 64u + (((uint32_t)h ^ sw) * 16u);
+    const uint32_t abase = smem_u32(smem + geo.off_A) + chunk_off((uint32_t)m, 2u * (uint32_t)h);
+    const int tail_blocks = nbr - 8 * (S - 1) - 2 * h;  // this thread's blocks in the last stage
 
     auto epilogue = [&](int jl_e) {
       const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
@@ -558,57 +563,91 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       }
     };
 
+    // The scale bytes of this thread's two blocks (one 16-bit load per stage), kPF stages ahead of
+    // their use: sfr[u] holds the stage q with q % kPF == u.
+    const uint32_t xlane = smem_u32(smem + geo.off_X) + (uint32_t)(h >> 1) * 512u + (uint32_t)lane * 16u +
+                           (uint32_t)sp * 4u + (uint32_t)(h & 1) * 2u;
+    uint32_t sfr[kPF];
+    int qp = 0, jl_p = 0, s_p = 0;
+    const unsigned short *srow = nullptr;  // row m's scales of the front job, from block 2h on
+    auto load_sf = [&](uint32_t &dst) {
+      if (qp >= nq) return;
+      if (s_p == 0) {
+        const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_p));
+        const int row = tile_row(jr, m);
+        srow = row >= 0 ? reinterpret_cast<const unsigned short *>(jr.sc + (size_t)row * nbr + 2 * h) : nullptr;
+      }
+      dst = srow != nullptr && 8 * s_p + 2 * h < nbr ? (uint32_t)__ldg(srow + 4 * s_p) : 0u;
+      qp++;
+      if (++s_p == S) {
+        s_p = 0;
+        jl_p++;
+      }
+    };
+#pragma unroll
+    for (int u = 0; u < kPF; u++) load_sf(sfr[u]);
+
     int jl = 0, s = 0, q = 0;
     uint32_t ws = 0, wph = 0, b = 0, eph = 0;  // word slot + phase bits, A slot + a_empty phase bits
-    for (; q < nq; q++) {
-      if (*abort_flag) break;
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(&w_full[ws], (wph >> ws) & 1u, tmo);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        *abort_flag = 1;
-        break;
-      }
-      wph ^= 1u << ws;
-      const uint32_t wa = wrow + ws * kWStage;
-      const uint4 c0 = lds_u4(wa + woff0), c1 = lds_u4(wa + woff1);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&w_empty[ws]);
-      ws = ws + 1 == kNW ? 0u : ws + 1;
-      uint32_t W[4][4];
-      planes_to_nibbles_interleaved(decode_block0(c0.x, c0.y), W[0][0], W[0][1], W[0][2], W[0][3]);
-      planes_to_nibbles_interleaved(decode_block0(c0.z, c0.w), W[1][0], W[1][1], W[1][2], W[1][3]);
-      planes_to_nibbles_interleaved(decode_block0(c1.x, c1.y), W[2][0], W[2][1], W[2][2], W[2][3]);
-      planes_to_nibbles_interleaved(decode_block0(c1.z, c1.w), W[3][0], W[3][1], W[3][2], W[3][3]);
-      if (q >= kNA) {
-        if (lane == 0) ok = mbar_wait(&a_empty[b], (eph >> b) & 1u, tmo);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        eph ^= 1u << b;
-        if (!ok) {
-          *abort_flag = 1;
+    bool stop = false;
+    for (int q0 = 0; q0 < nq && !stop; q0 += kPF) {
+#pragma unroll
+      for (int u = 0; u < kPF; u++) {
+        q = q0 + u;
+        if (q >= nq || *abort_flag) {
+          stop = true;
           break;
         }
-      }
-      const uint32_t ab = abase + b * kAStage;
-      const int nblk = s == S - 1 ? tail_blocks : 4;
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&w_full[ws], (wph >> ws) & 1u, tmo);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          *abort_flag = 1;
+          stop = true;
+          break;
+        }
+        wph ^= 1u << ws;
+        const uint4 c0 = lds_u4(wrow + ws * kWStage);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&w_empty[ws]);
+        ws = ws + 1 == kNW ? 0u : ws + 1;
+        uint32_t W[2][4];
+        planes_to_nibbles_interleaved(decode_block0(c0.x, c0.y), W[0][0], W[0][1], W[0][2], W[0][3]);
+        planes_to_nibbles_interleaved(decode_block0(c0.z, c0.w), W[1][0], W[1][1], W[1][2], W[1][3]);
+        if (q >= kNA) {
+          if (lane == 0) ok = mbar_wait(&a_empty[b], (eph >> b) & 1u, tmo);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          eph ^= 1u << b;
+          if (!ok) {
+            *abort_flag = 1;
+            stop = true;
+            break;
+          }
+        }
+        const uint32_t ab = abase + b * kAStage;
+        const int nblk = s == S - 1 ? tail_blocks : 2;
 #pragma unroll
-      for (int i = 0; i < 4; i++)
-        if (i < nblk) sts_u4(ab + (uint32_t)i * 128u, W[i][0], W[i][1], W[i][2], W[i][3]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[b]);
-      b = b + 1 == kNA ? 0u : b + 1;
-      if (warp < 4 && jl >= 1 && s == s_epi) epilogue(jl - 1);
-      if (++s == S) {
-        s = 0;
-        ++jl;
+        for (int i = 0; i < 2; i++)
+          if (i < nblk) sts_u4(ab + (uint32_t)i * 128u, W[i][0], W[i][1], W[i][2], W[i][3]);
+        sts_u16(xlane + b * 1024u, sfr[u]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[b]);
+        load_sf(sfr[u]);
+        b = b + 1 == kNA ? 0u : b + 1;
+        if (warp < 4 && jl >= 1 && s == s_epi) epilogue(jl - 1);
+        if (++s == S) {
+          s = 0;
+          ++jl;
+        }
       }
     }
+    if (!stop) q = nq;
     if (q == nq && nq > 0 && warp < 4 && !*abort_flag) epilogue(my_jobs - 1);
   } else if (warp == kLoadWarp) {
     // ---------------------------------------------------------------- loader warp
-    // TMA front: stage qi of job jl_i; scale staging: stage q of job jl.
-    const uint32_t wbase = smem_u32(smem + geo.off_W), xbase = smem_u32(smem + geo.off_X);
+    // TMA front: stage qi of job jl_i, up to kNW stages ahead of the decode warps.
+    const uint32_t wbase = smem_u32(smem + geo.off_W);
     unsigned char *my_maps = MODE == kModeGemv ? nullptr : a.maps + (size_t)blockIdx.x * kMapSlots * 128;
     int qi = 0, jl_i = 0, s_i = 0;
     uint32_t wi = 0, weph = 0;
@@ -649,56 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       return true;
     };
     bool ok = true;
-    while (ok && qi < nq && qi < kNW - 1) ok = issue_front();
-    int jl = 0, s = 0, q = 0;
-    uint32_t b = 0, eph = 0;
-    const uint8_t *rs[4] = {nullptr, nullptr, nullptr, nullptr};  // scale rows of this lane
-    for (; q < nq && ok; q++) {
-      if (*abort_flag) break;
-      if (qi < nq && !(ok = issue_front())) break;
-      if (s == 0) {
-        const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl));
-#pragma unroll
-        for (int r = 0; r < 4; r++) {
-          const int row = tile_row(jr, 32 * r + lane);
-          rs[r] = row >= 0 ? jr.sc + (size_t)row * nbr : nullptr;
-          if (rs[r] != nullptr)
-            for (int o = 0; o < nbr; o += 64) prefetch_l1(rs[r] + o);
-        }
-      }
-      if (q >= kNA) {
-        if (lane == 0) ok = mbar_wait(&a_empty[b], (eph >> b) & 1u, tmo);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        eph ^= 1u << b;
-        if (!ok) break;
-      }
-      // scale bytes of blocks 8s..8s+7 of rows lane, 32+lane, 64+lane, 96+lane (in pairs: nbr is
-      // even, so a pair of blocks is either whole or beyond the row)
-      uint32_t w0[4], w1[4];
-#pragma unroll
-      for (int r = 0; r < 4; r++) {
-        uint32_t p[4] = {0u, 0u, 0u, 0u};
-        if (rs[r] != nullptr) {
-          const unsigned short *src = reinterpret_cast<const unsigned short *>(rs[r] + 8 * s);
-#pragma unroll
-          for (int i = 0; i < 4; i++)
-            if (8 * s + 2 * i < nbr) p[i] = __ldg(src + i);
-        }
-        w0[r] = p[0] | (p[1] << 16);
-        w1[r] = p[2] | (p[3] << 16);
-      }
-      const uint32_t xb = xbase + b * 1024u + (uint32_t)lane * 16u;
-      sts_u4(xb, w0[0], w0[1], w0[2], w0[3]);
-      sts_u4(xb + 512u, w1[0], w1[1], w1[2], w1[3]);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[b]);
-      b = b + 1 == kNA ? 0u : b + 1;
-      if (++s == S) {
-        s = 0;
-        ++jl;
-      }
-    }
+    while (ok && qi < nq && !*abort_flag) ok = issue_front();
     if (!ok) *abort_flag = 1;
     // drain: the last min(kNW, qi) issued stages may still be in flight
     if (lane == 0)
@@ -731,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       int jl = 0, s = 0;
       uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : 16);
       uint32_t idesc0 = idesc_mxf4(ncols, 0u), idesc2 = idesc_mxf4(ncols, 2u);
-      uint32_t b = 0, bb = 0, aph = 0u, bph = 0u, beph = 0u, cph = 0u;
+      uint32_t b = 0, bb = 0, aph = 0u, bph = 0u, cph = 0u;
       const uint32_t a0 = smem_u32(smem + geo.off_A), b0 = smem_u32(smem + geo.off_B), x0 = smem_u32(smem + geo.off_X);
       bool ok = true;
       for (int q = 0; q < nq; q++) {
@@ -767,14 +757,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         tc_commit(&a_empty[b]);
         tc_commit(&b_empty[bb]);
         if (s == S - 1) tc_commit(&acc_full[jl & 1]);
-        // refill the B slot of stage q-1 once its MMAs are done (with stage q-1+kNB)
-        if (q >= 1 && issued_b < nq) {
-          const uint32_t pb = bb == 0 ? kNB - 1 : bb - 1;
-          if (!mbar_wait(&b_empty[pb], (beph >> pb) & 1u, tmo)) {
+        // refill the B slot of stage q-kBLag, whose MMAs were issued kBLag stages ago, with stage
+        // q-kBLag+kNB
+        if (q >= kBLag && issued_b < nq) {
+          const int qq = q - kBLag;
+          if (!mbar_wait(&b_empty[qq % kNB], (uint32_t)(qq / kNB) & 1u, tmo)) {
             ok = false;
             break;
           }
-          beph ^= 1u << pb;
           issue_b();
         }
         b = b + 1 == kNA ? 0u : b + 1;

@@ -11,10 +11,9 @@
 
 namespace tcf4 {
 
-// A wait gives up after kSpinLimit rounds of try_wait, each suspending for at most ~kSuspendNs:
-// about two seconds, far beyond any real wait (microseconds).
-constexpr uint32_t kSpinLimit = 1u << 20;
-constexpr uint32_t kSuspendNs = 2000u;
+// A wait gives up after about two seconds (kWaitCycles SM clock cycles), far beyond any real wait
+// (microseconds).
+constexpr long long kWaitCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -33,6 +32,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
+// One try_wait: the thread sleeps until the phase with the given parity completes (it is woken
+// then) or at most ~kSuspendNs; true once that phase has completed.
+constexpr uint32_t kSuspendNs = 1000000u;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -48,8 +50,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Bounded wait for the phase with the given parity to complete. Returns false on timeout, after
 // counting it in *timeouts.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *timeouts) {
-  for (uint32_t i = 0; i < kSpinLimit; i++)
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  do {
     if (mbar_try_wait(bar, parity)) return true;
+  } while (clock64() - t0 < kWaitCycles);
   atomicAdd(timeouts, 1u);
   return false;
 }
