@@ -8,21 +8,23 @@
 // residual expansion, see split_terms): B column kTerms*t + j holds term j of token t, and
 // y[t] = sum_j D[:, kTerms*t + j] in fp32.
 //
-// One persistent CTA per SM, over 128-row tiles ("jobs") of K stages of 256 (8 blocks of 32):
-//  * loader warp: lane 0 streams each stage's trellis words (128 rows x 64 bytes) into a ring of
-//    shared-memory slots with 2-D TMA tile loads (64-byte swizzle).
-//  * 16 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and K-blocks 2(w/4), 2(w/4)+1
-//    of a stage. It reads its 16 bytes of trellis words, decodes them in registers (bit-sliced),
-//    stores the two 16-byte E2M1 chunks into the stage's A tile, and stages the two blocks' scale
-//    bytes (loaded a few stages ahead) in the layout tcgen05.cp copies into TMEM.
-//  * MMA warp: lane 0 streams the activation terms (B) with bulk copies, copies the stage's scale
-//    factors into TMEM (tcgen05.cp) and issues the stage's 4 MMAs into a double-buffered TMEM
-//    accumulator.
+// One persistent CTA per SM, over 128-row tiles ("jobs") of K stages of 512 (16 blocks of 32):
+//  * word loader warp: lane 0 streams each stage's trellis words (128 rows x 128 bytes) into a ring
+//    of shared-memory slots with 2-D TMA tile loads (128-byte swizzle).
+//  * 16 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and the four K-blocks
+//    4(w/4)..4(w/4)+3 of a stage (one scale-factor group). It reads its 32 bytes of trellis words,
+//    decodes them in registers (bit-sliced), stores the four 16-byte E2M1 chunks into the stage's A
+//    tile, and writes the group's scale factors of its row (A) and of the B rows its lane stands
+//    for into TMEM (tcgen05.st into its own lane quarter; the scale bytes are loaded a few stages
+//    ahead).
+//  * B loader warp: lane 0 bulk-copies each stage's activation terms into the B slot of the stage.
+//  * MMA warp: lane 0 waits for a stage, issues its 8 MMAs into a double-buffered TMEM
+//    accumulator and releases the stage with one commit.
 //  * the epilogue of job i (tcgen05.ld, then the GEMV output, the SwiGLU of gate/up rows, or the MoE
 //    down rows and their combine) runs in decode warps 0-3 early in job i+1.
-// Every wait is a bounded mbarrier wait; a wait that gives up raises a shared abort flag that every
-// role polls once per stage, and each role drains its own asynchronous copies and MMAs before the
-// CTA frees its TMEM.
+// All tcgen05 MMAs of the CTA are issued by one thread. Every wait is a bounded mbarrier wait; a
+// wait that gives up raises a shared abort flag that every role polls once per stage, and each
+// role drains its own asynchronous copies and MMAs before the CTA frees its TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -36,30 +38,30 @@ namespace tcf4 {
 
 __device__ unsigned int g_tcf4_timeouts_mma = 0;
 
-constexpr int kNW = 6;               // trellis-word stages in flight (TMA ring)
-constexpr int kNA = 4;               // A stages (E2M1 tile + scale staging + TMEM scale slots)
-constexpr int kNB = 6;               // B stages (activation terms + their scales)
-constexpr int kBLag = 2;             // a B slot is refilled kBLag stages after its MMAs were issued
-constexpr int kPF = 4;               // stages of weight scale bytes a decode thread keeps in flight
+constexpr int kKB = 16;              // 32-blocks per row per stage (K = 512)
 constexpr int kTerms = 6;            // E2M1 terms per activation block
-constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> kNW jobs in flight)
-constexpr int kDecWarps = 16, kLoadWarp = 16, kMmaWarp = 17, kThreads = 576;
-constexpr uint32_t kWStage = 8192;   // 128 rows x 64 bytes of trellis words (two 64-row TMA boxes)
-constexpr uint32_t kAStage = 16384;  // 128 rows x 256 E2M1 elements, packed
-constexpr uint32_t kSbo = 1024;      // 8 rows x 8 chunks x 16 bytes: one 8-row group of a stage
+constexpr int kPF = 4;               // stages of scale factors a decode thread keeps in flight
+constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> jobs in flight)
+constexpr int kDecWarps = 16, kWLoadWarp = 16, kMmaWarp = 17, kBLoadWarp = 18, kThreads = 608;
+constexpr uint32_t kWStage = 16384;  // 128 rows x 128 bytes of trellis words (two 64-row TMA boxes)
+constexpr uint32_t kAStage = 32768;  // 128 rows x 512 E2M1 elements, packed
+constexpr uint32_t kSbo = 2048;      // 8 rows x 16 chunks x 16 bytes: one 8-row group of a stage
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
 
 template <int NMAX>
 struct Cfg {
+  static_assert(NMAX <= 128, "B scale factors of a 4-block group fit one 4-column TMEM slot");
   static constexpr int kTok = NMAX / kTerms;                   // tokens per group
   static constexpr int kSlots = (NMAX + kTerms - 1) / kTerms;  // token slots the split writes
-  static_assert(NMAX <= 128, "B scale factors of a 4-block group fit one 4-column TMEM slot");
-  static constexpr uint32_t kBTile = NMAX * 128u;              // NMAX rows x 256 E2M1
-  static constexpr uint32_t kBSlot = kBTile + 2u * 512u;       // + scales: one 32x128b copy per group
+  static constexpr int kC = (NMAX + 31) / 32;                  // B scale columns per 4-block group
+  static constexpr int kNW = 4;                                // word stages in flight
+  static constexpr int kNA = NMAX <= 32 ? 3 : 2;               // A / B / scale-factor stages
+  static constexpr uint32_t kBStage = NMAX * 256u;             // NMAX rows x 512 E2M1
+  static constexpr uint32_t kSfbStage = 4u * kC * 128u;        // [group][column][lane] u32
   static constexpr uint32_t kSfaCol = 2u * NMAX;               // TMEM: accumulators first
-  static constexpr uint32_t kSfbCol = kSfaCol + 8u * kNA;
-  static constexpr uint32_t kUsed = kSfbCol + 8u * kNA;
+  static constexpr uint32_t kSfbCol = kSfaCol + 16u * kNA;     // 16 columns per stage each
+  static constexpr uint32_t kUsed = kSfbCol + 16u * kNA;
   static constexpr uint32_t kTmemCols = kUsed <= 128 ? 128 : (kUsed <= 256 ? 256 : 512);
 };
 
@@ -68,8 +70,8 @@ struct Cfg {
 // 4j..4j+3 of the chunk (element 2b in the low nibble of byte b).
 __host__ __device__ constexpr int kpos_of_weight(int i) { return 8 * (i & 3) + (i >> 2); }
 
-// Byte offset of chunk c (0..7) of row n in a K-major, no-swizzle stage: core matrices of 8 rows
-// x 16 bytes, LBO = 128 (adjacent chunks), SBO = 1024 (adjacent 8-row groups).
+// Byte offset of chunk c (0..15) of row n in a K-major, no-swizzle stage: core matrices of 8 rows
+// x 16 bytes, LBO = 128 (adjacent chunks), SBO = 2048 (adjacent 8-row groups).
 __host__ __device__ constexpr uint32_t chunk_off(uint32_t n, uint32_t c) {
   return (n >> 3) * kSbo + c * 128u + (n & 7u) * 16u;
 }
@@ -146,18 +148,27 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
   return (c & 8u) ? -v : v;
 }
 
-// One 32-element block of one activation row (lane = element) -> kTerms E2M1 terms with UE8M0
-// scales, written as B rows kTerms*t .. kTerms*t+kTerms-1 of chunk kb of the group's B stages.
+// Per group of token slots, the activation terms of each stage: Bg [S][kBStage] (one K-major B
+// stage each) and Bsf [S][kSfbStage]: word (h, c, lane) of a stage holds the UE8M0 bytes of B row
+// 32c+lane for the stage's blocks 4h..4h+3 (byte i = block 4h+i).
+template <int NMAX>
+__host__ __device__ inline size_t terms_bytes(int S) {
+  return (size_t)S * (Cfg<NMAX>::kBStage + Cfg<NMAX>::kSfbStage);
+}
+
+// One 32-element block kb of one activation row (lane = element) -> kTerms E2M1 terms with UE8M0
+// scales, written as B rows kTerms*t .. kTerms*t+kTerms-1 of the group's terms (layout above).
 // Term j: with m the largest |residual| of the block, scale 2^S with S = ceil(log2(m / 6)) puts the
 // block in (3, 6]; each residual is rounded to the E2M1 grid (nearest even) and the rounded value
 // removed (exactly: Sterbenz). The largest residual shrinks by at least 5x per term, so after
 // kTerms terms |x - sum| <= 5^-6 max|x| over the block.
 template <int NMAX>
-__device__ __forceinline__ void split_terms(float v, int t, int kb, uint8_t *Bg) {
+__device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total, uint8_t *terms) {
   using C = Cfg<NMAX>;
   const int lane = threadIdx.x & 31;
-  const int s = kb >> 3, c = kb & 7, g = c >> 2;
-  uint8_t *slot = Bg + (size_t)s * C::kBSlot;
+  const int s = kb / kKB, c = kb - s * kKB, h = c >> 2;
+  uint8_t *bst = terms + (size_t)s * C::kBStage;
+  uint8_t *sfs = terms + (size_t)S_total * C::kBStage + (size_t)s * C::kSfbStage;
   const int kp = kpos_of_weight(lane);
   float r = v;
 #pragma unroll
@@ -175,9 +186,8 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, uint8_t *Bg)
     const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 4);
     if (n < NMAX) {
       if (((lane >> 2) & 1) == 0)
-        slot[chunk_off((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code | (partner << 4));
-      if (lane == 0)  // group g's copy: lane n%32, word n/32 (TMEM column 4g + n/32), byte = block in group
-        slot[C::kBTile + g * 512 + (n & 31) * 16 + (n >> 5) * 4 + (c & 3)] = (uint8_t)(S + 127);
+        bst[chunk_off((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code | (partner << 4));
+      if (lane == 0) sfs[((h * C::kC + (n >> 5)) * 32 + (n & 31)) * 4 + (c & 3)] = (uint8_t)(S + 127);
     }
   }
 }
@@ -185,13 +195,13 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, uint8_t *Bg)
 // Plain GEMV: one group, token slots 0..T-1 (slots up to kSlots are zero rows).
 template <int NMAX>
 __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
-                                                     uint8_t *__restrict__ Bg) {
-  const int nb = K >> 5, lane = threadIdx.x & 31;
+                                                     uint8_t *__restrict__ terms) {
+  const int nb = K >> 5, S = (nb + kKB - 1) / kKB, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < Cfg<NMAX>::kSlots * nb; wi += nwarps) {
     const int t = wi / nb, kb = wi - t * nb;
     const float v = t < T ? __uint_as_float((uint32_t)x[(size_t)t * K + kb * 32 + lane] << 16) : 0.f;
-    split_terms<NMAX>(v, t, kb, Bg);
+    split_terms<NMAX>(v, t, kb, S, terms);
   }
 }
 
@@ -200,13 +210,13 @@ __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict_
 // clears the down kernel's counters when `counters` is given.
 template <int NMAX>
 __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ ids, int P, int E, int div,
-                                                    const uint16_t *__restrict__ src, int K, uint8_t *__restrict__ Bg,
+                                                    const uint16_t *__restrict__ src, int K, uint8_t *__restrict__ terms,
                                                     int *__restrict__ counters, int n_counters) {
   __shared__ GroupPlan pl;
   if (counters != nullptr && blockIdx.x == 0)
     for (int c = threadIdx.x; c < n_counters; c += blockDim.x) counters[c] = 0;
   build_groups(pl, ids, P, E, Cfg<NMAX>::kTok);
-  const int nb = K >> 5, S = (nb + 7) >> 3;
+  const int nb = K >> 5, S = (nb + kKB - 1) / kKB;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int per_group = Cfg<NMAX>::kSlots * nb;
@@ -218,27 +228,27 @@ __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ 
       const int row = pl.list[pl.g_first[g] + t] / div;
       v = __uint_as_float((uint32_t)src[(size_t)row * K + kb * 32 + lane] << 16);
     }
-    split_terms<NMAX>(v, t, kb, Bg + (size_t)g * S * Cfg<NMAX>::kBSlot);
+    split_terms<NMAX>(v, t, kb, S, terms + (size_t)g * terms_bytes<NMAX>(S));
   }
 }
 
 // ------------------------------------------------------------------------------- geometry
 
-// Shared memory: barriers + tensor-map copy | word ring | A ring | scale staging | B ring
-// | gate/up exchange | group plan.
+// Shared memory: barriers + tensor-map copy | word ring | A ring | B ring | gate/up exchange
+// | group plan.
 struct MmaGeom {
-  uint32_t off_W, off_A, off_X, off_B, off_U, off_P, smem;
+  uint32_t off_W, off_A, off_B, off_U, off_P, smem;
 };
 
 template <int NMAX>
 __host__ __device__ inline MmaGeom mma_geom(int mode) {
+  using C = Cfg<NMAX>;
   MmaGeom g;
   g.off_W = 1024u;
-  g.off_A = g.off_W + kNW * kWStage;
-  g.off_X = g.off_A + kNA * kAStage;
-  g.off_B = g.off_X + kNA * 1024u;
-  g.off_U = g.off_B + kNB * Cfg<NMAX>::kBSlot;
-  g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)Cfg<NMAX>::kTok * 4u : 0u);
+  g.off_A = g.off_W + C::kNW * kWStage;
+  g.off_B = g.off_A + C::kNA * kAStage;
+  g.off_U = g.off_B + C::kNA * C::kBStage;
+  g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)C::kTok * 4u : 0u);
   g.smem = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
   return g;
 }
@@ -254,10 +264,6 @@ __device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__device__ __forceinline__ void sts_u16(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"((unsigned short)v) : "memory");
-}
-
 // 2-D TMA tile load (no multicast; the tensor map covers this GPU's memory only).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, int x, int y, uint64_t *bar) {
   asm volatile(
@@ -267,10 +273,9 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, int x
       : "memory");
 }
 
-// Shared memory (32 rows x 16 bytes) -> 4 TMEM columns of 32 lanes, replicated into all four lane
-// quarters.
-__device__ __forceinline__ void tmem_cp_32x128_x4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+// Warp-wide stores of one / four consecutive TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t a) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
 }
 
 // Instruction descriptor of a block-scaled kind::mxf4 MMA: A = B = E2M1, K-major, UE8M0 scales per
@@ -287,6 +292,8 @@ __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t N, uint32_t sf) {
   return d;                // bit 31 = 0: K = 64
 }
 
+// One thread: D[tmem] (+)= A[smem] x B[smem], block-scaled. The A scale factors of rows
+// 32q..32q+31 are read from lane quarter q at column sfa+q, those of B row n from column sfb + n/32.
 __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          uint32_t sfa_tmem, uint32_t sfb_tmem, bool accumulate) {
   asm volatile(
@@ -314,15 +321,13 @@ __device__ __forceinline__ void tmap_acquire(const void *gmap) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmap) : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l1(const void *p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
-
 // ------------------------------------------------------------------------------- kernel arguments
 
 struct MmaArgs {
   const uint8_t *scales;  // GEMV: the matrix's scales (MoE: from the table)
   int rows;               // GEMV rows
   int nbr;                // 32-blocks per row (K / 32)
-  const uint8_t *Bg;      // activation terms, per group [S][kBSlot]
+  const uint8_t *terms;   // activation terms, per group (terms_bytes each)
   int T;                  // GEMV tokens
   uint16_t *y;            // GEMV out [T][rows]
   const int32_t *ids;     // MoE routing [T][k]
@@ -336,8 +341,8 @@ struct MmaArgs {
 };
 
 // A job is one 128-row tile: tile rows [0, 64) are matrix rows y0.., tile rows [64, 128) matrix
-// rows y1..; na / nb of them valid. B group `group`, MMA width ncols; `cnt` tokens starting at
-// list index `first`.
+// rows y1..; na / nb of them valid. Activation group `group`, MMA width ncols; `cnt` tokens
+// starting at list index `first`.
 struct JobRows {
   const void *st;     // the matrix stream (MoE: the tensor map's address)
   const uint8_t *sc;  // its scales
@@ -407,19 +412,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
                                                      const __grid_constant__ MoeTable<MAXE> tab,
                                                      const __grid_constant__ CUtensorMap wmap) {
   using C = Cfg<NMAX>;
+  constexpr int kNW = C::kNW, kNA = C::kNA;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nbr = a.nbr, S = (nbr + 7) >> 3;
+  const int nbr = a.nbr, S = (nbr + kKB - 1) / kKB;
   const MmaGeom geo = mma_geom<NMAX>(MODE);
-  uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);
-  uint64_t *w_empty = w_full + 8, *a_full = w_full + 16, *a_empty = w_full + 20, *b_full = w_full + 24,
-           *b_empty = w_full + 32, *acc_full = w_full + 40, *acc_empty = w_full + 42, *u_full = w_full + 44,
-           *u_empty = w_full + 46, *drain = w_full + 48;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 448);  // barriers use bytes [0, 392)
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 452);
+  uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);  // 29 barriers in bytes [0, 232)
+  uint64_t *w_empty = w_full + 4, *a_full = w_full + 8, *a_empty = w_full + 12, *b_full = w_full + 16,
+           *acc_full = w_full + 20, *acc_empty = w_full + 22, *u_full = w_full + 24, *u_empty = w_full + 26,
+           *drain = w_full + 28;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 256);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 260);
   unsigned char *smap = smem + 512;  // shared-memory copy of the tensor map (grouped MoE)
   unsigned int *tmo = &g_tcf4_timeouts_mma;
   GroupPlan *pl = reinterpret_cast<GroupPlan *>(smem + geo.off_P);
+  const size_t tbytes = terms_bytes<NMAX>(S);
 
   if (tid == 0) {
     for (int i = 0; i < kNW; i++) {
@@ -429,10 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
     for (int i = 0; i < kNA; i++) {
       mbar_init(&a_full[i], kDecWarps);
       mbar_init(&a_empty[i], 1);
-    }
-    for (int i = 0; i < kNB; i++) {
       mbar_init(&b_full[i], 1);
-      mbar_init(&b_empty[i], 1);
     }
     for (int i = 0; i < 2; i++) {
       mbar_init(&acc_full[i], 1);
@@ -469,11 +473,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   if (warp < kDecWarps) {
     // ---------------------------------------------------------------- decode warps
     const int sp = warp & 3, h = warp >> 2, m = 32 * sp + lane;
-    const uint32_t rb = (uint32_t)(m & 63), sw = (rb >> 1) & 3u;  // row in its TMA box, 64-byte swizzle
-    const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * 4096u + rb * 64u + (((uint32_t)h ^ sw) * 16u);
-    const uint32_t abase = smem_u32(smem + geo.off_A) + chunk_off((uint32_t)m, 2u * (uint32_t)h);
-    const int tail_blocks = nbr - 8 * (S - 1) - 2 * h;  // this thread's blocks in the last stage
-
+    const uint32_t rb = (uint32_t)(m & 63), sw = rb & 7u;  // row in its TMA box, 128-byte swizzle
+    const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * 8192u + rb * 128u;
+    const uint32_t wo0 = ((2u * h) ^ sw) * 16u, wo1 = ((2u * h + 1u) ^ sw) * 16u;
+    const uint32_t abase = smem_u32(smem + geo.off_A) + chunk_off((uint32_t)m, 4u * (uint32_t)h);
+    const uint32_t tq = tbase + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lane quarter
+    const int tail_blocks = nbr - kKB * (S - 1) - 4 * h;      // this thread's blocks in the last stage
     auto epilogue = [&](int jl_e) {
       const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
       const int buf = jl_e & 1;
@@ -563,21 +568,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       }
     };
 
-    // The scale bytes of this thread's two blocks (one 16-bit load per stage), kPF stages ahead of
-    // their use: sfr[u] holds the stage q with q % kPF == u.
-    const uint32_t xlane = smem_u32(smem + geo.off_X) + (uint32_t)(h >> 1) * 512u + (uint32_t)lane * 16u +
-                           (uint32_t)sp * 4u + (uint32_t)(h & 1) * 2u;
-    uint32_t sfr[kPF];
+    // Scale factors of this thread's group of four blocks, kPF stages ahead of their use (slot u
+    // holds the stage q with q % kPF == u): its row's four UE8M0 bytes (two 16-bit loads) and the
+    // words of the B rows 32c + lane, c < kC.
+    uint32_t pa[kPF][2], pb[kPF][C::kC];
     int qp = 0, jl_p = 0, s_p = 0;
-    const unsigned short *srow = nullptr;  // row m's scales of the front job, from block 2h on
-    auto load_sf = [&](uint32_t &dst) {
+    const unsigned short *srow = nullptr;  // row m's scales of the front job, from block 4h on
+    const uint32_t *sfb_src = nullptr;     // the front job's B scale words of this lane
+    auto load_sf = [&](uint32_t(&da)[2], uint32_t(&db)[C::kC]) {
       if (qp >= nq) return;
       if (s_p == 0) {
         const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_p));
         const int row = tile_row(jr, m);
-        srow = row >= 0 ? reinterpret_cast<const unsigned short *>(jr.sc + (size_t)row * nbr + 2 * h) : nullptr;
+        srow = row >= 0 ? reinterpret_cast<const unsigned short *>(jr.sc + (size_t)row * nbr + 4 * h) : nullptr;
+        sfb_src = reinterpret_cast<const uint32_t *>(a.terms + (size_t)jr.group * tbytes + (size_t)S * C::kBStage) +
+                  (size_t)(h * C::kC) * 32 + lane;
       }
-      dst = srow != nullptr && 8 * s_p + 2 * h < nbr ? (uint32_t)__ldg(srow + 4 * s_p) : 0u;
+#pragma unroll
+      for (int i = 0; i < 2; i++)
+        da[i] = srow != nullptr && kKB * s_p + 4 * h + 2 * i < nbr ? (uint32_t)__ldg(srow + 8 * s_p + i) : 0u;
+#pragma unroll
+      for (int c = 0; c < C::kC; c++) db[c] = __ldg(sfb_src + (size_t)s_p * (C::kSfbStage / 4) + c * 32);
       qp++;
       if (++s_p == S) {
         s_p = 0;
@@ -585,10 +596,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       }
     };
 #pragma unroll
-    for (int u = 0; u < kPF; u++) load_sf(sfr[u]);
+    for (int u = 0; u < kPF; u++) load_sf(pa[u], pb[u]);
 
     int jl = 0, s = 0, q = 0;
-    uint32_t ws = 0, wph = 0, b = 0, eph = 0;  // word slot + phase bits, A slot + a_empty phase bits
+    uint32_t ws = 0, b = 0;
     bool stop = false;
     for (int q0 = 0; q0 < nq && !stop; q0 += kPF) {
 #pragma unroll
@@ -599,42 +610,50 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
           break;
         }
         bool ok = true;
-        if (lane == 0) ok = mbar_wait(&w_full[ws], (wph >> ws) & 1u, tmo);
+        if (lane == 0) ok = mbar_wait(&w_full[ws], (uint32_t)(q / kNW) & 1u, tmo);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
           *abort_flag = 1;
           stop = true;
           break;
         }
-        wph ^= 1u << ws;
-        const uint4 c0 = lds_u4(wrow + ws * kWStage);
+        const uint32_t wa = wrow + ws * kWStage;
+        const uint4 c0 = lds_u4(wa + wo0), c1 = lds_u4(wa + wo1);
         __syncwarp();
         if (lane == 0) mbar_arrive(&w_empty[ws]);
-        ws = ws + 1 == kNW ? 0u : ws + 1;
-        uint32_t W[2][4];
+        ws = ws + 1 == (uint32_t)kNW ? 0u : ws + 1;
+        uint32_t W[4][4];
         planes_to_nibbles_interleaved(decode_block0(c0.x, c0.y), W[0][0], W[0][1], W[0][2], W[0][3]);
         planes_to_nibbles_interleaved(decode_block0(c0.z, c0.w), W[1][0], W[1][1], W[1][2], W[1][3]);
+        planes_to_nibbles_interleaved(decode_block0(c1.x, c1.y), W[2][0], W[2][1], W[2][2], W[2][3]);
+        planes_to_nibbles_interleaved(decode_block0(c1.z, c1.w), W[3][0], W[3][1], W[3][2], W[3][3]);
         if (q >= kNA) {
-          if (lane == 0) ok = mbar_wait(&a_empty[b], (eph >> b) & 1u, tmo);
+          if (lane == 0) ok = mbar_wait(&a_empty[b], (uint32_t)((q - kNA) / kNA) & 1u, tmo);
           ok = __shfl_sync(0xffffffffu, ok, 0);
-          eph ^= 1u << b;
           if (!ok) {
             *abort_flag = 1;
             stop = true;
             break;
           }
+          tc_fence_after();
         }
         const uint32_t ab = abase + b * kAStage;
-        const int nblk = s == S - 1 ? tail_blocks : 2;
+        const int nblk = s == S - 1 ? tail_blocks : 4;
 #pragma unroll
-        for (int i = 0; i < 2; i++)
+        for (int i = 0; i < 4; i++)
           if (i < nblk) sts_u4(ab + (uint32_t)i * 128u, W[i][0], W[i][1], W[i][2], W[i][3]);
-        sts_u16(xlane + b * 1024u, sfr[u]);
+        // scale factors of the stage into TMEM: A of this row (its own quarter, column 4h + quarter)
+        // and B of rows 32c + lane (every quarter holds a copy)
+        tmem_st_x1(tq + C::kSfaCol + 16u * b + 4u * (uint32_t)h + (uint32_t)sp, pa[u][0] | (pa[u][1] << 16));
+#pragma unroll
+        for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + C::kSfbCol + 16u * b + 4u * (uint32_t)h + (uint32_t)c, pb[u][c]);
+        tmem_wait_st();
         fence_proxy_async_smem();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[b]);
-        load_sf(sfr[u]);
-        b = b + 1 == kNA ? 0u : b + 1;
+        load_sf(pa[u], pb[u]);
+        b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
         if (warp < 4 && jl >= 1 && s == s_epi) epilogue(jl - 1);
         if (++s == S) {
           s = 0;
@@ -644,109 +663,98 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
     }
     if (!stop) q = nq;
     if (q == nq && nq > 0 && warp < 4 && !*abort_flag) epilogue(my_jobs - 1);
-  } else if (warp == kLoadWarp) {
-    // ---------------------------------------------------------------- loader warp
+  } else if (warp == kWLoadWarp) {
+    // ---------------------------------------------------------------- word loader warp
     // TMA front: stage qi of job jl_i, up to kNW stages ahead of the decode warps.
     const uint32_t wbase = smem_u32(smem + geo.off_W);
     unsigned char *my_maps = MODE == kModeGemv ? nullptr : a.maps + (size_t)blockIdx.x * kMapSlots * 128;
     int qi = 0, jl_i = 0, s_i = 0;
-    uint32_t wi = 0, weph = 0;
+    uint32_t wi = 0;
     const void *map_i = &wmap;
     JobRows ji{};
-    auto start_front_job = [&]() {  // whole warp
-      ji = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_i));
-      if (MODE != kModeGemv) {
-        unsigned char *gm = my_maps + (size_t)(jl_i % kMapSlots) * 128;
-        if (lane == 0) tmap_set_address(smem_u32(smap), ji.st);
-        __syncwarp();
-        tmap_publish(gm, smem_u32(smap));
-        if (lane == 0) tmap_acquire(gm);
-        map_i = gm;
+    bool ok = true;
+    while (ok && qi < nq && !*abort_flag) {  // whole warp; lane 0 issues the two boxes of stage qi
+      if (s_i == 0) {
+        ji = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_i));
+        if (MODE != kModeGemv) {
+          unsigned char *gm = my_maps + (size_t)(jl_i % kMapSlots) * 128;
+          if (lane == 0) tmap_set_address(smem_u32(smap), ji.st);
+          __syncwarp();
+          tmap_publish(gm, smem_u32(smap));
+          if (lane == 0) tmap_acquire(gm);
+          map_i = gm;
+        }
       }
-    };
-    auto issue_front = [&]() -> bool {  // whole warp; lane 0 issues the two boxes of stage qi
-      if (s_i == 0) start_front_job();
-      bool ok = true;
       if (lane == 0) {
-        if (qi >= kNW) ok = mbar_wait(&w_empty[wi], (weph >> wi) & 1u, tmo);
+        if (qi >= kNW) ok = mbar_wait(&w_empty[wi], (uint32_t)((qi - kNW) / kNW) & 1u, tmo);
         if (ok) {
           mbar_arrive_expect_tx(&w_full[wi], kWStage);
           const uint32_t dst = wbase + wi * kWStage;
-          tma_load_2d(dst, map_i, 64 * s_i, ji.y0, &w_full[wi]);
-          tma_load_2d(dst + 4096u, map_i, 64 * s_i, ji.y1, &w_full[wi]);
+          tma_load_2d(dst, map_i, 128 * s_i, ji.y0, &w_full[wi]);
+          tma_load_2d(dst + 8192u, map_i, 128 * s_i, ji.y1, &w_full[wi]);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) return false;
-      if (qi >= kNW) weph ^= 1u << wi;
-      wi = wi + 1 == kNW ? 0u : wi + 1;
+      if (!ok) break;
+      wi = wi + 1 == (uint32_t)kNW ? 0u : wi + 1;
       qi++;
       if (++s_i == S) {
         s_i = 0;
         jl_i++;
       }
-      return true;
-    };
-    bool ok = true;
-    while (ok && qi < nq && !*abort_flag) ok = issue_front();
+    }
     if (!ok) *abort_flag = 1;
     // drain: the last min(kNW, qi) issued stages may still be in flight
     if (lane == 0)
       for (int d = qi - 1; d >= 0 && d >= qi - kNW; d--)
         if (!mbar_wait(&w_full[d % kNW], (uint32_t)(d / kNW) & 1u, tmo)) break;
     __syncwarp();
-  } else {
-    // ---------------------------------------------------------------- MMA warp
+  } else if (warp == kBLoadWarp) {
+    // ---------------------------------------------------------------- B loader warp
+    int issued = 0;
     if (lane == 0) {
-      const uint32_t bslot = C::kBSlot;
-      int issued_b = 0, jl_b = 0, s_b = 0;
-      const uint8_t *bsrc = a.Bg;
-      auto front_group = [&]() {
-        bsrc = a.Bg + (size_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_b)).group * S * bslot;
-      };
-      if (my_jobs) front_group();
-      uint32_t bb_i = 0;
-      auto issue_b = [&]() {
-        mbar_arrive_expect_tx(&b_full[bb_i], bslot);
-        bulk_g2s(smem + geo.off_B + bb_i * bslot, bsrc, bslot, &b_full[bb_i]);
-        bsrc += bslot;
-        if (++s_b == S) {
-          s_b = 0;
-          if (++jl_b < my_jobs) front_group();
-        }
-        bb_i = bb_i + 1 == kNB ? 0u : bb_i + 1;
-        issued_b++;
-      };
-      while (issued_b < kNB && issued_b < nq) issue_b();
       int jl = 0, s = 0;
-      uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : 16);
-      uint32_t idesc0 = idesc_mxf4(ncols, 0u), idesc2 = idesc_mxf4(ncols, 2u);
-      uint32_t b = 0, bb = 0, aph = 0u, bph = 0u, cph = 0u;
-      const uint32_t a0 = smem_u32(smem + geo.off_A), b0 = smem_u32(smem + geo.off_B), x0 = smem_u32(smem + geo.off_X);
+      const uint8_t *src = nullptr;
       bool ok = true;
       for (int q = 0; q < nq; q++) {
         if (*abort_flag) break;
-        ok = mbar_wait(&a_full[b], (aph >> b) & 1u, tmo);
-        aph ^= 1u << b;
-        ok = ok && mbar_wait(&b_full[bb], (bph >> bb) & 1u, tmo);
-        bph ^= 1u << bb;
-        if (ok && s == 0 && jl >= 2) {
-          ok = mbar_wait(&acc_empty[jl & 1], (cph >> (jl & 1)) & 1u, tmo);
-          cph ^= 1u << (jl & 1);
+        const int b = q % kNA;
+        if (s == 0) src = a.terms + (size_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl)).group * tbytes;
+        if (q >= kNA && !(ok = mbar_wait(&a_empty[b], (uint32_t)((q - kNA) / kNA) & 1u, tmo))) break;
+        mbar_arrive_expect_tx(&b_full[b], C::kBStage);
+        bulk_g2s(smem + geo.off_B + (uint32_t)b * C::kBStage, src + (size_t)s * C::kBStage, C::kBStage, &b_full[b]);
+        issued++;
+        if (++s == S) {
+          s = 0;
+          ++jl;
         }
+      }
+      if (!ok) *abort_flag = 1;
+      for (int d = issued - 1; d >= 0 && d >= issued - kNA; d--)
+        if (!mbar_wait(&b_full[d % kNA], (uint32_t)(d / kNA) & 1u, tmo)) break;
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- MMA warp
+    if (lane == 0) {
+      int jl = 0, s = 0;
+      uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : 16);
+      uint32_t idesc0 = idesc_mxf4(ncols, 0u), idesc2 = idesc_mxf4(ncols, 2u);
+      const uint32_t a0 = smem_u32(smem + geo.off_A), b0 = smem_u32(smem + geo.off_B);
+      bool ok = true;
+      for (int q = 0; q < nq; q++) {
+        if (*abort_flag) break;
+        const int b = q % kNA;
+        const uint32_t ph = (uint32_t)(q / kNA) & 1u;
+        ok = mbar_wait(&a_full[b], ph, tmo) && mbar_wait(&b_full[b], ph, tmo);
+        if (ok && s == 0 && jl >= 2) ok = mbar_wait(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo);
         if (!ok) break;
         tc_fence_after();
-        // the stage's scale factors into TMEM: A (2 groups x 4 lane quarters), then B
-        const uint32_t sfa = tbase + C::kSfaCol + 8u * b, sfb = tbase + C::kSfbCol + 8u * b;
-        const uint32_t xs = x0 + b * 1024u, bs = b0 + bb * bslot;
-        tmem_cp_32x128_x4(sfa, smem_desc(xs, 128u, 128u));
-        tmem_cp_32x128_x4(sfa + 4u, smem_desc(xs + 512u, 128u, 128u));
-        tmem_cp_32x128_x4(sfb, smem_desc(bs + C::kBTile, 128u, 128u));
-        tmem_cp_32x128_x4(sfb + 4u, smem_desc(bs + C::kBTile + 512u, 128u, 128u));
-        const int nmma = (nbr - 8 * s < 8 ? nbr - 8 * s : 8) >> 1;
-        uint64_t ad = smem_desc(a0 + b * kAStage, 128u, kSbo);
-        uint64_t bd = smem_desc(bs, 128u, kSbo);
+        const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
+        uint64_t ad = smem_desc(a0 + (uint32_t)b * kAStage, 128u, kSbo);
+        uint64_t bd = smem_desc(b0 + (uint32_t)b * C::kBStage, 128u, kSbo);
         const uint32_t d_t = tbase + (uint32_t)((jl & 1) * NMAX);
+        const uint32_t sfa = tbase + C::kSfaCol + 16u * (uint32_t)b, sfb = tbase + C::kSfbCol + 16u * (uint32_t)b;
         for (int j = 0; j < nmma; j++) {
           const uint32_t g = (uint32_t)(j >> 1), sf = (uint32_t)(j & 1) * 2u;
           mma_mxf4(d_t, ad, bd, sf ? idesc2 : idesc0, (sfa + 4u * g) | (sf << 30), (sfb + 4u * g) | (sf << 30),
@@ -755,20 +763,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
           bd += 16u;
         }
         tc_commit(&a_empty[b]);
-        tc_commit(&b_empty[bb]);
         if (s == S - 1) tc_commit(&acc_full[jl & 1]);
-        // refill the B slot of stage q-kBLag, whose MMAs were issued kBLag stages ago, with stage
-        // q-kBLag+kNB
-        if (q >= kBLag && issued_b < nq) {
-          const int qq = q - kBLag;
-          if (!mbar_wait(&b_empty[qq % kNB], (uint32_t)(qq / kNB) & 1u, tmo)) {
-            ok = false;
-            break;
-          }
-          issue_b();
-        }
-        b = b + 1 == kNA ? 0u : b + 1;
-        bb = bb + 1 == kNB ? 0u : bb + 1;
         if (++s == S) {
           s = 0;
           if (++jl < my_jobs) {
@@ -782,11 +777,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         }
       }
       if (!ok) *abort_flag = 1;
-      // drain: every tcgen05 operation issued so far, then the B copies that may be in flight
+      // drain: every tcgen05 operation issued so far
       tc_commit(drain);
       mbar_wait(drain, 0u, tmo);
-      for (int d = issued_b - 1; d >= 0 && d >= issued_b - kNB; d--)
-        if (!mbar_wait(&b_full[d % kNB], (uint32_t)(d / kNB) & 1u, tmo)) break;
     }
     __syncwarp();
   }
@@ -813,18 +806,18 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Tensor map of a trellis stream seen as a [rows][nbr*8] byte matrix, boxes of 64 rows x 64 bytes
-// with the 64-byte swizzle (the decode threads' 16-byte reads of consecutive rows then fall in
+// Tensor map of a trellis stream seen as a [rows][nbr*8] byte matrix, boxes of 64 rows x 128 bytes
+// with the 128-byte swizzle (the decode threads' 16-byte reads of consecutive rows then fall in
 // distinct banks); rows and columns beyond the matrix read as zero.
 static bool make_word_map(CUtensorMap *map, const void *stream, int rows, int nbr) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)nbr * 8u, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)nbr * 8u};
-  cuuint32_t box[2] = {64u, 64u};
+  cuuint32_t box[2] = {128u, 64u};
   cuuint32_t estr[2] = {1u, 1u};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(stream), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -844,16 +837,18 @@ static bool mma_fits(int NMAX, int mode) {
 // pitch that is a multiple of 16 bytes for the tensor map) and a 16-byte aligned stream.
 static bool k_ok(int nbr) { return nbr >= 2 && nbr % 2 == 0; }
 
+static size_t terms_for(int nbr, int NMAX) {
+  const int S = (nbr + kKB - 1) / kKB;
+  return NMAX == 32 ? terms_bytes<32>(S) : terms_bytes<96>(S);
+}
+
 bool gemv_mma_supported(const MatView &w, int T) {
   return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.stream) & 15u) == 0 && tensor_map_encoder() != nullptr &&
          mma_fits(nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv);
 }
 
 // Tokens beyond kGemvTok run as further passes, each with its own split of x.
-size_t gemv_mma_workspace(const MatView &w, int T) {
-  const int S = (w.nbr + 7) / 8;
-  return nmax_for(T < kGemvTok ? T : kGemvTok) == 32 ? (size_t)S * Cfg<32>::kBSlot : (size_t)S * Cfg<96>::kBSlot;
-}
+size_t gemv_mma_workspace(const MatView &w, int T) { return terms_for(w.nbr, nmax_for(T < kGemvTok ? T : kGemvTok)); }
 
 static int sm_count() {
   int dev = 0, nsm = 148;
@@ -865,9 +860,9 @@ static int sm_count() {
 template <int NMAX>
 static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, const uint16_t *x, int T, uint16_t *y,
                                     void *ws, cudaStream_t s) {
-  uint8_t *Bg = static_cast<uint8_t *>(ws);
+  uint8_t *terms = static_cast<uint8_t *>(ws);
   const int warps = Cfg<NMAX>::kSlots * w.nbr;
-  k_bsplit_gemv<NMAX><<<(warps + 7) / 8, 256, 0, s>>>(x, T, w.nbr * 32, Bg);
+  k_bsplit_gemv<NMAX><<<(warps + 7) / 8, 256, 0, s>>>(x, T, w.nbr * 32, terms);
   static unsigned long long attr = 0;
   cudaError_t e = ensure_max_dynamic_smem(k_mma<32, kModeGemv, NMAX>, attr);
   if (e != cudaSuccess) return e;
@@ -876,7 +871,7 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
   args.scales = w.scales;
   args.rows = w.rows;
   args.nbr = w.nbr;
-  args.Bg = Bg;
+  args.terms = terms;
   args.T = T;
   args.y = y;
   MoeTable<32> none{};
@@ -918,15 +913,13 @@ MoeMmaWorkspace moe_mma_workspace_layout(const tcf4_moe &m, int T, int k) {
   auto a256 = [](size_t v) { return (v + 255) & ~(size_t)255; };
   const int P = T * k, NMAX = nmax_for(T);
   const int G = moe_groups_max(m.E, P, NMAX == 32 ? Cfg<32>::kTok : Cfg<96>::kTok);
-  const size_t bslot = NMAX == 32 ? Cfg<32>::kBSlot : Cfg<96>::kBSlot;
-  const int S_gu = (m.H / 32 + 7) / 8, S_dn = (m.I / 32 + 7) / 8;
   MoeMmaWorkspace L;
   size_t off = 0;
   L.counters = off; off = a256(off + sizeof(int) * 4 * ((m.H + 127) / 128));
   L.hidden = off;   off = a256(off + sizeof(uint16_t) * (size_t)P * m.I);
   L.y = off;        off = a256(off + sizeof(float) * (size_t)P * m.H);
-  L.bg_gu = off;    off = a256(off + (size_t)G * S_gu * bslot);
-  L.bg_dn = off;    off = a256(off + (size_t)G * S_dn * bslot);
+  L.bg_gu = off;    off = a256(off + (size_t)G * terms_for(m.H / 32, NMAX));
+  L.bg_dn = off;    off = a256(off + (size_t)G * terms_for(m.I / 32, NMAX));
   L.maps = off;     off = a256(off + (size_t)sm_count() * kMapSlots * 128);
   L.total = off;
   return L;
@@ -968,32 +961,32 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
 
   // gate_up: split x per group (and clear the down counters), then decode + MMA + SwiGLU
   {
-    uint8_t *Bg = reinterpret_cast<uint8_t *>(base + L.bg_gu);
+    uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_gu);
     const int nbr = m.H / 32;
     const int warps = G * Cfg<NMAX>::kSlots * nbr;
     k_bsplit_moe<NMAX><<<(warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm, 256, 0, s>>>(
-        ids, P, m.E, k, x, m.H, Bg, args.counters, 4 * ((m.H + 127) / 128));
+        ids, P, m.E, k, x, m.H, terms, args.counters, 4 * ((m.H + 127) / 128));
     static unsigned long long attr = 0;
     cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, kModeGateUp, NMAX>, attr);
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
-    args.Bg = Bg;
+    args.terms = terms;
     const int jobs = G * ((m.I + 63) / 64);
     k_mma<MAXE, kModeGateUp, NMAX><<<jobs < nsm ? jobs : nsm, kThreads, mma_geom<NMAX>(kModeGateUp).smem, s>>>(
         args, tab, map_gu);
   }
   // down: split h per group, then decode + MMA, y to the workspace, last arriver per chunk combines
   {
-    uint8_t *Bg = reinterpret_cast<uint8_t *>(base + L.bg_dn);
+    uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_dn);
     const int nbr = m.I / 32;
     const int warps = G * Cfg<NMAX>::kSlots * nbr;
     k_bsplit_moe<NMAX><<<(warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm, 256, 0, s>>>(
-        ids, P, m.E, 1, args.hidden, m.I, Bg, nullptr, 0);
+        ids, P, m.E, 1, args.hidden, m.I, terms, nullptr, 0);
     static unsigned long long attr = 0;
     cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, kModeDown, NMAX>, attr);
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
-    args.Bg = Bg;
+    args.terms = terms;
     const int jobs = G * ((m.H + 127) / 128);
     k_mma<MAXE, kModeDown, NMAX><<<jobs < nsm ? jobs : nsm, kThreads, mma_geom<NMAX>(kModeDown).smem, s>>>(args, tab,
                                                                                                          map_dn);
