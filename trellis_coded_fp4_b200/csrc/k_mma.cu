@@ -13,13 +13,13 @@
 //    of shared-memory slots with 2-D TMA tile loads (128-byte swizzle).
 //  * 16 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and the four K-blocks
 //    4(w/4)..4(w/4)+3 of a stage (one scale-factor group). It reads its 32 bytes of trellis words,
-//    decodes them in registers (bit-sliced), stores the four 16-byte E2M1 chunks into the stage's A
-//    tile, and writes the group's scale factors of its row (A) and of the B rows its lane stands
-//    for into TMEM (tcgen05.st into its own lane quarter; the scale bytes are loaded a few stages
-//    ahead).
+//    decodes them in registers (bit-sliced) and stores the four blocks' E2M1 codes, packed eight per
+//    32-bit column, into the stage's A operand in TMEM, together with the group's scale factors of
+//    its row (A) and of the B rows its lane stands for (tcgen05.st into its own lane quarter; the
+//    scale bytes are loaded a few stages ahead). The decoded weights never touch shared memory.
 //  * B loader warp: lane 0 bulk-copies each stage's activation terms into the B slot of the stage.
-//  * MMA warp: lane 0 waits for a stage, issues its 8 MMAs into a double-buffered TMEM
-//    accumulator and releases the stage with one commit.
+//  * MMA warp: lane 0 waits for a stage, issues its 8 MMAs (A from TMEM, B from shared memory) into
+//    a double-buffered TMEM accumulator and releases the stage with one commit.
 //  * the epilogue of job i (tcgen05.ld, then the GEMV output, the SwiGLU of gate/up rows, or the MoE
 //    down rows and their combine) runs in decode warps 0-3 early in job i+1.
 // All tcgen05 MMAs of the CTA are issued by one thread. Every wait is a bounded mbarrier wait; a
@@ -44,8 +44,8 @@ constexpr int kPF = 4;               // stages of scale factors a decode thread 
 constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> jobs in flight)
 constexpr int kDecWarps = 16, kWLoadWarp = 16, kMmaWarp = 17, kBLoadWarp = 18, kThreads = 608;
 constexpr uint32_t kWStage = 16384;  // 128 rows x 128 bytes of trellis words (two 64-row TMA boxes)
-constexpr uint32_t kAStage = 32768;  // 128 rows x 512 E2M1 elements, packed
-constexpr uint32_t kSbo = 2048;      // 8 rows x 16 chunks x 16 bytes: one 8-row group of a stage
+constexpr uint32_t kACols = 64;      // TMEM columns of a stage's A operand: 512 E2M1 per lane, 8 per column
+constexpr uint32_t kSbo = 2048;      // B stage: 8 rows x 16 chunks x 16 bytes per 8-row group
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
 
@@ -55,12 +55,13 @@ struct Cfg {
   static constexpr int kTok = NMAX / kTerms;                   // tokens per group
   static constexpr int kSlots = (NMAX + kTerms - 1) / kTerms;  // token slots the split writes
   static constexpr int kC = (NMAX + 31) / 32;                  // B scale columns per 4-block group
-  static constexpr int kNW = 4;                                // word stages in flight
-  static constexpr int kNA = NMAX <= 32 ? 3 : 2;               // A / B / scale-factor stages
+  static constexpr int kNW = 6;                                // word stages in flight
+  static constexpr int kNA = NMAX <= 32 ? 4 : 3;               // A / B / scale-factor stages
   static constexpr uint32_t kBStage = NMAX * 256u;             // NMAX rows x 512 E2M1
   static constexpr uint32_t kSfbStage = 4u * kC * 128u;        // [group][column][lane] u32
-  static constexpr uint32_t kSfaCol = 2u * NMAX;               // TMEM: accumulators first
-  static constexpr uint32_t kSfbCol = kSfaCol + 16u * kNA;     // 16 columns per stage each
+  static constexpr uint32_t kACol = 2u * NMAX;                 // TMEM: accumulators first, then
+  static constexpr uint32_t kSfaCol = kACol + kACols * kNA;    // A stages, A scales (16 columns per
+  static constexpr uint32_t kSfbCol = kSfaCol + 16u * kNA;     // stage), B scales (16 per stage)
   static constexpr uint32_t kUsed = kSfbCol + 16u * kNA;
   static constexpr uint32_t kTmemCols = kUsed <= 128 ? 128 : (kUsed <= 256 ? 256 : 512);
 };
@@ -70,8 +71,9 @@ struct Cfg {
 // 4j..4j+3 of the chunk (element 2b in the low nibble of byte b).
 __host__ __device__ constexpr int kpos_of_weight(int i) { return 8 * (i & 3) + (i >> 2); }
 
-// Byte offset of chunk c (0..15) of row n in a K-major, no-swizzle stage: core matrices of 8 rows
-// x 16 bytes, LBO = 128 (adjacent chunks), SBO = 2048 (adjacent 8-row groups).
+// Byte offset of chunk c (0..15) of row n in a K-major, no-swizzle B stage: core matrices of 8 rows
+// x 16 bytes, LBO = 128 (adjacent chunks), SBO = 2048 (adjacent 8-row groups). In TMEM the A operand
+// holds the same 16-byte chunks, four 32-bit columns each (element e of a column in bits 4e..4e+3).
 __host__ __device__ constexpr uint32_t chunk_off(uint32_t n, uint32_t c) {
   return (n >> 3) * kSbo + c * 128u + (n & 7u) * 16u;
 }
@@ -234,10 +236,9 @@ __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ 
 
 // ------------------------------------------------------------------------------- geometry
 
-// Shared memory: barriers + tensor-map copy | word ring | A ring | B ring | gate/up exchange
-// | group plan.
+// Shared memory: barriers + tensor-map copy | word ring | B ring | gate/up exchange | group plan.
 struct MmaGeom {
-  uint32_t off_W, off_A, off_B, off_U, off_P, smem;
+  uint32_t off_W, off_B, off_U, off_P, smem;
 };
 
 template <int NMAX>
@@ -245,8 +246,7 @@ __host__ __device__ inline MmaGeom mma_geom(int mode) {
   using C = Cfg<NMAX>;
   MmaGeom g;
   g.off_W = 1024u;
-  g.off_A = g.off_W + C::kNW * kWStage;
-  g.off_B = g.off_A + C::kNA * kAStage;
+  g.off_B = g.off_W + C::kNW * kWStage;
   g.off_U = g.off_B + C::kNA * C::kBStage;
   g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)C::kTok * 4u : 0u);
   g.smem = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
@@ -259,9 +259,6 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
-}
-__device__ __forceinline__ void sts_u4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 // 2-D TMA tile load (no multicast; the tensor map covers this GPU's memory only).
@@ -278,6 +275,15 @@ __device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t a) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
 }
 
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[4][4]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0][0]), "r"(r[0][1]), "r"(r[0][2]), "r"(r[0][3]), "r"(r[1][0]), "r"(r[1][1]), "r"(r[1][2]), "r"(r[1][3]),
+      "r"(r[2][0]), "r"(r[2][1]), "r"(r[2][2]), "r"(r[2][3]), "r"(r[3][0]), "r"(r[3][1]), "r"(r[3][2]), "r"(r[3][3])
+      : "memory");
+}
+
 // Instruction descriptor of a block-scaled kind::mxf4 MMA: A = B = E2M1, K-major, UE8M0 scales per
 // 32, fp32 accumulation, M = 128, N columns; sf = scale-factor byte pair (0 or 2) of both operands.
 __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t N, uint32_t sf) {
@@ -292,15 +298,15 @@ __device__ __forceinline__ uint32_t idesc_mxf4(uint32_t N, uint32_t sf) {
   return d;                // bit 31 = 0: K = 64
 }
 
-// One thread: D[tmem] (+)= A[smem] x B[smem], block-scaled. The A scale factors of rows
+// One thread: D[tmem] (+)= A[tmem] x B[smem], block-scaled. The A scale factors of rows
 // 32q..32q+31 are read from lane quarter q at column sfa+q, those of B row n from column sfb + n/32.
-__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t sfa_tmem, uint32_t sfb_tmem, bool accumulate) {
+__device__ __forceinline__ void mma_mxf4_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, bool accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(sfa_tmem), "r"(sfb_tmem)
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], [%1], %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
 
@@ -417,12 +423,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = a.nbr, S = (nbr + kKB - 1) / kKB;
   const MmaGeom geo = mma_geom<NMAX>(MODE);
-  uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);  // 29 barriers in bytes [0, 232)
-  uint64_t *w_empty = w_full + 4, *a_full = w_full + 8, *a_empty = w_full + 12, *b_full = w_full + 16,
-           *acc_full = w_full + 20, *acc_empty = w_full + 22, *u_full = w_full + 24, *u_empty = w_full + 26,
-           *drain = w_full + 28;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 256);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 260);
+  static_assert(kNW <= 8 && kNA <= 4, "barrier block: 8 word slots, 4 operand slots");
+  uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);  // 37 barriers in bytes [0, 296)
+  uint64_t *w_empty = w_full + 8, *a_full = w_full + 16, *a_empty = w_full + 20, *b_full = w_full + 24,
+           *acc_full = w_full + 28, *acc_empty = w_full + 30, *u_full = w_full + 32, *u_empty = w_full + 34,
+           *drain = w_full + 36;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 448);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 452);
   unsigned char *smap = smem + 512;  // shared-memory copy of the tensor map (grouped MoE)
   unsigned int *tmo = &g_tcf4_timeouts_mma;
   GroupPlan *pl = reinterpret_cast<GroupPlan *>(smem + geo.off_P);
@@ -476,9 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
     const uint32_t rb = (uint32_t)(m & 63), sw = rb & 7u;  // row in its TMA box, 128-byte swizzle
     const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * 8192u + rb * 128u;
     const uint32_t wo0 = ((2u * h) ^ sw) * 16u, wo1 = ((2u * h + 1u) ^ sw) * 16u;
-    const uint32_t abase = smem_u32(smem + geo.off_A) + chunk_off((uint32_t)m, 4u * (uint32_t)h);
     const uint32_t tq = tbase + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lane quarter
-    const int tail_blocks = nbr - kKB * (S - 1) - 4 * h;      // this thread's blocks in the last stage
     auto epilogue = [&](int jl_e) {
       const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
       const int buf = jl_e & 1;
@@ -637,18 +642,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
           }
           tc_fence_after();
         }
-        const uint32_t ab = abase + b * kAStage;
-        const int nblk = s == S - 1 ? tail_blocks : 4;
-#pragma unroll
-        for (int i = 0; i < 4; i++)
-          if (i < nblk) sts_u4(ab + (uint32_t)i * 128u, W[i][0], W[i][1], W[i][2], W[i][3]);
-        // scale factors of the stage into TMEM: A of this row (its own quarter, column 4h + quarter)
-        // and B of rows 32c + lane (every quarter holds a copy)
+        // the four blocks' codes (columns 16h..16h+15 of the stage's A), the scale factors of this
+        // row (its own quarter, column 4h + quarter) and of B rows 32c + lane (every quarter holds a
+        // copy). Columns of blocks beyond the row's end hold the decode of the zero fill; no MMA reads them.
+        tmem_st_x16(tq + C::kACol + kACols * b + 16u * (uint32_t)h, W);
         tmem_st_x1(tq + C::kSfaCol + 16u * b + 4u * (uint32_t)h + (uint32_t)sp, pa[u][0] | (pa[u][1] << 16));
 #pragma unroll
         for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + C::kSfbCol + 16u * b + 4u * (uint32_t)h + (uint32_t)c, pb[u][c]);
         tmem_wait_st();
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[b]);
@@ -740,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       int jl = 0, s = 0;
       uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : 16);
       uint32_t idesc0 = idesc_mxf4(ncols, 0u), idesc2 = idesc_mxf4(ncols, 2u);
-      const uint32_t a0 = smem_u32(smem + geo.off_A), b0 = smem_u32(smem + geo.off_B);
+      const uint32_t b0 = smem_u32(smem + geo.off_B);
       bool ok = true;
       for (int q = 0; q < nq; q++) {
         if (*abort_flag) break;
@@ -751,16 +752,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         if (!ok) break;
         tc_fence_after();
         const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
-        uint64_t ad = smem_desc(a0 + (uint32_t)b * kAStage, 128u, kSbo);
+        const uint32_t at = tbase + C::kACol + kACols * (uint32_t)b;
         uint64_t bd = smem_desc(b0 + (uint32_t)b * C::kBStage, 128u, kSbo);
         const uint32_t d_t = tbase + (uint32_t)((jl & 1) * NMAX);
         const uint32_t sfa = tbase + C::kSfaCol + 16u * (uint32_t)b, sfb = tbase + C::kSfbCol + 16u * (uint32_t)b;
         for (int j = 0; j < nmma; j++) {
           const uint32_t g = (uint32_t)(j >> 1), sf = (uint32_t)(j & 1) * 2u;
-          mma_mxf4(d_t, ad, bd, sf ? idesc2 : idesc0, (sfa + 4u * g) | (sf << 30), (sfb + 4u * g) | (sf << 30),
-                   !(s == 0 && j == 0));
-          ad += 16u;  // +256 bytes: two chunks (the descriptor's start address counts 16-byte units)
-          bd += 16u;
+          mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd, sf ? idesc2 : idesc0, (sfa + 4u * g) | (sf << 30),
+                      (sfb + 4u * g) | (sf << 30), !(s == 0 && j == 0));
+          bd += 16u;  // +256 bytes: two chunks (the descriptor's start address counts 16-byte units)
         }
         tc_commit(&a_empty[b]);
         if (s == S - 1) tc_commit(&acc_full[jl & 1]);
