@@ -8,17 +8,18 @@
 // residual expansion, see split_terms): B column kTerms*t + j holds term j of token t, and
 // y[t] = sum_j D[:, kTerms*t + j] in fp32.
 //
-// One persistent CTA per SM, over 128-row tiles ("jobs") of K stages of 512 (16 blocks of 32):
-//  * word loader warp: lane 0 streams each stage's trellis words (128 rows x 128 bytes) into a ring
+// One persistent CTA per SM, over 128-row tiles ("jobs") of K stages of KB blocks of 32 (KB = 32 for
+// up to five tokens per group, else 16):
+//  * word loader warp: lane 0 streams each stage's trellis words (128 rows x 8 KB bytes) into a ring
 //    of shared-memory slots with 2-D TMA tile loads (128-byte swizzle).
-//  * 16 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and the four K-blocks
-//    4(w/4)..4(w/4)+3 of a stage (one scale-factor group). It reads its 32 bytes of trellis words,
-//    decodes them in registers (bit-sliced) and stores the four blocks' E2M1 codes, packed eight per
+//  * 16 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and the NBT = KB/4 K-blocks
+//    NBT(w/4).. of a stage (whole scale-factor groups). It reads its 8 NBT bytes of trellis words,
+//    decodes them in registers (bit-sliced) and stores the blocks' E2M1 codes, packed eight per
 //    32-bit column, into the stage's A operand in TMEM, together with the group's scale factors of
 //    its row (A) and of the B rows its lane stands for (tcgen05.st into its own lane quarter; the
 //    scale bytes are loaded a few stages ahead). The decoded weights never touch shared memory.
 //  * B loader warp: lane 0 bulk-copies each stage's activation terms into the B slot of the stage.
-//  * MMA warp: lane 0 waits for a stage, issues its 8 MMAs (A from TMEM, B from shared memory) into
+//  * MMA warp: lane 0 waits for a stage, issues its KB/2 MMAs (A from TMEM, B from shared memory) into
 //    a double-buffered TMEM accumulator and releases the stage with one commit.
 //  * the epilogue of job i (tcgen05.ld, then the GEMV output, the SwiGLU of gate/up rows, or the MoE
 //    down rows and their combine) runs in decode warps 0-3 early in job i+1.
@@ -38,14 +39,9 @@ namespace tcf4 {
 
 __device__ unsigned int g_tcf4_timeouts_mma = 0;
 
-constexpr int kKB = 16;              // 32-blocks per row per stage (K = 512)
 constexpr int kTerms = 6;            // E2M1 terms per activation block
-constexpr int kPF = 4;               // stages of scale factors a decode thread keeps in flight
 constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> jobs in flight)
 constexpr int kDecWarps = 16, kWLoadWarp = 16, kMmaWarp = 17, kBLoadWarp = 18, kThreads = 608;
-constexpr uint32_t kWStage = 16384;  // 128 rows x 128 bytes of trellis words (two 64-row TMA boxes)
-constexpr uint32_t kACols = 64;      // TMEM columns of a stage's A operand: 512 E2M1 per lane, 8 per column
-constexpr uint32_t kSbo = 2048;      // B stage: 8 rows x 16 chunks x 16 bytes per 8-row group
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
 
@@ -55,15 +51,24 @@ struct Cfg {
   static constexpr int kTok = NMAX / kTerms;                   // tokens per group
   static constexpr int kSlots = (NMAX + kTerms - 1) / kTerms;  // token slots the split writes
   static constexpr int kC = (NMAX + 31) / 32;                  // B scale columns per 4-block group
-  static constexpr int kNW = 6;                                // word stages in flight
-  static constexpr int kNA = NMAX <= 32 ? 4 : 3;               // A / B / scale-factor stages
-  static constexpr uint32_t kBStage = NMAX * 256u;             // NMAX rows x 512 E2M1
-  static constexpr uint32_t kSfbStage = 4u * kC * 128u;        // [group][column][lane] u32
+  static constexpr int kKB = NMAX <= 32 ? 32 : 16;             // 32-blocks per row per stage
+  static constexpr int kNBT = kKB / 4;                         // blocks per decode thread per stage
+  static constexpr int kNG = kNBT / 4;                         // scale groups per decode thread
+  static constexpr int kNW = kKB == 32 ? 3 : 6;                // word stages in flight
+  static constexpr int kNA = NMAX <= 32 ? 2 : 3;               // A / B / scale-factor stages
+  static constexpr int kPF = kKB == 32 ? 2 : 4;                // stages of scale factors in flight
+  static constexpr int kBoxCols = kKB / 16;                    // 128-byte TMA boxes per 64 rows
+  static constexpr uint32_t kWStage = 1024u * kKB;             // 128 rows x 8 KB bytes of words
+  static constexpr uint32_t kSbo = 128u * kKB;                 // B: 8 rows x KB chunks x 16 bytes
+  static constexpr uint32_t kBStage = NMAX * 16u * kKB;        // NMAX rows x 32 KB E2M1
+  static constexpr uint32_t kSfbStage = (kKB / 4) * kC * 128u;  // [group][column][lane] u32
+  static constexpr uint32_t kACols = 4u * kKB;                 // TMEM columns of a stage's A
   static constexpr uint32_t kACol = 2u * NMAX;                 // TMEM: accumulators first, then
-  static constexpr uint32_t kSfaCol = kACol + kACols * kNA;    // A stages, A scales (16 columns per
-  static constexpr uint32_t kSfbCol = kSfaCol + 16u * kNA;     // stage), B scales (16 per stage)
-  static constexpr uint32_t kUsed = kSfbCol + 16u * kNA;
+  static constexpr uint32_t kSfaCol = kACol + kACols * kNA;    // A stages, A scales (KB columns per
+  static constexpr uint32_t kSfbCol = kSfaCol + kKB * kNA;     // stage), B scales (KB per stage)
+  static constexpr uint32_t kUsed = kSfbCol + kKB * kNA;
   static constexpr uint32_t kTmemCols = kUsed <= 128 ? 128 : (kUsed <= 256 ? 256 : 512);
+  static_assert(kUsed <= 512, "TMEM budget");
 };
 
 // Position (0..31) inside a 32-element chunk of the MMA operand of weight i of the block: the
@@ -71,11 +76,13 @@ struct Cfg {
 // 4j..4j+3 of the chunk (element 2b in the low nibble of byte b).
 __host__ __device__ constexpr int kpos_of_weight(int i) { return 8 * (i & 3) + (i >> 2); }
 
-// Byte offset of chunk c (0..15) of row n in a K-major, no-swizzle B stage: core matrices of 8 rows
-// x 16 bytes, LBO = 128 (adjacent chunks), SBO = 2048 (adjacent 8-row groups). In TMEM the A operand
-// holds the same 16-byte chunks, four 32-bit columns each (element e of a column in bits 4e..4e+3).
+// Byte offset of chunk c (0..KB-1) of row n in a K-major, no-swizzle B stage: core matrices of 8
+// rows x 16 bytes, LBO = 128 (adjacent chunks), SBO = 128 KB (adjacent 8-row groups). In TMEM the A
+// operand holds the same 16-byte chunks, four 32-bit columns each (element e of a column in bits
+// 4e..4e+3).
+template <int NMAX>
 __host__ __device__ constexpr uint32_t chunk_off(uint32_t n, uint32_t c) {
-  return (n >> 3) * kSbo + c * 128u + (n & 7u) * 16u;
+  return (n >> 3) * Cfg<NMAX>::kSbo + c * 128u + (n & 7u) * 16u;
 }
 
 // ------------------------------------------------------------------------------- routing groups
@@ -151,8 +158,8 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
 }
 
 // Per group of token slots, the activation terms of each stage: Bg [S][kBStage] (one K-major B
-// stage each) and Bsf [S][kSfbStage]: word (h, c, lane) of a stage holds the UE8M0 bytes of B row
-// 32c+lane for the stage's blocks 4h..4h+3 (byte i = block 4h+i).
+// stage each) and Bsf [S][kSfbStage]: word (g, c, lane) of a stage holds the UE8M0 bytes of B row
+// 32c+lane for the stage's blocks 4g..4g+3 (byte i = block 4g+i).
 template <int NMAX>
 __host__ __device__ inline size_t terms_bytes(int S) {
   return (size_t)S * (Cfg<NMAX>::kBStage + Cfg<NMAX>::kSfbStage);
@@ -168,7 +175,7 @@ template <int NMAX>
 __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total, uint8_t *terms) {
   using C = Cfg<NMAX>;
   const int lane = threadIdx.x & 31;
-  const int s = kb / kKB, c = kb - s * kKB, h = c >> 2;
+  const int s = kb / C::kKB, c = kb - s * C::kKB, h = c >> 2;
   uint8_t *bst = terms + (size_t)s * C::kBStage;
   uint8_t *sfs = terms + (size_t)S_total * C::kBStage + (size_t)s * C::kSfbStage;
   const int kp = kpos_of_weight(lane);
@@ -188,7 +195,7 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
     const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 4);
     if (n < NMAX) {
       if (((lane >> 2) & 1) == 0)
-        bst[chunk_off((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code | (partner << 4));
+        bst[chunk_off<NMAX>((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code | (partner << 4));
       if (lane == 0) sfs[((h * C::kC + (n >> 5)) * 32 + (n & 31)) * 4 + (c & 3)] = (uint8_t)(S + 127);
     }
   }
@@ -198,7 +205,7 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
 template <int NMAX>
 __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
                                                      uint8_t *__restrict__ terms) {
-  const int nb = K >> 5, S = (nb + kKB - 1) / kKB, lane = threadIdx.x & 31;
+  const int nb = K >> 5, S = (nb + Cfg<NMAX>::kKB - 1) / Cfg<NMAX>::kKB, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < Cfg<NMAX>::kSlots * nb; wi += nwarps) {
     const int t = wi / nb, kb = wi - t * nb;
@@ -218,7 +225,7 @@ __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ 
   if (counters != nullptr && blockIdx.x == 0)
     for (int c = threadIdx.x; c < n_counters; c += blockDim.x) counters[c] = 0;
   build_groups(pl, ids, P, E, Cfg<NMAX>::kTok);
-  const int nb = K >> 5, S = (nb + kKB - 1) / kKB;
+  const int nb = K >> 5, S = (nb + Cfg<NMAX>::kKB - 1) / Cfg<NMAX>::kKB;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int per_group = Cfg<NMAX>::kSlots * nb;
@@ -246,7 +253,7 @@ __host__ __device__ inline MmaGeom mma_geom(int mode) {
   using C = Cfg<NMAX>;
   MmaGeom g;
   g.off_W = 1024u;
-  g.off_B = g.off_W + C::kNW * kWStage;
+  g.off_B = g.off_W + C::kNW * C::kWStage;
   g.off_U = g.off_B + C::kNA * C::kBStage;
   g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)C::kTok * 4u : 0u);
   g.smem = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
@@ -275,6 +282,9 @@ __device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t a) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(a) : "memory");
 }
 
+template <int NBT>
+__device__ __forceinline__ void tmem_st_codes(uint32_t taddr, const uint32_t (&r)[NBT][4]);
+
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[4][4]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
@@ -282,6 +292,29 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[
       "r"(r[0][0]), "r"(r[0][1]), "r"(r[0][2]), "r"(r[0][3]), "r"(r[1][0]), "r"(r[1][1]), "r"(r[1][2]), "r"(r[1][3]),
       "r"(r[2][0]), "r"(r[2][1]), "r"(r[2][2]), "r"(r[2][3]), "r"(r[3][0]), "r"(r[3][1]), "r"(r[3][2]), "r"(r[3][3])
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[8][4]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0][0]), "r"(r[0][1]), "r"(r[0][2]), "r"(r[0][3]),
+      "r"(r[1][0]), "r"(r[1][1]), "r"(r[1][2]), "r"(r[1][3]),
+      "r"(r[2][0]), "r"(r[2][1]), "r"(r[2][2]), "r"(r[2][3]),
+      "r"(r[3][0]), "r"(r[3][1]), "r"(r[3][2]), "r"(r[3][3]),
+      "r"(r[4][0]), "r"(r[4][1]), "r"(r[4][2]), "r"(r[4][3]),
+      "r"(r[5][0]), "r"(r[5][1]), "r"(r[5][2]), "r"(r[5][3]),
+      "r"(r[6][0]), "r"(r[6][1]), "r"(r[6][2]), "r"(r[6][3]),
+      "r"(r[7][0]), "r"(r[7][1]), "r"(r[7][2]), "r"(r[7][3])
+      : "memory");
+}
+
+template <>
+__device__ __forceinline__ void tmem_st_codes<4>(uint32_t taddr, const uint32_t (&r)[4][4]) {
+  tmem_st_x16(taddr, r);
+}
+template <>
+__device__ __forceinline__ void tmem_st_codes<8>(uint32_t taddr, const uint32_t (&r)[8][4]) {
+  tmem_st_x32(taddr, r);
 }
 
 // Instruction descriptor of a block-scaled kind::mxf4 MMA: A = B = E2M1, K-major, UE8M0 scales per
@@ -418,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
                                                      const __grid_constant__ MoeTable<MAXE> tab,
                                                      const __grid_constant__ CUtensorMap wmap) {
   using C = Cfg<NMAX>;
-  constexpr int kNW = C::kNW, kNA = C::kNA;
+  constexpr int kNW = C::kNW, kNA = C::kNA, kKB = C::kKB, kNBT = C::kNBT, kNG = C::kNG, kPF = C::kPF;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = a.nbr, S = (nbr + kKB - 1) / kKB;
@@ -480,9 +513,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   if (warp < kDecWarps) {
     // ---------------------------------------------------------------- decode warps
     const int sp = warp & 3, h = warp >> 2, m = 32 * sp + lane;
-    const uint32_t rb = (uint32_t)(m & 63), sw = rb & 7u;  // row in its TMA box, 128-byte swizzle
-    const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * 8192u + rb * 128u;
-    const uint32_t wo0 = ((2u * h) ^ sw) * 16u, wo1 = ((2u * h + 1u) ^ sw) * 16u;
+    // this thread's 8 kNBT bytes of a stage row: 16-byte chunks c0.. of TMA box column bc, 128-byte
+    // swizzle (chunk c of box row rb sits at chunk c ^ (rb & 7))
+    const uint32_t rb = (uint32_t)(m & 63), sw = rb & 7u;
+    const uint32_t bc = (uint32_t)(h * kNBT * 8) / 128u, c0 = ((uint32_t)(h * kNBT * 8) % 128u) / 16u;
+    const uint32_t wrow = smem_u32(smem + geo.off_W) + ((uint32_t)(m >> 6) * C::kBoxCols + bc) * 8192u + rb * 128u;
+    uint32_t wo[kNBT / 2];
+#pragma unroll
+    for (int i = 0; i < kNBT / 2; i++) wo[i] = ((c0 + (uint32_t)i) ^ sw) * 16u;
     const uint32_t tq = tbase + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lane quarter
     auto epilogue = [&](int jl_e) {
       const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
@@ -573,27 +611,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       }
     };
 
-    // Scale factors of this thread's group of four blocks, kPF stages ahead of their use (slot u
-    // holds the stage q with q % kPF == u): its row's four UE8M0 bytes (two 16-bit loads) and the
+    // Scale factors of this thread's kNG groups of four blocks, kPF stages ahead of their use (slot
+    // u holds the stage q with q % kPF == u): its row's bytes (16-bit loads of block pairs) and the
     // words of the B rows 32c + lane, c < kC.
-    uint32_t pa[kPF][2], pb[kPF][C::kC];
+    uint32_t pa[kPF][kNBT / 2], pb[kPF][kNG][C::kC];
     int qp = 0, jl_p = 0, s_p = 0;
-    const unsigned short *srow = nullptr;  // row m's scales of the front job, from block 4h on
+    const unsigned short *srow = nullptr;  // row m's scales of the front job, from block kNBT h on
     const uint32_t *sfb_src = nullptr;     // the front job's B scale words of this lane
-    auto load_sf = [&](uint32_t(&da)[2], uint32_t(&db)[C::kC]) {
+    auto load_sf = [&](uint32_t(&da)[kNBT / 2], uint32_t(&db)[kNG][C::kC]) {
       if (qp >= nq) return;
       if (s_p == 0) {
         const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_p));
         const int row = tile_row(jr, m);
-        srow = row >= 0 ? reinterpret_cast<const unsigned short *>(jr.sc + (size_t)row * nbr + 4 * h) : nullptr;
+        srow = row >= 0 ? reinterpret_cast<const unsigned short *>(jr.sc + (size_t)row * nbr + kNBT * h) : nullptr;
         sfb_src = reinterpret_cast<const uint32_t *>(a.terms + (size_t)jr.group * tbytes + (size_t)S * C::kBStage) +
-                  (size_t)(h * C::kC) * 32 + lane;
+                  (size_t)(h * kNG * C::kC) * 32 + lane;
       }
 #pragma unroll
-      for (int i = 0; i < 2; i++)
-        da[i] = srow != nullptr && kKB * s_p + 4 * h + 2 * i < nbr ? (uint32_t)__ldg(srow + 8 * s_p + i) : 0u;
+      for (int i = 0; i < kNBT / 2; i++)
+        da[i] = srow != nullptr && kKB * s_p + kNBT * h + 2 * i < nbr ? (uint32_t)__ldg(srow + (kKB / 2) * s_p + i) : 0u;
 #pragma unroll
-      for (int c = 0; c < C::kC; c++) db[c] = __ldg(sfb_src + (size_t)s_p * (C::kSfbStage / 4) + c * 32);
+      for (int g = 0; g < kNG; g++)
+#pragma unroll
+        for (int c = 0; c < C::kC; c++)
+          db[g][c] = __ldg(sfb_src + (size_t)s_p * (C::kSfbStage / 4) + (g * C::kC + c) * 32);
       qp++;
       if (++s_p == S) {
         s_p = 0;
@@ -622,16 +663,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
           stop = true;
           break;
         }
-        const uint32_t wa = wrow + ws * kWStage;
-        const uint4 c0 = lds_u4(wa + wo0), c1 = lds_u4(wa + wo1);
+        const uint32_t wa = wrow + ws * C::kWStage;
+        uint4 cw[kNBT / 2];
+#pragma unroll
+        for (int i = 0; i < kNBT / 2; i++) cw[i] = lds_u4(wa + wo[i]);
         __syncwarp();
         if (lane == 0) mbar_arrive(&w_empty[ws]);
         ws = ws + 1 == (uint32_t)kNW ? 0u : ws + 1;
-        uint32_t W[4][4];
-        planes_to_nibbles_interleaved(decode_block0(c0.x, c0.y), W[0][0], W[0][1], W[0][2], W[0][3]);
-        planes_to_nibbles_interleaved(decode_block0(c0.z, c0.w), W[1][0], W[1][1], W[1][2], W[1][3]);
-        planes_to_nibbles_interleaved(decode_block0(c1.x, c1.y), W[2][0], W[2][1], W[2][2], W[2][3]);
-        planes_to_nibbles_interleaved(decode_block0(c1.z, c1.w), W[3][0], W[3][1], W[3][2], W[3][3]);
+        uint32_t W[kNBT][4];
+#pragma unroll
+        for (int i = 0; i < kNBT / 2; i++) {
+          planes_to_nibbles_interleaved(decode_block0(cw[i].x, cw[i].y), W[2 * i][0], W[2 * i][1], W[2 * i][2],
+                                        W[2 * i][3]);
+          planes_to_nibbles_interleaved(decode_block0(cw[i].z, cw[i].w), W[2 * i + 1][0], W[2 * i + 1][1],
+                                        W[2 * i + 1][2], W[2 * i + 1][3]);
+        }
         if (q >= kNA) {
           if (lane == 0) ok = mbar_wait(&a_empty[b], (uint32_t)((q - kNA) / kNA) & 1u, tmo);
           ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -642,13 +688,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
           }
           tc_fence_after();
         }
-        // the four blocks' codes (columns 16h..16h+15 of the stage's A), the scale factors of this
-        // row (its own quarter, column 4h + quarter) and of B rows 32c + lane (every quarter holds a
-        // copy). Columns of blocks beyond the row's end hold the decode of the zero fill; no MMA reads them.
-        tmem_st_x16(tq + C::kACol + kACols * b + 16u * (uint32_t)h, W);
-        tmem_st_x1(tq + C::kSfaCol + 16u * b + 4u * (uint32_t)h + (uint32_t)sp, pa[u][0] | (pa[u][1] << 16));
+        // the blocks' codes (columns 4 kNBT h.. of the stage's A), the scale factors of this row
+        // (its own quarter, column 4g + quarter of group g) and of B rows 32c + lane (every quarter
+        // holds a copy). Columns of blocks beyond the row's end hold the decode of the zero fill; no
+        // MMA reads them.
+        tmem_st_codes<kNBT>(tq + C::kACol + C::kACols * b + 4u * kNBT * (uint32_t)h, W);
 #pragma unroll
-        for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + C::kSfbCol + 16u * b + 4u * (uint32_t)h + (uint32_t)c, pb[u][c]);
+        for (int g = 0; g < kNG; g++) {
+          const uint32_t gg = (uint32_t)(kNG * h + g);
+          tmem_st_x1(tq + C::kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[u][2 * g] | (pa[u][2 * g + 1] << 16));
+#pragma unroll
+          for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + C::kSfbCol + kKB * b + 4u * gg + (uint32_t)c, pb[u][g][c]);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -689,10 +740,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       if (lane == 0) {
         if (qi >= kNW) ok = mbar_wait(&w_empty[wi], (uint32_t)((qi - kNW) / kNW) & 1u, tmo);
         if (ok) {
-          mbar_arrive_expect_tx(&w_full[wi], kWStage);
-          const uint32_t dst = wbase + wi * kWStage;
-          tma_load_2d(dst, map_i, 128 * s_i, ji.y0, &w_full[wi]);
-          tma_load_2d(dst + 8192u, map_i, 128 * s_i, ji.y1, &w_full[wi]);
+          mbar_arrive_expect_tx(&w_full[wi], C::kWStage);
+          const uint32_t dst = wbase + wi * C::kWStage;
+#pragma unroll
+          for (int c = 0; c < C::kBoxCols; c++) {
+            tma_load_2d(dst + (uint32_t)c * 8192u, map_i, kKB * 8 * s_i + 128 * c, ji.y0, &w_full[wi]);
+            tma_load_2d(dst + (uint32_t)(C::kBoxCols + c) * 8192u, map_i, kKB * 8 * s_i + 128 * c, ji.y1, &w_full[wi]);
+          }
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -752,10 +806,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         if (!ok) break;
         tc_fence_after();
         const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
-        const uint32_t at = tbase + C::kACol + kACols * (uint32_t)b;
-        uint64_t bd = smem_desc(b0 + (uint32_t)b * C::kBStage, 128u, kSbo);
+        const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
+        uint64_t bd = smem_desc(b0 + (uint32_t)b * C::kBStage, 128u, C::kSbo);
         const uint32_t d_t = tbase + (uint32_t)((jl & 1) * NMAX);
-        const uint32_t sfa = tbase + C::kSfaCol + 16u * (uint32_t)b, sfb = tbase + C::kSfbCol + 16u * (uint32_t)b;
+        const uint32_t sfa = tbase + C::kSfaCol + kKB * (uint32_t)b, sfb = tbase + C::kSfbCol + kKB * (uint32_t)b;
         for (int j = 0; j < nmma; j++) {
           const uint32_t g = (uint32_t)(j >> 1), sf = (uint32_t)(j & 1) * 2u;
           mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd, sf ? idesc2 : idesc0, (sfa + 4u * g) | (sf << 30),
@@ -838,8 +892,8 @@ static bool mma_fits(int NMAX, int mode) {
 static bool k_ok(int nbr) { return nbr >= 2 && nbr % 2 == 0; }
 
 static size_t terms_for(int nbr, int NMAX) {
-  const int S = (nbr + kKB - 1) / kKB;
-  return NMAX == 32 ? terms_bytes<32>(S) : terms_bytes<96>(S);
+  return NMAX == 32 ? terms_bytes<32>((nbr + Cfg<32>::kKB - 1) / Cfg<32>::kKB)
+                    : terms_bytes<96>((nbr + Cfg<96>::kKB - 1) / Cfg<96>::kKB);
 }
 
 bool gemv_mma_supported(const MatView &w, int T) {
