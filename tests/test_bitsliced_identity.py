@@ -120,3 +120,24 @@ def test_interleaved_nibble_order():
     for j, w in enumerate((a, b, c, d)):
         for v in range(8):
             assert ((w >> np.uint64(4 * v)) & np.uint64(15) == codes[:, 4 * v + j]).all()
+
+
+def test_factored_segment_start_form():
+    # The segment-start decoder shifts shared XOR sums once (F = L ^ L<<2, U = L ^ L<<6,
+    # G = H ^ H<<2); restated here, it must equal the term-by-term planes for random blocks.
+    rng = np.random.default_rng(9)
+    L = rng.integers(0, 1 << 32, 4096, dtype=np.uint64)
+    H = rng.integers(0, 1 << 32, 4096, dtype=np.uint64)
+    z = np.zeros_like(L)
+    ref = _planes(L, H, z, z)
+
+    def s(x, d):
+        return (x << np.uint64(d)) & M32
+    F, U, H2 = L ^ s(L, 2), L ^ s(L, 6), s(H, 2)
+    G = H ^ H2
+    X = H ^ s(F, 2) ^ s(L, 7)
+    q1h = X ^ s(H, 1)
+    got = ((~(q1h ^ s(U, 1) ^ s(G, 4))) & M32, (~(X ^ s(F, 3) ^ s(H, 7))) & M32,
+           (~(q1h ^ U ^ s(G, 3) ^ H2)) & M32, (~q1h) & M32)
+    for a, b in zip(got, ref):
+        assert (a == b).all()
