@@ -268,6 +268,13 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
   return v;
 }
 
+// True in exactly one active lane of the warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(e));
+  return e != 0;
+}
+
 // 2-D TMA tile load (no multicast; the tensor map covers this GPU's memory only).
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, int x, int y, uint64_t *bar) {
   asm volatile(
@@ -791,47 +798,58 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- MMA warp
-    if (lane == 0) {
-      int jl = 0, s = 0;
-      uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : 16);
-      uint32_t idesc0 = idesc_mxf4(ncols, 0u), idesc2 = idesc_mxf4(ncols, 2u);
-      const uint32_t b0 = smem_u32(smem + geo.off_B);
-      bool ok = true;
-      for (int q = 0; q < nq; q++) {
-        if (*abort_flag) break;
-        const int b = q % kNA;
-        const uint32_t ph = (uint32_t)(q / kNA) & 1u;
-        ok = mbar_wait(&a_full[b], ph, tmo) && mbar_wait(&b_full[b], ph, tmo);
-        if (ok && s == 0 && jl >= 2) ok = mbar_wait(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo);
-        if (!ok) break;
-        tc_fence_after();
-        const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
-        const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
-        uint64_t bd = smem_desc(b0 + (uint32_t)b * C::kBStage, 128u, C::kSbo);
-        const uint32_t d_t = tbase + (uint32_t)((jl & 1) * NMAX);
-        const uint32_t sfa = tbase + C::kSfaCol + kKB * (uint32_t)b, sfb = tbase + C::kSfbCol + kKB * (uint32_t)b;
-        for (int j = 0; j < nmma; j++) {
-          const uint32_t g = (uint32_t)(j >> 1), sf = (uint32_t)(j & 1) * 2u;
-          mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd, sf ? idesc2 : idesc0, (sfa + 4u * g) | (sf << 30),
-                      (sfb + 4u * g) | (sf << 30), !(s == 0 && j == 0));
-          bd += 16u;  // +256 bytes: two chunks (the descriptor's start address counts 16-byte units)
+    // The whole warp runs the loop (its values are warp-uniform); one elected lane issues the
+    // tcgen05 operations.
+    const bool leader = elect_one();
+    int jl = 0, s = 0;
+    uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : 16);
+    uint32_t idesc0 = idesc_mxf4(ncols, 0u), idesc2 = idesc_mxf4(ncols, 2u);
+    const uint32_t b0 = smem_u32(smem + geo.off_B);
+    bool ok = true;
+    for (int q = 0; q < nq; q++) {
+      if (*abort_flag) break;
+      const int b = q % kNA;
+      const uint32_t ph = (uint32_t)(q / kNA) & 1u;
+      ok = mbar_wait(&a_full[b], ph, tmo) && mbar_wait(&b_full[b], ph, tmo);
+      if (ok && s == 0 && jl >= 2) ok = mbar_wait(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
+      const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
+      const uint64_t bd = smem_desc(b0 + (uint32_t)b * C::kBStage, 128u, C::kSbo);
+      const uint32_t d_t = tbase + (uint32_t)((jl & 1) * NMAX);
+      const uint32_t sfa = tbase + C::kSfaCol + kKB * (uint32_t)b, sfb = tbase + C::kSfbCol + kKB * (uint32_t)b;
+      if (leader) {
+#pragma unroll
+        for (int j = 0; j < kKB / 2; j++) {
+          if (j < nmma) {
+            const uint32_t sf = (uint32_t)(j & 1) * 2u;
+            // +256 bytes of B per MMA: the descriptor's start address counts 16-byte units
+            mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
+                        (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30), (sfb + 4u * (uint32_t)(j >> 1)) | (sf << 30),
+                        !(s == 0 && j == 0));
+          }
         }
         tc_commit(&a_empty[b]);
         if (s == S - 1) tc_commit(&acc_full[jl & 1]);
-        if (++s == S) {
-          s = 0;
-          if (++jl < my_jobs) {
-            const uint32_t nc = (uint32_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl)).ncols;
-            if (nc != ncols) {
-              ncols = nc;
-              idesc0 = idesc_mxf4(ncols, 0u);
-              idesc2 = idesc_mxf4(ncols, 2u);
-            }
+      }
+      __syncwarp();
+      if (++s == S) {
+        s = 0;
+        if (++jl < my_jobs) {
+          const uint32_t nc = (uint32_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl)).ncols;
+          if (nc != ncols) {
+            ncols = nc;
+            idesc0 = idesc_mxf4(ncols, 0u);
+            idesc2 = idesc_mxf4(ncols, 2u);
           }
         }
       }
-      if (!ok) *abort_flag = 1;
-      // drain: every tcgen05 operation issued so far
+    }
+    if (!ok && lane == 0) *abort_flag = 1;
+    // drain: every tcgen05 operation issued so far
+    if (leader) {
       tc_commit(drain);
       mbar_wait(drain, 0u, tmo);
     }
