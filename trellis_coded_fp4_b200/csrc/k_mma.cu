@@ -21,8 +21,9 @@
 //  * B loader warp: lane 0 bulk-copies each stage's activation terms into the B slot of the stage.
 //  * MMA warp: lane 0 waits for a stage, issues its KB/2 MMAs (A from TMEM, B from shared memory) into
 //    a double-buffered TMEM accumulator and releases the stage with one commit.
-//  * the epilogue of job i (tcgen05.ld, then the GEMV output, the SwiGLU of gate/up rows, or the MoE
-//    down rows and their combine) runs in decode warps 0-3 early in job i+1.
+//  * 4 epilogue warps (one per TMEM lane quarter): the epilogue of each job (tcgen05.ld, then the
+//    GEMV output, the SwiGLU of gate/up rows, or the MoE down rows and their combine), overlapping
+//    the next job's stages.
 // All tcgen05 MMAs of the CTA are issued by one thread. Every wait is a bounded mbarrier wait; a
 // wait that gives up raises a shared abort flag that every role polls once per stage, and each
 // role drains its own asynchronous copies and MMAs before the CTA frees its TMEM.
@@ -41,7 +42,7 @@ __device__ unsigned int g_tcf4_timeouts_mma = 0;
 
 constexpr int kTerms = 6;            // E2M1 terms per activation block
 constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> jobs in flight)
-constexpr int kDecWarps = 16, kWLoadWarp = 16, kMmaWarp = 17, kBLoadWarp = 18, kThreads = 608;
+constexpr int kDecWarps = 16, kWLoadWarp = 16, kMmaWarp = 17, kBLoadWarp = 18, kEpiWarp0 = 19, kThreads = 736;
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
 
@@ -515,7 +516,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   const int my_jobs = (int)blockIdx.x < njobs ? (njobs - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int nq = my_jobs * S;
   auto job_of = [&](int jl) { return (int)blockIdx.x + jl * (int)gridDim.x; };
-  const int s_epi = S > 1 ? 1 : 0;  // the epilogue of job jl-1 runs after the A stage (jl, s_epi)
 
   if (warp < kDecWarps) {
     // ---------------------------------------------------------------- decode warps
@@ -529,94 +529,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
 #pragma unroll
     for (int i = 0; i < kNBT / 2; i++) wo[i] = ((c0 + (uint32_t)i) ^ sw) * 16u;
     const uint32_t tq = tbase + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lane quarter
-    auto epilogue = [&](int jl_e) {
-      const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
-      const int buf = jl_e & 1;
-      if (!mbar_wait(&acc_full[buf], (uint32_t)(jl_e >> 1) & 1u, tmo)) {
-        *abort_flag = 1;
-        return;
-      }
-      tc_fence_after();
-      float v[C::kTok];
-#pragma unroll
-      for (int t = 0; t < C::kTok; t++) v[t] = 0.f;
-#pragma unroll
-      for (int c0 = 0; c0 < C::kTok * kTerms; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld_x16(tbase + ((uint32_t)(32 * warp) << 16) + (uint32_t)(buf * NMAX + c0), r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; i++)
-          if (c0 + i < C::kTok * kTerms) v[(c0 + i) / kTerms] += __uint_as_float(r[i]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
-      const int mrow = 32 * warp + lane;
-      if (MODE == kModeGemv) {
-        const int row = tile_row(jr, mrow);
-        if (row >= 0)
-#pragma unroll
-          for (int t = 0; t < C::kTok; t++)
-            if (t < a.T) a.y[(size_t)t * a.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v[t]));
-      } else if (MODE == kModeGateUp) {
-        float *U = reinterpret_cast<float *>(smem + geo.off_U) + (size_t)buf * 64 * C::kTok;
-        const uint32_t use = (uint32_t)(jl_e >> 1);
-        if (warp >= 2) {  // up rows: hand them to the gate rows' warps
-          if (use >= 1 && !mbar_wait(&u_empty[buf], (use - 1u) & 1u, tmo)) {
-            *abort_flag = 1;
-            return;
-          }
-#pragma unroll
-          for (int t = 0; t < C::kTok; t++) U[(mrow - 64) * C::kTok + t] = v[t];
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&u_full[buf]);
-        } else {
-          if (!mbar_wait(&u_full[buf], use & 1u, tmo)) {
-            *abort_flag = 1;
-            return;
-          }
-          if (mrow < jr.na)
-#pragma unroll
-            for (int t = 0; t < C::kTok; t++)
-              if (t < jr.cnt) {
-                const float g = v[t], u = U[mrow * C::kTok + t];
-                const int p = pl->list[jr.first + t];
-                a.hidden[(size_t)p * a.I + jr.row0 + mrow] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.0f + expf(-g)) * u));
-              }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&u_empty[buf]);
-        }
-      } else {
-        const int row = tile_row(jr, mrow);
-        if (row >= 0)
-#pragma unroll
-          for (int t = 0; t < C::kTok; t++)
-            if (t < jr.cnt) a.yws[(size_t)pl->list[jr.first + t] * a.H + row] = v[t];
-        __threadfence();
-        __syncwarp();
-        // the last group to finish this warp's 32 rows of the chunk combines them:
-        // out = sum_j w_j y_j over the token's routed pairs, in fixed j order
-        int last = 0;
-        if (lane == 0) last = atomicAdd(&a.counters[jr.chunk * 4 + warp], 1) == pl->n_groups - 1;
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          const int n = jr.row0 + mrow;
-          if (n < a.H)
-            for (int t = 0; t < a.Tm; t++) {
-              float acc = 0.f;
-              for (int jj = 0; jj < a.k; jj++) {
-                const int p = t * a.k + jj, ee = pl->ids[p];
-                if (ee < 0 || ee >= a.E) continue;
-                acc = fmaf(__ldg(a.wts + p), __ldcg(a.yws + (size_t)p * a.H + n), acc);
-              }
-              a.out[(size_t)t * a.H + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
-            }
-        }
-      }
-    };
 
     // Scale factors of this thread's kNG groups of four blocks, kPF stages ahead of their use (slot
     // u holds the stage q with q % kPF == u): its row's bytes (16-bit loads of block pairs) and the
@@ -651,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
 #pragma unroll
     for (int u = 0; u < kPF; u++) load_sf(pa[u], pb[u]);
 
-    int jl = 0, s = 0, q = 0;
+    int q = 0;
     uint32_t ws = 0, b = 0;
     bool stop = false;
     for (int q0 = 0; q0 < nq && !stop; q0 += kPF) {
@@ -713,15 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         if (lane == 0) mbar_arrive(&a_full[b]);
         load_sf(pa[u], pb[u]);
         b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
-        if (warp < 4 && jl >= 1 && s == s_epi) epilogue(jl - 1);
-        if (++s == S) {
-          s = 0;
-          ++jl;
-        }
       }
     }
-    if (!stop) q = nq;
-    if (q == nq && nq > 0 && warp < 4 && !*abort_flag) epilogue(my_jobs - 1);
   } else if (warp == kWLoadWarp) {
     // ---------------------------------------------------------------- word loader warp
     // TMA front: stage qi of job jl_i, up to kNW stages ahead of the decode warps.
@@ -796,6 +701,99 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         if (!mbar_wait(&b_full[d % kNA], (uint32_t)(d / kNA) & 1u, tmo)) break;
     }
     __syncwarp();
+  } else if (warp >= kEpiWarp0) {
+    // ---------------------------------------------------------------- epilogue warps
+    // Warp kEpiWarp0 + i reads TMEM lane quarter eq = warp % 4, i.e. tile rows 32 eq..32 eq + 31.
+    const int eq = warp & 3;
+    auto epilogue = [&](int jl_e) {
+      const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
+      const int buf = jl_e & 1;
+      if (!mbar_wait(&acc_full[buf], (uint32_t)(jl_e >> 1) & 1u, tmo)) {
+        *abort_flag = 1;
+        return;
+      }
+      tc_fence_after();
+      float v[C::kTok];
+#pragma unroll
+      for (int t = 0; t < C::kTok; t++) v[t] = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < C::kTok * kTerms; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_x16(tbase + ((uint32_t)(32 * eq) << 16) + (uint32_t)(buf * NMAX + c0), r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; i++)
+          if (c0 + i < C::kTok * kTerms) v[(c0 + i) / kTerms] += __uint_as_float(r[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      const int mrow = 32 * eq + lane;
+      if (MODE == kModeGemv) {
+        const int row = tile_row(jr, mrow);
+        if (row >= 0)
+#pragma unroll
+          for (int t = 0; t < C::kTok; t++)
+            if (t < a.T) a.y[(size_t)t * a.rows + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v[t]));
+      } else if (MODE == kModeGateUp) {
+        float *U = reinterpret_cast<float *>(smem + geo.off_U) + (size_t)buf * 64 * C::kTok;
+        const uint32_t use = (uint32_t)(jl_e >> 1);
+        if (eq >= 2) {  // up rows: hand them to the gate rows' warps
+          if (use >= 1 && !mbar_wait(&u_empty[buf], (use - 1u) & 1u, tmo)) {
+            *abort_flag = 1;
+            return;
+          }
+#pragma unroll
+          for (int t = 0; t < C::kTok; t++) U[(mrow - 64) * C::kTok + t] = v[t];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&u_full[buf]);
+        } else {
+          if (!mbar_wait(&u_full[buf], use & 1u, tmo)) {
+            *abort_flag = 1;
+            return;
+          }
+          if (mrow < jr.na)
+#pragma unroll
+            for (int t = 0; t < C::kTok; t++)
+              if (t < jr.cnt) {
+                const float g = v[t], u = U[mrow * C::kTok + t];
+                const int p = pl->list[jr.first + t];
+                a.hidden[(size_t)p * a.I + jr.row0 + mrow] =
+                    __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.0f + expf(-g)) * u));
+              }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&u_empty[buf]);
+        }
+      } else {
+        const int row = tile_row(jr, mrow);
+        if (row >= 0)
+#pragma unroll
+          for (int t = 0; t < C::kTok; t++)
+            if (t < jr.cnt) a.yws[(size_t)pl->list[jr.first + t] * a.H + row] = v[t];
+        __threadfence();
+        __syncwarp();
+        // the last group to finish this warp's 32 rows of the chunk combines them:
+        // out = sum_j w_j y_j over the token's routed pairs, in fixed j order
+        int last = 0;
+        if (lane == 0) last = atomicAdd(&a.counters[jr.chunk * 4 + eq], 1) == pl->n_groups - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          const int n = jr.row0 + mrow;
+          if (n < a.H)
+            for (int t = 0; t < a.Tm; t++) {
+              float acc = 0.f;
+              for (int jj = 0; jj < a.k; jj++) {
+                const int p = t * a.k + jj, ee = pl->ids[p];
+                if (ee < 0 || ee >= a.E) continue;
+                acc = fmaf(__ldg(a.wts + p), __ldcg(a.yws + (size_t)p * a.H + n), acc);
+              }
+              a.out[(size_t)t * a.H + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+            }
+        }
+      }
+    };
+    for (int jl = 0; jl < my_jobs && !*abort_flag; jl++) epilogue(jl);
   } else {
     // ---------------------------------------------------------------- MMA warp
     // The whole warp runs the loop (its values are warp-uniform); one elected lane issues the
