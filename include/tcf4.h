@@ -93,6 +93,21 @@ TCF4_API size_t trellis_gemv_workspace(tcf4_matrix w, int32_t T);
 TCF4_API tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *workspace,
                                   size_t ws_bytes, void *stream);
 
+/* trellis_gemv without a caller-provided workspace (the source pages have no counterpart; this is
+ * a convenience of this library). Same arguments, result and accuracy as trellis_gemv.
+ * For callers that cannot hand over device scratch memory: a host program that holds only the
+ * device pointers it was given and has no device allocator of its own, or a serving loop that must
+ * not allocate while it runs because its memory was reserved up front.
+ * The scratch is one 1 MiB array per device, inside this library. The first call on each device
+ * does a one-time setup: it looks up that array's address through the CUDA runtime, with the
+ * device current. Make that first call before beginning any stream capture. All calls on a device
+ * share the array and leave in it whatever they last wrote; nothing in it has to start at zero, as
+ * each call writes the scratch it reads. Calls that overlap in time on one device (other streams or
+ * host threads) race on the array: the caller must serialize them.
+ * Returns TCF4_ERR_WORKSPACE when the call would need more than 1 MiB of scratch (not reached
+ * within the limits of trellis_gemv), TCF4_ERR_CUDA when the one-time setup fails. */
+TCF4_API tcf4_status trellis_gemv_noalloc(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream);
+
 /* Router for the MoE layer: for each token, the k experts with the largest logits (ties to the
  * lower expert index) and softmax weights over those k logits (fp32).
  *   logits: fp32 [T][E]; topk_ids: int32 [T][k]; topk_w: fp32 [T][k].

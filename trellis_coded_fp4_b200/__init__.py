@@ -81,6 +81,17 @@ def gemv(w: TrellisMatrix, x: torch.Tensor, out=None, workspace=None):
     return out
 
 
+def gemv_noalloc(w: TrellisMatrix, x: torch.Tensor, out=None):
+    """gemv through trellis_gemv_noalloc: the scratch is the library's own per-device array."""
+    x = x if x.dim() == 2 else x.view(1, -1)
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, w.rows), dtype=torch.bfloat16, device=x.device)
+    _abi.check(_abi.load().trellis_gemv_noalloc(w.abi(), _ptr(x), T, _ptr(out), _stream_handle()),
+               "trellis_gemv_noalloc")
+    return out
+
+
 def moe_route(logits: torch.Tensor, k: int, ids=None, wts=None):
     """Top-k experts (ties to the lower index) and softmax weights over the selected logits."""
     T, E = logits.shape

@@ -10,7 +10,8 @@ STATUS_NAMES = {0: "TCF4_OK", 1: "TCF4_ERR_INVALID_ARG", 2: "TCF4_ERR_MISALIGNED
                 4: "TCF4_ERR_WORKSPACE", 5: "TCF4_ERR_CUDA"}
 
 # Every symbol include/tcf4.h declares.
-EXPORTED = ("trellis_decode_to_mxfp4", "trellis_gemv_workspace", "trellis_gemv", "trellis_moe_route", "trellis_grouped_moe_workspace",
+EXPORTED = ("trellis_decode_to_mxfp4", "trellis_gemv_workspace", "trellis_gemv", "trellis_gemv_noalloc",
+            "trellis_moe_route", "trellis_grouped_moe_workspace",
             "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "tcf4_device_timeouts",
             "tcf4_status_string")
 
@@ -46,6 +47,8 @@ def load(path: str = LIB_PATH):
     L.trellis_gemv_workspace.restype = sz
     L.trellis_gemv.argtypes = [Matrix, vp, i32, vp, vp, sz, vp]
     L.trellis_gemv.restype = ctypes.c_int
+    L.trellis_gemv_noalloc.argtypes = [Matrix, vp, i32, vp, vp]
+    L.trellis_gemv_noalloc.restype = ctypes.c_int
     L.trellis_moe_route.argtypes = [vp, i32, i32, i32, vp, vp, vp]
     L.trellis_moe_route.restype = ctypes.c_int
     L.trellis_grouped_moe_workspace.argtypes = [ctypes.POINTER(Moe), i32, i32]
