@@ -311,6 +311,19 @@ def cpu_baseline(layer, seed, stride=16):
 
 # ----------------------------------------------------------------------------- arms
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest x over all ranks (x itself on one process): replicas are timed by the slowest."""
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, weights_per_step: int, steps: int, ms_total: float) -> float:
+    """Decoded weights/s of the whole job: every replica decodes weights_per_step per step."""
+    return world * weights_per_step * steps / (ms_total * 1e-3)
+
+
 def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -402,11 +415,7 @@ def main():
     if dist is not None:
         dist.barrier()
     clocks = sampler.stop(tw0, tw1)
-    ms_total = start.elapsed_time(end)
-    ms_t = torch.tensor([ms_total], device=device, dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_total = float(ms_t.item())
+    ms_total = max_over_ranks(start.elapsed_time(end), dist, device)
     ms_per_step = ms_total / args.steps
 
     # per-call durations (events bracket each call on the launching stream)
@@ -435,7 +444,7 @@ def main():
                 "kernel": dom, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                 else "fallback 6650 GB/s"}
 
-    value = world * step.weights_per_step * args.steps / (ms_total * 1e-3)
+    value = job_value(world, step.weights_per_step, args.steps, ms_total)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
@@ -444,7 +453,8 @@ def main():
                        "intermediate": I, "seg_len": SEG, "decoded_weights_per_step": step.weights_per_step,
                        "l2": "inputs larger than L2 (each step streams >900 MB of stream/MXFP4 bytes through L2)",
                        "parallelism": f"replicas x{world}",
-                       "arithmetic": "decode: u32 bit logic; products: f32 accumulation of bf16 activations"},
+                       "arithmetic": "decode: u32 bit logic; products: block-scaled MXFP4 tensor-core MMA (activations as "
+                                     "six E2M1 terms per 32-block), fp32 accumulation"},
             "roofline": roofline, "kernels": kernels,
             "gpu_launches": step.launches_per_step * args.steps, "clocks": clocks}
 
