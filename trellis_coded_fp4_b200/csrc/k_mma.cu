@@ -151,11 +151,16 @@ __device__ __forceinline__ uint32_t to_e2m1(float v) {
   return r & 15u;
 }
 
-// E2M1 code -> value (exact).
+// E2M1 code (low nibble) -> value, exact (every E2M1 value is a binary16 value).
 __device__ __forceinline__ float e2m1_value(uint32_t c) {
-  const uint32_t mag = c & 7u;
-  const float v = mag < 2u ? 0.5f * (float)mag : ldexpf(1.f + 0.5f * (float)(mag & 1u), (int)(mag >> 1) - 1);
-  return (c & 8u) ? -v : v;
+  uint32_t h2;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "r"(c & 15u));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// 2^e for e in [-127, 127], exact.
+__device__ __forceinline__ float pow2f(int e) {
+  return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
 // Per group of token slots, the activation terms of each stage: Bg [S][kBStage] (one K-major B
@@ -185,14 +190,14 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
   for (int j = 0; j < kTerms; j++) {
     const int n = kTerms * t + j;
     const float m = warp_max(fabsf(r));
-    int S = -127;
-    if (m > 0.f) {
-      const int e = ilogbf(m);
-      S = scalbnf(m, -e) <= 1.5f ? e - 2 : e - 1;
-      S = S < -127 ? -127 : (S > 127 ? 127 : S);
-    }
-    const uint32_t code = to_e2m1(scalbnf(r, -S));
-    r -= scalbnf(e2m1_value(code), S);
+    // S from m's exponent field: m = 1.f * 2^e, and m / 2^e <= 1.5 iff the fraction <= 0.5.
+    // A subnormal or zero m gives S = -127. S <= 126 for any finite m (max|bf16| < 2^128).
+    const uint32_t mb = __float_as_uint(m);
+    const int e = (int)(mb >> 23) - 127;
+    int S = (mb >> 23) == 0u ? -127 : ((mb & 0x7FFFFFu) <= 0x400000u ? e - 2 : e - 1);
+    S = S < -127 ? -127 : S;
+    const uint32_t code = to_e2m1(r * pow2f(-S));
+    r -= e2m1_value(code) * pow2f(S);
     const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 4);
     if (n < NMAX) {
       if (((lane >> 2) & 1) == 0)
