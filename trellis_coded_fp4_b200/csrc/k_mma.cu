@@ -12,21 +12,24 @@
 // up to five tokens per group, else 16):
 //  * word loader warp: lane 0 streams each stage's trellis words (128 rows x 8 KB bytes) into a ring
 //    of shared-memory slots with 2-D TMA tile loads (128-byte swizzle).
-//  * 16 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and the NBT = KB/4 K-blocks
-//    NBT(w/4).. of a stage (whole scale-factor groups). It reads its 8 NBT bytes of trellis words,
-//    decodes them in registers (bit-sliced) and stores the blocks' E2M1 codes, packed eight per
-//    32-bit column, into the stage's A operand in TMEM, together with the group's scale factors of
-//    its row (A) and of the B rows its lane stands for (tcgen05.st into its own lane quarter; the
-//    scale bytes are loaded a few stages ahead). The decoded weights never touch shared memory.
-//  * B loader warp: lane 0 bulk-copies each stage's activation terms into the B slot of the stage.
-//  * MMA warp: lane 0 waits for a stage, issues its KB/2 MMAs (A from TMEM, B from shared memory) into
-//    a double-buffered TMEM accumulator and releases the stage with one commit.
+//  * KB/2 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and the 8 K-blocks 8(w/4)..
+//    of a stage (two scale-factor groups). It reads its 64 bytes of trellis words, decodes them in
+//    registers (bit-sliced) and stores the blocks' E2M1 codes, packed eight per 32-bit column, into
+//    the stage's A operand in TMEM, together with the groups' scale factors of its row (A) and of
+//    the B rows its lane stands for (tcgen05.st into its own lane quarter; the scale bytes are
+//    loaded one stage ahead). The decoded weights never touch shared memory. A stage's A operand
+//    is handed over in two halves (the first and last KB/2 blocks), each with its own barriers.
+//  * B loader warp: lane 0 bulk-copies each stage's activation terms into a 4-slot B ring, up to four
+//    stages ahead of the MMAs.
+//  * MMA warp(s): with up to five tokens per group two issuer warps, one per half stage, each into
+//    its own accumulator of a double-buffered pair (a single issuing thread sustains about one MMA
+//    per 60 cycles; two in different warps run concurrently); otherwise one warp issues both
+//    halves. A half's MMAs (A from TMEM, B from shared memory) are released with one commit.
 //  * 4 epilogue warps (one per TMEM lane quarter): the epilogue of each job (tcgen05.ld, then the
 //    GEMV output, the SwiGLU of gate/up rows, or the MoE down rows and their combine), overlapping
 //    the next job's stages.
-// All tcgen05 MMAs of the CTA are issued by one thread. Every wait is a bounded mbarrier wait; a
-// wait that gives up raises a shared abort flag that every role polls once per stage, and each
-// role drains its own asynchronous copies and MMAs before the CTA frees its TMEM.
+// Every wait is bounded; a wait that gives up raises a shared abort flag that the other roles see,
+// and each role drains its own asynchronous copies and MMAs before the CTA frees its TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -42,7 +45,12 @@ __device__ unsigned int g_tcf4_timeouts_mma = 0;
 
 constexpr int kTerms = 6;            // E2M1 terms per activation block
 constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> jobs in flight)
-constexpr int kDecWarps = 16, kWLoadWarp = 16, kMmaWarp = 17, kBLoadWarp = 18, kEpiWarp0 = 19, kThreads = 736;
+
+// Head start of the first half's decode warps (about half a stage).
+constexpr uint32_t kHalfLagNs = 600u;
+// Sleep between barrier tests of the idle roles. The loaders run stages ahead and the MMA issuers
+// have about two stages (~3 us) of slack, so these only bound how soon a completed phase is seen.
+constexpr uint32_t kLoaderSleepNs = 200u, kMmaSleepNs = 100u, kEpiSleepNs = 200u;
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
 
@@ -53,18 +61,28 @@ struct Cfg {
   static constexpr int kSlots = (NMAX + kTerms - 1) / kTerms;  // token slots the split writes
   static constexpr int kC = (NMAX + 31) / 32;                  // B scale columns per 4-block group
   static constexpr int kKB = NMAX <= 32 ? 32 : 16;             // 32-blocks per row per stage
-  static constexpr int kNBT = kKB / 4;                         // blocks per decode thread per stage
+  // Warps: kDecWarps decode warps (four per group of 8 blocks of a stage), then the word loader, two
+  // MMA issuer slots, the B loader and four epilogue warps.
+  static constexpr int kDecWarps = kKB / 2;
+  static constexpr int kWLoadWarp = kDecWarps, kMmaWarp = kDecWarps + 1, kBLoadWarp = kDecWarps + 3;
+  static constexpr int kEpiWarp0 = kDecWarps + 4, kThreads = 32 * (kDecWarps + 8);
+  static constexpr int kNBT = 8;                               // blocks per decode thread per stage
+  static constexpr int kNCh = kNBT / 8;                        // decoded in chunks of 8 blocks
   static constexpr int kNG = kNBT / 4;                         // scale groups per decode thread
   static constexpr int kNW = kKB == 32 ? 3 : 6;                // word stages in flight
-  static constexpr int kNA = NMAX <= 32 ? 2 : 3;               // A / B / scale-factor stages
-  static constexpr int kPF = kKB == 32 ? 2 : 4;                // stages of scale factors in flight
+  static constexpr int kNA = NMAX <= 32 ? 2 : 3;               // A / scale-factor stages (TMEM)
+  static constexpr int kNB = 4;                                // B stages (shared memory)
   static constexpr int kBoxCols = kKB / 16;                    // 128-byte TMA boxes per 64 rows
   static constexpr uint32_t kWStage = 1024u * kKB;             // 128 rows x 8 KB bytes of words
   static constexpr uint32_t kSbo = 128u * kKB;                 // B: 8 rows x KB chunks x 16 bytes
   static constexpr uint32_t kBStage = NMAX * 16u * kKB;        // NMAX rows x 32 KB E2M1
   static constexpr uint32_t kSfbStage = (kKB / 4) * kC * 128u;  // [group][column][lane] u32
+  // MMA issuers: one per half stage, each into its own accumulator, where TMEM has room for the
+  // two accumulator pairs (one issuing thread sustains about one MMA per 60 cycles; two of them in
+  // different warps run concurrently).
+  static constexpr int kNI = NMAX <= 32 ? 2 : 1;
   static constexpr uint32_t kACols = 4u * kKB;                 // TMEM columns of a stage's A
-  static constexpr uint32_t kACol = 2u * NMAX;                 // TMEM: accumulators first, then
+  static constexpr uint32_t kACol = 2u * kNI * NMAX;           // TMEM: accumulators first, then
   static constexpr uint32_t kSfaCol = kACol + kACols * kNA;    // A stages, A scales (KB columns per
   static constexpr uint32_t kSfbCol = kSfaCol + kKB * kNA;     // stage), B scales (KB per stage)
   static constexpr uint32_t kUsed = kSfbCol + kKB * kNA;
@@ -208,9 +226,16 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
 }
 
 // Plain GEMV: one group, token slots 0..T-1 (slots up to kSlots are zero rows).
+// Programmatic dependent launch: the GEMV's product kernel is launched while the activation split
+// still runs. It starts its TMEM setup and its first weight tiles (which do not depend on the split)
+// at once, and waits for the split's completion only before it reads the activation terms.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 template <int NMAX>
 __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
                                                      uint8_t *__restrict__ terms) {
+  grid_dep_release();  // the product kernel may start; it waits for this grid before reading terms
   const int nb = K >> 5, S = (nb + Cfg<NMAX>::kKB - 1) / Cfg<NMAX>::kKB, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < Cfg<NMAX>::kSlots * nb; wi += nwarps) {
@@ -260,7 +285,7 @@ __host__ __device__ inline MmaGeom mma_geom(int mode) {
   MmaGeom g;
   g.off_W = 1024u;
   g.off_B = g.off_W + C::kNW * C::kWStage;
-  g.off_U = g.off_B + C::kNA * C::kBStage;
+  g.off_U = g.off_B + C::kNB * C::kBStage;
   g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)C::kTok * 4u : 0u);
   g.smem = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
   return g;
@@ -272,6 +297,56 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
+}
+
+// One arrival on `bar` for the whole (converged) warp, from one elected lane; no branch.
+__device__ __forceinline__ void mbar_arrive_one(uint64_t *bar) {
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// Non-blocking test of a barrier phase (1 once the phase with the given parity has completed). Its
+// result is read later, so the test's latency overlaps other work.
+__device__ __forceinline__ uint32_t mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok;
+}
+
+// Bounded wait for a warp that has nothing else to do meanwhile (loaders, MMA issuers, the epilogue's
+// poller): it tests the barrier and sleeps about `ns` nanoseconds between tests. (A blocking try_wait
+// returns every few tens of nanoseconds while it waits, and the polls of several idle warps take
+// issue slots from the decode warps on the same SM sub-partitions.)
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, unsigned int *timeouts, uint32_t ns) {
+  if (mbar_test(bar, parity)) return true;
+  const long long t0 = clock64();
+  do {
+    __nanosleep(ns);
+    if (mbar_test(bar, parity)) return true;
+  } while (clock64() - t0 < kWaitCycles);
+  atomicAdd(timeouts, 1u);
+  return false;
+}
+
+// Bounded wait executed by the whole warp (one poll instruction serves all lanes; the result is made
+// warp-uniform). The shared abort flag is read only on the slow path, so a wait that succeeds at
+// once costs a poll and a vote.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, unsigned int *timeouts,
+                                          volatile int *abort_flag) {
+  bool ok = mbar_try_wait(bar, parity);
+  if (!__all_sync(0xffffffffu, ok)) {
+    const long long t0 = clock64();
+    ok = false;
+    while (!ok && !*abort_flag && clock64() - t0 < kWaitCycles) ok = mbar_try_wait(bar, parity);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok && (threadIdx.x & 31) == 0 && !*abort_flag) atomicAdd(timeouts, 1u);
+  }
+  return ok;
 }
 
 // True in exactly one active lane of the warp.
@@ -460,20 +535,22 @@ __device__ __forceinline__ int tile_row(const JobRows &j, int m) {
 // ------------------------------------------------------------------------------- the kernel
 
 template <int MAXE, int MODE, int NMAX>
-__global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
+__global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
                                                      const __grid_constant__ MoeTable<MAXE> tab,
                                                      const __grid_constant__ CUtensorMap wmap) {
   using C = Cfg<NMAX>;
-  constexpr int kNW = C::kNW, kNA = C::kNA, kKB = C::kKB, kNBT = C::kNBT, kNG = C::kNG, kPF = C::kPF;
+  constexpr int kNW = C::kNW, kNA = C::kNA, kKB = C::kKB, kNBT = C::kNBT, kNG = C::kNG;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = a.nbr, S = (nbr + kKB - 1) / kKB;
   const MmaGeom geo = mma_geom<NMAX>(MODE);
-  static_assert(kNW <= 8 && kNA <= 4, "barrier block: 8 word slots, 4 operand slots");
-  uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);  // 37 barriers in bytes [0, 296)
-  uint64_t *w_empty = w_full + 8, *a_full = w_full + 16, *a_empty = w_full + 20, *b_full = w_full + 24,
-           *acc_full = w_full + 28, *acc_empty = w_full + 30, *u_full = w_full + 32, *u_empty = w_full + 34,
-           *drain = w_full + 36;
+  static_assert(kNW <= 8 && kNA <= 4 && C::kNB <= 4, "barrier block: 8 word slots, 4 A and 4 B slots");
+  // 49 barriers in bytes [0, 392). The A operand of a stage is filled and released in two halves
+  // (blocks [0, KB/2) and [KB/2, KB), each by half of the decode warps): barrier 2 b + half.
+  uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *w_empty = w_full + 8, *a_full = w_full + 16, *a_empty = w_full + 24, *b_full = w_full + 32,
+           *b_empty = w_full + 36, *acc_full = w_full + 40, *acc_empty = w_full + 42, *u_full = w_full + 44,
+           *u_empty = w_full + 46, *drain = w_full + 48;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 448);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 452);
   unsigned char *smap = smem + 512;  // shared-memory copy of the tensor map (grouped MoE)
@@ -484,26 +561,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   if (tid == 0) {
     for (int i = 0; i < kNW; i++) {
       mbar_init(&w_full[i], 1);
-      mbar_init(&w_empty[i], kDecWarps);
+      mbar_init(&w_empty[i], C::kDecWarps);
     }
     for (int i = 0; i < kNA; i++) {
-      mbar_init(&a_full[i], kDecWarps);
-      mbar_init(&a_empty[i], 1);
+      for (int hh = 0; hh < 2; hh++) {
+        mbar_init(&a_full[2 * i + hh], C::kDecWarps / 2);
+        mbar_init(&a_empty[2 * i + hh], 1);
+      }
+    }
+    for (int i = 0; i < C::kNB; i++) {
       mbar_init(&b_full[i], 1);
+      mbar_init(&b_empty[i], C::kNI);  // every issuer releases the slot after its MMAs of the stage
     }
     for (int i = 0; i < 2; i++) {
-      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_full[i], C::kNI);
       mbar_init(&acc_empty[i], 4);
       mbar_init(&u_full[i], 2);
       mbar_init(&u_empty[i], 2);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, C::kNI);
     *abort_flag = 0;
     mbar_fence_init();
   }
   if (MODE != kModeGemv && tid < 32)
     reinterpret_cast<uint32_t *>(smap)[tid] = reinterpret_cast<const uint32_t *>(&wmap)[tid];
-  if (warp == kMmaWarp) {
+  if (warp == C::kMmaWarp) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
@@ -522,23 +604,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   const int nq = my_jobs * S;
   auto job_of = [&](int jl) { return (int)blockIdx.x + jl * (int)gridDim.x; };
 
-  if (warp < kDecWarps) {
+  if (warp < C::kDecWarps) {
     // ---------------------------------------------------------------- decode warps
+    // Thread (warp w, lane l) owns tile row m = 32 (w % 4) + l and the kNBT blocks kNBT (w / 4).. of
+    // each stage, decoded in chunks of eight (64 bytes of words, four 16-byte reads).
     const int sp = warp & 3, h = warp >> 2, m = 32 * sp + lane;
-    // this thread's 8 kNBT bytes of a stage row: 16-byte chunks c0.. of TMA box column bc, 128-byte
-    // swizzle (chunk c of box row rb sits at chunk c ^ (rb & 7))
+    const int hf = 2 * kNBT * h / kKB;  // the half of the stage this warp's blocks lie in
+    // 16-byte chunk c of box row rb sits at chunk c ^ (rb & 7) (128-byte swizzle). A chunk of eight
+    // blocks is 64 bytes at an offset that is a multiple of 64, so its four reads are chunks
+    // c0 + i (c0 = 0 or 4) of one box row: at (c0 ^ (sw & 4)) | (i ^ (sw & 3)).
     const uint32_t rb = (uint32_t)(m & 63), sw = rb & 7u;
-    const uint32_t bc = (uint32_t)(h * kNBT * 8) / 128u, c0 = ((uint32_t)(h * kNBT * 8) % 128u) / 16u;
-    const uint32_t wrow = smem_u32(smem + geo.off_W) + ((uint32_t)(m >> 6) * C::kBoxCols + bc) * 8192u + rb * 128u;
-    uint32_t wo[kNBT / 2];
+    const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * C::kBoxCols * 8192u + rb * 128u;
+    uint32_t wlo[4];
 #pragma unroll
-    for (int i = 0; i < kNBT / 2; i++) wo[i] = ((c0 + (uint32_t)i) ^ sw) * 16u;
+    for (int i = 0; i < 4; i++) wlo[i] = ((uint32_t)i ^ (sw & 3u)) * 16u;
     const uint32_t tq = tbase + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lane quarter
 
-    // Scale factors of this thread's kNG groups of four blocks, kPF stages ahead of their use (slot
-    // u holds the stage q with q % kPF == u): its row's bytes (16-bit loads of block pairs) and the
-    // words of the B rows 32c + lane, c < kC.
-    uint32_t pa[kPF][kNBT / 2], pb[kPF][kNG][C::kC];
+    // Scale factors of this thread's kNG groups of four blocks, loaded one stage ahead of their use:
+    // its row's bytes (16-bit loads of block pairs) and the words of the B rows 32c + lane, c < kC.
+    uint32_t pa[kNBT / 2], pb[kNG][C::kC];
     int qp = 0, jl_p = 0, s_p = 0;
     const unsigned short *srow = nullptr;  // row m's scales of the front job, from block kNBT h on
     const uint32_t *sfb_src = nullptr;     // the front job's B scale words of this lane
@@ -551,9 +635,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         sfb_src = reinterpret_cast<const uint32_t *>(a.terms + (size_t)jr.group * tbytes + (size_t)S * C::kBStage) +
                   (size_t)(h * kNG * C::kC) * 32 + lane;
       }
+      const int lim = nbr - kKB * s_p - kNBT * h;  // blocks of this thread's range inside the row
 #pragma unroll
       for (int i = 0; i < kNBT / 2; i++)
-        da[i] = srow != nullptr && kKB * s_p + kNBT * h + 2 * i < nbr ? (uint32_t)__ldg(srow + (kKB / 2) * s_p + i) : 0u;
+        da[i] = srow != nullptr && 2 * i < lim ? (uint32_t)__ldg(srow + (kKB / 2) * s_p + i) : 0u;
 #pragma unroll
       for (int g = 0; g < kNG; g++)
 #pragma unroll
@@ -565,74 +650,82 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         jl_p++;
       }
     };
-#pragma unroll
-    for (int u = 0; u < kPF; u++) load_sf(pa[u], pb[u]);
+    grid_dep_wait();  // the activation terms (B scales) come from the preceding split kernel
+    load_sf(pa, pb);
 
-    int q = 0;
+    // Barrier latencies are hidden: the release of this stage's A slot and the arrival of the next
+    // stage's words are tested (non-blocking) before a chunk's decode and their results read after
+    // it; only a barrier found incomplete costs a blocking wait.
     uint32_t ws = 0, b = 0;
-    bool stop = false;
-    for (int q0 = 0; q0 < nq && !stop; q0 += kPF) {
+    bool ok = true, wf_ready = false;
+    // The halves start about half a stage apart, so that one half's warps decode while the other's
+    // wait on barriers and store scale factors.
+    if (hf == 1) __nanosleep(kHalfLagNs);
+#pragma unroll 1
+    for (int q = 0; q < nq; q++) {
+      if (!wf_ready && !(ok = warp_wait(&w_full[ws], (uint32_t)(q / kNW) & 1u, tmo, abort_flag))) break;
+      uint32_t na[kNBT / 2], nb[kNG][C::kC];
+      load_sf(na, nb);  // the next stage's scale factors; their latency hides behind this stage
+      const uint32_t wa = wrow + ws * C::kWStage;
+      const uint32_t ws1 = ws + 1 == (uint32_t)kNW ? 0u : ws + 1;
+      uint32_t ae = 1u, wf = 0u;
+#pragma unroll 1
+      for (int ch = 0; ch < C::kNCh; ch++) {
+        const uint32_t byte0 = (uint32_t)(kNBT * h + 8 * ch) * 8u;  // the chunk's offset in the stage row
+        const uint32_t wc = wa + (byte0 >> 7) * 8192u + ((((byte0 >> 4) & 7u) ^ (sw & 4u)) * 16u);
+        uint4 cw[4];
 #pragma unroll
-      for (int u = 0; u < kPF; u++) {
-        q = q0 + u;
-        if (q >= nq || *abort_flag) {
-          stop = true;
-          break;
-        }
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(&w_full[ws], (uint32_t)(q / kNW) & 1u, tmo);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          *abort_flag = 1;
-          stop = true;
-          break;
-        }
-        const uint32_t wa = wrow + ws * C::kWStage;
-        uint4 cw[kNBT / 2];
+        for (int i = 0; i < 4; i++) cw[i] = lds_u4(wc + wlo[i]);
+        if (ch == 0 && q >= kNA) ae = mbar_test(&a_empty[2 * b + hf], (uint32_t)((q - kNA) / kNA) & 1u);
+        if (ch == C::kNCh - 1 && q + 1 < nq) wf = mbar_test(&w_full[ws1], (uint32_t)((q + 1) / kNW) & 1u);
+        uint32_t W[8][4];
 #pragma unroll
-        for (int i = 0; i < kNBT / 2; i++) cw[i] = lds_u4(wa + wo[i]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&w_empty[ws]);
-        ws = ws + 1 == (uint32_t)kNW ? 0u : ws + 1;
-        uint32_t W[kNBT][4];
-#pragma unroll
-        for (int i = 0; i < kNBT / 2; i++) {
+        for (int i = 0; i < 4; i++) {
           planes_to_nibbles_interleaved(decode_block0(cw[i].x, cw[i].y), W[2 * i][0], W[2 * i][1], W[2 * i][2],
                                         W[2 * i][3]);
           planes_to_nibbles_interleaved(decode_block0(cw[i].z, cw[i].w), W[2 * i + 1][0], W[2 * i + 1][1],
                                         W[2 * i + 1][2], W[2 * i + 1][3]);
         }
-        if (q >= kNA) {
-          if (lane == 0) ok = mbar_wait(&a_empty[b], (uint32_t)((q - kNA) / kNA) & 1u, tmo);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) {
-            *abort_flag = 1;
-            stop = true;
+        if (ch == C::kNCh - 1) {  // every word of the stage has been read (and used): free the slot
+          __syncwarp();
+          mbar_arrive_one(&w_empty[ws]);
+        }
+        if (ch == 0 && q >= kNA) {
+          if (!__all_sync(0xffffffffu, ae != 0u) &&
+              !(ok = warp_wait(&a_empty[2 * b + hf], (uint32_t)((q - kNA) / kNA) & 1u, tmo, abort_flag)))
             break;
-          }
           tc_fence_after();
         }
-        // the blocks' codes (columns 4 kNBT h.. of the stage's A), the scale factors of this row
-        // (its own quarter, column 4g + quarter of group g) and of B rows 32c + lane (every quarter
-        // holds a copy). Columns of blocks beyond the row's end hold the decode of the zero fill; no
-        // MMA reads them.
-        tmem_st_codes<kNBT>(tq + C::kACol + C::kACols * b + 4u * kNBT * (uint32_t)h, W);
-#pragma unroll
-        for (int g = 0; g < kNG; g++) {
-          const uint32_t gg = (uint32_t)(kNG * h + g);
-          tmem_st_x1(tq + C::kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[u][2 * g] | (pa[u][2 * g + 1] << 16));
-#pragma unroll
-          for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + C::kSfbCol + kKB * b + 4u * gg + (uint32_t)c, pb[u][g][c]);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[b]);
-        load_sf(pa[u], pb[u]);
-        b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
+        // the chunk's codes: columns 4 (kNBT h + 8 ch).. of the stage's A. Columns of blocks beyond
+        // the row's end hold the decode of the zero fill; no MMA reads them.
+        tmem_st_codes<8>(tq + C::kACol + C::kACols * b + 4u * (uint32_t)(kNBT * h + 8 * ch), W);
       }
+      if (!ok) break;
+      wf_ready = __all_sync(0xffffffffu, wf != 0u);
+      ws = ws1;
+      // the scale factors of this row (its own quarter, column 4g + quarter of group g) and of B
+      // rows 32c + lane (every quarter holds a copy)
+#pragma unroll
+      for (int g = 0; g < kNG; g++) {
+        const uint32_t gg = (uint32_t)(kNG * h + g);
+        tmem_st_x1(tq + C::kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[2 * g] | (pa[2 * g + 1] << 16));
+#pragma unroll
+        for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + C::kSfbCol + kKB * b + 4u * gg + (uint32_t)c, pb[g][c]);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      mbar_arrive_one(&a_full[2 * b + hf]);
+#pragma unroll
+      for (int i = 0; i < kNBT / 2; i++) pa[i] = na[i];
+#pragma unroll
+      for (int g = 0; g < kNG; g++)
+#pragma unroll
+        for (int c = 0; c < C::kC; c++) pb[g][c] = nb[g][c];
+      b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
     }
-  } else if (warp == kWLoadWarp) {
+    if (!ok) *abort_flag = 1;
+  } else if (warp == C::kWLoadWarp) {
     // ---------------------------------------------------------------- word loader warp
     // TMA front: stage qi of job jl_i, up to kNW stages ahead of the decode warps.
     const uint32_t wbase = smem_u32(smem + geo.off_W);
@@ -655,7 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         }
       }
       if (lane == 0) {
-        if (qi >= kNW) ok = mbar_wait(&w_empty[wi], (uint32_t)((qi - kNW) / kNW) & 1u, tmo);
+        if (qi >= kNW) ok = mbar_wait_sleep(&w_empty[wi], (uint32_t)((qi - kNW) / kNW) & 1u, tmo, kLoaderSleepNs);
         if (ok) {
           mbar_arrive_expect_tx(&w_full[wi], C::kWStage);
           const uint32_t dst = wbase + wi * C::kWStage;
@@ -681,20 +774,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       for (int d = qi - 1; d >= 0 && d >= qi - kNW; d--)
         if (!mbar_wait(&w_full[d % kNW], (uint32_t)(d / kNW) & 1u, tmo)) break;
     __syncwarp();
-  } else if (warp == kBLoadWarp) {
+  } else if (warp == C::kBLoadWarp) {
     // ---------------------------------------------------------------- B loader warp
     int issued = 0;
+    grid_dep_wait();  // the activation terms come from the preceding split kernel
     if (lane == 0) {
       int jl = 0, s = 0;
       const uint8_t *src = nullptr;
       bool ok = true;
       for (int q = 0; q < nq; q++) {
         if (*abort_flag) break;
-        const int b = q % kNA;
+        const int bb = q % C::kNB;
         if (s == 0) src = a.terms + (size_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl)).group * tbytes;
-        if (q >= kNA && !(ok = mbar_wait(&a_empty[b], (uint32_t)((q - kNA) / kNA) & 1u, tmo))) break;
-        mbar_arrive_expect_tx(&b_full[b], C::kBStage);
-        bulk_g2s(smem + geo.off_B + (uint32_t)b * C::kBStage, src + (size_t)s * C::kBStage, C::kBStage, &b_full[b]);
+        // up to kNB stages ahead of the MMAs: the slot is free once its last use was released
+        if (q >= C::kNB && !(ok = mbar_wait_sleep(&b_empty[bb], (uint32_t)((q - C::kNB) / C::kNB) & 1u, tmo,
+                                                  kLoaderSleepNs)))
+          break;
+        mbar_arrive_expect_tx(&b_full[bb], C::kBStage);
+        bulk_g2s(smem + geo.off_B + (uint32_t)bb * C::kBStage, src + (size_t)s * C::kBStage, C::kBStage, &b_full[bb]);
         issued++;
         if (++s == S) {
           s = 0;
@@ -702,33 +799,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
         }
       }
       if (!ok) *abort_flag = 1;
-      for (int d = issued - 1; d >= 0 && d >= issued - kNA; d--)
-        if (!mbar_wait(&b_full[d % kNA], (uint32_t)(d / kNA) & 1u, tmo)) break;
+      for (int d = issued - 1; d >= 0 && d >= issued - C::kNB; d--)
+        if (!mbar_wait(&b_full[d % C::kNB], (uint32_t)(d / C::kNB) & 1u, tmo)) break;
     }
     __syncwarp();
-  } else if (warp >= kEpiWarp0) {
+  } else if (warp >= C::kEpiWarp0) {
     // ---------------------------------------------------------------- epilogue warps
-    // Warp kEpiWarp0 + i reads TMEM lane quarter eq = warp % 4, i.e. tile rows 32 eq..32 eq + 31.
+    // Warp C::kEpiWarp0 + i reads TMEM lane quarter eq = warp % 4, i.e. tile rows 32 eq..32 eq + 31.
     const int eq = warp & 3;
     auto epilogue = [&](int jl_e) {
       const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
       const int buf = jl_e & 1;
-      if (!mbar_wait(&acc_full[buf], (uint32_t)(jl_e >> 1) & 1u, tmo)) {
-        *abort_flag = 1;
-        return;
+      // one warp polls; the others wait at a named barrier (no issue slots taken meanwhile)
+      if (warp == C::kEpiWarp0) {
+        if (!mbar_wait_sleep(&acc_full[buf], (uint32_t)(jl_e >> 1) & 1u, tmo, kEpiSleepNs)) *abort_flag = 1;
       }
+      named_bar(1, 128);
+      if (*abort_flag) return;
       tc_fence_after();
       float v[C::kTok];
 #pragma unroll
       for (int t = 0; t < C::kTok; t++) v[t] = 0.f;
+      // with two issuers the second accumulator holds the second halves of the stages; it was never
+      // written when the rows fit in half a stage
+      const int nacc = C::kNI == 2 && nbr > kKB / 2 ? 2 : 1;
+      for (int ia = 0; ia < nacc; ia++) {
 #pragma unroll
-      for (int c0 = 0; c0 < C::kTok * kTerms; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld_x16(tbase + ((uint32_t)(32 * eq) << 16) + (uint32_t)(buf * NMAX + c0), r);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < C::kTok * kTerms; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld_x16(tbase + ((uint32_t)(32 * eq) << 16) + (uint32_t)((buf * C::kNI + ia) * NMAX + c0), r);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; i++)
-          if (c0 + i < C::kTok * kTerms) v[(c0 + i) / kTerms] += __uint_as_float(r[i]);
+          for (int i = 0; i < 16; i++)
+            if (c0 + i < C::kTok * kTerms) v[(c0 + i) / kTerms] += __uint_as_float(r[i]);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -799,11 +903,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       }
     };
     for (int jl = 0; jl < my_jobs && !*abort_flag; jl++) epilogue(jl);
-  } else {
-    // ---------------------------------------------------------------- MMA warp
+  } else if (warp - C::kMmaWarp < C::kNI) {
+    // ---------------------------------------------------------------- MMA warp(s)
     // The whole warp runs the loop (its values are warp-uniform); one elected lane issues the
-    // tcgen05 operations.
+    // tcgen05 operations. With two issuers, warp C::kMmaWarp + i issues the MMAs of half i of every
+    // stage into accumulator i of the job's pair; with one, warp C::kMmaWarp issues both halves.
     const bool leader = elect_one();
+    const int h_lo = C::kNI == 2 ? warp - C::kMmaWarp : 0, h_hi = C::kNI == 2 ? h_lo + 1 : 2;
     int jl = 0, s = 0;
     uint32_t ncols = (uint32_t)(my_jobs ? job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(0)).ncols : 16);
     uint32_t idesc0 = idesc_mxf4(ncols, 0u), idesc2 = idesc_mxf4(ncols, 2u);
@@ -813,30 +919,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       if (*abort_flag) break;
       const int b = q % kNA;
       const uint32_t ph = (uint32_t)(q / kNA) & 1u;
-      ok = mbar_wait(&a_full[b], ph, tmo) && mbar_wait(&b_full[b], ph, tmo);
-      if (ok && s == 0 && jl >= 2) ok = mbar_wait(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
+      const int bb = q % C::kNB;
+      ok = mbar_wait_sleep(&b_full[bb], (uint32_t)(q / C::kNB) & 1u, tmo, kMmaSleepNs);
+      if (ok && s == 0 && jl >= 2)
+        ok = mbar_wait_sleep(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo, kMmaSleepNs);
       const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
       const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
-      const uint64_t bd = smem_desc(b0 + (uint32_t)b * C::kBStage, 128u, C::kSbo);
-      const uint32_t d_t = tbase + (uint32_t)((jl & 1) * NMAX);
+      const uint64_t bd = smem_desc(b0 + (uint32_t)bb * C::kBStage, 128u, C::kSbo);
       const uint32_t sfa = tbase + C::kSfaCol + kKB * (uint32_t)b, sfb = tbase + C::kSfbCol + kKB * (uint32_t)b;
-      if (leader) {
 #pragma unroll
-        for (int j = 0; j < kKB / 2; j++) {
-          if (j < nmma) {
-            const uint32_t sf = (uint32_t)(j & 1) * 2u;
-            // +256 bytes of B per MMA: the descriptor's start address counts 16-byte units
-            mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
-                        (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30), (sfb + 4u * (uint32_t)(j >> 1)) | (sf << 30),
-                        !(s == 0 && j == 0));
+      for (int hh = h_lo; hh < h_hi; hh++) {  // this issuer's halves of the stage, in order
+        ok = __all_sync(0xffffffffu, ok && mbar_wait_sleep(&a_full[2 * b + hh], ph, tmo, kMmaSleepNs));
+        if (!ok) break;
+        tc_fence_after();
+        const int jfirst = C::kNI == 2 ? hh * kKB / 4 : 0;  // this issuer's first MMA of a job
+        const uint32_t d_t = tbase + (uint32_t)(((jl & 1) * C::kNI + (C::kNI == 2 ? hh : 0)) * NMAX);
+        if (leader) {
+#pragma unroll
+          for (int j = hh * kKB / 4; j < (hh + 1) * kKB / 4; j++) {
+            if (j < nmma) {
+              const uint32_t sf = (uint32_t)(j & 1) * 2u;
+              // +256 bytes of B per MMA: the descriptor's start address counts 16-byte units
+              mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
+                          (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30), (sfb + 4u * (uint32_t)(j >> 1)) | (sf << 30),
+                          !(s == 0 && j == jfirst));
+            }
+          }
+          tc_commit(&a_empty[2 * b + hh]);
+          if (hh == h_hi - 1) {
+            tc_commit(&b_empty[bb]);
+            if (s == S - 1) tc_commit(&acc_full[jl & 1]);
           }
         }
-        tc_commit(&a_empty[b]);
-        if (s == S - 1) tc_commit(&acc_full[jl & 1]);
       }
+      if (!ok) break;
       __syncwarp();
       if (++s == S) {
         s = 0;
@@ -851,7 +967,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
       }
     }
     if (!ok && lane == 0) *abort_flag = 1;
-    // drain: every tcgen05 operation issued so far
+    // drain: every tcgen05 operation this issuer started (the barrier completes once every issuer
+    // has committed)
     if (leader) {
       tc_commit(drain);
       mbar_wait(drain, 0u, tmo);
@@ -861,7 +978,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_mma(const __grid_constant__ Mma
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_dealloc(tbase, C::kTmemCols);
+  if (warp == C::kMmaWarp) tmem_dealloc(tbase, C::kTmemCols);
 }
 
 // ------------------------------------------------------------------------------- host side
@@ -950,9 +1067,17 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
   args.T = T;
   args.y = y;
   MoeTable<32> none{};
-  k_mma<32, kModeGemv, NMAX><<<ntiles < nsm ? ntiles : nsm, kThreads, mma_geom<NMAX>(kModeGemv).smem, s>>>(args, none,
-                                                                                                          map);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(ntiles < nsm ? ntiles : nsm);
+  cfg.blockDim = dim3(Cfg<NMAX>::kThreads);
+  cfg.dynamicSmemBytes = mma_geom<NMAX>(kModeGemv).smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap with the split kernel
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_mma<32, kModeGemv, NMAX>, args, none, map);
 }
 
 cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
@@ -1047,7 +1172,7 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
     args.nbr = nbr;
     args.terms = terms;
     const int jobs = G * ((m.I + 63) / 64);
-    k_mma<MAXE, kModeGateUp, NMAX><<<jobs < nsm ? jobs : nsm, kThreads, mma_geom<NMAX>(kModeGateUp).smem, s>>>(
+    k_mma<MAXE, kModeGateUp, NMAX><<<jobs < nsm ? jobs : nsm, Cfg<NMAX>::kThreads, mma_geom<NMAX>(kModeGateUp).smem, s>>>(
         args, tab, map_gu);
   }
   // down: split h per group, then decode + MMA, y to the workspace, last arriver per chunk combines
@@ -1063,7 +1188,7 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
     args.nbr = nbr;
     args.terms = terms;
     const int jobs = G * ((m.H + 127) / 128);
-    k_mma<MAXE, kModeDown, NMAX><<<jobs < nsm ? jobs : nsm, kThreads, mma_geom<NMAX>(kModeDown).smem, s>>>(args, tab,
+    k_mma<MAXE, kModeDown, NMAX><<<jobs < nsm ? jobs : nsm, Cfg<NMAX>::kThreads, mma_geom<NMAX>(kModeDown).smem, s>>>(args, tab,
                                                                                                          map_dn);
   }
   return cudaGetLastError();
