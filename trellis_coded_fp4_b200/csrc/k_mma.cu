@@ -46,8 +46,6 @@ __device__ unsigned int g_tcf4_timeouts_mma = 0;
 constexpr int kTerms = 6;            // E2M1 terms per activation block
 constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> jobs in flight)
 
-// Head start of the first half's decode warps (about half a stage).
-constexpr uint32_t kHalfLagNs = 600u;
 // Sleep between barrier tests of the idle roles. The loaders run stages ahead and the MMA issuers
 // have about two stages (~3 us) of slack, so these only bound how soon a completed phase is seen.
 constexpr uint32_t kLoaderSleepNs = 200u, kMmaSleepNs = 100u, kEpiSleepNs = 200u;
@@ -658,9 +656,6 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
     // it; only a barrier found incomplete costs a blocking wait.
     uint32_t ws = 0, b = 0;
     bool ok = true, wf_ready = false;
-    // The halves start about half a stage apart, so that one half's warps decode while the other's
-    // wait on barriers and store scale factors.
-    if (hf == 1) __nanosleep(kHalfLagNs);
 #pragma unroll 1
     for (int q = 0; q < nq; q++) {
       if (!wf_ready && !(ok = warp_wait(&w_full[ws], (uint32_t)(q / kNW) & 1u, tmo, abort_flag))) break;
