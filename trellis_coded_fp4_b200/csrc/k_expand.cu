@@ -32,6 +32,8 @@ __global__ void __launch_bounds__(256) k_expand(const uint2 *__restrict__ stream
                                                 uint32_t blocks_per_row, uint32_t seg_blocks,
                                                 uint4 *__restrict__ out, const uint8_t *__restrict__ scales,
                                                 uint8_t *__restrict__ out_scales, int scales_aligned16) {
+  grid_dep_wait();  // out may still be read by the preceding kernel
+  grid_dep_release();
   const uint32_t pair = blockIdx.x * blockDim.x + threadIdx.x;
   const uint32_t npairs = (nblocks + 1u) >> 1;
   const uint32_t g0 = 2u * pair;
@@ -102,13 +104,12 @@ cudaError_t launch_expand(const MatView &w, uint8_t *out_nibbles, uint8_t *out_s
   const uint32_t grid = (nthreads + 255u) / 256u;
   auto *out = reinterpret_cast<uint4 *>(out_nibbles);
   if (w.seg_blocks == 1) {
-    k_expand<true><<<grid, 256, 0, s>>>(w.stream, nblocks, (uint32_t)w.nbr, 1u, out, w.scales, out_scales,
-                                        aligned ? 1 : 0);
+    return launch_dependent(k_expand<true>, dim3(grid), dim3(256), 0, s, w.stream, nblocks, (uint32_t)w.nbr, 1u, out,
+                            w.scales, out_scales, aligned ? 1 : 0);
   } else {
-    k_expand<false><<<grid, 256, 0, s>>>(w.stream, nblocks, (uint32_t)w.nbr, (uint32_t)w.seg_blocks, out,
-                                         w.scales, out_scales, aligned ? 1 : 0);
+    return launch_dependent(k_expand<false>, dim3(grid), dim3(256), 0, s, w.stream, nblocks, (uint32_t)w.nbr,
+                            (uint32_t)w.seg_blocks, out, w.scales, out_scales, aligned ? 1 : 0);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace tcf4

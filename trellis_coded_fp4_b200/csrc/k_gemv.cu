@@ -34,6 +34,8 @@ template <int TT, bool SEG32, int R>
 __global__ void __launch_bounds__(256) k_gemv(MatView w, const uint16_t *__restrict__ x, int T,
                                               uint16_t *__restrict__ y, int bulk_scales) {
   extern __shared__ __align__(128) unsigned char smem[];
+  grid_dep_wait();  // x may come from, and y may still be read by, the preceding kernel
+  grid_dep_release();
   constexpr int RPW = R / 8;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = w.nbr, K = nbr * 32;
@@ -119,8 +121,7 @@ static cudaError_t launch_gemv_t(const MatView &w, const uint16_t *x, int T, uin
   const int nslab = (w.rows + R - 1) / R;
   const int grid = nslab < nsm * occ ? nslab : nsm * occ;
   const int bulk_scales = ((reinterpret_cast<uintptr_t>(w.scales) & 15u) == 0 && (R * w.nbr) % 16 == 0) ? 1 : 0;
-  k_gemv<TT, SEG32, R><<<grid, 256, geo.smem, s>>>(w, x, T, y, bulk_scales);
-  return cudaGetLastError();
+  return launch_dependent(k_gemv<TT, SEG32, R>, dim3(grid), dim3(256), geo.smem, s, w, x, T, y, bulk_scales);
 }
 
 template <int TT, bool SEG32>

@@ -224,15 +224,13 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
 }
 
 // Plain GEMV: one group, token slots 0..T-1 (slots up to kSlots are zero rows).
-// Programmatic dependent launch: the GEMV's product kernel is launched while the activation split
-// still runs. It starts its TMEM setup and its first weight tiles (which do not depend on the split)
-// at once, and waits for the split's completion only before it reads the activation terms.
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
+// The GEMV's product kernel is launched as a programmatic dependent of this split: it starts its
+// TMEM setup and its first weight tiles (which do not depend on the split) at once and waits for
+// the split's completion only before it reads the activation terms.
 template <int NMAX>
 __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
                                                      uint8_t *__restrict__ terms) {
+  grid_dep_wait();     // x may come from, and terms may still be read by, the preceding kernel
   grid_dep_release();  // the product kernel may start; it waits for this grid before reading terms
   const int nb = K >> 5, S = (nb + Cfg<NMAX>::kKB - 1) / Cfg<NMAX>::kKB, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -251,6 +249,8 @@ __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ 
                                                     const uint16_t *__restrict__ src, int K, uint8_t *__restrict__ terms,
                                                     int *__restrict__ counters, int n_counters) {
   __shared__ GroupPlan pl;
+  grid_dep_wait();  // every input (routing, x or h) and the workspace come from preceding kernels
+  grid_dep_release();
   if (counters != nullptr && blockIdx.x == 0)
     for (int c = threadIdx.x; c < n_counters; c += blockDim.x) counters[c] = 0;
   build_groups(pl, ids, P, E, Cfg<NMAX>::kTok);
@@ -772,7 +772,8 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   } else if (warp == C::kBLoadWarp) {
     // ---------------------------------------------------------------- B loader warp
     int issued = 0;
-    grid_dep_wait();  // the activation terms come from the preceding split kernel
+    grid_dep_wait();     // the activation terms come from the preceding split kernel
+    grid_dep_release();  // a dependent launch may start its prologue now
     if (lane == 0) {
       int jl = 0, s = 0;
       const uint8_t *src = nullptr;
@@ -1049,9 +1050,10 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
                                     void *ws, cudaStream_t s) {
   uint8_t *terms = static_cast<uint8_t *>(ws);
   const int warps = Cfg<NMAX>::kSlots * w.nbr;
-  k_bsplit_gemv<NMAX><<<(warps + 7) / 8, 256, 0, s>>>(x, T, w.nbr * 32, terms);
+  cudaError_t e = launch_dependent(k_bsplit_gemv<NMAX>, dim3((warps + 7) / 8), dim3(256), 0, s, x, T, w.nbr * 32, terms);
+  if (e != cudaSuccess) return e;
   static unsigned long long attr = 0;
-  cudaError_t e = ensure_max_dynamic_smem(k_mma<32, kModeGemv, NMAX>, attr);
+  e = ensure_max_dynamic_smem(k_mma<32, kModeGemv, NMAX>, attr);
   if (e != cudaSuccess) return e;
   const int ntiles = (w.rows + 127) / 128, nsm = sm_count();
   MmaArgs args{};
@@ -1062,17 +1064,8 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
   args.T = T;
   args.y = y;
   MoeTable<32> none{};
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(ntiles < nsm ? ntiles : nsm);
-  cfg.blockDim = dim3(Cfg<NMAX>::kThreads);
-  cfg.dynamicSmemBytes = mma_geom<NMAX>(kModeGemv).smem;
-  cfg.stream = s;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap with the split kernel
-  at[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_mma<32, kModeGemv, NMAX>, args, none, map);
+  return launch_dependent(k_mma<32, kModeGemv, NMAX>, dim3(ntiles < nsm ? ntiles : nsm), dim3(Cfg<NMAX>::kThreads),
+                          mma_geom<NMAX>(kModeGemv).smem, s, args, none, map);
 }
 
 cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
@@ -1115,7 +1108,9 @@ MoeMmaWorkspace moe_mma_workspace_layout(const tcf4_moe &m, int T, int k) {
   L.y = off;        off = a256(off + sizeof(float) * (size_t)P * m.H);
   L.bg_gu = off;    off = a256(off + (size_t)G * terms_for(m.H / 32, NMAX));
   L.bg_dn = off;    off = a256(off + (size_t)G * terms_for(m.I / 32, NMAX));
-  L.maps = off;     off = a256(off + (size_t)sm_count() * kMapSlots * 128);
+  // tensor-map slots: one region for the gate/up kernel and one for the down kernel (the down kernel
+  // may start while gate/up CTAs still run)
+  L.maps = off;     off = a256(off + 2 * (size_t)sm_count() * kMapSlots * 128);
   L.total = off;
   return L;
 }
@@ -1159,32 +1154,39 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
     uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_gu);
     const int nbr = m.H / 32;
     const int warps = G * Cfg<NMAX>::kSlots * nbr;
-    k_bsplit_moe<NMAX><<<(warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm, 256, 0, s>>>(
-        ids, P, m.E, k, x, m.H, terms, args.counters, 4 * ((m.H + 127) / 128));
+    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
+                                     dim3(256), 0, s, ids, P, m.E, k, x, m.H, terms, args.counters,
+                                     4 * ((m.H + 127) / 128));
+    if (e != cudaSuccess) return e;
     static unsigned long long attr = 0;
-    cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, kModeGateUp, NMAX>, attr);
+    e = ensure_max_dynamic_smem(k_mma<MAXE, kModeGateUp, NMAX>, attr);
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
     const int jobs = G * ((m.I + 63) / 64);
-    k_mma<MAXE, kModeGateUp, NMAX><<<jobs < nsm ? jobs : nsm, Cfg<NMAX>::kThreads, mma_geom<NMAX>(kModeGateUp).smem, s>>>(
-        args, tab, map_gu);
+    e = launch_dependent(k_mma<MAXE, kModeGateUp, NMAX>, dim3(jobs < nsm ? jobs : nsm), dim3(Cfg<NMAX>::kThreads),
+                         mma_geom<NMAX>(kModeGateUp).smem, s, args, tab, map_gu);
+    if (e != cudaSuccess) return e;
   }
   // down: split h per group, then decode + MMA, y to the workspace, last arriver per chunk combines
   {
     uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_dn);
     const int nbr = m.I / 32;
     const int warps = G * Cfg<NMAX>::kSlots * nbr;
-    k_bsplit_moe<NMAX><<<(warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm, 256, 0, s>>>(
-        ids, P, m.E, 1, args.hidden, m.I, terms, nullptr, 0);
+    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
+                                     dim3(256), 0, s, ids, P, m.E, 1, (const uint16_t *)args.hidden, m.I, terms,
+                                     (int *)nullptr, 0);
+    if (e != cudaSuccess) return e;
     static unsigned long long attr = 0;
-    cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, kModeDown, NMAX>, attr);
+    e = ensure_max_dynamic_smem(k_mma<MAXE, kModeDown, NMAX>, attr);
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
+    args.maps += (size_t)nsm * kMapSlots * 128;  // the down kernel's own tensor-map slots
     const int jobs = G * ((m.H + 127) / 128);
-    k_mma<MAXE, kModeDown, NMAX><<<jobs < nsm ? jobs : nsm, Cfg<NMAX>::kThreads, mma_geom<NMAX>(kModeDown).smem, s>>>(args, tab,
-                                                                                                         map_dn);
+    e = launch_dependent(k_mma<MAXE, kModeDown, NMAX>, dim3(jobs < nsm ? jobs : nsm), dim3(Cfg<NMAX>::kThreads),
+                         mma_geom<NMAX>(kModeDown).smem, s, args, tab, map_dn);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -110,6 +110,8 @@ __global__ void __launch_bounds__(256) k_moe_gateup(const __grid_constant__ MoeT
                                                     uint16_t *__restrict__ hidden, int *__restrict__ counters,
                                                     int n_counters, int bulk_scales) {
   extern __shared__ __align__(128) unsigned char smem[];
+  grid_dep_wait();  // inputs and workspace come from, or are still read by, the preceding kernel
+  grid_dep_release();
   constexpr int RPW = R / 8;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = H >> 5;
@@ -214,6 +216,8 @@ __global__ void __launch_bounds__(256) k_moe_down(const __grid_constant__ MoeTab
                                                   int *__restrict__ counters, uint16_t *__restrict__ out,
                                                   int bulk_scales) {
   extern __shared__ __align__(128) unsigned char smem[];
+  grid_dep_wait();  // inputs and workspace come from, or are still read by, the preceding kernel
+  grid_dep_release();
   constexpr int RPW = R / 8;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = I >> 5;
@@ -359,9 +363,8 @@ static cudaError_t launch_gateup(const MoeLaunch<MAXE> &ml, const tcf4_moe &m, i
   if (grid > items) grid = items;
   const int bulk = ml.scales_aligned && (R * nbr) % 16 == 0 && ((size_t)m.I * nbr) % 16 == 0;
   const int n_counters = (m.H + kMoeRMin - 1) / kMoeRMin;
-  k_moe_gateup<MAXE, TT, SEG32, R><<<grid, 256, g.smem, s>>>(ml.tab, ids, T * k, m.E, k, m.H, m.I, seg, x, ml.hidden,
-                                                             ml.counters, n_counters, bulk);
-  return cudaGetLastError();
+  return launch_dependent(k_moe_gateup<MAXE, TT, SEG32, R>, dim3(grid), dim3(256), g.smem, s, ml.tab, ids, T * k, m.E,
+                          k, m.H, m.I, seg, x, ml.hidden, ml.counters, n_counters, bulk);
 }
 
 template <int MAXE, int TT, bool SEG32, int R>
@@ -381,9 +384,8 @@ static cudaError_t launch_down(const MoeLaunch<MAXE> &ml, const tcf4_moe &m, int
   const int items = max_active * ((m.H + R - 1) / R);
   if (grid > items) grid = items;
   const int bulk = ml.scales_aligned && (R * nbr) % 16 == 0;
-  k_moe_down<MAXE, TT, SEG32, R><<<grid, 256, g.smem, s>>>(ml.tab, ids, wts, T * k, m.E, k, T, m.H, m.I, seg,
-                                                           ml.hidden, ml.yws, ml.counters, out, bulk);
-  return cudaGetLastError();
+  return launch_dependent(k_moe_down<MAXE, TT, SEG32, R>, dim3(grid), dim3(256), g.smem, s, ml.tab, ids, wts, T * k,
+                          m.E, k, T, m.H, m.I, seg, (const uint16_t *)ml.hidden, ml.yws, ml.counters, out, bulk);
 }
 
 // Dispatch (TT, seg_len == 32, R) to a compiled instance.

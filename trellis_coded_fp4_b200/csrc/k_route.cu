@@ -10,6 +10,8 @@ namespace tcf4 {
 
 __global__ void __launch_bounds__(256) k_route(const float *__restrict__ logits, int T, int E, int k,
                                                int32_t *__restrict__ ids, float *__restrict__ wts) {
+  grid_dep_wait();  // the logits come from the preceding kernel
+  grid_dep_release();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
   if (t >= T) return;
@@ -63,8 +65,7 @@ __global__ void __launch_bounds__(256) k_route(const float *__restrict__ logits,
 }
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *wts, cudaStream_t s) {
-  k_route<<<(T + 7) / 8, 256, 0, s>>>(logits, T, E, k, ids, wts);
-  return cudaGetLastError();
+  return launch_dependent(k_route, dim3((T + 7) / 8), dim3(256), 0, s, logits, T, E, k, ids, wts);
 }
 
 }  // namespace tcf4

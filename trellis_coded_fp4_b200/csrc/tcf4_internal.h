@@ -3,10 +3,35 @@
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include "tcf4.h"
 
 namespace tcf4 {
+
+// Programmatic dependent launch. Every kernel of the library is launched with programmatic stream
+// serialization. Each kernel calls grid_dep_wait before it touches anything a preceding kernel
+// writes or still reads, and releases its successor (grid_dep_release) only after that wait: so a
+// kernel overlaps at most its immediate predecessor, and only with work that depends on nothing in
+// flight (launch latency, setup, loads of resident weights).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... P, typename... A>
+inline cudaError_t launch_dependent(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                    A &&...args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTokens = 32;
