@@ -52,6 +52,7 @@ def lib():
         L.oracle_decode_codes.argtypes = [u32p, i64, i64, i64, u8p]
         L.oracle_decode_values.argtypes = [u32p, u8p, i64, i64, i64, f64p]
         L.oracle_expand_mxfp4.argtypes = [u32p, u8p, i64, i64, i64, u8p, u8p]
+        L.oracle_mxfp4_gemv.argtypes = [u8p, u8p, i64, i64, u16p, i64, i64p, i64, f64p, f64p]
         L.oracle_bf16_value.argtypes = [ctypes.c_uint16]
         L.oracle_bf16_value.restype = ctypes.c_double
         L.oracle_bf16_round.argtypes = [ctypes.c_double]
@@ -199,6 +200,31 @@ def gemv(stream, scales, rows, cols, seg_len, x_bits, row_ids=None):
     return y, wn
 
 
+def mxfp4_gemv(nibbles, scales, rows, cols, x_bits, row_ids=None):
+    """y[T][nr] (fp64) and ||w_row||_2 [nr] from a resident MXFP4 tensor (HEPH mode 2 consumer):
+    nibbles uint8 [rows][cols/2], scales uint8 [rows][cols/32], bf16 bits x [T][cols]."""
+    nibbles = np.ascontiguousarray(nibbles, np.uint8).reshape(-1)
+    scales = np.ascontiguousarray(scales, np.uint8).reshape(-1)
+    if nibbles.size != rows * (cols // 2) or scales.size != rows * (cols // 32):
+        raise ValueError("nibbles must be [rows][cols/2] and scales [rows][cols/32]")
+    x_bits = np.ascontiguousarray(np.atleast_2d(x_bits), np.uint16)
+    T = x_bits.shape[0]
+    if x_bits.shape[1] != cols:
+        raise ValueError("x must be [T][cols]")
+    if row_ids is None:
+        nr, rid = rows, None
+    else:
+        rid = np.ascontiguousarray(row_ids, np.int64)
+        nr = rid.size
+    y = np.zeros((T, nr), np.float64)
+    wn = np.zeros(nr, np.float64)
+    _check(lib().oracle_mxfp4_gemv(_ptr(nibbles, ctypes.c_uint8), _ptr(scales, ctypes.c_uint8), rows, cols,
+                                   _ptr(x_bits, ctypes.c_uint16), T,
+                                   None if rid is None else _ptr(rid, ctypes.c_int64), nr,
+                                   _ptr(y, ctypes.c_double), _ptr(wn, ctypes.c_double)), "mxfp4_gemv")
+    return y, wn
+
+
 # ----------------------------------------------------------------------------- encoder
 
 def viterbi_encode(target, D, scale):
@@ -262,6 +288,14 @@ def silu(g):
         return g / (1.0 + np.exp(-g))
 
 
+def _product(layer, kind, e, rows, cols, seg_len, xb):
+    """One expert matrix's product: the trellis stream decoded (mode 1) or, when the layer carries
+    expanded tensors (attributes gu_nibbles / dn_nibbles), the resident MXFP4 tensor (mode 2)."""
+    if hasattr(layer, kind + "_nibbles"):
+        return mxfp4_gemv(getattr(layer, kind + "_nibbles")[e], getattr(layer, kind + "_mx_scales")[e], rows, cols, xb)
+    return gemv(getattr(layer, kind + "_stream")[e], getattr(layer, kind + "_scales")[e], rows, cols, seg_len, xb)
+
+
 def moe_hidden(layer, x_bits, ids, seg_len):
     """Exact gate/up products and h = bf16(silu(g) * u) for every (t, j): returns
     g, u [T][k][I] fp64, h_bits [T][k][I] uint16, and the gate/up row norms [T][k][2I]."""
@@ -274,7 +308,7 @@ def moe_hidden(layer, x_bits, ids, seg_len):
     for t in range(T):
         for j in range(k):
             e = int(ids[t, j])
-            y, wn = gemv(layer.gu_stream[e], layer.gu_scales[e], 2 * I, H, seg_len, x_bits[t:t + 1])
+            y, wn = _product(layer, "gu", e, 2 * I, H, seg_len, x_bits[t:t + 1])
             g[t, j], u[t, j] = y[0, :I], y[0, I:]
             norms[t, j] = wn
     h_bits = bf16_round_array(silu(g) * u)
@@ -292,7 +326,7 @@ def moe_down(layer, h_bits, ids, w, seg_len):
         for j in range(k):
             e = int(ids[t, j])
             hb = np.asarray(h_bits[t, j], np.uint16)[None, :]
-            y, wn = gemv(layer.dn_stream[e], layer.dn_scales[e], H, I, seg_len, hb)
+            y, wn = _product(layer, "dn", e, H, I, seg_len, hb)
             hn = np.linalg.norm(bf16_bits_to_f64(hb))
             out[t] += w[t, j] * y[0]
             bound[t] += abs(w[t, j]) * wn * hn

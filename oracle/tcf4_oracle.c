@@ -258,6 +258,50 @@ int oracle_gemv(const uint32_t *stream, const uint8_t *scales, int64_t rows, int
     return ORACLE_OK;
 }
 
+/* [HEPH] mode 2, consumer side: the same products from a resident MXFP4 tensor. By the OCP MX
+ * definition ([TTP] section 2.1) element k of row n is E2M1(code) * 2^(E-127), code = nibble k of
+ * the row (low nibble of byte k/2 for even k), E = scales[n][k/32]. y[t][i] = sum_k w x in fp64, in
+ * k order, for the rows in row_ids (all rows when NULL, nr = rows); wnorm as in oracle_gemv. */
+int oracle_mxfp4_gemv(const uint8_t *nibbles, const uint8_t *scales, int64_t rows, int64_t cols, const uint16_t *x,
+                      int64_t T, const int64_t *row_ids, int64_t nr, double *y, double *wnorm) {
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || T < 0 || nr < 0) return ORACLE_EINVAL;
+    if (row_ids == NULL && nr != rows) return ORACLE_EINVAL;
+    double *w = (double *)malloc(sizeof(double) * (size_t)(cols > 0 ? cols : 1));
+    double *xv = (double *)malloc(sizeof(double) * (size_t)(T * cols > 0 ? T * cols : 1));
+    if (!w || !xv) {
+        free(w);
+        free(xv);
+        return ORACLE_ENOMEM;
+    }
+    for (int64_t i = 0; i < T * cols; i++) xv[i] = oracle_bf16_value(x[i]);
+    for (int64_t i = 0; i < nr; i++) {
+        int64_t n = row_ids ? row_ids[i] : i;
+        if (n < 0 || n >= rows) {
+            free(w);
+            free(xv);
+            return ORACLE_EINVAL;
+        }
+        for (int64_t k = 0; k < cols; k++) {
+            uint8_t byte = nibbles[n * (cols / 2) + k / 2];
+            uint8_t code = (k % 2 == 0) ? (uint8_t)(byte & 0xF) : (uint8_t)(byte >> 4);
+            w[k] = oracle_e2m1_value(code) * oracle_ue8m0_value(scales[n * (cols / 32) + k / 32]);
+        }
+        if (wnorm) {
+            double ss = 0.0;
+            for (int64_t k = 0; k < cols; k++) ss += w[k] * w[k];
+            wnorm[i] = sqrt(ss);
+        }
+        for (int64_t t = 0; t < T; t++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < cols; k++) acc += w[k] * xv[t * cols + k];
+            y[t * nr + i] = acc;
+        }
+    }
+    free(w);
+    free(xv);
+    return ORACLE_OK;
+}
+
 /* [XT] Viterbi bullet: the D-weighted additive distortion of one segment,
  *   cost = sum_k D[k] * (target[k] - P(s_k) * scale[k])^2,
  * minimised over the 4^L branch sequences of a segment that starts in state 0 and may end in
