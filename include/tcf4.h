@@ -150,6 +150,58 @@ TCF4_API tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, i
 /* Byte offset of h (bf16 [T*k][I]) inside the workspace of trellis_grouped_moe. */
 TCF4_API size_t trellis_grouped_moe_hidden_offset(const tcf4_moe *m, int32_t T, int32_t k);
 
+/* ------------------------------------------------------------------------------------------------
+ * HEPH abstract, second serving mode, consumer side: products straight from the resident MXFP4
+ * tensor that trellis_decode_to_mxfp4 writes (expand once, then every product reads 4.25 bits per
+ * weight with no decode). Same operations and accuracy contract as trellis_gemv and
+ * trellis_grouped_moe, on the tensor cores (block-scaled MXFP4 x MXFP4 MMA with the activations
+ * written as six E2M1 terms per 32-block; the same workspaces).
+ * ------------------------------------------------------------------------------------------------ */
+
+/* One resident MXFP4 matrix W [rows][cols]:
+ *   nibbles: uint8 [rows][cols/2], byte u of a row holds element 2u in its low nibble and element
+ *            2u+1 in its high nibble (OCP E2M1 codes); 16-byte aligned.
+ *   scales:  uint8 [rows][cols/32] UE8M0, element k of a row scaled by 2^(scales[k/32] - 127);
+ *            2-byte aligned.
+ *   cols:    a multiple of 64 (whole K = 64 MMAs), at most 16384. Device memory owned by the
+ *            caller. */
+typedef struct {
+  const uint8_t *nibbles;
+  const uint8_t *scales;
+  int64_t rows;
+  int64_t cols;
+} tcf4_mxfp4;
+
+/* y[t][n] = bf16( sum_k w[n][k] * x[t][k] ), fp32 accumulation; x bf16 bits [T][cols], y bf16 bits
+ * [T][rows], 1 <= T <= 32 (T == 0 is a no-op); x and y 16-byte aligned.
+ *   workspace: device scratch of at least mxfp4_gemv_workspace(w, T) bytes, 256-byte aligned, owned
+ *   by the caller. Accuracy: |y - exact| <= 2e-3 * ||w_row||_2 * ||x_t||_2 plus the bf16 rounding.
+ * Errors: TCF4_ERR_UNSUPPORTED when cols is not a multiple of 64 or exceeds 16384, or when T > 32;
+ * TCF4_ERR_MISALIGNED for pointers that break the alignment above. */
+TCF4_API size_t mxfp4_gemv_workspace(tcf4_mxfp4 w, int32_t T);
+TCF4_API tcf4_status mxfp4_gemv(tcf4_mxfp4 w, const uint16_t *x, int32_t T, uint16_t *y, void *workspace,
+                                size_t ws_bytes, void *stream);
+
+/* A routed MoE layer of resident MXFP4 experts: gate_up[e] is [2I][H] (gate rows 0..I-1, up rows
+ * I..2I-1), down[e] is [H][I]; host arrays of E descriptors. */
+typedef struct {
+  const tcf4_mxfp4 *gate_up;
+  const tcf4_mxfp4 *down;
+  int32_t E;
+  int32_t H;
+  int32_t I;
+} tcf4_mxfp4_moe;
+
+/* The same layer computation as trellis_grouped_moe (SwiGLU between gate/up and down, fp32
+ * combine of the k routed experts, bf16 out) from resident MXFP4 experts. Limits: 1 <= T <= 32,
+ * 1 <= k <= 8, E <= 256, H and I multiples of 64 up to 16384. The workspace holds h as bf16
+ * [T*k][I] in (t, j) order at offset mxfp4_grouped_moe_hidden_offset(m, T, k) after the call. */
+TCF4_API size_t mxfp4_grouped_moe_workspace(const tcf4_mxfp4_moe *m, int32_t T, int32_t k);
+TCF4_API size_t mxfp4_grouped_moe_hidden_offset(const tcf4_mxfp4_moe *m, int32_t T, int32_t k);
+TCF4_API tcf4_status mxfp4_grouped_moe(const tcf4_mxfp4_moe *m, const uint16_t *x, int32_t T,
+                                       const int32_t *topk_ids, const float *topk_w, int32_t k, uint16_t *out,
+                                       void *workspace, size_t ws_bytes, void *stream);
+
 /* Bounded waits that gave up inside the library's kernels since the last call, then resets the
  * count. Kernels that stage weights with bulk copies wait on shared-memory barriers with an
  * iteration limit; a wait that runs out is counted and the affected outputs are invalid. Never

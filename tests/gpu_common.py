@@ -39,14 +39,36 @@ def xnorms(x_bits):
     return np.linalg.norm(oracle.bf16_bits_to_f64(x_bits), axis=1)
 
 
-def check_moe(layer, W, x, ids, wts, out, ws, k, seg_gu, seg_dn=None, rows_h=None, rows_out=None):
+def upload_mx(nib, sc):
+    """A resident MXFP4 matrix from numpy nibbles [rows][cols/2] and scales [rows][cols/32]."""
+    rows, half = nib.shape
+    return tc.Mxfp4Matrix(torch.from_numpy(np.ascontiguousarray(nib)).cuda(),
+                          torch.from_numpy(np.ascontiguousarray(sc)).cuda(), rows, 2 * half)
+
+
+def _trellis_product(layer, kind, e, rows, cols, seg, xb, row_ids):
+    return oracle.gemv(getattr(layer, kind + "_stream")[e], getattr(layer, kind + "_scales")[e], rows, cols, seg, xb,
+                       row_ids=row_ids)
+
+
+def mx_product(mx):
+    """Oracle products of expert matrices given as MXFP4 numpy pairs: mx["gu"][e], mx["dn"][e]."""
+    def product(layer, kind, e, rows, cols, seg, xb, row_ids):
+        nib, sc = mx[kind][e]
+        return oracle.mxfp4_gemv(nib, sc, rows, cols, xb, row_ids=row_ids)
+    return product
+
+
+def check_moe(layer, W, x, ids, wts, out, ws, k, seg_gu, seg_dn=None, rows_h=None, rows_out=None,
+              product=_trellis_product):
     """Two-stage check of a grouped-MoE call.
 
     (i) h (read back from the workspace) against h_exact = silu(g) u from exact g, u, within the
         bound propagated from the product tolerance on g and u plus one bf16 rounding;
     (ii) out against sum_j w_j (down_j . h_gpu_j) computed exactly from the GPU's own h, within
         2e-3 sum_j |w_j| ||down_row|| ||h_j||.
-    rows_h / rows_out: optional subsets of intermediate / output rows (sampled checks)."""
+    rows_h / rows_out: optional subsets of intermediate / output rows (sampled checks).
+    product: the oracle's expert products (default: the trellis stream of `layer`)."""
     T = x.shape[0]
     H, I = layer.H, layer.I
     seg_dn = seg_gu if seg_dn is None else seg_dn
@@ -64,8 +86,7 @@ def check_moe(layer, W, x, ids, wts, out, ws, k, seg_gu, seg_dn=None, rows_h=Non
             if not 0 <= e < layer.E:
                 continue
             gu_rows = np.concatenate([ri, I + ri])
-            y, wn = oracle.gemv(layer.gu_stream[e], layer.gu_scales[e], 2 * I, H, seg_gu, x_bits[t:t + 1],
-                                row_ids=gu_rows)
+            y, wn = product(layer, "gu", e, 2 * I, H, seg_gu, x_bits[t:t + 1], gu_rows)
             g, u = y[0, :len(ri)], y[0, len(ri):]
             dg, du = TOL * wn[:len(ri)] * xn[t], TOL * wn[len(ri):] * xn[t]
             sg = oracle.silu(g)
@@ -83,7 +104,7 @@ def check_moe(layer, W, x, ids, wts, out, ws, k, seg_gu, seg_dn=None, rows_h=Non
             if not 0 <= e < layer.E:
                 continue
             hb = h_gpu[t, j][None, :]
-            y, wn = oracle.gemv(layer.dn_stream[e], layer.dn_scales[e], H, I, seg_dn, hb, row_ids=rn)
+            y, wn = product(layer, "dn", e, H, I, seg_dn, hb, rn)
             acc += w_np[t, j] * y[0]
             bnd += abs(w_np[t, j]) * wn * np.linalg.norm(oracle.bf16_bits_to_f64(hb))
         bad = np.abs(out_got[t, rn] - acc) > TOL * bnd + 1e-30

@@ -137,6 +137,79 @@ class MoEWeights:
         return int(_abi.load().trellis_grouped_moe_hidden_offset(ctypes.byref(self._moe), T, k))
 
 
+class Mxfp4Matrix:
+    """A resident MXFP4 matrix W [rows][cols]: nibbles uint8 [rows][cols/2] (element 2u in the low
+    nibble of byte u) and UE8M0 scales uint8 [rows][cols/32], both on the GPU (the output of
+    decode_to_mxfp4)."""
+
+    def __init__(self, nibbles: torch.Tensor, scales: torch.Tensor, rows: int, cols: int):
+        self.nibbles, self.scales = nibbles, scales
+        self.rows, self.cols = int(rows), int(cols)
+
+    @classmethod
+    def expand(cls, w: "TrellisMatrix"):
+        """Expand a trellis matrix once into a resident MXFP4 tensor."""
+        nib, sc = decode_to_mxfp4(w)
+        return cls(nib, sc, w.rows, w.cols)
+
+    def abi(self) -> _abi.Mxfp4:
+        return _abi.Mxfp4(self.nibbles.data_ptr(), self.scales.data_ptr(), self.rows, self.cols)
+
+
+def mxfp4_gemv_workspace_bytes(w: Mxfp4Matrix, T: int) -> int:
+    return int(_abi.load().mxfp4_gemv_workspace(w.abi(), T))
+
+
+def mxfp4_gemv(w: Mxfp4Matrix, x: torch.Tensor, out=None, workspace=None):
+    """y = bf16(W x) from the resident MXFP4 tensor, bf16 activations x [T][cols] (T <= 32)."""
+    x = x if x.dim() == 2 else x.view(1, -1)
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, w.rows), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(mxfp4_gemv_workspace_bytes(w, T), 1), dtype=torch.uint8, device=x.device)
+    _abi.check(_abi.load().mxfp4_gemv(w.abi(), _ptr(x), T, _ptr(out), _ptr(workspace), workspace.numel(),
+                                      _stream_handle()), "mxfp4_gemv")
+    return out
+
+
+class Mxfp4MoEWeights:
+    """E experts of one MoE layer as resident MXFP4: gate_up [2I][H] and down [H][I] per expert."""
+
+    def __init__(self, gate_up, down, H: int, I: int):
+        assert len(gate_up) == len(down)
+        self.gate_up, self.down = list(gate_up), list(down)
+        self.E, self.H, self.I = len(gate_up), int(H), int(I)
+        self._gu = (_abi.Mxfp4 * self.E)(*[m.abi() for m in self.gate_up])
+        self._dn = (_abi.Mxfp4 * self.E)(*[m.abi() for m in self.down])
+        self._moe = _abi.Mxfp4Moe(self._gu, self._dn, self.E, self.H, self.I)
+
+    @classmethod
+    def expand(cls, m: "MoEWeights"):
+        """Expand every expert of a trellis MoE layer once."""
+        return cls([Mxfp4Matrix.expand(w) for w in m.gate_up], [Mxfp4Matrix.expand(w) for w in m.down], m.H, m.I)
+
+    def workspace_bytes(self, T: int, k: int) -> int:
+        return int(_abi.load().mxfp4_grouped_moe_workspace(ctypes.byref(self._moe), T, k))
+
+    def hidden_offset(self, T: int, k: int) -> int:
+        return int(_abi.load().mxfp4_grouped_moe_hidden_offset(ctypes.byref(self._moe), T, k))
+
+
+def mxfp4_grouped_moe(m: Mxfp4MoEWeights, x: torch.Tensor, ids: torch.Tensor, wts: torch.Tensor, out=None,
+                      workspace=None):
+    """The grouped MoE layer of grouped_moe, from resident MXFP4 experts."""
+    T, k = ids.shape
+    if out is None:
+        out = torch.empty((T, m.H), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(m.workspace_bytes(T, k), 1), dtype=torch.uint8, device=x.device)
+    _abi.check(_abi.load().mxfp4_grouped_moe(ctypes.byref(m._moe), _ptr(x), T, _ptr(ids), _ptr(wts), k, _ptr(out),
+                                             _ptr(workspace), workspace.numel(), _stream_handle()),
+               "mxfp4_grouped_moe")
+    return out, workspace
+
+
 def moe_workspace_bytes(m: MoEWeights, T: int, k: int) -> int:
     return m.workspace_bytes(T, k)
 

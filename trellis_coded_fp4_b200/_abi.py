@@ -12,8 +12,9 @@ STATUS_NAMES = {0: "TCF4_OK", 1: "TCF4_ERR_INVALID_ARG", 2: "TCF4_ERR_MISALIGNED
 # Every symbol include/tcf4.h declares.
 EXPORTED = ("trellis_decode_to_mxfp4", "trellis_gemv_workspace", "trellis_gemv", "trellis_gemv_noalloc",
             "trellis_moe_route", "trellis_grouped_moe_workspace",
-            "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "tcf4_device_timeouts",
-            "tcf4_status_string")
+            "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "mxfp4_gemv_workspace", "mxfp4_gemv",
+            "mxfp4_grouped_moe_workspace", "mxfp4_grouped_moe_hidden_offset", "mxfp4_grouped_moe",
+            "tcf4_device_timeouts", "tcf4_status_string")
 
 
 class Matrix(ctypes.Structure):
@@ -25,6 +26,18 @@ class Matrix(ctypes.Structure):
 class Moe(ctypes.Structure):
     """tcf4_moe"""
     _fields_ = [("gate_up", ctypes.POINTER(Matrix)), ("down", ctypes.POINTER(Matrix)), ("E", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("I", ctypes.c_int32)]
+
+
+class Mxfp4(ctypes.Structure):
+    """tcf4_mxfp4"""
+    _fields_ = [("nibbles", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("cols", ctypes.c_int64)]
+
+
+class Mxfp4Moe(ctypes.Structure):
+    """tcf4_mxfp4_moe"""
+    _fields_ = [("gate_up", ctypes.POINTER(Mxfp4)), ("down", ctypes.POINTER(Mxfp4)), ("E", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("I", ctypes.c_int32)]
 
 
@@ -57,6 +70,16 @@ def load(path: str = LIB_PATH):
     L.trellis_grouped_moe_hidden_offset.restype = sz
     L.trellis_grouped_moe.argtypes = [ctypes.POINTER(Moe), vp, i32, vp, vp, i32, vp, vp, sz, vp]
     L.trellis_grouped_moe.restype = ctypes.c_int
+    L.mxfp4_gemv_workspace.argtypes = [Mxfp4, i32]
+    L.mxfp4_gemv_workspace.restype = sz
+    L.mxfp4_gemv.argtypes = [Mxfp4, vp, i32, vp, vp, sz, vp]
+    L.mxfp4_gemv.restype = ctypes.c_int
+    L.mxfp4_grouped_moe_workspace.argtypes = [ctypes.POINTER(Mxfp4Moe), i32, i32]
+    L.mxfp4_grouped_moe_workspace.restype = sz
+    L.mxfp4_grouped_moe_hidden_offset.argtypes = [ctypes.POINTER(Mxfp4Moe), i32, i32]
+    L.mxfp4_grouped_moe_hidden_offset.restype = sz
+    L.mxfp4_grouped_moe.argtypes = [ctypes.POINTER(Mxfp4Moe), vp, i32, vp, vp, i32, vp, vp, sz, vp]
+    L.mxfp4_grouped_moe.restype = ctypes.c_int
     L.tcf4_device_timeouts.argtypes = []
     L.tcf4_device_timeouts.restype = ctypes.c_uint
     L.tcf4_status_string.argtypes = [ctypes.c_int]

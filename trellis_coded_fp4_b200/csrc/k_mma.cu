@@ -86,6 +86,16 @@ struct Cfg {
   static constexpr uint32_t kUsed = kSfbCol + kKB * kNA;
   static constexpr uint32_t kTmemCols = kUsed <= 128 ? 128 : (kUsed <= 256 ? 256 : 512);
   static_assert(kUsed <= 512, "TMEM budget");
+  // Resident-MXFP4 source (the expanded tensor): the A operand is a shared-memory tile of nibbles
+  // (128 rows x 16 KB bytes, 128-byte-swizzled TMA boxes) and TMEM holds only the accumulators and
+  // the scale factors.
+  static constexpr int kNWX = NMAX <= 32 ? 2 : 3;              // A-tile stages in flight
+  static constexpr uint32_t kWStageX = 2048u * kKB;
+  static constexpr uint32_t kSfaColX = 2u * kNI * NMAX;
+  static constexpr uint32_t kSfbColX = kSfaColX + kKB * kNA;
+  static constexpr uint32_t kUsedX = kSfbColX + kKB * kNA;
+  static constexpr uint32_t kTmemColsX = kUsedX <= 128 ? 128 : (kUsedX <= 256 ? 256 : 512);
+  static_assert(kUsedX <= 512, "TMEM budget");
 };
 
 // Position (0..31) inside a 32-element chunk of the MMA operand of weight i of the block: the
@@ -193,14 +203,15 @@ __host__ __device__ inline size_t terms_bytes(int S) {
 // block in (3, 6]; each residual is rounded to the E2M1 grid (nearest even) and the rounded value
 // removed (exactly: Sterbenz). The largest residual shrinks by at least 5x per term, so after
 // kTerms terms |x - sum| <= 5^-6 max|x| over the block.
-template <int NMAX>
+// NAT: natural K order within a block (the MXFP4 tensor's), else the decoder's interleaved order.
+template <int NMAX, bool NAT = false>
 __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total, uint8_t *terms) {
   using C = Cfg<NMAX>;
   const int lane = threadIdx.x & 31;
   const int s = kb / C::kKB, c = kb - s * C::kKB, h = c >> 2;
   uint8_t *bst = terms + (size_t)s * C::kBStage;
   uint8_t *sfs = terms + (size_t)S_total * C::kBStage + (size_t)s * C::kSfbStage;
-  const int kp = kpos_of_weight(lane);
+  const int kp = NAT ? lane : kpos_of_weight(lane);
   float r = v;
 #pragma unroll
   for (int j = 0; j < kTerms; j++) {
@@ -214,9 +225,10 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
     S = S < -127 ? -127 : S;
     const uint32_t code = to_e2m1(r * pow2f(-S));
     r -= e2m1_value(code) * pow2f(S);
-    const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, 4);
+    // the element sharing this one's byte: K positions kp and kp ^ 1
+    const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, NAT ? 1 : 4);
     if (n < NMAX) {
-      if (((lane >> 2) & 1) == 0)
+      if ((kp & 1) == 0)
         bst[chunk_off<NMAX>((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code | (partner << 4));
       if (lane == 0) sfs[((h * C::kC + (n >> 5)) * 32 + (n & 31)) * 4 + (c & 3)] = (uint8_t)(S + 127);
     }
@@ -227,7 +239,7 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
 // The GEMV's product kernel is launched as a programmatic dependent of this split: it starts its
 // TMEM setup and its first weight tiles (which do not depend on the split) at once and waits for
 // the split's completion only before it reads the activation terms.
-template <int NMAX>
+template <int NMAX, bool NAT>
 __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
                                                      uint8_t *__restrict__ terms) {
   grid_dep_wait();     // x may come from, and terms may still be read by, the preceding kernel
@@ -237,14 +249,14 @@ __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict_
   for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < Cfg<NMAX>::kSlots * nb; wi += nwarps) {
     const int t = wi / nb, kb = wi - t * nb;
     const float v = t < T ? __uint_as_float((uint32_t)x[(size_t)t * K + kb * 32 + lane] << 16) : 0.f;
-    split_terms<NMAX>(v, t, kb, S, terms);
+    split_terms<NMAX, NAT>(v, t, kb, S, terms);
   }
 }
 
 // MoE: group g's token slot i is pair list[g_first + i]; its activation row is src[pair / div]
 // (gate_up reads x rows of tokens: div = k; down reads h rows of pairs: div = 1). Block 0 also
 // clears the down kernel's counters when `counters` is given.
-template <int NMAX>
+template <int NMAX, bool NAT>
 __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ ids, int P, int E, int div,
                                                     const uint16_t *__restrict__ src, int K, uint8_t *__restrict__ terms,
                                                     int *__restrict__ counters, int n_counters) {
@@ -266,7 +278,7 @@ __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ 
       const int row = pl.list[pl.g_first[g] + t] / div;
       v = __uint_as_float((uint32_t)src[(size_t)row * K + kb * 32 + lane] << 16);
     }
-    split_terms<NMAX>(v, t, kb, S, terms + (size_t)g * terms_bytes<NMAX>(S));
+    split_terms<NMAX, NAT>(v, t, kb, S, terms + (size_t)g * terms_bytes<NMAX>(S));
   }
 }
 
@@ -278,11 +290,11 @@ struct MmaGeom {
 };
 
 template <int NMAX>
-__host__ __device__ inline MmaGeom mma_geom(int mode) {
+__host__ __device__ inline MmaGeom mma_geom(int mode, bool mx = false) {
   using C = Cfg<NMAX>;
   MmaGeom g;
   g.off_W = 1024u;
-  g.off_B = g.off_W + C::kNW * C::kWStage;
+  g.off_B = g.off_W + (mx ? C::kNWX * C::kWStageX : C::kNW * C::kWStage);
   g.off_U = g.off_B + C::kNB * C::kBStage;
   g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)C::kTok * 4u : 0u);
   g.smem = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
@@ -429,6 +441,31 @@ __device__ __forceinline__ void mma_mxf4_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// The same MMA with A from shared memory (descriptor a_desc).
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand tile in the 128-byte-swizzled layout a SWIZZLE_128B
+// TMA box of 128-byte rows produces (layout type 2; SBO = 1 KB between 8-row groups; LBO unused).
+// A K step of 64 E2M1 elements (32 bytes) inside the 128-byte swizzle row advances the start
+// address by 32 bytes.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;  // descriptor version for tcgen05
+  d |= (uint64_t)2u << 61;  // SWIZZLE_128B
+  return d;
+}
+
 // Per-job tensor maps of the grouped MoE: lane 0 rewrites the global address of the shared-memory
 // copy, then the whole warp publishes it to the CTA's global slot for the TMA unit.
 __device__ __forceinline__ void tmap_set_address(uint32_t smap, const void *addr) {
@@ -532,19 +569,27 @@ __device__ __forceinline__ int tile_row(const JobRows &j, int m) {
 
 // ------------------------------------------------------------------------------- the kernel
 
-template <int MAXE, int MODE, int NMAX>
+// MX: the weights are a resident MXFP4 tensor (nibbles [rows][K/2], scales [rows][K/32]) instead of a
+// trellis stream; the word loader then brings 128-byte-swizzled nibble tiles that the MMAs read as
+// the A operand straight from shared memory, and four scale-factor warps replace the decode warps.
+template <int MAXE, int MODE, int NMAX, bool MX>
 __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
                                                      const __grid_constant__ MoeTable<MAXE> tab,
                                                      const __grid_constant__ CUtensorMap wmap) {
   using C = Cfg<NMAX>;
-  constexpr int kNW = C::kNW, kNA = C::kNA, kKB = C::kKB, kNBT = C::kNBT, kNG = C::kNG;
+  constexpr int kNW = MX ? C::kNWX : C::kNW, kNA = C::kNA, kKB = C::kKB, kNBT = C::kNBT, kNG = C::kNG;
+  constexpr uint32_t kWStage = MX ? C::kWStageX : C::kWStage;
+  constexpr uint32_t kSfaCol = MX ? C::kSfaColX : C::kSfaCol, kSfbCol = MX ? C::kSfbColX : C::kSfbCol;
+  constexpr uint32_t kTmemCols = MX ? C::kTmemColsX : C::kTmemCols;
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = a.nbr, S = (nbr + kKB - 1) / kKB;
-  const MmaGeom geo = mma_geom<NMAX>(MODE);
-  static_assert(kNW <= 8 && kNA <= 4 && C::kNB <= 4, "barrier block: 8 word slots, 4 A and 4 B slots");
+  const MmaGeom geo = mma_geom<NMAX>(MODE, MX);
+  static_assert((MX ? 2 * kNW : kNW) <= 8 && kNA <= 4 && C::kNB <= 4,
+                "barrier block: 8 word slots, 4 A and 4 B slots");
   // 49 barriers in bytes [0, 392). The A operand of a stage is filled and released in two halves
-  // (blocks [0, KB/2) and [KB/2, KB), each by half of the decode warps): barrier 2 b + half.
+  // (blocks [0, KB/2) and [KB/2, KB), each by half of the decode warps): barrier 2 b + half. With
+  // MX the word slots are also split in halves (barrier 2 ws + half), each released by its MMAs.
   uint64_t *w_full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *w_empty = w_full + 8, *a_full = w_full + 16, *a_empty = w_full + 24, *b_full = w_full + 32,
            *b_empty = w_full + 36, *acc_full = w_full + 40, *acc_empty = w_full + 42, *u_full = w_full + 44,
@@ -557,13 +602,13 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   const size_t tbytes = terms_bytes<NMAX>(S);
 
   if (tid == 0) {
-    for (int i = 0; i < kNW; i++) {
+    for (int i = 0; i < (MX ? 2 * kNW : kNW); i++) {
       mbar_init(&w_full[i], 1);
-      mbar_init(&w_empty[i], C::kDecWarps);
+      mbar_init(&w_empty[i], MX ? 1 : C::kDecWarps);
     }
     for (int i = 0; i < kNA; i++) {
       for (int hh = 0; hh < 2; hh++) {
-        mbar_init(&a_full[2 * i + hh], C::kDecWarps / 2);
+        mbar_init(&a_full[2 * i + hh], MX ? 4 : C::kDecWarps / 2);
         mbar_init(&a_empty[2 * i + hh], 1);
       }
     }
@@ -584,7 +629,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   if (MODE != kModeGemv && tid < 32)
     reinterpret_cast<uint32_t *>(smap)[tid] = reinterpret_cast<const uint32_t *>(&wmap)[tid];
   if (warp == C::kMmaWarp) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   int njobs;
@@ -602,7 +647,78 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   const int nq = my_jobs * S;
   auto job_of = [&](int jl) { return (int)blockIdx.x + jl * (int)gridDim.x; };
 
-  if (warp < C::kDecWarps) {
+  if (MX && warp < C::kDecWarps) {
+    // ---------------------------------------------------------------- scale-factor warps (MX)
+    // Warp w < 4 writes, for every stage, the scale factors of tile rows 32w..32w+31 (its lane
+    // quarter): each row's KB UE8M0 bytes (A) and this lane's B scale words (every quarter holds a
+    // copy). The next stage's bytes are loaded while the current stage's are stored.
+    if (warp < 4) {
+      constexpr int kG = kKB / 4;  // scale groups per stage
+      const int m = 32 * warp + lane;
+      const uint32_t tq = tbase + ((uint32_t)(32 * warp) << 16);
+      uint32_t pa[kKB / 2], pb[kG][C::kC];
+      int qp = 0, jl_p = 0, s_p = 0;
+      const unsigned short *srow = nullptr;
+      const uint32_t *sfb_src = nullptr;
+      auto load_sf = [&](uint32_t(&da)[kKB / 2], uint32_t(&db)[kG][C::kC]) {
+        if (qp >= nq) return;
+        if (s_p == 0) {
+          const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_p));
+          const int row = tile_row(jr, m);
+          srow = row >= 0 ? reinterpret_cast<const unsigned short *>(jr.sc + (size_t)row * nbr) : nullptr;
+          sfb_src = reinterpret_cast<const uint32_t *>(a.terms + (size_t)jr.group * tbytes + (size_t)S * C::kBStage) + lane;
+        }
+        const int lim = nbr - kKB * s_p;  // blocks of the stage inside the row
+#pragma unroll
+        for (int i = 0; i < kKB / 2; i++)
+          da[i] = srow != nullptr && 2 * i < lim ? (uint32_t)__ldg(srow + (kKB / 2) * s_p + i) : 0u;
+#pragma unroll
+        for (int g = 0; g < kG; g++)
+#pragma unroll
+          for (int c = 0; c < C::kC; c++)
+            db[g][c] = __ldg(sfb_src + (size_t)s_p * (C::kSfbStage / 4) + (g * C::kC + c) * 32);
+        qp++;
+        if (++s_p == S) {
+          s_p = 0;
+          jl_p++;
+        }
+      };
+      grid_dep_wait();  // the activation terms (B scales) come from the preceding split kernel
+      load_sf(pa, pb);
+      uint32_t b = 0;
+      bool ok = true;
+#pragma unroll 1
+      for (int q = 0; q < nq; q++) {
+        uint32_t na[kKB / 2], nb[kG][C::kC];
+        load_sf(na, nb);
+        if (q >= kNA) {
+          const uint32_t ph = (uint32_t)((q - kNA) / kNA) & 1u;
+          if (!(ok = warp_wait(&a_empty[2 * b], ph, tmo, abort_flag) && warp_wait(&a_empty[2 * b + 1], ph, tmo, abort_flag)))
+            break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int g = 0; g < kG; g++) {
+          tmem_st_x1(tq + kSfaCol + kKB * b + 4u * (uint32_t)g + (uint32_t)warp, pa[2 * g] | (pa[2 * g + 1] << 16));
+#pragma unroll
+          for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + kSfbCol + kKB * b + 4u * (uint32_t)g + (uint32_t)c, pb[g][c]);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        mbar_arrive_one(&a_full[2 * b]);
+        mbar_arrive_one(&a_full[2 * b + 1]);
+#pragma unroll
+        for (int i = 0; i < kKB / 2; i++) pa[i] = na[i];
+#pragma unroll
+        for (int g = 0; g < kG; g++)
+#pragma unroll
+          for (int c = 0; c < C::kC; c++) pb[g][c] = nb[g][c];
+        b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
+      }
+      if (!ok) *abort_flag = 1;
+    }
+  } else if (warp < C::kDecWarps) {
     // ---------------------------------------------------------------- decode warps
     // Thread (warp w, lane l) owns tile row m = 32 (w % 4) + l and the kNBT blocks kNBT (w / 4).. of
     // each stage, decoded in chunks of eight (64 bytes of words, four 16-byte reads).
@@ -661,7 +777,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       if (!wf_ready && !(ok = warp_wait(&w_full[ws], (uint32_t)(q / kNW) & 1u, tmo, abort_flag))) break;
       uint32_t na[kNBT / 2], nb[kNG][C::kC];
       load_sf(na, nb);  // the next stage's scale factors; their latency hides behind this stage
-      const uint32_t wa = wrow + ws * C::kWStage;
+      const uint32_t wa = wrow + ws * kWStage;
       const uint32_t ws1 = ws + 1 == (uint32_t)kNW ? 0u : ws + 1;
       uint32_t ae = 1u, wf = 0u;
 #pragma unroll 1
@@ -703,9 +819,9 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
 #pragma unroll
       for (int g = 0; g < kNG; g++) {
         const uint32_t gg = (uint32_t)(kNG * h + g);
-        tmem_st_x1(tq + C::kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[2 * g] | (pa[2 * g + 1] << 16));
+        tmem_st_x1(tq + kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[2 * g] | (pa[2 * g + 1] << 16));
 #pragma unroll
-        for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + C::kSfbCol + kKB * b + 4u * gg + (uint32_t)c, pb[g][c]);
+        for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + kSfbCol + kKB * b + 4u * gg + (uint32_t)c, pb[g][c]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -743,14 +859,36 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         }
       }
       if (lane == 0) {
-        if (qi >= kNW) ok = mbar_wait_sleep(&w_empty[wi], (uint32_t)((qi - kNW) / kNW) & 1u, tmo, kLoaderSleepNs);
-        if (ok) {
-          mbar_arrive_expect_tx(&w_full[wi], C::kWStage);
-          const uint32_t dst = wbase + wi * C::kWStage;
+        if constexpr (MX) {
+          // two halves of KB/2 blocks, each its own barrier pair: column box c (128 bytes = 8 blocks)
+          // of rows y0.. at (2c) x 8 KB and of rows y1.. at (2c + 1) x 8 KB, so each column's 128
+          // rows form one SBO = 1 KB operand tile
+          const uint32_t dst = wbase + wi * kWStage;
 #pragma unroll
-          for (int c = 0; c < C::kBoxCols; c++) {
-            tma_load_2d(dst + (uint32_t)c * 8192u, map_i, kKB * 8 * s_i + 128 * c, ji.y0, &w_full[wi]);
-            tma_load_2d(dst + (uint32_t)(C::kBoxCols + c) * 8192u, map_i, kKB * 8 * s_i + 128 * c, ji.y1, &w_full[wi]);
+          for (int hh = 0; hh < 2; hh++) {
+            if (qi >= kNW && ok)
+              ok = mbar_wait_sleep(&w_empty[2 * wi + hh], (uint32_t)((qi - kNW) / kNW) & 1u, tmo, kLoaderSleepNs);
+            if (ok) {
+              mbar_arrive_expect_tx(&w_full[2 * wi + hh], kWStage / 2);
+#pragma unroll
+              for (int c = hh * kKB / 16; c < (hh + 1) * kKB / 16; c++) {
+                tma_load_2d(dst + (uint32_t)(2 * c) * 8192u, map_i, kKB * 16 * s_i + 128 * c, ji.y0, &w_full[2 * wi + hh]);
+                tma_load_2d(dst + (uint32_t)(2 * c + 1) * 8192u, map_i, kKB * 16 * s_i + 128 * c, ji.y1,
+                            &w_full[2 * wi + hh]);
+              }
+            }
+          }
+        } else {
+          if (qi >= kNW) ok = mbar_wait_sleep(&w_empty[wi], (uint32_t)((qi - kNW) / kNW) & 1u, tmo, kLoaderSleepNs);
+          if (ok) {
+            mbar_arrive_expect_tx(&w_full[wi], kWStage);
+            const uint32_t dst = wbase + wi * kWStage;
+#pragma unroll
+            for (int c = 0; c < C::kBoxCols; c++) {
+              tma_load_2d(dst + (uint32_t)c * 8192u, map_i, kKB * 8 * s_i + 128 * c, ji.y0, &w_full[wi]);
+              tma_load_2d(dst + (uint32_t)(C::kBoxCols + c) * 8192u, map_i, kKB * 8 * s_i + 128 * c, ji.y1,
+                          &w_full[wi]);
+            }
           }
         }
       }
@@ -766,8 +904,10 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
     if (!ok) *abort_flag = 1;
     // drain: the last min(kNW, qi) issued stages may still be in flight
     if (lane == 0)
-      for (int d = qi - 1; d >= 0 && d >= qi - kNW; d--)
-        if (!mbar_wait(&w_full[d % kNW], (uint32_t)(d / kNW) & 1u, tmo)) break;
+      for (int d = qi - 1; d >= 0 && d >= qi - kNW; d--) {
+        if (!mbar_wait(&w_full[MX ? 2 * (d % kNW) : d % kNW], (uint32_t)(d / kNW) & 1u, tmo)) break;
+        if (MX && !mbar_wait(&w_full[2 * (d % kNW) + 1], (uint32_t)(d / kNW) & 1u, tmo)) break;
+      }
     __syncwarp();
   } else if (warp == C::kBLoadWarp) {
     // ---------------------------------------------------------------- B loader warp
@@ -922,10 +1062,15 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
       const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
       const uint64_t bd = smem_desc(b0 + (uint32_t)bb * C::kBStage, 128u, C::kSbo);
-      const uint32_t sfa = tbase + C::kSfaCol + kKB * (uint32_t)b, sfb = tbase + C::kSfbCol + kKB * (uint32_t)b;
+      const uint32_t sfa = tbase + kSfaCol + kKB * (uint32_t)b, sfb = tbase + kSfbCol + kKB * (uint32_t)b;
+      const int wsx = q % kNW;  // MX: the stage's word slot
+      const uint64_t ad0 = MX ? desc_sw128(smem_u32(smem + geo.off_W) + (uint32_t)wsx * kWStage) : 0ull;
 #pragma unroll
       for (int hh = h_lo; hh < h_hi; hh++) {  // this issuer's halves of the stage, in order
         ok = __all_sync(0xffffffffu, ok && mbar_wait_sleep(&a_full[2 * b + hh], ph, tmo, kMmaSleepNs));
+        if (MX && ok)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait_sleep(&w_full[2 * wsx + hh], (uint32_t)(q / kNW) & 1u, tmo, kMmaSleepNs));
         if (!ok) break;
         tc_fence_after();
         const int jfirst = C::kNI == 2 ? hh * kKB / 4 : 0;  // this issuer's first MMA of a job
@@ -936,12 +1081,18 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
             if (j < nmma) {
               const uint32_t sf = (uint32_t)(j & 1) * 2u;
               // +256 bytes of B per MMA: the descriptor's start address counts 16-byte units
-              mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
-                          (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30), (sfb + 4u * (uint32_t)(j >> 1)) | (sf << 30),
-                          !(s == 0 && j == jfirst));
+              if constexpr (MX)  // A: column box j / 4 (16 KB apart), 32 bytes per MMA inside it
+                mma_mxf4_ss(d_t, ad0 + (uint64_t)((j >> 2) * 1024 + 2 * (j & 3)), bd + 16u * (uint64_t)j,
+                            (j & 1) ? idesc2 : idesc0, (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30),
+                            (sfb + 4u * (uint32_t)(j >> 1)) | (sf << 30), !(s == 0 && j == jfirst));
+              else
+                mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
+                            (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30), (sfb + 4u * (uint32_t)(j >> 1)) | (sf << 30),
+                            !(s == 0 && j == jfirst));
             }
           }
           tc_commit(&a_empty[2 * b + hh]);
+          if (MX) tc_commit(&w_empty[2 * wsx + hh]);
           if (hh == h_hi - 1) {
             tc_commit(&b_empty[bb]);
             if (s == S - 1) tc_commit(&acc_full[jl & 1]);
@@ -974,7 +1125,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == C::kMmaWarp) tmem_dealloc(tbase, C::kTmemCols);
+  if (warp == C::kMmaWarp) tmem_dealloc(tbase, kTmemCols);
 }
 
 // ------------------------------------------------------------------------------- host side
@@ -994,14 +1145,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Tensor map of a trellis stream seen as a [rows][nbr*8] byte matrix, boxes of 64 rows x 128 bytes
-// with the 128-byte swizzle (the decode threads' 16-byte reads of consecutive rows then fall in
-// distinct banks); rows and columns beyond the matrix read as zero.
-static bool make_word_map(CUtensorMap *map, const void *stream, int rows, int nbr) {
+// Tensor map of a trellis stream seen as a [rows][nbr*8] byte matrix (bpb = 8 bytes per block), or
+// of a resident MXFP4 nibble matrix [rows][nbr*16] (bpb = 16): boxes of 64 rows x 128 bytes with
+// the 128-byte swizzle (the decode threads' 16-byte reads of consecutive rows then fall in distinct
+// banks; for MXFP4 it is the MMA's K-major A layout); rows and columns beyond the matrix read as
+// zero.
+static bool make_word_map(CUtensorMap *map, const void *stream, int rows, int nbr, int bpb = 8) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)nbr * 8u, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)nbr * 8u};
+  cuuint64_t dims[2] = {(cuuint64_t)nbr * (cuuint64_t)bpb, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)nbr * (cuuint64_t)bpb};
   cuuint32_t box[2] = {128u, 64u};
   cuuint32_t estr[2] = {1u, 1u};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(stream), dims, strides, box, estr,
@@ -1013,11 +1166,11 @@ static bool make_word_map(CUtensorMap *map, const void *stream, int rows, int nb
 constexpr int kGemvTok = Cfg<96>::kTok;
 static int nmax_for(int tokens_per_group) { return tokens_per_group <= Cfg<32>::kTok ? 32 : 96; }
 
-static bool mma_fits(int NMAX, int mode) {
+static bool mma_fits(int NMAX, int mode, bool mx = false) {
   int dev = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
-  const uint32_t need = NMAX == 32 ? mma_geom<32>(mode).smem : mma_geom<96>(mode).smem;
+  const uint32_t need = NMAX == 32 ? mma_geom<32>(mode, mx).smem : mma_geom<96>(mode, mx).smem;
   return need <= (uint32_t)optin;
 }
 
@@ -1030,9 +1183,17 @@ static size_t terms_for(int nbr, int NMAX) {
                     : terms_bytes<96>((nbr + Cfg<96>::kKB - 1) / Cfg<96>::kKB);
 }
 
+// The scale-factor threads read a row's scale bytes in pairs (16-bit loads): the scales must be
+// 2-byte aligned (rows are, with an even block count).
 bool gemv_mma_supported(const MatView &w, int T) {
-  return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.stream) & 15u) == 0 && tensor_map_encoder() != nullptr &&
+  return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.stream) & 15u) == 0 &&
+         (reinterpret_cast<uintptr_t>(w.scales) & 1u) == 0 && tensor_map_encoder() != nullptr &&
          mma_fits(nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv);
+}
+bool mx_gemv_supported(const MatView &w, int T) {
+  return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.stream) & 15u) == 0 &&
+         (reinterpret_cast<uintptr_t>(w.scales) & 1u) == 0 && tensor_map_encoder() != nullptr &&
+         mma_fits(nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv, true);
 }
 
 // Tokens beyond kGemvTok run as further passes, each with its own split of x.
@@ -1045,15 +1206,16 @@ static int sm_count() {
   return nsm;
 }
 
-template <int NMAX>
+template <int NMAX, bool MX>
 static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, const uint16_t *x, int T, uint16_t *y,
                                     void *ws, cudaStream_t s) {
   uint8_t *terms = static_cast<uint8_t *>(ws);
   const int warps = Cfg<NMAX>::kSlots * w.nbr;
-  cudaError_t e = launch_dependent(k_bsplit_gemv<NMAX>, dim3((warps + 7) / 8), dim3(256), 0, s, x, T, w.nbr * 32, terms);
+  cudaError_t e =
+      launch_dependent(k_bsplit_gemv<NMAX, MX>, dim3((warps + 7) / 8), dim3(256), 0, s, x, T, w.nbr * 32, terms);
   if (e != cudaSuccess) return e;
   static unsigned long long attr = 0;
-  e = ensure_max_dynamic_smem(k_mma<32, kModeGemv, NMAX>, attr);
+  e = ensure_max_dynamic_smem(k_mma<32, kModeGemv, NMAX, MX>, attr);
   if (e != cudaSuccess) return e;
   const int ntiles = (w.rows + 127) / 128, nsm = sm_count();
   MmaArgs args{};
@@ -1064,23 +1226,31 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
   args.T = T;
   args.y = y;
   MoeTable<32> none{};
-  return launch_dependent(k_mma<32, kModeGemv, NMAX>, dim3(ntiles < nsm ? ntiles : nsm), dim3(Cfg<NMAX>::kThreads),
-                          mma_geom<NMAX>(kModeGemv).smem, s, args, none, map);
+  return launch_dependent(k_mma<32, kModeGemv, NMAX, MX>, dim3(ntiles < nsm ? ntiles : nsm), dim3(Cfg<NMAX>::kThreads),
+                          mma_geom<NMAX>(kModeGemv, MX).smem, s, args, none, map);
 }
 
-cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
+template <bool MX>
+static cudaError_t launch_gemv_t(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
   CUtensorMap map;
-  if (!make_word_map(&map, w.stream, w.rows, w.nbr)) return cudaErrorInvalidValue;
+  if (!make_word_map(&map, w.stream, w.rows, w.nbr, MX ? 16 : 8)) return cudaErrorInvalidValue;
   const bool n32 = nmax_for(T < kGemvTok ? T : kGemvTok) == 32;
   for (int t0 = 0; t0 < T; t0 += kGemvTok) {
     const int n = T - t0 < kGemvTok ? T - t0 : kGemvTok;
     const uint16_t *xp = x + (size_t)t0 * w.nbr * 32;
     uint16_t *yp = y + (size_t)t0 * w.rows;
     cudaError_t e =
-        n32 ? launch_gemv_pass<32>(w, map, xp, n, yp, ws, s) : launch_gemv_pass<96>(w, map, xp, n, yp, ws, s);
+        n32 ? launch_gemv_pass<32, MX>(w, map, xp, n, yp, ws, s) : launch_gemv_pass<96, MX>(w, map, xp, n, yp, ws, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
+  return launch_gemv_t<false>(w, x, T, y, ws, s);
+}
+cudaError_t launch_mx_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
+  return launch_gemv_t<true>(w, x, T, y, ws, s);
 }
 
 // ----------------------------------------------------------------------------- MoE on the tensor cores
@@ -1091,10 +1261,21 @@ bool moe_mma_supported(const tcf4_moe &m, int gu_seg, int dn_seg, int T) {
   if (gu_seg != 1 || dn_seg != 1) return false;
   if (!k_ok(m.H / 32) || !k_ok(m.I / 32) || tensor_map_encoder() == nullptr) return false;
   for (int e = 0; e < m.E; e++)
-    if ((reinterpret_cast<uintptr_t>(m.gate_up[e].stream) | reinterpret_cast<uintptr_t>(m.down[e].stream)) & 15u)
+    if (((reinterpret_cast<uintptr_t>(m.gate_up[e].stream) | reinterpret_cast<uintptr_t>(m.down[e].stream)) & 15u) ||
+        ((reinterpret_cast<uintptr_t>(m.gate_up[e].scales) | reinterpret_cast<uintptr_t>(m.down[e].scales)) & 1u))
       return false;
   const int NMAX = nmax_for(T);
   return mma_fits(NMAX, kModeGateUp) && mma_fits(NMAX, kModeDown);
+}
+// The same layer as resident MXFP4 (stream fields point at the nibble matrices).
+bool moe_mx_supported(const tcf4_moe &m, int T) {
+  if (!k_ok(m.H / 32) || !k_ok(m.I / 32) || tensor_map_encoder() == nullptr) return false;
+  for (int e = 0; e < m.E; e++)
+    if (((reinterpret_cast<uintptr_t>(m.gate_up[e].stream) | reinterpret_cast<uintptr_t>(m.down[e].stream)) & 15u) ||
+        ((reinterpret_cast<uintptr_t>(m.gate_up[e].scales) | reinterpret_cast<uintptr_t>(m.down[e].scales)) & 1u))
+      return false;
+  const int NMAX = nmax_for(T);
+  return mma_fits(NMAX, kModeGateUp, true) && mma_fits(NMAX, kModeDown, true);
 }
 
 MoeMmaWorkspace moe_mma_workspace_layout(const tcf4_moe &m, int T, int k) {
@@ -1115,7 +1296,7 @@ MoeMmaWorkspace moe_mma_workspace_layout(const tcf4_moe &m, int T, int k) {
   return L;
 }
 
-template <int MAXE, int NMAX>
+template <int MAXE, int NMAX, bool MX>
 static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids,
                                     const float *wts, int k, uint16_t *out, void *ws, cudaStream_t s) {
   MoeTable<MAXE> tab;
@@ -1127,8 +1308,8 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
     tab.dns[e] = ok ? m.down[e].scales : nullptr;
   }
   CUtensorMap map_gu, map_dn;  // templates from expert 0 (every expert's matrices have the same shape)
-  if (!make_word_map(&map_gu, m.gate_up[0].stream, 2 * m.I, m.H / 32) ||
-      !make_word_map(&map_dn, m.down[0].stream, m.H, m.I / 32))
+  if (!make_word_map(&map_gu, m.gate_up[0].stream, 2 * m.I, m.H / 32, MX ? 16 : 8) ||
+      !make_word_map(&map_dn, m.down[0].stream, m.H, m.I / 32, MX ? 16 : 8))
     return cudaErrorInvalidValue;
   const MoeMmaWorkspace L = moe_mma_workspace_layout(m, T, k);
   char *base = static_cast<char *>(ws);
@@ -1154,18 +1335,18 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
     uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_gu);
     const int nbr = m.H / 32;
     const int warps = G * Cfg<NMAX>::kSlots * nbr;
-    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
+    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX, MX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
                                      dim3(256), 0, s, ids, P, m.E, k, x, m.H, terms, args.counters,
                                      4 * ((m.H + 127) / 128));
     if (e != cudaSuccess) return e;
     static unsigned long long attr = 0;
-    e = ensure_max_dynamic_smem(k_mma<MAXE, kModeGateUp, NMAX>, attr);
+    e = ensure_max_dynamic_smem(k_mma<MAXE, kModeGateUp, NMAX, MX>, attr);
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
     const int jobs = G * ((m.I + 63) / 64);
-    e = launch_dependent(k_mma<MAXE, kModeGateUp, NMAX>, dim3(jobs < nsm ? jobs : nsm), dim3(Cfg<NMAX>::kThreads),
-                         mma_geom<NMAX>(kModeGateUp).smem, s, args, tab, map_gu);
+    e = launch_dependent(k_mma<MAXE, kModeGateUp, NMAX, MX>, dim3(jobs < nsm ? jobs : nsm), dim3(Cfg<NMAX>::kThreads),
+                         mma_geom<NMAX>(kModeGateUp, MX).smem, s, args, tab, map_gu);
     if (e != cudaSuccess) return e;
   }
   // down: split h per group, then decode + MMA, y to the workspace, last arriver per chunk combines
@@ -1173,32 +1354,41 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
     uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_dn);
     const int nbr = m.I / 32;
     const int warps = G * Cfg<NMAX>::kSlots * nbr;
-    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
+    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX, MX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
                                      dim3(256), 0, s, ids, P, m.E, 1, (const uint16_t *)args.hidden, m.I, terms,
                                      (int *)nullptr, 0);
     if (e != cudaSuccess) return e;
     static unsigned long long attr = 0;
-    e = ensure_max_dynamic_smem(k_mma<MAXE, kModeDown, NMAX>, attr);
+    e = ensure_max_dynamic_smem(k_mma<MAXE, kModeDown, NMAX, MX>, attr);
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
     args.maps += (size_t)nsm * kMapSlots * 128;  // the down kernel's own tensor-map slots
     const int jobs = G * ((m.H + 127) / 128);
-    e = launch_dependent(k_mma<MAXE, kModeDown, NMAX>, dim3(jobs < nsm ? jobs : nsm), dim3(Cfg<NMAX>::kThreads),
-                         mma_geom<NMAX>(kModeDown).smem, s, args, tab, map_dn);
+    e = launch_dependent(k_mma<MAXE, kModeDown, NMAX, MX>, dim3(jobs < nsm ? jobs : nsm), dim3(Cfg<NMAX>::kThreads),
+                         mma_geom<NMAX>(kModeDown, MX).smem, s, args, tab, map_dn);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_moe_mma(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts, int k,
-                           uint16_t *out, void *ws, cudaStream_t s) {
+template <bool MX>
+static cudaError_t launch_moe_t(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts,
+                                int k, uint16_t *out, void *ws, cudaStream_t s) {
   const bool n32 = nmax_for(T) == 32;
   if (m.E <= 32)
-    return n32 ? launch_moe_mma_t<32, 32>(m, x, T, ids, wts, k, out, ws, s)
-               : launch_moe_mma_t<32, 96>(m, x, T, ids, wts, k, out, ws, s);
-  return n32 ? launch_moe_mma_t<256, 32>(m, x, T, ids, wts, k, out, ws, s)
-             : launch_moe_mma_t<256, 96>(m, x, T, ids, wts, k, out, ws, s);
+    return n32 ? launch_moe_mma_t<32, 32, MX>(m, x, T, ids, wts, k, out, ws, s)
+               : launch_moe_mma_t<32, 96, MX>(m, x, T, ids, wts, k, out, ws, s);
+  return n32 ? launch_moe_mma_t<256, 32, MX>(m, x, T, ids, wts, k, out, ws, s)
+             : launch_moe_mma_t<256, 96, MX>(m, x, T, ids, wts, k, out, ws, s);
+}
+cudaError_t launch_moe_mma(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts, int k,
+                           uint16_t *out, void *ws, cudaStream_t s) {
+  return launch_moe_t<false>(m, x, T, ids, wts, k, out, ws, s);
+}
+cudaError_t launch_moe_mx(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts, int k,
+                          uint16_t *out, void *ws, cudaStream_t s) {
+  return launch_moe_t<true>(m, x, T, ids, wts, k, out, ws, s);
 }
 
 unsigned int take_timeouts_mma() {

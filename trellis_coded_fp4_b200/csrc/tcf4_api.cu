@@ -38,6 +38,36 @@ MatView view(const tcf4_matrix &w) {
 
 tcf4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? TCF4_OK : TCF4_ERR_CUDA; }
 
+tcf4_status check_mx(const tcf4_mxfp4 &w) {
+  if (w.rows < 0 || w.cols < 0 || w.cols % 32 != 0) return TCF4_ERR_INVALID_ARG;
+  if (w.rows == 0 || w.cols == 0) return TCF4_OK;
+  if (w.nibbles == nullptr || w.scales == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(w.nibbles) || (reinterpret_cast<uintptr_t>(w.scales) & 1u) != 0) return TCF4_ERR_MISALIGNED;
+  if (w.cols % 64 != 0 || w.cols > kMaxCols || w.rows > INT32_MAX) return TCF4_ERR_UNSUPPORTED;
+  return TCF4_OK;
+}
+
+// The MXFP4 consumers reuse the trellis views: stream points at the nibble matrix.
+MatView mx_view(const tcf4_mxfp4 &w) {
+  MatView v;
+  v.stream = reinterpret_cast<const uint2 *>(w.nibbles);
+  v.scales = w.scales;
+  v.rows = (int32_t)w.rows;
+  v.nbr = (int32_t)(w.cols / 32);
+  v.seg_blocks = 1;
+  return v;
+}
+
+tcf4_matrix mx_as_matrix(const tcf4_mxfp4 &w) {
+  tcf4_matrix m;
+  m.stream = reinterpret_cast<const uint32_t *>(w.nibbles);
+  m.scales = w.scales;
+  m.rows = w.rows;
+  m.cols = w.cols;
+  m.seg_len = 32;
+  return m;
+}
+
 // A non-sticky error left pending by earlier, unrelated CUDA calls would otherwise be reported
 // as this call's launch failure; clear it before launching (documented in tcf4.h).
 void clear_pending_error() { (void)cudaGetLastError(); }
@@ -177,6 +207,83 @@ tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, int32_t T,
     return from_cuda(launch_moe_mma(*m, x, T, topk_ids, topk_w, k, out, workspace, static_cast<cudaStream_t>(stream)));
   return from_cuda(launch_moe(*m, gu_seg, dn_seg, x, T, topk_ids, topk_w, k, out, workspace,
                               static_cast<cudaStream_t>(stream)));
+}
+
+size_t mxfp4_gemv_workspace(tcf4_mxfp4 w, int32_t T) {
+  if (check_mx(w) != TCF4_OK || T <= 0 || T > kMaxTokens || w.rows == 0 || w.cols == 0) return 0;
+  return gemv_mma_workspace(mx_view(w), T);
+}
+
+tcf4_status mxfp4_gemv(tcf4_mxfp4 w, const uint16_t *x, int32_t T, uint16_t *y, void *workspace, size_t ws_bytes,
+                       void *stream) {
+  tcf4_status st = check_mx(w);
+  if (st != TCF4_OK) return st;
+  if (T < 0) return TCF4_ERR_INVALID_ARG;
+  if (T == 0 || w.rows == 0) return TCF4_OK;
+  if (T > kMaxTokens) return TCF4_ERR_UNSUPPORTED;
+  if (w.cols == 0) return TCF4_ERR_INVALID_ARG;
+  if (x == nullptr || y == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return TCF4_ERR_MISALIGNED;
+  const MatView v = mx_view(w);
+  if (!mx_gemv_supported(v, T)) return TCF4_ERR_UNSUPPORTED;
+  if (workspace == nullptr || ws_bytes < gemv_mma_workspace(v, T)) return TCF4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
+  clear_pending_error();
+  return from_cuda(launch_mx_gemv(v, x, T, y, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+// The layer as a tcf4_moe whose stream fields point at the nibble matrices (host arrays of this
+// thread, valid until its next MXFP4 MoE call).
+static tcf4_status mx_moe_view(const tcf4_mxfp4_moe *m, int32_t T, int32_t k, tcf4_moe *out) {
+  static thread_local tcf4_matrix gu[kMaxExperts], dn[kMaxExperts];
+  if (m == nullptr || m->gate_up == nullptr || m->down == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (m->E < 1 || m->H < 32 || m->I < 32 || m->H % 32 != 0 || m->I % 32 != 0) return TCF4_ERR_INVALID_ARG;
+  if (T < 0 || k < 1 || k > m->E) return TCF4_ERR_INVALID_ARG;
+  if (m->E > kMaxExperts || k > kMaxTopK || T > kMaxTokens || m->H > kMaxCols || m->I > kMaxCols)
+    return TCF4_ERR_UNSUPPORTED;
+  for (int e = 0; e < m->E; e++) {
+    const tcf4_mxfp4 &g = m->gate_up[e], &d = m->down[e];
+    if (g.rows != 2 * (int64_t)m->I || g.cols != m->H || d.rows != m->H || d.cols != m->I) return TCF4_ERR_INVALID_ARG;
+    tcf4_status s1 = check_mx(g), s2 = check_mx(d);
+    if (s1 != TCF4_OK) return s1;
+    if (s2 != TCF4_OK) return s2;
+    gu[e] = mx_as_matrix(g);
+    dn[e] = mx_as_matrix(d);
+  }
+  out->gate_up = gu;
+  out->down = dn;
+  out->E = m->E;
+  out->H = m->H;
+  out->I = m->I;
+  return TCF4_OK;
+}
+
+size_t mxfp4_grouped_moe_workspace(const tcf4_mxfp4_moe *m, int32_t T, int32_t k) {
+  tcf4_moe v;
+  if (mx_moe_view(m, T, k, &v) != TCF4_OK || T == 0) return 0;
+  return moe_mma_workspace_layout(v, T, k).total;
+}
+
+size_t mxfp4_grouped_moe_hidden_offset(const tcf4_mxfp4_moe *m, int32_t T, int32_t k) {
+  tcf4_moe v;
+  if (mx_moe_view(m, T, k, &v) != TCF4_OK || T == 0) return 0;
+  return moe_mma_workspace_layout(v, T, k).hidden;
+}
+
+tcf4_status mxfp4_grouped_moe(const tcf4_mxfp4_moe *m, const uint16_t *x, int32_t T, const int32_t *topk_ids,
+                              const float *topk_w, int32_t k, uint16_t *out, void *workspace, size_t ws_bytes,
+                              void *stream) {
+  tcf4_moe v;
+  tcf4_status st = mx_moe_view(m, T, k, &v);
+  if (st != TCF4_OK) return st;
+  if (T == 0) return TCF4_OK;
+  if (x == nullptr || topk_ids == nullptr || topk_w == nullptr || out == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return TCF4_ERR_MISALIGNED;
+  if (!moe_mx_supported(v, T)) return TCF4_ERR_UNSUPPORTED;
+  if (workspace == nullptr || ws_bytes < moe_mma_workspace_layout(v, T, k).total) return TCF4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
+  clear_pending_error();
+  return from_cuda(launch_moe_mx(v, x, T, topk_ids, topk_w, k, out, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 unsigned int tcf4_device_timeouts(void) {

@@ -101,6 +101,13 @@ struct MoeMmaWorkspace {
   size_t counters, hidden, y, bg_gu, bg_dn, maps, total;
 };
 bool moe_mma_supported(const tcf4_moe &m, int gu_seg, int dn_seg, int T);
+// Resident MXFP4 consumers (the tensor-core kernel reading nibble tiles): the views' stream fields
+// point at the nibble matrices [rows][cols/2]. Workspaces are the same as the trellis paths'.
+bool mx_gemv_supported(const MatView &w, int T);
+cudaError_t launch_mx_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s);
+bool moe_mx_supported(const tcf4_moe &m, int T);
+cudaError_t launch_moe_mx(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts, int k,
+                          uint16_t *out, void *ws, cudaStream_t s);
 MoeMmaWorkspace moe_mma_workspace_layout(const tcf4_moe &m, int T, int k);
 cudaError_t launch_moe_mma(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts, int k,
                            uint16_t *out, void *ws, cudaStream_t s);
