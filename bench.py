@@ -168,7 +168,8 @@ class Step:
         self.ws = torch.empty(self.M.workspace_bytes(T, K_TOP), dtype=torch.uint8, device=device)
         self.wsG = torch.empty(max(1, tc.gemv_workspace_bytes(self.G, T)), dtype=torch.uint8, device=device)
         self.wsD = torch.empty(max(1, tc.gemv_workspace_bytes(self.D, T)), dtype=torch.uint8, device=device)
-        self.launches_per_step = 2 + 1 + 4 + 2
+        # expansion 2, route 1, grouped MoE 4 (two splits, two products), GEMV 2 x (split + product)
+        self.launches_per_step = 2 + 1 + 4 + 4
         self.nG, self.nD = E * 2 * I * H, E * H * I
         self.moe_weights = K_TOP * (2 * I * H + H * I)  # distinct experts at T = 1: exactly k
         self.weights_per_step = self.nG + self.nD + self.moe_weights + self.nG + self.nD
@@ -205,6 +206,38 @@ class Step:
         mark("gemv_down")
         tc.gemv(self.D, self.xd[v], self.yD, self.wsD)
         mark("end")
+
+    # the next row beyond the step: products read straight from the resident MXFP4 tensors that the
+    # step's expansion calls wrote (HEPH serving mode 2, consumer side)
+    def mx_weights(self):
+        tc = self.tc
+        if not hasattr(self, "_mxG"):
+            self._mxG = tc.Mxfp4Matrix(self.nibG, self.scG, E * 2 * I, H)
+            self._mxD = tc.Mxfp4Matrix(self.nibD, self.scD, E * H, I)
+            ng, sg, nd, sd = self.nibG.view(E, -1), self.scG.view(E, -1), self.nibD.view(E, -1), self.scD.view(E, -1)
+            self._mxM = tc.Mxfp4MoEWeights([tc.Mxfp4Matrix(ng[e], sg[e], 2 * I, H) for e in range(E)],
+                                           [tc.Mxfp4Matrix(nd[e], sd[e], H, I) for e in range(E)], H, I)
+            self._mxws = torch.empty(max(1, self._mxM.workspace_bytes(T, K_TOP)), dtype=torch.uint8,
+                                     device=self.nibG.device)
+        return self._mxG, self._mxD, self._mxM
+
+    def run_mx(self, name, i):
+        tc = self.tc
+        G, D, M = self.mx_weights()
+        v = i % len(self.x)
+        if name == "mxfp4_gemv_gate_up":
+            tc.mxfp4_gemv(G, self.x[v], self.yG, self.wsG)
+        elif name == "mxfp4_gemv_down":
+            tc.mxfp4_gemv(D, self.xd[v], self.yD, self.wsD)
+        else:
+            tc.moe_route(self.logits[v], K_TOP, self.ids, self.wts)
+            tc.mxfp4_grouped_moe(M, self.x[v], self.ids, self.wts, self.out, self._mxws)
+
+    def mx_algo_bytes(self):
+        def gemv(rows, cols):
+            return rows * cols // 2 + rows * cols // 32 + 2 * cols * T + 2 * rows * T
+        return {"mxfp4_gemv_gate_up": gemv(E * 2 * I, H), "mxfp4_gemv_down": gemv(E * H, I),
+                "mxfp4_grouped_moe": K_TOP * (gemv(2 * I, H) + gemv(H, I))}
 
     # algorithmic bytes per call (what the method must move)
     def algo_bytes(self):
@@ -358,7 +391,7 @@ def reference_arm(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)  # ~0.3 s timed: several clock samples
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="tcf4", choices=["tcf4", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -457,6 +490,28 @@ def main():
                                      "six E2M1 terms per 32-block), fp32 accumulation"},
             "roofline": roofline, "kernels": kernels,
             "gpu_launches": step.launches_per_step * args.steps, "clocks": clocks}
+
+    # the next row (outside the step): products from the resident MXFP4 tensors, each call timed on
+    # its own with CUDA events after warm-up, inputs > L2 (the tensors are 423 MB)
+    mx = {}
+    for name, nbytes in step.mx_algo_bytes().items():
+        for i in range(3):
+            step.run_mx(name, i)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_mx = max(10, args.steps // 4)
+        e0.record()
+        for i in range(n_mx):
+            step.run_mx(name, i)
+        e1.record()
+        torch.cuda.synchronize()
+        us = 1e3 * e0.elapsed_time(e1) / n_mx
+        gbs = nbytes / (us * 1e-6) / 1e9
+        mx[name] = {"avg_us": round(us, 3), "algo_bytes": nbytes, "gb_s": round(gbs, 1),
+                    "frac_of_measured_hbm": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / 8000.0, 4),
+                    "calls": n_mx, "note": "includes route" if name == "mxfp4_grouped_moe" else ""}
+    line["next_rows"] = {"mxfp4_consumer": mx, "description": "products read straight from the resident MXFP4 "
+                         "tensors the step's expansion wrote (HEPH serving mode 2); outside the step and its value"}
 
     if rank == 0:
         line["e2e"] = run_e2e(step, args.e2e_steps, device)
