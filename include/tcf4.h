@@ -80,8 +80,9 @@ TCF4_API tcf4_status trellis_decode_to_mxfp4(tcf4_matrix w, uint8_t *out_nibbles
 /* HEPH abstract, first serving mode: fused decode + product.
  *   y[t][n] = bf16( sum_k w[n][k] * x[t][k] ), fp32 accumulation, round to nearest even.
  *   x: bf16 bits [T][cols]; y: bf16 bits [T][rows]; 1 <= T <= 32 (T == 0 is a no-op).
- * Two kernels behind one call: when seg_len == 32 and cols is a multiple of 64, the product runs on
- * the tensor cores (block-scaled MXFP4 x MXFP4 MMA: each 32-block of x is written as a sum of six
+ * Two kernels behind one call: when cols is a multiple of 64 (any seg_len; segments longer than a
+ * block carry the trellis state from block to block) and the scales are 2-byte aligned, the product
+ * runs on the tensor cores (block-scaled MXFP4 x MXFP4 MMA: each 32-block of x is written as a sum of six
  * E2M1 terms with their own UE8M0 scales, which leaves at most 5^-6 of the block's largest |x|
  * unrepresented) and needs `workspace`; otherwise it runs on CUDA cores and needs none.
  * trellis_gemv_workspace tells which (0 bytes = none needed).

@@ -86,6 +86,22 @@ def test_gemv_small(rows, cols, T):
         assert_products_close(y, y_exact, wn, xnorms(xb), f"{rows}x{cols} T={T} seg={seg}")
 
 
+@pytest.mark.parametrize("seg", [64, 96, 160, 288, 480, 2880])
+@pytest.mark.parametrize("T", [1, 6])
+def test_gemv_long_segments_on_tensor_cores(seg, T):
+    # K = 2880 (90 blocks): segments of 2, 3, 5, 9, 15 and 90 blocks start inside a decode thread's
+    # 8 blocks, at a thread's first block and across stages; 300 rows leave a ragged last tile
+    rows, cols = 300, 2880
+    st, sc, W = upload_matrix(rows, cols, seed=2500 + seg + T, seg_len=seg)
+    assert tc.gemv_workspace_bytes(W, T) > 0  # the tensor-core path takes it
+    x = synth.activations(T, cols, seed=2500 + T)
+    y = tc.gemv(W, x.cuda())
+    torch.cuda.synchronize()
+    xb = synth.bf16_bits(x)
+    y_exact, wn = oracle.gemv(st, sc, rows, cols, seg, xb)
+    assert_products_close(y, y_exact, wn, xnorms(xb), f"seg={seg} T={T}")
+
+
 @pytest.mark.parametrize("seg", [32, 2048])
 def test_gemv_2048_square_batch1(seg):
     rows = cols = 2048

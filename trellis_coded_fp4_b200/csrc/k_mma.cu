@@ -486,6 +486,8 @@ __device__ __forceinline__ void tmap_acquire(const void *gmap) {
 // ------------------------------------------------------------------------------- kernel arguments
 
 struct MmaArgs {
+  const uint2 *stream;    // GEMV: the matrix's stream words (MoE: from the table)
+  int seg_blocks;         // trellis segment length in 32-blocks (carry path: > 1)
   const uint8_t *scales;  // GEMV: the matrix's scales (MoE: from the table)
   int rows;               // GEMV rows
   int nbr;                // 32-blocks per row (K / 32)
@@ -517,7 +519,7 @@ __device__ __forceinline__ JobRows job_rows(const MmaArgs &a, const MoeTable<MAX
   JobRows j;
   if (MODE == kModeGemv) {
     const int r0 = job * 128;
-    j.st = nullptr;
+    j.st = a.stream;
     j.sc = a.scales;
     j.y0 = r0;
     j.y1 = r0 + 64;
@@ -572,7 +574,9 @@ __device__ __forceinline__ int tile_row(const JobRows &j, int m) {
 // MX: the weights are a resident MXFP4 tensor (nibbles [rows][K/2], scales [rows][K/32]) instead of a
 // trellis stream; the word loader then brings 128-byte-swizzled nibble tiles that the MMAs read as
 // the A operand straight from shared memory, and four scale-factor warps replace the decode warps.
-template <int MAXE, int MODE, int NMAX, bool MX>
+// CARRY: trellis segments longer than a block (seg_len = 32 * seg_blocks): each block's state
+// continues from the previous block of its segment.
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY>
 __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
                                                      const __grid_constant__ MoeTable<MAXE> tab,
                                                      const __grid_constant__ CUtensorMap wmap) {
@@ -772,9 +776,37 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
     // it; only a barrier found incomplete costs a blocking wait.
     uint32_t ws = 0, b = 0;
     bool ok = true, wf_ready = false;
+    // carry path: this thread's first block of the stage is block kKB s_c + kNBT h of its row, at
+    // position r_c of its segment (r_c = 0: a segment starts there); srow_w = the row's words
+    const int segb = CARRY ? a.seg_blocks : 1, seg_inc = CARRY ? kKB % segb : 0;
+    int s_c = 0, jl_c = 0, r_c = 0;
+    const uint2 *srow_w = nullptr;
 #pragma unroll 1
     for (int q = 0; q < nq; q++) {
       if (!wf_ready && !(ok = warp_wait(&w_full[ws], (uint32_t)(q / kNW) & 1u, tmo, abort_flag))) break;
+      uint32_t cL = 0u, cH = 0u, smask = 0xFFu;  // carry into the first block; blocks that start a segment
+      if constexpr (CARRY) {
+        if (s_c == 0) {
+          const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_c));
+          const int row = tile_row(jr, m);
+          srow_w = row >= 0 ? reinterpret_cast<const uint2 *>(jr.st) + (size_t)row * nbr : nullptr;
+          r_c = (kNBT * h) % segb;
+        }
+        smask = 0u;
+        for (int k = r_c == 0 ? 0 : segb - r_c; k < kNBT; k += segb) smask |= 1u << k;
+        if (r_c != 0) {
+          if (h > 0) {  // the block before this thread's range is in the same tile
+            const uint32_t byte = (uint32_t)(kNBT * h - 1) * 8u;
+            const uint2 v = lds_u2(wrow + ws * kWStage + (byte >> 7) * 8192u + ((((byte >> 4) & 7u) ^ sw) * 16u) + 8u);
+            cL = v.x;
+            cH = v.y;
+          } else if (srow_w != nullptr) {  // the previous stage's last block of the row
+            const uint2 v = __ldg(srow_w + (size_t)kKB * s_c - 1);
+            cL = v.x;
+            cH = v.y;
+          }
+        }
+      }
       uint32_t na[kNBT / 2], nb[kNG][C::kC];
       load_sf(na, nb);  // the next stage's scale factors; their latency hides behind this stage
       const uint32_t wa = wrow + ws * kWStage;
@@ -790,12 +822,23 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         if (ch == 0 && q >= kNA) ae = mbar_test(&a_empty[2 * b + hf], (uint32_t)((q - kNA) / kNA) & 1u);
         if (ch == C::kNCh - 1 && q + 1 < nq) wf = mbar_test(&w_full[ws1], (uint32_t)((q + 1) / kNW) & 1u);
         uint32_t W[8][4];
+        if constexpr (CARRY) {
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-          planes_to_nibbles_interleaved(decode_block0(cw[i].x, cw[i].y), W[2 * i][0], W[2 * i][1], W[2 * i][2],
-                                        W[2 * i][3]);
-          planes_to_nibbles_interleaved(decode_block0(cw[i].z, cw[i].w), W[2 * i + 1][0], W[2 * i + 1][1],
-                                        W[2 * i + 1][2], W[2 * i + 1][3]);
+          for (int i = 0; i < 8; i++) {
+            const uint32_t L = (i & 1) ? cw[i >> 1].z : cw[i >> 1].x, Hh = (i & 1) ? cw[i >> 1].w : cw[i >> 1].y;
+            if ((smask >> i) & 1u) cL = cH = 0u;
+            planes_to_nibbles_interleaved(decode_block(L, Hh, cL, cH), W[i][0], W[i][1], W[i][2], W[i][3]);
+            cL = L;
+            cH = Hh;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            planes_to_nibbles_interleaved(decode_block0(cw[i].x, cw[i].y), W[2 * i][0], W[2 * i][1], W[2 * i][2],
+                                          W[2 * i][3]);
+            planes_to_nibbles_interleaved(decode_block0(cw[i].z, cw[i].w), W[2 * i + 1][0], W[2 * i + 1][1],
+                                          W[2 * i + 1][2], W[2 * i + 1][3]);
+          }
         }
         if (ch == C::kNCh - 1) {  // every word of the stage has been read (and used): free the slot
           __syncwarp();
@@ -834,6 +877,14 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
 #pragma unroll
         for (int c = 0; c < C::kC; c++) pb[g][c] = nb[g][c];
       b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
+      if constexpr (CARRY) {
+        r_c += seg_inc;
+        if (r_c >= segb) r_c -= segb;
+        if (++s_c == S) {
+          s_c = 0;
+          jl_c++;
+        }
+      }
     }
     if (!ok) *abort_flag = 1;
   } else if (warp == C::kWLoadWarp) {
@@ -1206,6 +1257,27 @@ static int sm_count() {
   return nsm;
 }
 
+// One launch of a product kernel instance (dynamic shared memory attribute set once per instance).
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY>
+static cudaError_t launch_product(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
+                                  cudaStream_t s) {
+  static unsigned long long attr = 0;
+  cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, MODE, NMAX, MX, CARRY>, attr);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(k_mma<MAXE, MODE, NMAX, MX, CARRY>, dim3(grid), dim3(Cfg<NMAX>::kThreads),
+                          mma_geom<NMAX>(MODE, MX).smem, s, args, tab, map);
+}
+template <int MAXE, int MODE, int NMAX, bool MX>
+static cudaError_t launch_product_seg(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
+                                      cudaStream_t s) {
+  if constexpr (MX) {
+    return launch_product<MAXE, MODE, NMAX, true, false>(grid, args, tab, map, s);
+  } else {
+    return args.seg_blocks > 1 ? launch_product<MAXE, MODE, NMAX, false, true>(grid, args, tab, map, s)
+                               : launch_product<MAXE, MODE, NMAX, false, false>(grid, args, tab, map, s);
+  }
+}
+
 template <int NMAX, bool MX>
 static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, const uint16_t *x, int T, uint16_t *y,
                                     void *ws, cudaStream_t s) {
@@ -1214,11 +1286,10 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
   cudaError_t e =
       launch_dependent(k_bsplit_gemv<NMAX, MX>, dim3((warps + 7) / 8), dim3(256), 0, s, x, T, w.nbr * 32, terms);
   if (e != cudaSuccess) return e;
-  static unsigned long long attr = 0;
-  e = ensure_max_dynamic_smem(k_mma<32, kModeGemv, NMAX, MX>, attr);
-  if (e != cudaSuccess) return e;
   const int ntiles = (w.rows + 127) / 128, nsm = sm_count();
   MmaArgs args{};
+  args.stream = w.stream;
+  args.seg_blocks = MX ? 1 : w.seg_blocks;
   args.scales = w.scales;
   args.rows = w.rows;
   args.nbr = w.nbr;
@@ -1226,8 +1297,7 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
   args.T = T;
   args.y = y;
   MoeTable<32> none{};
-  return launch_dependent(k_mma<32, kModeGemv, NMAX, MX>, dim3(ntiles < nsm ? ntiles : nsm), dim3(Cfg<NMAX>::kThreads),
-                          mma_geom<NMAX>(kModeGemv, MX).smem, s, args, none, map);
+  return launch_product_seg<32, kModeGemv, NMAX, MX>(ntiles < nsm ? ntiles : nsm, args, none, map, s);
 }
 
 template <bool MX>
@@ -1258,7 +1328,8 @@ cudaError_t launch_mx_gemv(const MatView &w, const uint16_t *x, int T, uint16_t 
 static int moe_groups_max(int E, int P, int gmax) { return (E < P ? E : P) + P / gmax + 1; }
 
 bool moe_mma_supported(const tcf4_moe &m, int gu_seg, int dn_seg, int T) {
-  if (gu_seg != 1 || dn_seg != 1) return false;
+  (void)gu_seg;  // any segment length: blocks after a segment's first carry the state (CARRY)
+  (void)dn_seg;
   if (!k_ok(m.H / 32) || !k_ok(m.I / 32) || tensor_map_encoder() == nullptr) return false;
   for (int e = 0; e < m.E; e++)
     if (((reinterpret_cast<uintptr_t>(m.gate_up[e].stream) | reinterpret_cast<uintptr_t>(m.down[e].stream)) & 15u) ||
@@ -1339,14 +1410,11 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
                                      dim3(256), 0, s, ids, P, m.E, k, x, m.H, terms, args.counters,
                                      4 * ((m.H + 127) / 128));
     if (e != cudaSuccess) return e;
-    static unsigned long long attr = 0;
-    e = ensure_max_dynamic_smem(k_mma<MAXE, kModeGateUp, NMAX, MX>, attr);
-    if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
+    args.seg_blocks = MX ? 1 : (int)(m.gate_up[0].seg_len / 32);
     const int jobs = G * ((m.I + 63) / 64);
-    e = launch_dependent(k_mma<MAXE, kModeGateUp, NMAX, MX>, dim3(jobs < nsm ? jobs : nsm), dim3(Cfg<NMAX>::kThreads),
-                         mma_geom<NMAX>(kModeGateUp, MX).smem, s, args, tab, map_gu);
+    e = launch_product_seg<MAXE, kModeGateUp, NMAX, MX>(jobs < nsm ? jobs : nsm, args, tab, map_gu, s);
     if (e != cudaSuccess) return e;
   }
   // down: split h per group, then decode + MMA, y to the workspace, last arriver per chunk combines
@@ -1358,15 +1426,12 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
                                      dim3(256), 0, s, ids, P, m.E, 1, (const uint16_t *)args.hidden, m.I, terms,
                                      (int *)nullptr, 0);
     if (e != cudaSuccess) return e;
-    static unsigned long long attr = 0;
-    e = ensure_max_dynamic_smem(k_mma<MAXE, kModeDown, NMAX, MX>, attr);
-    if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
+    args.seg_blocks = MX ? 1 : (int)(m.down[0].seg_len / 32);
     args.maps += (size_t)nsm * kMapSlots * 128;  // the down kernel's own tensor-map slots
     const int jobs = G * ((m.H + 127) / 128);
-    e = launch_dependent(k_mma<MAXE, kModeDown, NMAX, MX>, dim3(jobs < nsm ? jobs : nsm), dim3(Cfg<NMAX>::kThreads),
-                         mma_geom<NMAX>(kModeDown, MX).smem, s, args, tab, map_dn);
+    e = launch_product_seg<MAXE, kModeDown, NMAX, MX>(jobs < nsm ? jobs : nsm, args, tab, map_dn, s);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();

@@ -110,10 +110,10 @@ static tcf4_status check_gemv(const tcf4_matrix &w, int32_t T) {
   return TCF4_OK;
 }
 
-// The tensor-core path runs whenever it applies (seg_len 32, see gemv_mma_supported); it needs
+// The tensor-core path runs whenever it applies (any seg_len; see gemv_mma_supported); it needs
 // the workspace for the activation split. Other shapes run the CUDA-core kernel without one.
 static bool gemv_uses_mma(const tcf4_matrix &w, int32_t T) {
-  return w.seg_len == 32 && w.rows > 0 && T > 0 && gemv_mma_supported(view(w), T);
+  return w.rows > 0 && T > 0 && gemv_mma_supported(view(w), T);
 }
 
 size_t trellis_gemv_workspace(tcf4_matrix w, int32_t T) {
