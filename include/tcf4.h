@@ -203,6 +203,30 @@ TCF4_API tcf4_status mxfp4_grouped_moe(const tcf4_mxfp4_moe *m, const uint16_t *
                                        const int32_t *topk_ids, const float *topk_w, int32_t k, uint16_t *out,
                                        void *workspace, size_t ws_bytes, void *stream);
 
+/* ------------------------------------------------------------------------------------------------
+ * The upstream (offline) step: "XOR-Trellis: Hadamard-free FP4 LLM quantization" news page, bullet
+ * "Curvature-aware Viterbi objective". Each segment of seg_len weights of a row is encoded as the
+ * trellis path, starting in state 0 and ending in any state, that minimises
+ *   sum_k D[k] * (target[k] - value_k * 2^(E_k - 127))^2
+ * where value_k is the palette value of the state after symbol k (the decoder of trellis_gemv) and
+ * E_k the UE8M0 scale byte of weight k's 32-block (chosen by the caller, e.g. the grid-aligned
+ * convention: the block's own MXFP4 exponent). The sum is evaluated in fp64, term by term in that
+ * order with no fused operations. Among equal-cost paths the lower predecessor window (the 7
+ * previous symbols read as a number, newest symbol in the top bits) wins at each step, and the
+ * lowest final window at the end.
+ *   target, D:  fp64 [rows][cols], device.       scales: uint8 [rows][cols/32], device.
+ *   stream_out: uint32 [rows][cols/32][2] planar words (the layout of tcf4_matrix.stream), device.
+ *   cost_out:   fp64 [rows][cols/seg_len], the minimum of each segment, device (may be NULL).
+ *   workspace:  device scratch; trellis_encode_workspace(rows, cols, seg_len) bytes run one segment
+ *               per SM at a time, fewer bytes (at least seg_len * 4 KiB) fewer segments. 256-byte
+ *               aligned, owned by the caller.
+ * Compute-bound: 2^16 candidate paths per weight. Limits: cols a multiple of 32, seg_len a
+ * multiple of 32 dividing cols, rows * cols < 2^31. */
+TCF4_API size_t trellis_encode_workspace(int64_t rows, int64_t cols, int32_t seg_len);
+TCF4_API tcf4_status trellis_encode(const double *target, const double *D, const uint8_t *scales, int64_t rows,
+                                    int64_t cols, int32_t seg_len, uint32_t *stream_out, double *cost_out,
+                                    void *workspace, size_t ws_bytes, void *stream);
+
 /* Bounded waits that gave up inside the library's kernels since the last call, then resets the
  * count. Kernels that stage weights with bulk copies wait on shared-memory barriers with an
  * iteration limit; a wait that runs out is counted and the affected outputs are invalid. Never

@@ -210,6 +210,25 @@ def mxfp4_grouped_moe(m: Mxfp4MoEWeights, x: torch.Tensor, ids: torch.Tensor, wt
     return out, workspace
 
 
+def encode_workspace_bytes(rows: int, cols: int, seg_len: int) -> int:
+    return int(_abi.load().trellis_encode_workspace(rows, cols, seg_len))
+
+
+def encode(target: torch.Tensor, D: torch.Tensor, scales: torch.Tensor, seg_len: int = 32, workspace=None):
+    """D-weighted Viterbi encoding of fp64 target [rows][cols] under UE8M0 block scales [rows][cols/32]:
+    returns (a TrellisMatrix holding the stream and those scales, per-segment minimum costs fp64)."""
+    rows, cols = target.shape
+    st = torch.empty(rows * (cols // 32) * 2, dtype=torch.int32, device=target.device)
+    cost = torch.empty((rows, cols // seg_len), dtype=torch.float64, device=target.device)
+    if workspace is None:
+        workspace = torch.empty(max(encode_workspace_bytes(rows, cols, seg_len), 1), dtype=torch.uint8,
+                                device=target.device)
+    _abi.check(_abi.load().trellis_encode(_ptr(target), _ptr(D), _ptr(scales), rows, cols, seg_len, _ptr(st),
+                                          _ptr(cost), _ptr(workspace), workspace.numel(), _stream_handle()),
+               "trellis_encode")
+    return TrellisMatrix(st, scales.reshape(-1), rows, cols, seg_len), cost
+
+
 def moe_workspace_bytes(m: MoEWeights, T: int, k: int) -> int:
     return m.workspace_bytes(T, k)
 

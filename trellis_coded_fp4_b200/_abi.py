@@ -14,6 +14,7 @@ EXPORTED = ("trellis_decode_to_mxfp4", "trellis_gemv_workspace", "trellis_gemv",
             "trellis_moe_route", "trellis_grouped_moe_workspace",
             "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "mxfp4_gemv_workspace", "mxfp4_gemv",
             "mxfp4_grouped_moe_workspace", "mxfp4_grouped_moe_hidden_offset", "mxfp4_grouped_moe",
+            "trellis_encode_workspace", "trellis_encode",
             "tcf4_device_timeouts", "tcf4_status_string")
 
 
@@ -80,6 +81,10 @@ def load(path: str = LIB_PATH):
     L.mxfp4_grouped_moe_hidden_offset.restype = sz
     L.mxfp4_grouped_moe.argtypes = [ctypes.POINTER(Mxfp4Moe), vp, i32, vp, vp, i32, vp, vp, sz, vp]
     L.mxfp4_grouped_moe.restype = ctypes.c_int
+    L.trellis_encode_workspace.argtypes = [i64, i64, i32]
+    L.trellis_encode_workspace.restype = sz
+    L.trellis_encode.argtypes = [vp, vp, vp, i64, i64, i32, vp, vp, vp, sz, vp]
+    L.trellis_encode.restype = ctypes.c_int
     L.tcf4_device_timeouts.argtypes = []
     L.tcf4_device_timeouts.restype = ctypes.c_uint
     L.tcf4_status_string.argtypes = [ctypes.c_int]

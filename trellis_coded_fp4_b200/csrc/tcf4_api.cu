@@ -286,6 +286,36 @@ tcf4_status mxfp4_grouped_moe(const tcf4_mxfp4_moe *m, const uint16_t *x, int32_
   return from_cuda(launch_moe_mx(v, x, T, topk_ids, topk_w, k, out, workspace, static_cast<cudaStream_t>(stream)));
 }
 
+static tcf4_status check_encode(int64_t rows, int64_t cols, int32_t seg_len) {
+  if (rows < 0 || cols < 0 || cols % 32 != 0) return TCF4_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return TCF4_OK;
+  if (seg_len <= 0 || seg_len % 32 != 0 || cols % seg_len != 0) return TCF4_ERR_INVALID_ARG;
+  if (rows * cols >= ((int64_t)1 << 31)) return TCF4_ERR_UNSUPPORTED;
+  return TCF4_OK;
+}
+
+size_t trellis_encode_workspace(int64_t rows, int64_t cols, int32_t seg_len) {
+  if (check_encode(rows, cols, seg_len) != TCF4_OK || rows == 0 || cols == 0) return 0;
+  return encode_workspace((int)rows, (int)cols, seg_len);
+}
+
+tcf4_status trellis_encode(const double *target, const double *D, const uint8_t *scales, int64_t rows, int64_t cols,
+                           int32_t seg_len, uint32_t *stream_out, double *cost_out, void *workspace, size_t ws_bytes,
+                           void *stream) {
+  tcf4_status st = check_encode(rows, cols, seg_len);
+  if (st != TCF4_OK) return st;
+  if (rows == 0 || cols == 0) return TCF4_OK;
+  if (target == nullptr || D == nullptr || scales == nullptr || stream_out == nullptr) return TCF4_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(target) | reinterpret_cast<uintptr_t>(D)) & 7u) return TCF4_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(stream_out) & 7u) || (reinterpret_cast<uintptr_t>(cost_out) & 7u))
+    return TCF4_ERR_MISALIGNED;
+  if (workspace == nullptr || ws_bytes < encode_cta_bytes(seg_len)) return TCF4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
+  clear_pending_error();
+  return from_cuda(launch_encode(target, D, scales, (int)rows, (int)cols, seg_len, stream_out, cost_out, workspace,
+                                 ws_bytes, static_cast<cudaStream_t>(stream)));
+}
+
 unsigned int tcf4_device_timeouts(void) {
   cudaDeviceSynchronize();
   return take_timeouts_gemv() + take_timeouts_moe() + take_timeouts_mma();

@@ -101,6 +101,12 @@ struct MoeMmaWorkspace {
   size_t counters, hidden, y, bg_gu, bg_dn, maps, total;
 };
 bool moe_mma_supported(const tcf4_moe &m, int gu_seg, int dn_seg, int T);
+// D-weighted Viterbi encoder (k_encode.cu): back-pointer bytes of one CTA, the workspace for one
+// segment per SM, and the launch (as many concurrent segments as ws_bytes holds, at most one per SM).
+size_t encode_cta_bytes(int seg);
+size_t encode_workspace(int rows, int cols, int seg);
+cudaError_t launch_encode(const double *target, const double *D, const uint8_t *scales, int rows, int cols, int seg,
+                          uint32_t *out_stream, double *out_cost, void *ws, size_t ws_bytes, cudaStream_t s);
 // Resident MXFP4 consumers (the tensor-core kernel reading nibble tiles): the views' stream fields
 // point at the nibble matrices [rows][cols/2]. Workspaces are the same as the trellis paths'.
 bool mx_gemv_supported(const MatView &w, int T);
