@@ -14,7 +14,7 @@
 //  * the E2M1 code of the full 16-bit state (window, new symbol) is fixed per window: each thread
 //    derives its 64 codes once from the decoder (bit 7 of the planes of a block whose first eight
 //    symbols are the state), and each step needs only the 16 distortions D_k (t_k - v_c s_k)^2, one
-//    per E2M1 code c, computed by 16 threads;
+//    per E2M1 code c, computed for 256 steps at a time by all threads;
 //  * the chosen predecessor of every new window (2 bits) goes to a per-CTA workspace in global
 //    memory (4 KB per step); after the last step one thread walks the path back from the cheapest
 //    final window (lowest index on ties) and writes the planar stream words.
@@ -33,10 +33,10 @@ namespace tcf4 {
 
 constexpr int kEncThreads = 1024;
 constexpr int kWindows = 1 << 14;
-constexpr int kEncChunk = 512;  // steps whose (target, D) pairs are staged in shared memory at a time
-// shared memory: costs | 16 distortions | staged (target, D) pairs | codes of every thread's groups |
+constexpr int kEncChunk = 256;  // steps whose 16 distortions are computed ahead, all at once
+// shared memory: costs | distortions of a chunk [step][E2M1 code] | codes of every thread's groups |
 // reduction scratch
-constexpr size_t kEncSmem = sizeof(double) * kWindows + sizeof(double) * 16 + sizeof(double2) * kEncChunk +
+constexpr size_t kEncSmem = sizeof(double) * kWindows + sizeof(double) * 16 * kEncChunk +
                             sizeof(uint64_t) * 4 * kEncThreads + 1024;
 
 // E2M1 code of the state s (symbol m of the window at bits 2m, 2m+1; the newest at bits 14-15):
@@ -65,9 +65,8 @@ __global__ void __launch_bounds__(kEncThreads, 1)
              uint32_t *__restrict__ back) {
   extern __shared__ __align__(16) unsigned char smem[];
   double *cost = reinterpret_cast<double *>(smem);
-  double *dist = cost + kWindows;
-  double2 *td = reinterpret_cast<double2 *>(dist + 16);
-  uint64_t *codes_s = reinterpret_cast<uint64_t *>(td + kEncChunk);  // [4][1024]
+  double *dist = cost + kWindows;                                       // [kEncChunk][16]
+  uint64_t *codes_s = reinterpret_cast<uint64_t *>(dist + 16 * kEncChunk);  // [4][1024]
   double *red_c = reinterpret_cast<double *>(codes_s + 4 * kEncThreads);  // 32 warp minima
   int *red_w = reinterpret_cast<int *>(red_c + 32);
   grid_dep_wait();  // the inputs may come from, and the outputs still be read by, preceding kernels
@@ -92,20 +91,19 @@ __global__ void __launch_bounds__(kEncThreads, 1)
     for (int w = t; w < kWindows; w += kEncThreads) cost[w] = w == 0 ? 0.0 : INFINITY;
     for (int kc = 0; kc < seg; kc += kEncChunk) {
       const int n = seg - kc < kEncChunk ? seg - kc : kEncChunk;
-      __syncthreads();  // the previous chunk's pairs are no longer read
-      for (int j = t; j < n; j += kEncThreads) {
-        const size_t at = (size_t)row * cols + k0 + kc + j;
-        td[j] = make_double2(target[at], Dw[at]);
+      __syncthreads();  // the previous chunk's distortions are no longer read
+      for (int j = t; j < 16 * n; j += kEncThreads) {
+        const int kk = j >> 4, c = j & 15, k = k0 + kc + kk;
+        const size_t at = (size_t)row * cols + k;
+        const uint32_t E = scales[(size_t)row * nbr + k / 32];
+        const double sc = E == 255u ? __longlong_as_double(0x7FF8000000000000ll) : ldexp(1.0, (int)E - 127);
+        const double d = __dsub_rn(target[at], __dmul_rn(e2m1_f64((uint32_t)c), sc));
+        dist[j] = __dmul_rn(__dmul_rn(Dw[at], d), d);
       }
       for (int kk = 0; kk < n; kk++) {
         const int k = k0 + kc + kk;
-        __syncthreads();  // pairs staged; the previous step's costs written
-        if (t < 16) {
-          const uint32_t E = scales[(size_t)row * nbr + k / 32];
-          const double sc = E == 255u ? __longlong_as_double(0x7FF8000000000000ll) : ldexp(1.0, (int)E - 127);
-          const double d = __dsub_rn(td[kk].x, __dmul_rn(e2m1_f64((uint32_t)t), sc));
-          dist[t] = __dmul_rn(__dmul_rn(td[kk].y, d), d);
-        }
+        const double *dk = dist + 16 * kk;
+        __syncthreads();  // distortions ready; the previous step's costs written
         double oc[4][4];
 #pragma unroll
         for (int i = 0; i < 4; i++) {
@@ -116,7 +114,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
           oc[i][2] = v1.x;
           oc[i][3] = v1.y;
         }
-        __syncthreads();  // every old cost read, the distortions written
+        __syncthreads();  // every old cost read
         uint32_t bp = 0;
 #pragma unroll
         for (int i = 0; i < 4; i++) {
@@ -128,7 +126,7 @@ __global__ void __launch_bounds__(kEncThreads, 1)
             uint32_t br = 0;
 #pragma unroll
             for (int r = 0; r < 4; r++) {  // predecessors in increasing order: the first minimum wins
-              const double c = __dadd_rn(oc[i][r], dist[(codes >> (4 * (4 * b + r))) & 15u]);
+              const double c = __dadd_rn(oc[i][r], dk[(codes >> (4 * (4 * b + r))) & 15u]);
               if (c < best) {
                 best = c;
                 br = (uint32_t)r;
