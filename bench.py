@@ -510,8 +510,29 @@ def main():
         mx[name] = {"avg_us": round(us, 3), "algo_bytes": nbytes, "gb_s": round(gbs, 1),
                     "frac_of_measured_hbm": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / 8000.0, 4),
                     "calls": n_mx, "note": "includes route" if name == "mxfp4_grouped_moe" else ""}
-    line["next_rows"] = {"mxfp4_consumer": mx, "description": "products read straight from the resident MXFP4 "
-                         "tensors the step's expansion wrote (HEPH serving mode 2); outside the step and its value"}
+    # the upstream encoder (D-weighted Viterbi): 296 rows of the gate_up matrix re-encoded from their
+    # decoded values with random D, segments of 32 weights; compute-bound, timed over 3 calls
+    enc_rows, enc_cols = 296, H
+    gen = torch.Generator(device=device).manual_seed(seed)
+    et = torch.randn(enc_rows, enc_cols, dtype=torch.float64, device=device, generator=gen)
+    eD = torch.rand(enc_rows, enc_cols, dtype=torch.float64, device=device, generator=gen) + 0.1
+    esc = step.G.scales[: enc_rows * (enc_cols // 32)]
+    step.tc.encode(et, eD, esc, 32)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(3):
+        step.tc.encode(et, eD, esc, 32)
+    e1.record()
+    torch.cuda.synchronize()
+    enc_ms = e0.elapsed_time(e1) / 3
+    encoder = {"ms_per_call": round(enc_ms, 3), "weights": enc_rows * enc_cols, "seg_len": 32,
+               "weights_per_s": enc_rows * enc_cols / (enc_ms * 1e-3), "bound": "alu",
+               "note": "2^16 candidate paths per weight, fp64 costs evaluated exactly (no fused operations)"}
+    line["next_rows"] = {"mxfp4_consumer": mx, "encoder": encoder,
+                         "description": "products read straight from the resident MXFP4 tensors the step's "
+                         "expansion wrote (HEPH serving mode 2), and the D-weighted Viterbi encoder; outside "
+                         "the step and its value"}
 
     if rank == 0:
         line["e2e"] = run_e2e(step, args.e2e_steps, device)
