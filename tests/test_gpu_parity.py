@@ -51,6 +51,20 @@ def test_expand_unaligned_scale_pointers():
     assert (out_sc.cpu().numpy().reshape(rows, -1) == ref_sc).all()
 
 
+def test_expand_output_16_byte_aligned_only():
+    # an output 16 bytes past a 32-byte boundary takes the 16-byte stores instead of the 32-byte ones
+    rows, cols = 9, 2880
+    st, sc, W = upload_matrix(rows, cols, seed=78)
+    buf = torch.zeros(rows * cols // 2 + 32, dtype=torch.uint8, device="cuda")
+    assert buf.data_ptr() % 32 == 0
+    out = buf[16:16 + rows * cols // 2].view(rows, cols // 2)
+    nib, osc = tc.decode_to_mxfp4(W, out_nibbles=out)
+    torch.cuda.synchronize()
+    ref_nib, ref_sc = oracle.expand_mxfp4(st, sc, rows, cols, 32)
+    assert (nib.cpu().numpy() == ref_nib).all() and (osc.cpu().numpy() == ref_sc).all()
+    assert (buf[:16].cpu().numpy() == 0).all() and (buf[16 + rows * cols // 2:].cpu().numpy() == 0).all()
+
+
 def test_expand_full_moe_layer_sampled():
     # The 32-expert, hidden-2880 layer (gate_up 32x5760x2880, down 32x2880x2880) in the launch
     # configuration the bench times: one call per kind; sampled rows checked bit-exactly, scales

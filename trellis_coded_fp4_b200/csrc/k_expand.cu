@@ -26,11 +26,19 @@ __device__ __forceinline__ void st_stream(uint4 *p, uint4 v) {
                : "memory");
 }
 
+// One 32-byte streaming store (both blocks of a pair; p 32-byte aligned).
+__device__ __forceinline__ void st_stream2(uint4 *p, uint4 a, uint4 b) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w),
+               "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
 // SEG32: every block starts a segment (state 0), so no carry between blocks. PT: pairs per thread;
 // a CTA covers 256 * PT consecutive pairs, thread t the pairs t, t + 256, ... of them (each round
 // coalesced across the warp), and issues all its PT loads before it decodes, so that enough bytes
 // are in flight per SM to cover the memory latency.
-template <bool SEG32, int PT>
+// V8: the output is 32-byte aligned, so a pair's two blocks go out as one 32-byte store.
+template <bool SEG32, int PT, bool V8>
 __global__ void __launch_bounds__(256) k_expand(const uint2 *__restrict__ stream, uint32_t nblocks,
                                                 uint32_t blocks_per_row, uint32_t seg_blocks,
                                                 uint4 *__restrict__ out, const uint8_t *__restrict__ scales,
@@ -62,10 +70,16 @@ __global__ void __launch_bounds__(256) k_expand(const uint2 *__restrict__ stream
     if (SEG32) {
       if (valid) {
         planes_to_nibbles_natural(decode_block0(v[j].x, v[j].y), o.x, o.y, o.z, o.w);
-        st_stream(out + g0, o);
-        if (has2) {
-          planes_to_nibbles_natural(decode_block0(v[j].z, v[j].w), o.x, o.y, o.z, o.w);
-          st_stream(out + g0 + 1u, o);
+        if (V8 && has2) {
+          uint4 o2;
+          planes_to_nibbles_natural(decode_block0(v[j].z, v[j].w), o2.x, o2.y, o2.z, o2.w);
+          st_stream2(out + g0, o, o2);
+        } else {
+          st_stream(out + g0, o);
+          if (has2) {
+            planes_to_nibbles_natural(decode_block0(v[j].z, v[j].w), o.x, o.y, o.z, o.w);
+            st_stream(out + g0 + 1u, o);
+          }
         }
       }
     } else {
@@ -116,11 +130,14 @@ cudaError_t launch_expand(const MatView &w, uint8_t *out_nibbles, uint8_t *out_s
   const uint32_t npairs = (nblocks + 1u) / 2u;
   const uint32_t grid = (npairs + 256u * kExpandPairs - 1u) / (256u * kExpandPairs);
   auto *out = reinterpret_cast<uint4 *>(out_nibbles);
+  const bool out32 = (reinterpret_cast<uintptr_t>(out_nibbles) & 31u) == 0;
   if (w.seg_blocks == 1) {
-    return launch_dependent(k_expand<true, kExpandPairs>, dim3(grid), dim3(256), 0, s, w.stream, nblocks,
-                            (uint32_t)w.nbr, 1u, out, w.scales, out_scales, aligned ? 1 : 0);
+    return out32 ? launch_dependent(k_expand<true, kExpandPairs, true>, dim3(grid), dim3(256), 0, s, w.stream, nblocks,
+                                    (uint32_t)w.nbr, 1u, out, w.scales, out_scales, aligned ? 1 : 0)
+                 : launch_dependent(k_expand<true, kExpandPairs, false>, dim3(grid), dim3(256), 0, s, w.stream, nblocks,
+                                    (uint32_t)w.nbr, 1u, out, w.scales, out_scales, aligned ? 1 : 0);
   } else {
-    return launch_dependent(k_expand<false, kExpandPairs>, dim3(grid), dim3(256), 0, s, w.stream, nblocks,
+    return launch_dependent(k_expand<false, kExpandPairs, false>, dim3(grid), dim3(256), 0, s, w.stream, nblocks,
                             (uint32_t)w.nbr, (uint32_t)w.seg_blocks, out, w.scales, out_scales, aligned ? 1 : 0);
   }
 }
