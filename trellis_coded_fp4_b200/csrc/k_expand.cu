@@ -26,6 +26,13 @@ __device__ __forceinline__ void st_stream(uint4 *p, uint4 v) {
                : "memory");
 }
 
+// One 32-byte non-allocating load (four blocks of words; p 32-byte aligned).
+__device__ __forceinline__ void ld_stream2(const uint4 *p, uint4 &a, uint4 &b) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+               : "l"(p));
+}
+
 // One 32-byte streaming store (both blocks of a pair; p 32-byte aligned).
 __device__ __forceinline__ void st_stream2(uint4 *p, uint4 a, uint4 b) {
   asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w),
@@ -124,6 +131,38 @@ __global__ void __launch_bounds__(256) k_expand(const uint2 *__restrict__ stream
 // 184320 x 2880 gate_up matrix: 77.3 us with one pair, 77.5 with two, 82.5 with four).
 constexpr int kExpandPairs = 1;
 
+// Segments of one block with 32-byte aligned stream and output: a thread takes four consecutive
+// blocks, one 32-byte load and two 32-byte stores (the last partial quad block by block).
+__global__ void __launch_bounds__(256) k_expand_q(const uint2 *__restrict__ stream, uint32_t nblocks,
+                                                  uint4 *__restrict__ out, const uint8_t *__restrict__ scales,
+                                                  uint8_t *__restrict__ out_scales, int scales_aligned16) {
+  grid_dep_wait();  // out may still be read by the preceding kernel
+  grid_dep_release();
+  const uint32_t g0 = 4u * (blockIdx.x * 256u + threadIdx.x);
+  if (g0 + 3u < nblocks) {
+    uint4 a, b, o0, o1;
+    ld_stream2(reinterpret_cast<const uint4 *>(stream + g0), a, b);
+    planes_to_nibbles_natural(decode_block0(a.x, a.y), o0.x, o0.y, o0.z, o0.w);
+    planes_to_nibbles_natural(decode_block0(a.z, a.w), o1.x, o1.y, o1.z, o1.w);
+    st_stream2(out + g0, o0, o1);
+    planes_to_nibbles_natural(decode_block0(b.x, b.y), o0.x, o0.y, o0.z, o0.w);
+    planes_to_nibbles_natural(decode_block0(b.z, b.w), o1.x, o1.y, o1.z, o1.w);
+    st_stream2(out + g0 + 2u, o0, o1);
+  } else {
+    for (uint32_t g = g0; g < nblocks; g++) {
+      const uint2 t = stream[g];
+      uint4 o;
+      planes_to_nibbles_natural(decode_block0(t.x, t.y), o.x, o.y, o.z, o.w);
+      st_stream(out + g, o);
+    }
+  }
+  const uint32_t tg = blockIdx.x * 256u + threadIdx.x, nth = gridDim.x * 256u;
+  const uint32_t nchunk = scales_aligned16 ? nblocks >> 4 : 0u;
+  for (uint32_t c = tg; c < nchunk; c += nth)
+    reinterpret_cast<uint4 *>(out_scales)[c] = reinterpret_cast<const uint4 *>(scales)[c];
+  for (uint32_t b = (nchunk << 4) + tg; b < nblocks; b += nth) out_scales[b] = scales[b];
+}
+
 cudaError_t launch_expand(const MatView &w, uint8_t *out_nibbles, uint8_t *out_scales, cudaStream_t s) {
   const uint32_t nblocks = (uint32_t)((int64_t)w.rows * w.nbr);
   const bool aligned = ((reinterpret_cast<uintptr_t>(w.scales) | reinterpret_cast<uintptr_t>(out_scales)) & 15u) == 0;
@@ -131,6 +170,9 @@ cudaError_t launch_expand(const MatView &w, uint8_t *out_nibbles, uint8_t *out_s
   const uint32_t grid = (npairs + 256u * kExpandPairs - 1u) / (256u * kExpandPairs);
   auto *out = reinterpret_cast<uint4 *>(out_nibbles);
   const bool out32 = (reinterpret_cast<uintptr_t>(out_nibbles) & 31u) == 0;
+  if (w.seg_blocks == 1 && out32 && (reinterpret_cast<uintptr_t>(w.stream) & 31u) == 0)
+    return launch_dependent(k_expand_q, dim3((nblocks + 1023u) / 1024u), dim3(256), 0, s, w.stream, nblocks, out,
+                            w.scales, out_scales, aligned ? 1 : 0);
   if (w.seg_blocks == 1) {
     return out32 ? launch_dependent(k_expand<true, kExpandPairs, true>, dim3(grid), dim3(256), 0, s, w.stream, nblocks,
                                     (uint32_t)w.nbr, 1u, out, w.scales, out_scales, aligned ? 1 : 0)
