@@ -168,8 +168,9 @@ class Step:
         self.ws = torch.empty(self.M.workspace_bytes(T, K_TOP), dtype=torch.uint8, device=device)
         self.wsG = torch.empty(max(1, tc.gemv_workspace_bytes(self.G, T)), dtype=torch.uint8, device=device)
         self.wsD = torch.empty(max(1, tc.gemv_workspace_bytes(self.D, T)), dtype=torch.uint8, device=device)
-        # expansion 2, route 1, grouped MoE 4 (two splits, two products), GEMV 2 x (split + product)
-        self.launches_per_step = 2 + 1 + 4 + 4
+        # expansion 2, route 1, grouped MoE 3 (the split of x, gate/up whose epilogue also splits h,
+        # down), GEMV 2 x (split + product)
+        self.launches_per_step = 2 + 1 + 3 + 4
         self.nG, self.nD = E * 2 * I * H, E * H * I
         self.moe_weights = K_TOP * (2 * I * H + H * I)  # distinct experts at T = 1: exactly k
         self.weights_per_step = self.nG + self.nD + self.moe_weights + self.nG + self.nD

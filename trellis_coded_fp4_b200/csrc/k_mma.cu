@@ -57,6 +57,7 @@ struct Cfg {
   static_assert(NMAX <= 128, "B scale factors of a 4-block group fit one 4-column TMEM slot");
   static constexpr int kTok = NMAX / kTerms;                   // tokens per group
   static constexpr int kSlots = (NMAX + kTerms - 1) / kTerms;  // token slots the split writes
+  static constexpr int kSplitNT = kTok <= 6 ? kTok : 4;        // slots split side by side
   static constexpr int kC = (NMAX + 31) / 32;                  // B scale columns per 4-block group
   static constexpr int kKB = NMAX <= 32 ? 32 : 16;             // 32-blocks per row per stage
   // Warps: kDecWarps decode warps (four per group of 8 blocks of a stage), then the word loader, two
@@ -197,42 +198,60 @@ __host__ __device__ inline size_t terms_bytes(int S) {
   return (size_t)S * (Cfg<NMAX>::kBStage + Cfg<NMAX>::kSfbStage);
 }
 
-// One 32-element block kb of one activation row (lane = element) -> kTerms E2M1 terms with UE8M0
-// scales, written as B rows kTerms*t .. kTerms*t+kTerms-1 of the group's terms (layout above).
-// Term j: with m the largest |residual| of the block, scale 2^S with S = ceil(log2(m / 6)) puts the
-// block in (3, 6]; each residual is rounded to the E2M1 grid (nearest even) and the rounded value
-// removed (exactly: Sterbenz). The largest residual shrinks by at least 5x per term, so after
-// kTerms terms |x - sum| <= 5^-6 max|x| over the block.
+// One 32-element block kb of NT activation rows (lane = element; v[i] is slot t0 + i) -> kTerms
+// E2M1 terms each with UE8M0 scales, written as B rows kTerms*t .. kTerms*t+kTerms-1 of the
+// group's terms (layout above). Term j: with m the largest |residual| of the block, scale 2^S with
+// S = ceil(log2(m / 6)) puts the block in (3, 6]; each residual is rounded to the E2M1 grid
+// (nearest even) and the rounded value removed (exactly: Sterbenz). The largest residual shrinks
+// by at least 5x per term, so after kTerms terms |x - sum| <= 5^-6 max|x| over the block.
+// The NT slots are split side by side (their dependent chains overlap); slots at or past `nvalid`
+// are computed but not stored.
 // NAT: natural K order within a block (the MXFP4 tensor's), else the decoder's interleaved order.
-template <int NMAX, bool NAT = false>
-__device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total, uint8_t *terms) {
+template <int NMAX, bool NAT, int NT>
+__device__ __forceinline__ void split_terms_n(const float *v, int t0, int nvalid, int kb, int S_total,
+                                              uint8_t *terms) {
   using C = Cfg<NMAX>;
   const int lane = threadIdx.x & 31;
   const int s = kb / C::kKB, c = kb - s * C::kKB, h = c >> 2;
   uint8_t *bst = terms + (size_t)s * C::kBStage;
   uint8_t *sfs = terms + (size_t)S_total * C::kBStage + (size_t)s * C::kSfbStage;
   const int kp = NAT ? lane : kpos_of_weight(lane);
-  float r = v;
+  float r[NT];
+#pragma unroll
+  for (int i = 0; i < NT; i++) r[i] = v[i];
 #pragma unroll
   for (int j = 0; j < kTerms; j++) {
-    const int n = kTerms * t + j;
-    const float m = warp_max(fabsf(r));
-    // S from m's exponent field: m = 1.f * 2^e, and m / 2^e <= 1.5 iff the fraction <= 0.5.
-    // A subnormal or zero m gives S = -127. S <= 126 for any finite m (max|bf16| < 2^128).
-    const uint32_t mb = __float_as_uint(m);
-    const int e = (int)(mb >> 23) - 127;
-    int S = (mb >> 23) == 0u ? -127 : ((mb & 0x7FFFFFu) <= 0x400000u ? e - 2 : e - 1);
-    S = S < -127 ? -127 : S;
-    const uint32_t code = to_e2m1(r * pow2f(-S));
-    r -= e2m1_value(code) * pow2f(S);
-    // the element sharing this one's byte: K positions kp and kp ^ 1
-    const uint32_t partner = __shfl_xor_sync(0xffffffffu, code, NAT ? 1 : 4);
-    if (n < NMAX) {
-      if ((kp & 1) == 0)
-        bst[chunk_off<NMAX>((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code | (partner << 4));
-      if (lane == 0) sfs[((h * C::kC + (n >> 5)) * 32 + (n & 31)) * 4 + (c & 3)] = (uint8_t)(S + 127);
+    uint32_t code[NT];
+    int S[NT];
+#pragma unroll
+    for (int i = 0; i < NT; i++) {
+      // the largest |residual|: for non-negative floats the bit patterns order as the values do
+      const uint32_t mb = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(r[i])));
+      // S from m's exponent field: m = 1.f * 2^e, and m / 2^e <= 1.5 iff the fraction <= 0.5.
+      // A subnormal or zero m gives S = -127. S <= 126 for any finite m (max|bf16| < 2^128).
+      const int e = (int)(mb >> 23) - 127;
+      int Si = (mb >> 23) == 0u ? -127 : ((mb & 0x7FFFFFu) <= 0x400000u ? e - 2 : e - 1);
+      S[i] = Si < -127 ? -127 : Si;
+      code[i] = to_e2m1(r[i] * pow2f(-S[i]));
+      r[i] -= e2m1_value(code[i]) * pow2f(S[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < NT; i++) {
+      // the element sharing this one's byte: K positions kp and kp ^ 1
+      const uint32_t partner = __shfl_xor_sync(0xffffffffu, code[i], NAT ? 1 : 4);
+      const int n = kTerms * (t0 + i) + j;
+      if (t0 + i < nvalid && n < NMAX) {
+        if ((kp & 1) == 0)
+          bst[chunk_off<NMAX>((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code[i] | (partner << 4));
+        if (lane == 0) sfs[((h * C::kC + (n >> 5)) * 32 + (n & 31)) * 4 + (c & 3)] = (uint8_t)(S[i] + 127);
+      }
     }
   }
+}
+
+template <int NMAX, bool NAT = false>
+__device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total, uint8_t *terms) {
+  split_terms_n<NMAX, NAT, 1>(&v, t, t + 1, kb, S_total, terms);
 }
 
 // Plain GEMV: one group, token slots 0..T-1 (slots up to kSlots are zero rows).
@@ -498,6 +517,7 @@ struct MmaArgs {
   const float *wts;
   int P, E, k, Tm, H, I;
   uint16_t *hidden;       // [P][I] bf16
+  uint8_t *terms_dn;      // gate/up: the down kernel's activation terms, written by its epilogue
   float *yws;             // [P][H] fp32
   int *counters;          // 4 per 128-row chunk of H
   uint16_t *out;          // [T][H] bf16
@@ -1048,15 +1068,30 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
             *abort_flag = 1;
             return;
           }
-          if (mrow < jr.na)
+          // h = bf16(silu(g) u) of this warp's 32 rows, which are one 32-block of the down product's
+          // K, for every token of the group: written out, and split here into the down kernel's
+          // activation terms. The B rows of empty slots are not written: an MMA column depends on
+          // its own B row only, and the down epilogue reads the columns of the group's tokens.
+          constexpr int NT = C::kSplitNT, kTokPad = (C::kTok + NT - 1) / NT * NT;
+          float hv[kTokPad];
 #pragma unroll
-            for (int t = 0; t < C::kTok; t++)
-              if (t < jr.cnt) {
-                const float g = v[t], u = U[mrow * C::kTok + t];
-                const int p = pl->list[jr.first + t];
-                a.hidden[(size_t)p * a.I + jr.row0 + mrow] =
-                    __bfloat16_as_ushort(__float2bfloat16_rn(g / (1.0f + expf(-g)) * u));
-              }
+          for (int t = 0; t < kTokPad; t++) {
+            hv[t] = 0.f;
+            if (t < C::kTok && t < jr.cnt && mrow < jr.na) {
+              const float g = v[t], u = U[mrow * C::kTok + t];
+              const int p = pl->list[jr.first + t];
+              const __nv_bfloat16 hb = __float2bfloat16_rn(g / (1.0f + expf(-g)) * u);
+              a.hidden[(size_t)p * a.I + jr.row0 + mrow] = __bfloat16_as_ushort(hb);
+              hv[t] = __bfloat162float(hb);
+            }
+          }
+          if (jr.row0 + 32 * eq < a.I) {  // warp-uniform
+            const int S_dn = (a.I / 32 + kKB - 1) / kKB, kb_dn = jr.row0 / 32 + eq;
+            uint8_t *tg = a.terms_dn + (size_t)jr.group * terms_bytes<NMAX>(S_dn);
+#pragma unroll
+            for (int t0 = 0; t0 < kTokPad; t0 += NT)
+              if (t0 < jr.cnt) split_terms_n<NMAX, MX, NT>(hv + t0, t0, jr.cnt, kb_dn, S_dn, tg);
+          }
           __syncwarp();
           if (lane == 0) mbar_arrive(&u_empty[buf]);
         }
@@ -1412,26 +1447,23 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
+    args.terms_dn = reinterpret_cast<uint8_t *>(base + L.bg_dn);
     args.seg_blocks = MX ? 1 : (int)(m.gate_up[0].seg_len / 32);
     const int jobs = G * ((m.I + 63) / 64);
     e = launch_product_seg<MAXE, kModeGateUp, NMAX, MX>(jobs < nsm ? jobs : nsm, args, tab, map_gu, s);
     if (e != cudaSuccess) return e;
   }
-  // down: split h per group, then decode + MMA, y to the workspace, last arriver per chunk combines
+  // down: decode + MMA of the terms the gate/up epilogue wrote, y to the workspace, last arriver per
+  // chunk combines
   {
     uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_dn);
     const int nbr = m.I / 32;
-    const int warps = G * Cfg<NMAX>::kSlots * nbr;
-    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX, MX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
-                                     dim3(256), 0, s, ids, P, m.E, 1, (const uint16_t *)args.hidden, m.I, terms,
-                                     (int *)nullptr, 0);
-    if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
     args.seg_blocks = MX ? 1 : (int)(m.down[0].seg_len / 32);
     args.maps += (size_t)nsm * kMapSlots * 128;  // the down kernel's own tensor-map slots
     const int jobs = G * ((m.H + 127) / 128);
-    e = launch_product_seg<MAXE, kModeDown, NMAX, MX>(jobs < nsm ? jobs : nsm, args, tab, map_dn, s);
+    const cudaError_t e = launch_product_seg<MAXE, kModeDown, NMAX, MX>(jobs < nsm ? jobs : nsm, args, tab, map_dn, s);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
