@@ -52,6 +52,8 @@ def lib():
         L.oracle_decode_codes.argtypes = [u32p, i64, i64, i64, u8p]
         L.oracle_decode_values.argtypes = [u32p, u8p, i64, i64, i64, f64p]
         L.oracle_expand_mxfp4.argtypes = [u32p, u8p, i64, i64, i64, u8p, u8p]
+        L.oracle_decode_codes_interleaved.argtypes = [u32p, i64, i64, i64, u8p]
+        L.oracle_repack_interleaved.argtypes = [u32p, i64, i64, u32p]
         L.oracle_mxfp4_gemv.argtypes = [u8p, u8p, i64, i64, u16p, i64, i64p, i64, f64p, f64p]
         L.oracle_bf16_value.argtypes = [ctypes.c_uint16]
         L.oracle_bf16_value.restype = ctypes.c_double
@@ -165,6 +167,24 @@ def decode_values(stream, scales, rows, cols, seg_len):
     _check(lib().oracle_decode_values(_ptr(stream, ctypes.c_uint32), _ptr(scales, ctypes.c_uint8),
                                       rows, cols, seg_len, _ptr(w, ctypes.c_double)), "decode_values")
     return w
+
+
+def decode_codes_interleaved(il, rows, cols, seg_len):
+    """Codes [rows][cols] of an interleaved-packed stream, from 16-bit windows of its bit string."""
+    il, _ = _stream_args(il, None, rows, cols)
+    codes = np.zeros((rows, cols), np.uint8)
+    _check(lib().oracle_decode_codes_interleaved(_ptr(il, ctypes.c_uint32), rows, cols, seg_len,
+                                                 _ptr(codes, ctypes.c_uint8)), "decode_codes_interleaved")
+    return codes
+
+
+def repack_interleaved(il, rows, cols):
+    """Planar stream words [rows][cols/32][2] of an interleaved-packed stream of the same shape."""
+    il, _ = _stream_args(il, None, rows, cols)
+    out = np.zeros((rows, cols // 32, 2), np.uint32)
+    _check(lib().oracle_repack_interleaved(_ptr(il, ctypes.c_uint32), rows, cols, _ptr(out, ctypes.c_uint32)),
+           "repack_interleaved")
+    return out
 
 
 def expand_mxfp4(stream, scales, rows, cols, seg_len):

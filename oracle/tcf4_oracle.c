@@ -33,7 +33,9 @@
  *     low bits of symbols 0..31, bit i = symbol i; word 1 the high bits)  [unpinned];
  *   - the state is 0 at the start of every segment of seg_len weights along a row;
  *   - P3's zero is -0 (code 0x8), so the 16 palette slots are the 16 E2M1 codes;
- *   - an MXFP4 byte holds element 2u in its low nibble and 2u+1 in its high nibble.
+ *   - an MXFP4 byte holds element 2u in its low nibble and 2u+1 in its high nibble;
+ *   - the second, interleaved packing (below) stores each row as one bit string, two bits per
+ *     symbol, low bit first, LSB-first in 32-bit words  [unpinned, like the planar packing].
  */
 #include <math.h>
 #include <stdint.h>
@@ -184,6 +186,54 @@ int oracle_expand_mxfp4(const uint32_t *stream, const uint8_t *scales, int64_t r
         }
     }
     memcpy(out_scales, scales, (size_t)(rows * (cols / 32)));
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------- interleaved packing
+ * A second packing of the same stream (a reading; the pages fix none): each row is one bit string
+ * in which symbol k takes bits 2k (its low bit) and 2k+1 (its high bit), stored LSB-first in 32-bit
+ * words, so block j of a row owns words 2j (its symbols 0..15) and 2j+1 (symbols 16..31).
+ * Under this packing the [XT] "16-bit sliding state" is literally a window of the bit string. */
+
+/* Bit p of row n's bit string. */
+static uint32_t il_bit(const uint32_t *il, int64_t cols, int64_t n, int64_t p) {
+    return (il[n * (cols / 16) + p / 32] >> (p % 32)) & 1u;
+}
+
+/* [XT] decoder bullet, read on the interleaved bit string: the state of weight k is the 16 bits of
+ * the row's string that end with symbol k's high bit (bit m of the state = string bit 2k - 14 + m),
+ * with every bit before the start of k's segment read as 0. No symbol recurrence is used here. */
+int oracle_decode_codes_interleaved(const uint32_t *il, int64_t rows, int64_t cols, int64_t seg_len,
+                                    uint8_t *codes) {
+    if (check_shape(rows, cols, seg_len)) return ORACLE_EINVAL;
+    for (int64_t n = 0; n < rows; n++)
+        for (int64_t k = 0; k < cols; k++) {
+            int64_t start = 2 * (k - k % seg_len);
+            uint32_t s = 0;
+            for (int m = 0; m < 16; m++) {
+                int64_t p = 2 * k - 14 + m;
+                if (p >= start) s |= il_bit(il, cols, n, p) << m;
+            }
+            codes[n * cols + k] = oracle_state_code(s);
+        }
+    return ORACLE_OK;
+}
+
+/* Interleaved -> planar: symbol k of a row (bits 2k, 2k+1 of its string) becomes bit k % 32 of the
+ * low and high words of its block. */
+int oracle_repack_interleaved(const uint32_t *il, int64_t rows, int64_t cols, uint32_t *planar) {
+    if (rows < 0 || cols < 0 || cols % 32 != 0) return ORACLE_EINVAL;
+    for (int64_t n = 0; n < rows; n++)
+        for (int64_t j = 0; j < cols / 32; j++) {
+            uint32_t lo = 0, hi = 0;
+            for (int64_t i = 0; i < 32; i++) {
+                int64_t k = 32 * j + i;
+                lo |= il_bit(il, cols, n, 2 * k) << i;
+                hi |= il_bit(il, cols, n, 2 * k + 1) << i;
+            }
+            planar[2 * (n * (cols / 32) + j)] = lo;
+            planar[2 * (n * (cols / 32) + j) + 1] = hi;
+        }
     return ORACLE_OK;
 }
 
