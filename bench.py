@@ -537,10 +537,31 @@ def main():
     encoder = {"ms_per_call": round(enc_ms, 3), "weights": enc_rows * enc_cols, "seg_len": 32,
                "weights_per_s": enc_rows * enc_cols / (enc_ms * 1e-3), "bound": "alu",
                "note": "2^16 candidate paths per weight, fp64 costs evaluated exactly (no fused operations)"}
-    line["next_rows"] = {"mxfp4_consumer": mx, "encoder": encoder,
+    # the interleaved-packing repack of the gate_up stream (184320 x 2880: 133 MB read, 133 MB
+    # written per call, more than L2 holds), back to back after warm-up
+    rp_out = torch.empty_like(step.G.stream)
+    rp_rows, rp_cols = step.G.rows, step.G.cols
+    for _ in range(3):
+        step.tc.repack_interleaved(step.G.stream, rp_rows, rp_cols, out=rp_out)
+    torch.cuda.synchronize()
+    n_rp = max(10, args.steps // 4)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_rp):
+        step.tc.repack_interleaved(step.G.stream, rp_rows, rp_cols, out=rp_out)
+    e1.record()
+    torch.cuda.synchronize()
+    rp_us = 1e3 * e0.elapsed_time(e1) / n_rp
+    rp_bytes = 16 * rp_rows * (rp_cols // 32)
+    rp_gbs = rp_bytes / (rp_us * 1e-6) / 1e9
+    repack = {"avg_us": round(rp_us, 3), "algo_bytes": rp_bytes, "gb_s": round(rp_gbs, 1),
+              "frac_of_measured_hbm": round(rp_gbs / peak, 4), "frac_of_8tbs": round(rp_gbs / 8000.0, 4),
+              "calls": n_rp, "bound": "hbm", "note": "8 bytes read + 8 written per 32-weight block"}
+    del rp_out
+    line["next_rows"] = {"mxfp4_consumer": mx, "encoder": encoder, "repack_interleaved": repack,
                          "description": "products read straight from the resident MXFP4 tensors the step's "
-                         "expansion wrote (HEPH serving mode 2), and the D-weighted Viterbi encoder; outside "
-                         "the step and its value"}
+                         "expansion wrote (HEPH serving mode 2), the D-weighted Viterbi encoder, and the "
+                         "interleaved-to-planar stream repack; outside the step and its value"}
 
     if rank == 0:
         line["e2e"] = run_e2e(step, args.e2e_steps, device)

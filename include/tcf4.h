@@ -77,6 +77,18 @@ typedef struct {
 TCF4_API tcf4_status trellis_decode_to_mxfp4(tcf4_matrix w, uint8_t *out_nibbles, uint8_t *out_scales,
                                     void *stream);
 
+/* The second stream packing: each row one bit string, symbol k at bits 2k (its low bit) and 2k+1
+ * (its high bit), LSB-first in 32-bit words, so block j of a row owns words 2j (its symbols 0..15)
+ * and 2j+1 (symbols 16..31). The XOR-Trellis page's 16-bit sliding state ("XOR-Trellis FP4
+ * decoder" bullet) is then a window of that string. Every other call here reads the planar packing
+ * (tcf4_matrix.stream); this call converts, bit for bit, once at load time.
+ *   in:  uint32 [rows][cols/32][2] interleaved words (device); out: the same shape, planar words.
+ *   in == out converts in place; otherwise the two buffers must not overlap (TCF4_ERR_INVALID_ARG).
+ *   Both pointers 8-byte aligned (TCF4_ERR_MISALIGNED); 32-byte alignment of both takes the widest
+ *   accesses. rows * cols / 32 < 2^31 (TCF4_ERR_UNSUPPORTED). rows or cols 0: nothing to do. */
+TCF4_API tcf4_status trellis_repack_interleaved(const uint32_t *in, int64_t rows, int64_t cols, uint32_t *out,
+                                                void *stream);
+
 /* HEPH abstract, first serving mode: fused decode + product.
  *   y[t][n] = bf16( sum_k w[n][k] * x[t][k] ), fp32 accumulation, round to nearest even.
  *   x: bf16 bits [T][cols]; y: bf16 bits [T][rows]; 1 <= T <= 32 (T == 0 is a no-op).

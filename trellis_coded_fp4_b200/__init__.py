@@ -61,6 +61,16 @@ def decode_to_mxfp4(w: TrellisMatrix, out_nibbles=None, out_scales=None):
     return out_nibbles, out_scales
 
 
+def repack_interleaved(stream: torch.Tensor, rows: int, cols: int, out=None):
+    """Interleaved-packed stream words (each row one bit string, two bits per symbol, low bit first)
+    -> the planar words TrellisMatrix holds; int32 [rows][cols/32][2]. out=stream converts in place."""
+    if out is None:
+        out = torch.empty((rows, cols // 32, 2), dtype=torch.int32, device=stream.device)
+    _abi.check(_abi.load().trellis_repack_interleaved(_ptr(stream), rows, cols, _ptr(out), _stream_handle()),
+               "trellis_repack_interleaved")
+    return out
+
+
 def gemv_workspace_bytes(w: TrellisMatrix, T: int) -> int:
     """Scratch bytes trellis_gemv needs for T tokens (0: the call needs none)."""
     return int(_abi.load().trellis_gemv_workspace(w.abi(), T))

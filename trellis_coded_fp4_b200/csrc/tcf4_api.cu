@@ -99,6 +99,21 @@ tcf4_status trellis_decode_to_mxfp4(tcf4_matrix w, uint8_t *out_nibbles, uint8_t
   return from_cuda(launch_expand(view(w), out_nibbles, out_scales, static_cast<cudaStream_t>(stream)));
 }
 
+tcf4_status trellis_repack_interleaved(const uint32_t *in, int64_t rows, int64_t cols, uint32_t *out, void *stream) {
+  if (rows < 0 || cols < 0 || cols % 32 != 0) return TCF4_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return TCF4_OK;
+  if (in == nullptr || out == nullptr) return TCF4_ERR_INVALID_ARG;
+  const uintptr_t ib = reinterpret_cast<uintptr_t>(in), ob = reinterpret_cast<uintptr_t>(out);
+  if (((ib | ob) & 7u) != 0) return TCF4_ERR_MISALIGNED;
+  if (rows > INT32_MAX || cols / 32 > INT32_MAX || rows * (cols / 32) >= ((int64_t)1 << 31))
+    return TCF4_ERR_UNSUPPORTED;
+  const int64_t nblocks = rows * (cols / 32);
+  const uintptr_t nbytes = (uintptr_t)nblocks * 8u;
+  if (ib != ob && ib < ob + nbytes && ob < ib + nbytes) return TCF4_ERR_INVALID_ARG;
+  clear_pending_error();
+  return from_cuda(launch_repack(in, out, (uint32_t)nblocks, static_cast<cudaStream_t>(stream)));
+}
+
 static tcf4_status check_gemv(const tcf4_matrix &w, int32_t T) {
   tcf4_status st = check_matrix(w);
   if (st != TCF4_OK) return st;
