@@ -42,6 +42,10 @@ def lib():
         L.oracle_e2m1_value.restype = ctypes.c_double
         L.oracle_ue8m0_value.argtypes = [ctypes.c_uint8]
         L.oracle_ue8m0_value.restype = ctypes.c_double
+        L.oracle_e5m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e5m3_value.restype = ctypes.c_double
+        L.oracle_decode_values_e5m3.argtypes = [u32p, u8p, i64, i64, i64, f64p]
+        L.oracle_gemv_e5m3.argtypes = [u32p, u8p, i64, i64, i64, u16p, i64, i64p, i64, f64p, f64p]
         L.oracle_state_push.argtypes = [ctypes.c_uint32, ctypes.c_uint32]
         L.oracle_state_push.restype = ctypes.c_uint32
         L.oracle_state_decode.argtypes = [ctypes.c_uint32, P(ctypes.c_int), P(ctypes.c_int)]
@@ -95,6 +99,11 @@ def e2m1_value(code):
 
 def ue8m0_value(E):
     return lib().oracle_ue8m0_value(int(E))
+
+
+def e5m3_value(b):
+    """E5M3 block scale (the reading: no sign, bias 15, subnormals, exponent 31 = NaN)."""
+    return lib().oracle_e5m3_value(int(b))
 
 
 def state_push(s, b):
@@ -161,11 +170,12 @@ def decode_codes(stream, rows, cols, seg_len):
     return codes
 
 
-def decode_values(stream, scales, rows, cols, seg_len):
+def decode_values(stream, scales, rows, cols, seg_len, scale_fmt="ue8m0"):
     stream, scales = _stream_args(stream, scales, rows, cols)
     w = np.zeros((rows, cols), np.float64)
-    _check(lib().oracle_decode_values(_ptr(stream, ctypes.c_uint32), _ptr(scales, ctypes.c_uint8),
-                                      rows, cols, seg_len, _ptr(w, ctypes.c_double)), "decode_values")
+    fn = lib().oracle_decode_values_e5m3 if scale_fmt == "e5m3" else lib().oracle_decode_values
+    _check(fn(_ptr(stream, ctypes.c_uint32), _ptr(scales, ctypes.c_uint8), rows, cols, seg_len,
+              _ptr(w, ctypes.c_double)), "decode_values")
     return w
 
 
@@ -199,8 +209,9 @@ def expand_mxfp4(stream, scales, rows, cols, seg_len):
 
 # ----------------------------------------------------------------------------- products
 
-def gemv(stream, scales, rows, cols, seg_len, x_bits, row_ids=None):
-    """y[T][nr] (fp64) and ||w_row||_2 [nr] for bf16 activations x_bits [T][cols] (uint16)."""
+def gemv(stream, scales, rows, cols, seg_len, x_bits, row_ids=None, scale_fmt="ue8m0"):
+    """y[T][nr] (fp64) and ||w_row||_2 [nr] for bf16 activations x_bits [T][cols] (uint16);
+    scale_fmt "e5m3" reads the scale bytes as E5M3 block scales."""
     stream, scales = _stream_args(stream, scales, rows, cols)
     x_bits = np.ascontiguousarray(np.atleast_2d(x_bits), np.uint16)
     T = x_bits.shape[0]
@@ -213,10 +224,10 @@ def gemv(stream, scales, rows, cols, seg_len, x_bits, row_ids=None):
         nr = rid.size
     y = np.zeros((T, nr), np.float64)
     wn = np.zeros(nr, np.float64)
-    _check(lib().oracle_gemv(_ptr(stream, ctypes.c_uint32), _ptr(scales, ctypes.c_uint8), rows, cols,
-                             seg_len, _ptr(x_bits, ctypes.c_uint16), T,
-                             None if rid is None else _ptr(rid, ctypes.c_int64), nr,
-                             _ptr(y, ctypes.c_double), _ptr(wn, ctypes.c_double)), "gemv")
+    fn = lib().oracle_gemv_e5m3 if scale_fmt == "e5m3" else lib().oracle_gemv
+    _check(fn(_ptr(stream, ctypes.c_uint32), _ptr(scales, ctypes.c_uint8), rows, cols, seg_len,
+              _ptr(x_bits, ctypes.c_uint16), T, None if rid is None else _ptr(rid, ctypes.c_int64), nr,
+              _ptr(y, ctypes.c_double), _ptr(wn, ctypes.c_double)), "gemv")
     return y, wn
 
 

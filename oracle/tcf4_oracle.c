@@ -86,6 +86,24 @@ int oracle_e2m1_code(double v, uint8_t *code) {
 /* [TTP]/OCP MX: an E8M0 (UE8M0) scale byte E means 2^(E-127); E = 0xFF is NaN. */
 double oracle_ue8m0_value(uint8_t E) { return E == 0xFF ? NAN : ldexp(1.0, (int)E - 127); }
 
+/* The XOR-Trellis news page's paragraph on the grouping format pairs E2M1 elements with E5M3 block
+ * scales and gives no encoding for the scale. Reading: 8 bits, no sign bit (block scales are positive), exponent
+ * in bits 7..3 with bias 15, mantissa in bits 2..0; exponent 0 is subnormal (2^-14 * m/8), exponent
+ * 31 is NaN; one scale per 32-weight block, as for UE8M0. */
+double oracle_e5m3_value(uint8_t b) {
+    int e = b >> 3, m = b & 7;
+    if (e == 31) return NAN;
+    if (e == 0) return ldexp((double)m / 8.0, -14);
+    return ldexp(1.0 + (double)m / 8.0, e - 15);
+}
+
+#define SCALE_UE8M0 0
+#define SCALE_E5M3 1
+
+static double scale_value(uint8_t b, int fmt) {
+    return fmt == SCALE_E5M3 ? oracle_e5m3_value(b) : oracle_ue8m0_value(b);
+}
+
 static int parity16(uint32_t v) {
     int p = 0;
     for (int i = 0; i < 16; i++) p ^= (int)((v >> i) & 1u);
@@ -149,22 +167,33 @@ int oracle_decode_codes(const uint32_t *stream, int64_t rows, int64_t cols, int6
     return ORACLE_OK;
 }
 
-/* One decoded row in fp64: palette value times its block's scale ([HEPH] grid-aligned). */
+/* One decoded row in fp64: palette value times its block's scale ([HEPH] grid-aligned; or the
+ * E5M3 block scale of the XOR-Trellis page's grouping format when fmt is SCALE_E5M3). */
 static void decode_row(const uint32_t *stream, const uint8_t *scales, int64_t cols, int64_t seg_len,
-                       int64_t n, double *w) {
+                       int64_t n, double *w, int fmt) {
     uint32_t s = 0;
     for (int64_t k = 0; k < cols; k++) {
         if (k % seg_len == 0) s = 0;
         s = oracle_state_push(s, symbol_at(stream, cols, n, k));
-        w[k] = oracle_state_value(s) * oracle_ue8m0_value(scales[n * (cols / 32) + k / 32]);
+        w[k] = oracle_state_value(s) * scale_value(scales[n * (cols / 32) + k / 32], fmt);
     }
+}
+
+static int decode_values_fmt(const uint32_t *stream, const uint8_t *scales, int64_t rows, int64_t cols,
+                             int64_t seg_len, double *w, int fmt) {
+    if (check_shape(rows, cols, seg_len)) return ORACLE_EINVAL;
+    for (int64_t n = 0; n < rows; n++) decode_row(stream, scales, cols, seg_len, n, w + n * cols, fmt);
+    return ORACLE_OK;
 }
 
 int oracle_decode_values(const uint32_t *stream, const uint8_t *scales, int64_t rows, int64_t cols,
                          int64_t seg_len, double *w) {
-    if (check_shape(rows, cols, seg_len)) return ORACLE_EINVAL;
-    for (int64_t n = 0; n < rows; n++) decode_row(stream, scales, cols, seg_len, n, w + n * cols);
-    return ORACLE_OK;
+    return decode_values_fmt(stream, scales, rows, cols, seg_len, w, SCALE_UE8M0);
+}
+
+int oracle_decode_values_e5m3(const uint32_t *stream, const uint8_t *scales, int64_t rows, int64_t cols,
+                              int64_t seg_len, double *w) {
+    return decode_values_fmt(stream, scales, rows, cols, seg_len, w, SCALE_E5M3);
 }
 
 /* [HEPH] mode 2: packed MXFP4, [rows][cols/2] bytes (even element in the low nibble) plus the
@@ -272,8 +301,9 @@ uint16_t oracle_bf16_bits(double v) {
  * listed in row_ids (all rows in order when row_ids is NULL, nr = rows). Also returns the
  * Euclidean norm of each listed decoded row in wnorm (may be NULL). x holds bf16 bits [T][cols].
  * The sum's rounding error is at most cols * 2^-53 * sum |w x|. */
-int oracle_gemv(const uint32_t *stream, const uint8_t *scales, int64_t rows, int64_t cols, int64_t seg_len,
-                const uint16_t *x, int64_t T, const int64_t *row_ids, int64_t nr, double *y, double *wnorm) {
+static int gemv_fmt(const uint32_t *stream, const uint8_t *scales, int64_t rows, int64_t cols, int64_t seg_len,
+                    const uint16_t *x, int64_t T, const int64_t *row_ids, int64_t nr, double *y, double *wnorm,
+                    int fmt) {
     if (check_shape(rows, cols, seg_len) || T < 0 || nr < 0) return ORACLE_EINVAL;
     if (row_ids == NULL && nr != rows) return ORACLE_EINVAL;
     double *w = (double *)malloc(sizeof(double) * (size_t)(cols > 0 ? cols : 1));
@@ -291,7 +321,7 @@ int oracle_gemv(const uint32_t *stream, const uint8_t *scales, int64_t rows, int
             free(xv);
             return ORACLE_EINVAL;
         }
-        decode_row(stream, scales, cols, seg_len, n, w);
+        decode_row(stream, scales, cols, seg_len, n, w, fmt);
         if (wnorm) {
             double ss = 0.0;
             for (int64_t k = 0; k < cols; k++) ss += w[k] * w[k];
@@ -306,6 +336,17 @@ int oracle_gemv(const uint32_t *stream, const uint8_t *scales, int64_t rows, int
     free(w);
     free(xv);
     return ORACLE_OK;
+}
+
+int oracle_gemv(const uint32_t *stream, const uint8_t *scales, int64_t rows, int64_t cols, int64_t seg_len,
+                const uint16_t *x, int64_t T, const int64_t *row_ids, int64_t nr, double *y, double *wnorm) {
+    return gemv_fmt(stream, scales, rows, cols, seg_len, x, T, row_ids, nr, y, wnorm, SCALE_UE8M0);
+}
+
+/* The same products with E5M3 block scales (reading above oracle_e5m3_value). */
+int oracle_gemv_e5m3(const uint32_t *stream, const uint8_t *scales, int64_t rows, int64_t cols, int64_t seg_len,
+                     const uint16_t *x, int64_t T, const int64_t *row_ids, int64_t nr, double *y, double *wnorm) {
+    return gemv_fmt(stream, scales, rows, cols, seg_len, x, T, row_ids, nr, y, wnorm, SCALE_E5M3);
 }
 
 /* [HEPH] mode 2, consumer side: the same products from a resident MXFP4 tensor. By the OCP MX
