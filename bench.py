@@ -558,10 +558,37 @@ def main():
               "frac_of_measured_hbm": round(rp_gbs / peak, 4), "frac_of_8tbs": round(rp_gbs / 8000.0, 4),
               "calls": n_rp, "bound": "hbm", "note": "8 bytes read + 8 written per 32-weight block"}
     del rp_out
+    # the E5M3 block-scale variant: the gate_up stream (184320 x 2880) with E5M3 scale bytes of the
+    # same binades as its UE8M0 ones and random mantissas, batch 1, on the CUDA-core kernel
+    g5 = torch.Generator(device=device).manual_seed(seed + 5)
+    m5 = torch.randint(0, 8, step.G.scales.shape, dtype=torch.int32, device=device, generator=g5)
+    sc5 = (((step.G.scales.to(torch.int32) - 112) << 3) | m5).to(torch.uint8)
+    W5 = step.tc.TrellisMatrix(step.G.stream, sc5, step.G.rows, step.G.cols, step.G.seg_len)
+    y5 = torch.empty((T, W5.rows), dtype=torch.bfloat16, device=device)
+    for i in range(3):
+        step.tc.gemv_e5m3(W5, step.x[i % len(step.x)], out=y5)
+    torch.cuda.synchronize()
+    n5 = max(10, args.steps // 20)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n5):
+        step.tc.gemv_e5m3(W5, step.x[i % len(step.x)], out=y5)
+    e1.record()
+    torch.cuda.synchronize()
+    g5_us = 1e3 * e0.elapsed_time(e1) / n5
+    g5_bytes = step.algo_bytes()["gemv_gate_up"]
+    g5_gbs = g5_bytes / (g5_us * 1e-6) / 1e9
+    e5m3 = {"avg_us": round(g5_us, 3), "algo_bytes": g5_bytes, "gb_s": round(g5_gbs, 1),
+            "frac_of_measured_hbm": round(g5_gbs / peak, 4), "frac_of_8tbs": round(g5_gbs / 8000.0, 4),
+            "decoded_weights_per_s": W5.rows * W5.cols / (g5_us * 1e-6), "calls": n5,
+            "note": "CUDA-core kernel (a block-scaled MMA takes power-of-two scales only)"}
+    del W5, sc5, m5, y5
     line["next_rows"] = {"mxfp4_consumer": mx, "encoder": encoder, "repack_interleaved": repack,
+                         "gemv_e5m3_gate_up": e5m3,
                          "description": "products read straight from the resident MXFP4 tensors the step's "
-                         "expansion wrote (HEPH serving mode 2), the D-weighted Viterbi encoder, and the "
-                         "interleaved-to-planar stream repack; outside the step and its value"}
+                         "expansion wrote (HEPH serving mode 2), the D-weighted Viterbi encoder, the "
+                         "interleaved-to-planar stream repack and the E5M3 block-scale GEMV; outside the "
+                         "step and its value"}
 
     if rank == 0:
         line["e2e"] = run_e2e(step, args.e2e_steps, device)

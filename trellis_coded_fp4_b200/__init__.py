@@ -91,6 +91,16 @@ def gemv(w: TrellisMatrix, x: torch.Tensor, out=None, workspace=None):
     return out
 
 
+def gemv_e5m3(w: TrellisMatrix, x: torch.Tensor, out=None):
+    """y = bf16(W x) with w.scales read as E5M3 block scales (CUDA-core kernel): bf16 [T][rows]."""
+    x = x if x.dim() == 2 else x.view(1, -1)
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, w.rows), dtype=torch.bfloat16, device=x.device)
+    _abi.check(_abi.load().trellis_gemv_e5m3(w.abi(), _ptr(x), T, _ptr(out), _stream_handle()), "trellis_gemv_e5m3")
+    return out
+
+
 def gemv_noalloc(w: TrellisMatrix, x: torch.Tensor, out=None):
     """gemv through trellis_gemv_noalloc: the scratch is the library's own per-device array."""
     x = x if x.dim() == 2 else x.view(1, -1)

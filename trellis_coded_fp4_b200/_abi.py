@@ -14,7 +14,7 @@ EXPORTED = ("trellis_decode_to_mxfp4", "trellis_gemv_workspace", "trellis_gemv",
             "trellis_moe_route", "trellis_grouped_moe_workspace",
             "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "mxfp4_gemv_workspace", "mxfp4_gemv",
             "mxfp4_grouped_moe_workspace", "mxfp4_grouped_moe_hidden_offset", "mxfp4_grouped_moe",
-            "trellis_encode_workspace", "trellis_encode", "trellis_repack_interleaved",
+            "trellis_encode_workspace", "trellis_encode", "trellis_repack_interleaved", "trellis_gemv_e5m3",
             "tcf4_device_timeouts", "tcf4_status_string")
 
 
@@ -58,6 +58,8 @@ def load(path: str = LIB_PATH):
     L.trellis_decode_to_mxfp4.argtypes = [Matrix, vp, vp, vp]
     L.trellis_decode_to_mxfp4.restype = ctypes.c_int
     L.trellis_repack_interleaved.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, vp]
+    L.trellis_gemv_e5m3.argtypes = [Matrix, vp, ctypes.c_int32, vp, vp]
+    L.trellis_gemv_e5m3.restype = ctypes.c_int
     L.trellis_repack_interleaved.restype = ctypes.c_int
     L.trellis_gemv_workspace.argtypes = [Matrix, i32]
     L.trellis_gemv_workspace.restype = sz

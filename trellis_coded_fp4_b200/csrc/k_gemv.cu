@@ -30,7 +30,7 @@ __host__ __device__ inline GemvGeom gemv_geom(int nbr, int TT, int R) {
   return g;
 }
 
-template <int TT, bool SEG32, int R>
+template <int TT, bool SEG32, int R, bool E5M3>
 __global__ void __launch_bounds__(256) k_gemv(MatView w, const uint16_t *__restrict__ x, int T,
                                               uint16_t *__restrict__ y, int bulk_scales) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -90,7 +90,7 @@ __global__ void __launch_bounds__(256) k_gemv(MatView w, const uint16_t *__restr
           rok[q] = rid[q] < (int)s.nrows;
         }
         float acc[RPW][TT];
-        rows_dot_smem<RPW, TT, SEG32>(st_base, st_base + ring.sc_off, nbr, w.seg_blocks, rid, rok, smem_u32(xs),
+        rows_dot_smem<RPW, TT, SEG32, E5M3>(st_base, st_base + ring.sc_off, nbr, w.seg_blocks, rid, rok, smem_u32(xs),
                                       acc);
         const int r0 = ((int)blockIdx.x + j * (int)gridDim.x) * R;
 #pragma unroll
@@ -106,32 +106,33 @@ __global__ void __launch_bounds__(256) k_gemv(MatView w, const uint16_t *__restr
   }
 }
 
-template <int TT, bool SEG32, int R>
+template <int TT, bool SEG32, int R, bool E5M3>
 static cudaError_t launch_gemv_t(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s) {
   const GemvGeom geo = gemv_geom(w.nbr, TT, R);
   static unsigned long long attr_done = 0;  // benign race: setting the same attribute twice is harmless
-  cudaError_t e = ensure_max_dynamic_smem(k_gemv<TT, SEG32, R>, attr_done);
+  cudaError_t e = ensure_max_dynamic_smem(k_gemv<TT, SEG32, R, E5M3>, attr_done);
   if (e != cudaSuccess) return e;
   int dev = 0, nsm = 148, occ = 1;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<TT, SEG32, R>, 256, geo.smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_gemv<TT, SEG32, R, E5M3>, 256, geo.smem);
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   const int nslab = (w.rows + R - 1) / R;
   const int grid = nslab < nsm * occ ? nslab : nsm * occ;
   const int bulk_scales = ((reinterpret_cast<uintptr_t>(w.scales) & 15u) == 0 && (R * w.nbr) % 16 == 0) ? 1 : 0;
-  return launch_dependent(k_gemv<TT, SEG32, R>, dim3(grid), dim3(256), geo.smem, s, w, x, T, y, bulk_scales);
+  return launch_dependent(k_gemv<TT, SEG32, R, E5M3>, dim3(grid), dim3(256), geo.smem, s, w, x, T, y, bulk_scales);
 }
 
-template <int TT, bool SEG32>
+template <int TT, bool SEG32, bool E5M3>
 static cudaError_t launch_gemv_r(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s) {
   // 16 rows per slab while a slab stays within ~36 KB, else 8
-  if ((size_t)16 * w.nbr * 9 <= 36 * 1024) return launch_gemv_t<TT, SEG32, 16>(w, x, T, y, s);
-  return launch_gemv_t<TT, SEG32, 8>(w, x, T, y, s);
+  if ((size_t)16 * w.nbr * 9 <= 36 * 1024) return launch_gemv_t<TT, SEG32, 16, E5M3>(w, x, T, y, s);
+  return launch_gemv_t<TT, SEG32, 8, E5M3>(w, x, T, y, s);
 }
 
-cudaError_t launch_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s) {
+template <bool E5M3>
+static cudaError_t launch_gemv_f(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s) {
   const int K = w.nbr * 32;
   int TT = T >= 3 ? 4 : T;
   // activations of TT tokens plus 4 slab buffers must fit in shared memory
@@ -139,10 +140,14 @@ cudaError_t launch_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y,
   (void)K;
   const bool seg32 = w.seg_blocks == 1;
   switch (TT) {
-    case 1: return seg32 ? launch_gemv_r<1, true>(w, x, T, y, s) : launch_gemv_r<1, false>(w, x, T, y, s);
-    case 2: return seg32 ? launch_gemv_r<2, true>(w, x, T, y, s) : launch_gemv_r<2, false>(w, x, T, y, s);
-    default: return seg32 ? launch_gemv_r<4, true>(w, x, T, y, s) : launch_gemv_r<4, false>(w, x, T, y, s);
+    case 1: return seg32 ? launch_gemv_r<1, true, E5M3>(w, x, T, y, s) : launch_gemv_r<1, false, E5M3>(w, x, T, y, s);
+    case 2: return seg32 ? launch_gemv_r<2, true, E5M3>(w, x, T, y, s) : launch_gemv_r<2, false, E5M3>(w, x, T, y, s);
+    default: return seg32 ? launch_gemv_r<4, true, E5M3>(w, x, T, y, s) : launch_gemv_r<4, false, E5M3>(w, x, T, y, s);
   }
+}
+
+cudaError_t launch_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s, bool e5m3) {
+  return e5m3 ? launch_gemv_f<true>(w, x, T, y, s) : launch_gemv_f<false>(w, x, T, y, s);
 }
 
 unsigned int take_timeouts_gemv() {

@@ -154,6 +154,16 @@ tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *
   return from_cuda(launch_gemv(v, x, T, y, static_cast<cudaStream_t>(stream)));
 }
 
+tcf4_status trellis_gemv_e5m3(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream) {
+  tcf4_status st = check_gemv(w, T);
+  if (st != TCF4_OK) return st;
+  if (T == 0 || w.rows == 0) return TCF4_OK;
+  if (x == nullptr || y == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return TCF4_ERR_MISALIGNED;
+  clear_pending_error();
+  return from_cuda(launch_gemv(view(w), x, T, y, static_cast<cudaStream_t>(stream), true));
+}
+
 tcf4_status trellis_moe_route(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *topk_ids,
                               float *topk_w, void *stream) {
   if (T < 0 || k < 1 || E < k) return TCF4_ERR_INVALID_ARG;

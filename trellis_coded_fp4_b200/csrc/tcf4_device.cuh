@@ -125,6 +125,16 @@ __device__ __forceinline__ float ue8m0_to_float(uint32_t E) {
                                                               : __uint_as_float(E << 23));
 }
 
+// E5M3 block scale -> float, exact. The XOR-Trellis news page pairs E2M1 elements with E5M3 block
+// scales (its paragraph on the grouping format) and gives no encoding; read as: no sign, exponent
+// bits 7..3 with bias 15, mantissa bits 2..0, exponent 0 subnormal (m * 2^-17), exponent 31 NaN.
+// A normal byte b is the float with exponent field (b >> 3) + 112 and mantissa bits (b & 7) << 20.
+__device__ __forceinline__ float e5m3_to_float(uint32_t b) {
+  if (b >= 0xF8u) return __uint_as_float(0x7FC00000u);
+  if (b < 8u) return (float)b * __uint_as_float(110u << 23);  // m * 2^-17
+  return __uint_as_float((b << 20) + (112u << 23));
+}
+
 // Eight E2M1 codes (a word, byte u = codes 2u and 2u+1, low nibble first) -> four half2
 // (exact: every E2M1 value is a binary16 value).
 __device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t &h0, uint32_t &h1, uint32_t &h2,

@@ -86,7 +86,8 @@ cudaError_t ensure_max_dynamic_smem(F *func, unsigned long long &done) {
 cudaError_t launch_expand(const MatView &w, uint8_t *out_nibbles, uint8_t *out_scales, cudaStream_t s);
 // Interleaved -> planar stream words of nblocks 32-weight blocks (in == out allowed).
 cudaError_t launch_repack(const uint32_t *in, uint32_t *out, uint32_t nblocks, cudaStream_t s);
-cudaError_t launch_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s);
+// CUDA-core fused decode GEMV; e5m3: the scale bytes are E5M3 block scales instead of UE8M0.
+cudaError_t launch_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, cudaStream_t s, bool e5m3 = false);
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *wts, cudaStream_t s);
 cudaError_t launch_moe(const tcf4_moe &m, int gu_seg, int dn_seg, const uint16_t *x, int T, const int32_t *ids,
                        const float *wts, int k, uint16_t *out, void *ws, cudaStream_t s);

@@ -57,8 +57,9 @@ __device__ __forceinline__ void stage_x(float2 *xs, const uint16_t *__restrict__
 //   st_base / sc_base: shared addresses of row 0's stream words / scales (row stride nbr*8 / nbr);
 //   rows: warp-local row indices row_id[q] (q < RPW), valid when row_ok[q];
 //   xs_base: shared address of the staged activations (token stride nbr*16 float2).
-// Returns in every lane acc[q][t] = full dot product.
-template <int RPW, int TT, bool SEG32>
+// Returns in every lane acc[q][t] = full dot product. E5M3: the scale bytes are E5M3 block scales
+// (not exact powers of two, so the scaled partial sum is rounded once to fp32).
+template <int RPW, int TT, bool SEG32, bool E5M3 = false>
 __device__ __forceinline__ void rows_dot_smem(uint32_t st_base, uint32_t sc_base, int nbr, int seg_blocks,
                                               const int *row_id, const bool *row_ok, uint32_t xs_base,
                                               float (&acc)[RPW][TT]) {
@@ -102,7 +103,7 @@ __device__ __forceinline__ void rows_dot_smem(uint32_t st_base, uint32_t sc_base
         P = decode_block(v.x, v.y, pL, pH);
       }
       planes_to_nibbles_interleaved(P, W[q][0], W[q][1], W[q][2], W[q][3]);
-      sc[q] = ue8m0_to_float(E);
+      sc[q] = E5M3 ? e5m3_to_float(E) : ue8m0_to_float(E);
     }
     if (vj) {
       float bsum[RPW][TT];
