@@ -52,6 +52,10 @@ constexpr uint32_t kLoaderSleepNs = 200u, kMmaSleepNs = 100u, kEpiSleepNs = 200u
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
 
+// Register split of the NMAX = 32 decode GEMV (see k_mma): registers per thread at launch, of the
+// decode warps and of the other warps after the split.
+constexpr int kRsLaunchRegs = 80, kRsDecRegs = 96, kRsOtherRegs = 48;
+
 template <int NMAX>
 struct Cfg {
   static_assert(NMAX <= 128, "B scale factors of a 4-block group fit one 4-column TMEM slot");
@@ -596,7 +600,12 @@ __device__ __forceinline__ int tile_row(const JobRows &j, int m) {
 // the A operand straight from shared memory, and four scale-factor warps replace the decode warps.
 // CARRY: trellis segments longer than a block (seg_len = 32 * seg_blocks): each block's state
 // continues from the previous block of its segment.
-template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY>
+// RS: register split. The launch gives every thread the same registers (768 threads x 80 = 61440
+// at NMAX = 32); the decode warps, which carry eight blocks' words and codes, take 96 each and the
+// eight other warps give theirs down to 48 (16 x 32 x 96 + 8 x 32 x 48 = 61440). Launched only after
+// the host has checked that the compiled kernel's registers cover that sum, since a larger request
+// than the launch holds would never be granted.
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS = false>
 __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
                                                      const __grid_constant__ MoeTable<MAXE> tab,
                                                      const __grid_constant__ CUtensorMap wmap) {
@@ -670,6 +679,16 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   const int my_jobs = (int)blockIdx.x < njobs ? (njobs - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int nq = my_jobs * S;
   auto job_of = [&](int jl) { return (int)blockIdx.x + jl * (int)gridDim.x; };
+  if constexpr (RS) {
+    static_assert(!MX && C::kThreads == 768 && C::kDecWarps == 16 && C::kDecWarps % 4 == 0 &&
+                      C::kDecWarps * 32 * kRsDecRegs + (C::kThreads - C::kDecWarps * 32) * kRsOtherRegs ==
+                          C::kThreads * kRsLaunchRegs,
+                  "register split: the shares add up to the launch's registers");
+    if (warp < C::kDecWarps)
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRsDecRegs));
+    else
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRsOtherRegs));
+  }
 
   if (MX && warp < C::kDecWarps) {
     // ---------------------------------------------------------------- scale-factor warps (MX)
@@ -1293,14 +1312,38 @@ static int sm_count() {
 }
 
 // One launch of a product kernel instance (dynamic shared memory attribute set once per instance).
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS>
+static cudaError_t launch_product_rs(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
+                                     cudaStream_t s) {
+  static unsigned long long attr = 0;
+  cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS>, attr);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS>, dim3(grid), dim3(Cfg<NMAX>::kThreads),
+                          mma_geom<NMAX>(MODE, MX).smem, s, args, tab, map);
+}
+
+// True when the register-split instance was compiled with at least kRsLaunchRegs registers per
+// thread, so that its split can be granted (checked once per instance).
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY>
+static bool register_split_ok() {
+  static int ok = -1;
+  if (ok < 0) {
+    cudaFuncAttributes fa;
+    ok = cudaFuncGetAttributes(&fa, k_mma<MAXE, MODE, NMAX, MX, CARRY, true>) == cudaSuccess &&
+         fa.numRegs >= kRsLaunchRegs;
+  }
+  return ok == 1;
+}
+
+// The decode GEMV at NMAX = 32 takes the register split when its compiled registers allow it.
 template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY>
 static cudaError_t launch_product(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
                                   cudaStream_t s) {
-  static unsigned long long attr = 0;
-  cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, MODE, NMAX, MX, CARRY>, attr);
-  if (e != cudaSuccess) return e;
-  return launch_dependent(k_mma<MAXE, MODE, NMAX, MX, CARRY>, dim3(grid), dim3(Cfg<NMAX>::kThreads),
-                          mma_geom<NMAX>(MODE, MX).smem, s, args, tab, map);
+  if constexpr (MODE == kModeGemv && NMAX == 32 && !MX) {
+    if (register_split_ok<MAXE, MODE, NMAX, MX, CARRY>())
+      return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, true>(grid, args, tab, map, s);
+  }
+  return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, false>(grid, args, tab, map, s);
 }
 template <int MAXE, int MODE, int NMAX, bool MX>
 static cudaError_t launch_product_seg(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
