@@ -44,7 +44,7 @@ FALLBACK_HBM_GBS = 6650.0
 # decoded weight, for the kernel as it is now; None when not yet measured for this kernel version.
 # gemv: 153,369,088 bytes over the 530,841,600 weights of the gate_up launch; expand:
 # 375,607,040 bytes over the same weights (profiles/k_mma_gemv_gate_up.md, profiles/k_expand_gate_up.md).
-NCU_TRAFFIC_B_PER_WEIGHT = {"expand": 375607040 / 530841600, "gemv": 153369088 / 530841600}
+NCU_TRAFFIC_B_PER_WEIGHT = {"expand": 375607040 / 530841600, "gemv": 153748224 / 530841600}
 
 
 def measured_hbm_peak():
