@@ -128,6 +128,43 @@ def test_gemv_2048_square_batch1(seg):
     assert_products_close(y, y_exact, wn, xnorms(xb), "2048^2")
 
 
+@pytest.mark.parametrize("T", [1, 32])
+def test_gemv_full_moe_layer_sampled(T):
+    # Every expert matrix of the 32-expert hidden-2880 layer stacked (gate_up 184320 x 2880, down
+    # 92160 x 2880): the shapes and launch configuration the bench times at T = 1 (register-split
+    # instance), and T = 32 (the largest batch, two passes of the 16-token instance). 64 sampled
+    # rows per matrix against the oracle, plus every output finite.
+    E, H, I = 32, 2880, 2880
+    layer = synth.moe_layer(E, H, I, seed=synth.SEED_BASE + 1)
+    r = np.random.default_rng(6 + T)
+    x = synth.activations(T, H, seed=60 + T)
+    xb = synth.bf16_bits(x)
+    for st, sc, rows, cols in ((layer.gu_stream, layer.gu_scales, E * 2 * I, H),
+                               (layer.dn_stream, layer.dn_scales, E * H, I)):
+        W = tc.TrellisMatrix.from_numpy(st, sc, rows, cols, 32)
+        assert tc.gemv_workspace_bytes(W, T) > 0
+        y = tc.gemv(W, x.cuda())
+        torch.cuda.synchronize()
+        assert torch.isfinite(y.float()).all()
+        sample = np.concatenate([[0, rows - 1], r.choice(rows, 62, replace=False)])
+        y_exact, wn = oracle.gemv(st, sc, rows, cols, 32, xb, row_ids=sample)
+        assert_products_close(y[:, torch.from_numpy(sample).cuda()], y_exact, wn, xnorms(xb),
+                              f"{rows}x{cols} T={T}")
+
+
+@pytest.mark.parametrize("T", [1, 32])
+def test_gemv_largest_cols(T):
+    # cols = 16384, the largest trellis_gemv takes (512 blocks, 16 stages per row)
+    rows, cols = 130, 16384
+    st, sc, W = upload_matrix(rows, cols, seed=2600 + T)
+    x = synth.activations(T, cols, seed=2600 + T)
+    y = tc.gemv(W, x.cuda())
+    torch.cuda.synchronize()
+    xb = synth.bf16_bits(x)
+    y_exact, wn = oracle.gemv(st, sc, rows, cols, 32, xb)
+    assert_products_close(y, y_exact, wn, xnorms(xb), f"cols={cols} T={T}")
+
+
 def test_gemv_one_hot_returns_exact_columns():
     rows, cols = 67, 256
     st, sc, W = upload_matrix(rows, cols, seed=31, seg_len=128)
