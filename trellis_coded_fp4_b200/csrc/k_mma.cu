@@ -277,8 +277,9 @@ __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict_
 }
 
 // MoE: group g's token slot i is pair list[g_first + i]; its activation row is src[pair / div]
-// (gate_up reads x rows of tokens: div = k; down reads h rows of pairs: div = 1). Block 0 also
-// clears the down kernel's counters when `counters` is given.
+// (rows of tokens: div = k, as for x before gate/up; rows of pairs: div = 1). The down product's
+// terms do not come from here: the gate/up epilogue writes them. Block 0 also clears the down
+// kernel's counters when `counters` is given.
 template <int NMAX, bool NAT>
 __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ ids, int P, int E, int div,
                                                     const uint16_t *__restrict__ src, int K, uint8_t *__restrict__ terms,
@@ -726,7 +727,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
           jl_p++;
         }
       };
-      grid_dep_wait();  // the activation terms (B scales) come from the preceding split kernel
+      grid_dep_wait();  // the activation terms (B scales) come from the preceding kernel (a split, or gate/up)
       load_sf(pa, pb);
       uint32_t b = 0;
       bool ok = true;
@@ -807,7 +808,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         jl_p++;
       }
     };
-    grid_dep_wait();  // the activation terms (B scales) come from the preceding split kernel
+    grid_dep_wait();  // the activation terms (B scales) come from the preceding kernel (a split, or gate/up)
     load_sf(pa, pb);
 
     // Barrier latencies are hidden: the release of this stage's A slot and the arrival of the next
@@ -1002,7 +1003,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   } else if (warp == C::kBLoadWarp) {
     // ---------------------------------------------------------------- B loader warp
     int issued = 0;
-    grid_dep_wait();     // the activation terms come from the preceding split kernel
+    grid_dep_wait();     // the activation terms come from the preceding kernel (a split, or gate/up)
     grid_dep_release();  // a dependent launch may start its prologue now
     if (lane == 0) {
       int jl = 0, s = 0;
