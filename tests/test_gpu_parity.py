@@ -1,6 +1,6 @@
 """GPU parity: the CUDA library (through its C ABI) against the CPU oracle on the same inputs.
 
-Bit-exact for the MXFP4 expansion (nibbles and scales); the benchmark spec's tolerance
+Bit-exact for the MXFP4 expansion (nibbles and scales); the stated tolerance
 |y - exact| <= 2e-3 ||w_row|| ||x|| for products; exact ids for routing.
 """
 import numpy as np
