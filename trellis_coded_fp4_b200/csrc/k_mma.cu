@@ -258,7 +258,8 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
   split_terms_n<NMAX, NAT, 1>(&v, t, t + 1, kb, S_total, terms);
 }
 
-// Plain GEMV: one group, token slots 0..T-1 (slots up to kSlots are zero rows).
+// Plain GEMV: one group, token slots 0..T-1. The B rows of the other slots are not written: an MMA
+// column depends only on its own B row (and its scale), and no output reads those columns.
 // The GEMV's product kernel is launched as a programmatic dependent of this split: it starts its
 // TMEM setup and its first weight tiles (which do not depend on the split) at once and waits for
 // the split's completion only before it reads the activation terms.
@@ -269,17 +270,17 @@ __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict_
   grid_dep_release();  // the product kernel may start; it waits for this grid before reading terms
   const int nb = K >> 5, S = (nb + Cfg<NMAX>::kKB - 1) / Cfg<NMAX>::kKB, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < Cfg<NMAX>::kSlots * nb; wi += nwarps) {
+  for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < T * nb; wi += nwarps) {
     const int t = wi / nb, kb = wi - t * nb;
-    const float v = t < T ? __uint_as_float((uint32_t)x[(size_t)t * K + kb * 32 + lane] << 16) : 0.f;
-    split_terms<NMAX, NAT>(v, t, kb, S, terms);
+    split_terms<NMAX, NAT>(__uint_as_float((uint32_t)x[(size_t)t * K + kb * 32 + lane] << 16), t, kb, S, terms);
   }
 }
 
 // MoE: group g's token slot i is pair list[g_first + i]; its activation row is src[pair / div]
-// (rows of tokens: div = k, as for x before gate/up; rows of pairs: div = 1). The down product's
-// terms do not come from here: the gate/up epilogue writes them. Block 0 also clears the down
-// kernel's counters when `counters` is given.
+// (rows of tokens: div = k, as for x before gate/up; rows of pairs: div = 1). Only the slots that
+// hold a pair are split (the B rows of empty slots feed MMA columns nothing reads). The down
+// product's terms do not come from here: the gate/up epilogue writes them. Block 0 also clears the
+// down kernel's counters when `counters` is given.
 template <int NMAX, bool NAT>
 __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ ids, int P, int E, int div,
                                                     const uint16_t *__restrict__ src, int K, uint8_t *__restrict__ terms,
@@ -293,16 +294,19 @@ __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ 
   const int nb = K >> 5, S = (nb + Cfg<NMAX>::kKB - 1) / Cfg<NMAX>::kKB;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int per_group = Cfg<NMAX>::kSlots * nb;
-  for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < pl.n_groups * per_group; wi += nwarps) {
-    const int g = wi / per_group, r = wi - g * per_group;
-    const int t = r / nb, kb = r - t * nb;
-    float v = 0.f;
-    if (t < pl.g_cnt[g]) {
-      const int row = pl.list[pl.g_first[g] + t] / div;
-      v = __uint_as_float((uint32_t)src[(size_t)row * K + kb * 32 + lane] << 16);
+  // the routed pairs in list order: entry i belongs to the group g with g_first[g] <= i (groups are
+  // consecutive runs of the list, in order), as slot i - g_first[g]
+  const int npairs = pl.n_groups > 0 ? pl.g_first[pl.n_groups - 1] + pl.g_cnt[pl.n_groups - 1] : 0;
+  for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < npairs * nb; wi += nwarps) {
+    const int i = wi / nb, kb = wi - i * nb;
+    int lo = 0, hi = pl.n_groups - 1;  // the last group whose first entry is <= i
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pl.g_first[mid] <= i) lo = mid; else hi = mid - 1;
     }
-    split_terms<NMAX, NAT>(v, t, kb, S, terms + (size_t)g * terms_bytes<NMAX>(S));
+    const int row = pl.list[i] / div;
+    split_terms<NMAX, NAT>(__uint_as_float((uint32_t)src[(size_t)row * K + kb * 32 + lane] << 16), i - pl.g_first[lo],
+                           kb, S, terms + (size_t)lo * terms_bytes<NMAX>(S));
   }
 }
 
@@ -1361,7 +1365,7 @@ template <int NMAX, bool MX>
 static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, const uint16_t *x, int T, uint16_t *y,
                                     void *ws, cudaStream_t s) {
   uint8_t *terms = static_cast<uint8_t *>(ws);
-  const int warps = Cfg<NMAX>::kSlots * w.nbr;
+  const int warps = T * w.nbr;
   cudaError_t e =
       launch_dependent(k_bsplit_gemv<NMAX, MX>, dim3((warps + 7) / 8), dim3(256), 0, s, x, T, w.nbr * 32, terms);
   if (e != cudaSuccess) return e;
@@ -1484,7 +1488,7 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
   {
     uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_gu);
     const int nbr = m.H / 32;
-    const int warps = G * Cfg<NMAX>::kSlots * nbr;
+    const int warps = P * nbr;  // one warp per routed pair and 32-block
     cudaError_t e = launch_dependent(k_bsplit_moe<NMAX, MX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
                                      dim3(256), 0, s, ids, P, m.E, k, x, m.H, terms, args.counters,
                                      4 * ((m.H + 127) / 128));
