@@ -98,3 +98,49 @@ def test_moe_workspace_and_checks(lib):
     mixed = _abi.Moe(gu, dn2, E, H, I)                                        # mixed seg_len
     assert lib.trellis_grouped_moe(ctypes.byref(mixed), p, 3, p, p, 2, p, p, ws, s0) == 3
     assert lib.trellis_grouped_moe(ctypes.byref(m), p, 0, p, p, 2, p, p, ws, s0) == 0
+
+
+def test_repack_argument_checks(lib):
+    s0 = ctypes.c_void_p(0)
+    a, b = ctypes.c_void_p(4096), ctypes.c_void_p(1 << 20)
+    rp = lib.trellis_repack_interleaved
+    assert rp(a, 2, 48, b, s0) == 1                        # cols % 32
+    assert rp(a, -1, 32, b, s0) == 1                       # rows < 0
+    assert rp(ctypes.c_void_p(0), 2, 32, b, s0) == 1       # null input
+    assert rp(a, 2, 32, ctypes.c_void_p(0), s0) == 1       # null output
+    assert rp(ctypes.c_void_p(4100), 2, 32, b, s0) == 2    # 4-byte aligned input
+    assert rp(a, 2, 32, ctypes.c_void_p((1 << 20) + 4), s0) == 2
+    assert rp(a, 4, 32, ctypes.c_void_p(4096 + 8), s0) == 1   # partial overlap (32 bytes from 4096)
+    assert rp(ctypes.c_void_p(4096 + 24), 4, 32, a, s0) == 1  # overlap from the other side
+    assert rp(a, 1 << 31, 32 * 2, b, s0) == 3              # 2^32 blocks
+    assert rp(a, 0, 32, b, s0) == 0 and rp(a, 3, 0, b, s0) == 0   # nothing to do
+
+
+def test_e5m3_gemv_argument_checks(lib):
+    s0 = ctypes.c_void_p(0)
+    ok_x, ok_y = ctypes.c_void_p(4096), ctypes.c_void_p(8192)
+    g = lib.trellis_gemv_e5m3
+    assert g(_mat(cols=48), ok_x, 1, ok_y, s0) == 1
+    assert g(_mat(seg=96), ok_x, 1, ok_y, s0) == 1
+    assert g(_mat(stream=8), ok_x, 1, ok_y, s0) == 2
+    assert g(_mat(), ctypes.c_void_p(4098), 1, ok_y, s0) == 2
+    assert g(_mat(), ok_x, 1, ctypes.c_void_p(8200), s0) == 2
+    assert g(_mat(), ok_x, 33, ok_y, s0) == 3
+    assert g(_mat(), ok_x, -1, ok_y, s0) == 1
+    assert g(_mat(), ctypes.c_void_p(0), 1, ok_y, s0) == 1
+    assert g(_mat(), ok_x, 0, ok_y, s0) == 0 and g(_mat(rows=0), ok_x, 1, ok_y, s0) == 0
+
+
+def test_encode_argument_checks(lib):
+    s0 = ctypes.c_void_p(0)
+    p8, p16 = ctypes.c_void_p(8 * 512), ctypes.c_void_p(16 * 512)
+    ws = ctypes.c_void_p(256 * 64)
+    e = lib.trellis_encode
+    assert e(p8, p8, p16, 2, 64, 48, p8, s0, ws, 1 << 20, s0) == 1    # seg % 32
+    assert e(p8, p8, p16, 2, 64, 128, p8, s0, ws, 1 << 20, s0) == 1   # seg > cols
+    assert e(p8, p8, p16, 2, 48, 32, p8, s0, ws, 1 << 20, s0) == 1    # cols % 32
+    assert e(ctypes.c_void_p(8 * 512 + 4), p8, p16, 2, 64, 32, p8, s0, ws, 1 << 20, s0) == 2
+    assert e(p8, p8, p16, 2, 64, 32, p8, s0, s0, 0, s0) == 4          # no workspace
+    assert e(p8, p8, p16, 2, 64, 32, p8, s0, ctypes.c_void_p(256 * 64 + 128), 1 << 20, s0) == 2
+    assert e(p8, p8, p16, 1 << 20, 1 << 12, 32, p8, s0, ws, 1 << 20, s0) == 3   # 2^32 weights
+    assert e(p8, p8, p16, 0, 64, 32, p8, s0, s0, 0, s0) == 0
