@@ -256,6 +256,46 @@ class Step:
                 "gemv_gate_up": self.nG, "gemv_down": self.nD}
 
 
+def batch_sweep(step, device, n):
+    """Fused decode GEMV and MXFP4 GEMV of the 184320 x 2880 gate_up matrix at T = 1 .. 32: CUDA-event
+    time per call over n calls back to back after warm-up, algorithmic bytes (stream or nibbles, scales,
+    activations and outputs) per second, and the fraction of the measured copy peak."""
+    tc = step.tc
+    peak, _ = measured_hbm_peak()
+    G = step.G
+    Gm = tc.Mxfp4Matrix(step.nibG, step.scG, G.rows, G.cols)
+    tc.decode_to_mxfp4(G, step.nibG, step.scG)
+    out = {"sweep": "gemv gate_up 184320x2880", "calls": n, "peak_gb_s": peak, "rows": []}
+    for T in (1, 2, 4, 8, 16, 32):
+        x = synth_activations(T, G.cols, device)
+        y = torch.empty((T, G.rows), dtype=torch.bfloat16, device=device)
+        row = {"T": T}
+        for name, fn, w, wbytes in (("fused", tc.gemv, G, G.rows * G.cols // 4),
+                                    ("mxfp4", tc.mxfp4_gemv, Gm, G.rows * G.cols // 2)):
+            ws = torch.empty(max(1, tc.gemv_workspace_bytes(G, T)), dtype=torch.uint8, device=device)
+            for _ in range(3):
+                fn(w, x, y, ws)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(n):
+                fn(w, x, y, ws)
+            e1.record()
+            torch.cuda.synchronize()
+            us = 1e3 * e0.elapsed_time(e1) / n
+            nbytes = wbytes + G.rows * G.cols // 32 + 2 * G.cols * T + 2 * G.rows * T
+            gbs = nbytes / (us * 1e-6) / 1e9
+            row[name] = {"us": round(us, 2), "gb_s": round(gbs, 1), "frac": round(gbs / peak, 3)}
+        out["rows"].append(row)
+    out["timeouts"] = tc.device_timeouts()
+    return out
+
+
+def synth_activations(T, cols, device):
+    from trellis_coded_fp4_b200 import synth
+    return synth.activations(T, cols, seed=synth.SEED_BASE + 90 + T).to(device)
+
+
 def run_e2e(step, steps, device):
     """The same step through the public API with HOST buffers: every input (stream words, scales,
     activations, logits) is copied from pinned host memory and every output (MXFP4 nibbles and
@@ -399,6 +439,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", default=None,
                     help="run only this call of the step (e.g. gemv_gate_up), for profiling one kernel")
+    ap.add_argument("--sweep", action="store_true",
+                    help="batch sweep instead of the step: fused decode GEMV and MXFP4 GEMV of the gate_up "
+                         "matrix at T = 1, 2, 4, 8, 16, 32 (one JSON line, not a bench line)")
     args = ap.parse_args()
     if args.impl == "reference":
         return reference_arm(args)
@@ -418,6 +461,9 @@ def main():
     build.build()
     seed = synth.SEED_BASE + 1 + rank
     step = Step(seed, device)
+    if args.sweep:
+        print(json.dumps(batch_sweep(step, device, max(10, args.steps // 10))))
+        return 0
     if args.only is not None:  # profiling mode: a few launches of one call, no timing line
         for i in range(args.warmup + args.steps):
             step.run(i, only=args.only)
