@@ -297,7 +297,13 @@ def pack_symbols(sym, rows, cols):
 # ----------------------------------------------------------------------------- routing and MoE
 
 def route(logits, k):
-    """Top-k experts per token (ties -> lower index) and fp64 softmax over the selected logits."""
+    """Top-k experts per token and fp64 softmax over the selected logits.
+
+    Ranking: larger logit first, ties -> lower index; a NaN logit ranks below every number
+    (-inf included), so k valid expert ids always come out. Weights: softmax over the k selected
+    logits with NaN read as -inf; when the largest selected logit is -inf every weight is 0 (the
+    token routes nowhere), and when it is +inf the +inf logits share the weight equally (the limit
+    of the softmax)."""
     logits = np.asarray(logits, np.float64)
     T, E = logits.shape
     if not 1 <= k <= E:
@@ -305,11 +311,18 @@ def route(logits, k):
     ids = np.zeros((T, k), np.int32)
     w = np.zeros((T, k), np.float64)
     for t in range(T):
-        order = sorted(range(E), key=lambda e: (-logits[t, e], e))[:k]
-        sel = np.array([logits[t, e] for e in order])
-        ex = np.exp(sel - sel.max())
+        order = sorted(range(E), key=lambda e: (bool(np.isnan(logits[t, e])),
+                                                0.0 if np.isnan(logits[t, e]) else -logits[t, e], e))[:k]
+        sel = np.array([-np.inf if np.isnan(logits[t, e]) else logits[t, e] for e in order])
         ids[t] = order
-        w[t] = ex / ex.sum()
+        mx = sel.max()
+        if mx == -np.inf:
+            w[t] = 0.0
+        elif mx == np.inf:
+            w[t] = (sel == np.inf) / np.count_nonzero(sel == np.inf)
+        else:
+            ex = np.exp(sel - mx)
+            w[t] = ex / ex.sum()
     return ids, w
 
 

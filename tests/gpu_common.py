@@ -1,7 +1,19 @@
 """Shared helpers for the GPU parity tests: upload synthetic inputs, compare with the oracle.
 
 Tolerance for products (fp32 accumulation, bf16 out): |y_gpu - y_exact| <= 2e-3 ||w_row|| ||x_t||
-per output, against the unrounded exact product.
+per output, against the unrounded exact product (the stated target). A second, tighter check
+holds the kernels to the error their own design allows:
+
+    |y_gpu - y_exact| <= (sqrt(32) 5^-6 + 1.5 max((K/32 + 16) 2^-20, K 2^-24)) ||w|| ||x|| + ulp(y)/2
+
+* sqrt(32) 5^-6: the tensor-core path writes each bf16 32-block of x as six E2M1 terms; every
+  element is then off by at most 5^-6 of its block's largest magnitude, so the block's error
+  vector has norm <= sqrt(32) 5^-6 ||x_block||;
+* the fp32 accumulation, with room to spare: at most K/32 + 16 roundings of at most 2^-20 of the
+  running sum on the tensor cores (blocks are summed exactly inside an MMA), or K roundings of
+  2^-24 for the CUDA-core kernels' sequential FMA chain; the running sums are bounded by
+  sum |w_k| sum_j |term_jk| <= 1.5 ||w|| ||x||;
+* half a bf16 unit in the last place of the output.
 """
 import numpy as np
 import torch
@@ -11,6 +23,18 @@ import trellis_coded_fp4_b200 as tc
 from trellis_coded_fp4_b200 import synth
 
 TOL = 2e-3
+
+
+def tight_tol(cols):
+    """The design's own relative bound for K = cols (the ulp term is added per output)."""
+    return 32 ** 0.5 * 5.0 ** -6 + 1.5 * max((cols / 32 + 16) * 2.0 ** -20, cols * 2.0 ** -24)
+
+
+def half_ulp_bf16(v):
+    """Half a bf16 ulp at |v| (0 at v = 0)."""
+    a = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - 8), 0.0)
 
 
 def upload_matrix(rows, cols, seed, seg_len=32, lo=120, hi=126):
@@ -23,16 +47,36 @@ def bf16_to_f64(t):
     return oracle.bf16_bits_to_f64(synth.bf16_bits(t.cpu()))
 
 
-def assert_products_close(y_gpu, y_exact, wnorm, xnorm, what=""):
-    """y_gpu: bf16 tensor [T][n]; y_exact [T][n] fp64; wnorm [n]; xnorm [T]."""
+def assert_products_close(y_gpu, y_exact, wnorm, xnorm, what="", cols=None):
+    """y_gpu: bf16 tensor [T][n]; y_exact [T][n] fp64; wnorm [n]; xnorm [T].
+    cols: the reduction length K; when given, the design bound (module docstring) is checked too."""
     got = bf16_to_f64(y_gpu)
-    bound = TOL * np.outer(xnorm, wnorm)
+    wx = np.outer(xnorm, wnorm)
+    bound = TOL * wx
     err = np.abs(got - y_exact)
     bad = err > bound
     if bad.any():
         i = np.argwhere(bad)[0]
         raise AssertionError(f"{what}: {bad.sum()} outputs out of tolerance; first {tuple(i)}: gpu {got[tuple(i)]!r} "
                              f"exact {y_exact[tuple(i)]!r} bound {bound[tuple(i)]!r}")
+    if cols is not None:
+        tight = tight_tol(cols) * wx + half_ulp_bf16(np.maximum(np.abs(got), np.abs(y_exact)))
+        bad = err > tight
+        if bad.any():
+            i = np.argwhere(bad)[0]
+            raise AssertionError(f"{what}: {bad.sum()} outputs outside the design bound; first {tuple(i)}: gpu "
+                                 f"{got[tuple(i)]!r} exact {y_exact[tuple(i)]!r} bound {tight[tuple(i)]!r}")
+
+
+def assert_mostly_correctly_rounded(y_gpu, y_exact, what="", max_frac=0.02):
+    """For N(0,1) inputs the kernels' error is ~1e-6 of ||w|| ||x||, far below a bf16 ulp of y, so
+    almost every output must be the correctly rounded exact product; an error the size of a
+    dropped activation term or a wrong code in a small-scale block moves many of them."""
+    got = bf16_to_f64(y_gpu)
+    ref = torch.from_numpy(np.ascontiguousarray(y_exact)).to(torch.float32).to(torch.bfloat16).double().numpy()
+    # y_exact -> fp32 is one extra rounding; only outputs within 2^-24 relative of a tie can differ
+    frac = float((got != ref).mean())
+    assert frac <= max_frac, f"{what}: {frac:.4f} of outputs are not the correctly rounded product"
 
 
 def xnorms(x_bits):

@@ -33,7 +33,7 @@ def test_e5m3_gemv_matches_oracle(rows, cols, T):
         torch.cuda.synchronize()
         xb = synth.bf16_bits(x.cpu())
         y_ex, wn = oracle.gemv(st, sc, rows, cols, seg, xb, scale_fmt="e5m3")
-        assert_products_close(y, y_ex, wn, xnorms(xb), f"e5m3 {rows}x{cols} T={T} seg={seg}")
+        assert_products_close(y, y_ex, wn, xnorms(xb), f"e5m3 {rows}x{cols} T={T} seg={seg}", cols=cols)
 
 
 def test_zero_mantissa_is_bit_identical_to_ue8m0():
@@ -76,7 +76,8 @@ def test_e5m3_full_size_sampled():
     sample = np.concatenate([[0, rows - 1], np.random.default_rng(4).choice(rows, 62, replace=False)])
     xb = synth.bf16_bits(x.cpu())
     y_ex, wn = oracle.gemv(st, sc, rows, cols, 32, xb, row_ids=sample, scale_fmt="e5m3")
-    assert_products_close(y[:, torch.from_numpy(sample).cuda()], y_ex, wn, xnorms(xb), "e5m3 full size")
+    assert_products_close(y[:, torch.from_numpy(sample).cuda()], y_ex, wn, xnorms(xb), "e5m3 full size",
+                          cols=cols)
 
 
 def test_e5m3_argument_errors():

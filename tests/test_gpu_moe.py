@@ -59,7 +59,7 @@ def test_moe_32_experts_hidden_2880_batch1():
     check_moe(layer, W, x, ids, wts, out, ws, k, 32)
 
 
-@pytest.mark.parametrize("T", [2, 8, 32])
+@pytest.mark.parametrize("T", [2, 4, 8, 16, 32])
 def test_moe_32_experts_batch_sweep_sampled(T):
     E, H, I, k = 32, 2880, 2880, 4
     layer = synth.moe_layer(E, H, I, seed=synth.SEED_BASE + 3)
@@ -69,14 +69,25 @@ def test_moe_32_experts_batch_sweep_sampled(T):
               rows_out=r.choice(H, 48, replace=False))
 
 
-@pytest.mark.parametrize("T", [1, 8])
-def test_moe_256_experts_hidden_7168_sampled(T):
-    E, H, I, k = 256, 7168, 2048, 8
+@pytest.fixture(scope="module")
+def layer_7168():
+    # 256 experts, hidden 7168, intermediate 2048 (11.3 G weights, 3.17 GB resident), built once
+    E, H, I = 256, 7168, 2048
     layer = synth.moe_layer(E, H, I, seed=synth.SEED_BASE + 4, lo=118, hi=126)
-    W, x, ids, wts, out, ws = _run(layer, T, k, synth.SEED_BASE + 4 + T)
+    return layer, tc.MoEWeights.from_layer(layer, seg_len=32)
+
+
+@pytest.mark.parametrize("T", [1, 8, 32])
+def test_moe_256_experts_hidden_7168_sampled(layer_7168, T):
+    layer, W = layer_7168
+    k = 8
+    x = synth.activations(T, layer.H, seed=synth.SEED_BASE + 4 + T).cuda()
+    ids, wts = tc.moe_route(synth.logits(T, layer.E, seed=synth.SEED_BASE + 4 + T).cuda(), k)
+    out, ws = tc.grouped_moe(W, x, ids, wts)
+    torch.cuda.synchronize()
     r = np.random.default_rng(100 + T)
-    check_moe(layer, W, x, ids, wts, out, ws, k, 32, rows_h=r.choice(I, 24, replace=False),
-              rows_out=r.choice(H, 24, replace=False))
+    check_moe(layer, W, x, ids, wts, out, ws, k, 32, rows_h=r.choice(layer.I, 24, replace=False),
+              rows_out=r.choice(layer.H, 24, replace=False))
 
 
 def test_moe_tensor_core_path_many_tokens_per_expert():

@@ -13,7 +13,8 @@ import oracle
 import trellis_coded_fp4_b200 as tc
 from trellis_coded_fp4_b200 import _abi, synth
 
-from gpu_common import assert_products_close, check_moe, mx_product, upload_mx, xnorms
+from gpu_common import (assert_products_close, bf16_to_f64, check_moe, half_ulp_bf16, mx_product, upload_matrix,
+                        upload_mx, xnorms)
 
 pytestmark = pytest.mark.gpu
 
@@ -36,7 +37,7 @@ def test_mxfp4_gemv_small(rows, cols, T):
     torch.cuda.synchronize()
     xb = synth.bf16_bits(x.cpu())
     ye, wn = oracle.mxfp4_gemv(nib, sc, rows, cols, xb)
-    assert_products_close(y, ye, wn, xnorms(xb), f"mxfp4_gemv {rows}x{cols} T={T}")
+    assert_products_close(y, ye, wn, xnorms(xb), f"mxfp4_gemv {rows}x{cols} T={T}", cols=cols)
 
 
 def test_mxfp4_gemv_one_hot_returns_exact_elements():
@@ -64,7 +65,7 @@ def test_mxfp4_gemv_of_expanded_trellis_matrix():
     torch.cuda.synchronize()
     xb = synth.bf16_bits(x.cpu())
     ye, wn = oracle.gemv(st, sc, rows, cols, 32, xb)
-    assert_products_close(y, ye, wn, xnorms(xb), "expanded 2048x2048")
+    assert_products_close(y, ye, wn, xnorms(xb), "expanded 2048x2048", cols=cols)
 
 
 @pytest.mark.parametrize("T", [1, 8])
@@ -79,7 +80,7 @@ def test_mxfp4_gemv_gate_up_size_sampled(T):
     rid = np.sort(np.random.default_rng(T).choice(rows, 400, replace=False))
     xb = synth.bf16_bits(x.cpu())
     ye, wn = oracle.mxfp4_gemv(nib, sc, rows, cols, xb, row_ids=rid)
-    assert_products_close(y[:, torch.from_numpy(rid).cuda()], ye, wn, xnorms(xb), "gate_up size")
+    assert_products_close(y[:, torch.from_numpy(rid).cuda()], ye, wn, xnorms(xb), "gate_up size", cols=cols)
 
 
 def test_mxfp4_gemv_argument_errors():
@@ -169,3 +170,48 @@ def test_mxfp4_moe_32_experts_batch_sweep_sampled(T):
 
 def test_mxfp4_no_bounded_wait_gave_up():
     assert tc.device_timeouts() == 0
+
+
+def _wide_range_activations(T, cols, seed):
+    """bf16 activations whose 32-blocks each span ~2^-24 .. 2^6 with full 8-bit significands: the
+    case where the six-term E2M1 split of a block has the most to do."""
+    r = np.random.default_rng(seed)
+    mant = 1.0 + r.integers(0, 128, (T, cols)) / 128.0
+    expo = r.integers(-24, 7, (T, cols))
+    sign = np.where(r.random((T, cols)) < 0.5, -1.0, 1.0)
+    return torch.from_numpy(sign * mant * 2.0 ** expo).to(torch.float32).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("T", [1, 5, 16])
+def test_activation_split_within_its_bound(T):
+    # Identity weights (E2M1 1.0 at [n][n], zeros elsewhere, scale 2^0) make y[t][n] the kernel's
+    # reconstruction of x[t][n] from its E2M1 terms. Each element must lie within 5^-6 of its
+    # block's largest magnitude (the six-term bound) plus half a bf16 ulp of the output; a split
+    # with fewer terms, or terms dropped from the sum, misses it by orders of magnitude here.
+    n = 1024
+    nib = np.zeros((n, n // 2), np.uint8)
+    idx = np.arange(n)
+    nib[idx, idx // 2] = np.where(idx % 2 == 0, 0x02, 0x20).astype(np.uint8)  # E2M1 code 2 = +1.0
+    sc = np.full((n, n // 32), 127, np.uint8)
+    W = upload_mx(nib, sc)
+    x = _wide_range_activations(T, n, 7600 + T)
+    y = bf16_to_f64(tc.mxfp4_gemv(W, x.cuda()))
+    torch.cuda.synchronize()
+    xv = x.double().numpy()
+    blk_max = np.repeat(np.abs(xv).reshape(T, n // 32, 32).max(axis=2), 32, axis=1)
+    bound = 5.0 ** -6 * blk_max + half_ulp_bf16(np.maximum(np.abs(y), np.abs(xv)))
+    bad = np.abs(y - xv) > bound
+    assert not bad.any(), f"{bad.sum()} elements outside the split bound, first {np.argwhere(bad)[0].tolist()}"
+
+
+@pytest.mark.parametrize("seg", [32, 2880])
+def test_fused_gemv_wide_range_activations(seg):
+    # the trellis GEMV on the same kind of activations, held to the design bound
+    rows, cols, T = 300, 2880, 3
+    st, sc, Wt = upload_matrix(rows, cols, seed=7700 + seg, seg_len=seg)
+    x = _wide_range_activations(T, cols, 7700)
+    y = tc.gemv(Wt, x.cuda())
+    torch.cuda.synchronize()
+    xb = synth.bf16_bits(x)
+    ye, wn = oracle.gemv(st, sc, rows, cols, seg, xb)
+    assert_products_close(y, ye, wn, xnorms(xb), f"wide-range x seg={seg}", cols=cols)

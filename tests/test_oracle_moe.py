@@ -24,6 +24,33 @@ def test_route_matches_stable_argsort_and_softmax():
     assert oracle.route(lg, 4)[0][3, 0] == 5 and oracle.route(lg, 4)[0][3, 1] == 9
 
 
+def test_route_nan_and_infinite_logits():
+    # hand-worked cases of the reading: NaN ranks below every number (-inf included) and weighs as
+    # -inf; a token whose best selected logit is -inf gets zero weights; +inf winners share equally
+    nan, inf = np.nan, np.inf
+    lg = np.array([[nan, -inf, 1.0, nan],
+                   [nan, nan, nan, nan],
+                   [inf, 0.0, inf, -1.0],
+                   [-inf, -inf, nan, -inf],
+                   [2.0, nan, 2.0, 0.0]])
+    ids, w = oracle.route(lg, 3)
+    assert ids.tolist() == [[2, 1, 0], [0, 1, 2], [0, 2, 1], [0, 1, 3], [0, 2, 3]]
+    assert w[0].tolist() == [1.0, 0.0, 0.0]
+    assert w[1].tolist() == [0.0, 0.0, 0.0] and w[3].tolist() == [0.0, 0.0, 0.0]
+    assert w[2].tolist() == [0.5, 0.5, 0.0]
+    assert np.allclose(w[4], scipy.special.softmax([2.0, 2.0, 0.0]), rtol=1e-15, atol=0)
+    # random NaN placement: ranking equals a lexicographic sort on (is NaN, -logit, index)
+    lg = synth.logits(8, 32, seed=43).numpy().astype(np.float64)
+    lg[np.random.default_rng(43).random(lg.shape) < 0.3] = nan
+    for k in (1, 4, 8):
+        ids, w = oracle.route(lg, k)
+        for t in range(lg.shape[0]):
+            ref = np.lexsort((np.arange(32), -np.nan_to_num(lg[t], nan=0.0), np.isnan(lg[t])))[:k]
+            assert ids[t].tolist() == ref.tolist()
+            sel = np.where(np.isnan(lg[t, ref]), -inf, lg[t, ref])
+            assert np.allclose(w[t], scipy.special.softmax(sel), rtol=1e-15, atol=0)
+
+
 def _dense_mlp(layer, e, x_bits, seg_len):
     """Decoded down matrix and the exact gate/up products of expert e, by numpy matmul."""
     H, I = layer.H, layer.I

@@ -6,8 +6,10 @@
 // the scales are copied unchanged.
 //
 // HBM-bound streaming kernel: per 32-weight block it reads 8 bytes of stream and writes 16 bytes
-// of nibbles (plus one scale byte read and written): 0.8125 B/weight. A thread handles pairs of
-// consecutive blocks: one 16-byte load and two 16-byte stores per pair, coalesced across the warp.
+// of nibbles (plus one scale byte read and written): 0.8125 B/weight. When the stream and the
+// output are 32-byte aligned a thread takes four consecutive blocks (one 32-byte load, two 32-byte
+// stores); otherwise pairs of blocks (one 16-byte load, two 16-byte stores). Accesses are
+// coalesced across the warp.
 #include "tcf4_device.cuh"
 #include "tcf4_internal.h"
 

@@ -1,19 +1,14 @@
-// tcf4_tc.cuh -- thin wrappers over the sm_100a tensor-core (tcgen05) and async-copy instructions.
+// tcf4_tc.cuh -- thin wrappers over the sm_100a tensor-core (tcgen05) instructions: TMEM
+// allocation, loads and waits, the shared-memory operand descriptor, commits and barriers.
 //
-// Operand layouts follow the UMMA canonical K-major, no-swizzle form: a tile is made of "core
-// matrices" of 8 rows x 16 bytes (rows 16 bytes apart); SBO is the byte distance between
-// core matrices adjacent along M/N (8-row groups) and LBO between the two 16-byte K chunks of one
-// K=32 MMA step. An E2M1 operand of kind::mxf8f6f4 sits in shared memory unpacked: each 16-byte
-// row chunk holds 16 elements packed in its first 8 bytes (element e in byte e/2, low nibble for
-// even e), the other 8 bytes unused.
+// A shared-memory operand in the UMMA canonical K-major, no-swizzle form is made of "core
+// matrices" of 8 rows x 16 bytes (rows 16 bytes apart); SBO is the byte distance between core
+// matrices adjacent along M/N (8-row groups) and LBO between core matrices adjacent along K.
 #pragma once
 #include <cstdint>
 
 namespace tcf4 {
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -33,14 +28,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 
 // Warp-wide stores/loads between registers and this warp's 32 TMEM lanes (32x32b shape: thread i
 // <-> lane base+i, consecutive 32-bit columns).
-__device__ __forceinline__ void tmem_st_x2(uint32_t taddr, uint32_t a, uint32_t b) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a), "r"(b) : "memory");
-}
-__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -64,31 +51,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   return d;
 }
 
-// Instruction descriptor of a block-scaled kind::mxf8f6f4 MMA: A = E2M1, B = E4M3, both K-major,
-// UE8M0 scale factors, fp32 accumulation (M = 128), N columns, scale-factor bytes a_sf / b_sf.
-__device__ __forceinline__ uint32_t idesc_mxf8f6f4_e2m1_e4m3(uint32_t N, uint32_t a_sf, uint32_t b_sf) {
-  uint32_t d = 0;
-  d |= (b_sf & 3u) << 4;     // B scale-factor id
-  d |= 5u << 7;              // A format: E2M1
-  d |= 0u << 10;             // B format: E4M3
-  d |= (N >> 3) << 17;       // N / 8
-  d |= 1u << 23;             // scale format: UE8M0
-  d |= (128u >> 4) << 24;    // M / 16
-  d |= (a_sf & 3u) << 29;    // A scale-factor id
-  return d;
-}
-
-// One thread: D[tmem] (+)= A[smem] x B[smem] with per-32 block scales from TMEM.
-__device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t sfa_tmem, uint32_t sfb_tmem, bool accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
 // The mbarrier gets one arrival when all tcgen05 operations issued so far by this thread are done.
 __device__ __forceinline__ void tc_commit(uint64_t *bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -100,17 +62,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(bar)))
                : "memory");
 }
-
-// 16-byte async copy global -> shared; only src_bytes (0..16) are read, the rest is zero-filled.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Named barrier among `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar(uint32_t id, uint32_t count) {
