@@ -1,23 +1,34 @@
 #!/usr/bin/env python
-"""Benchmark of the trellis-coded FP4 hot path on B200.
+"""Benchmark of the batch-1 fused trellis-decode GEMV on B200, with every other row of the path.
 
-One step = every step of the path over one batch on the 32-expert, hidden-2880 MoE layer
-(per expert gate_up 5760x2880 and down 2880x2880; 2 bits/weight trellis streams, one UE8M0 scale
-per 32 weights, seg_len 32), inputs resident in HBM:
-  1. expansion of every expert into a resident packed MXFP4 tensor (HEPH serving mode 2):
-     trellis_decode_to_mxfp4 on gate_up [32*5760][2880] and down [32*2880][2880];
-  2. routing of one token (N(0,1) logits, top-4, softmax) and the fused-decode grouped MoE at
-     batch 1 (HEPH serving mode 1): trellis_moe_route + trellis_grouped_moe;
-  3. the batch-1 fused decode GEMV over every expert matrix of the layer: trellis_gemv on
-     gate_up [32*5760][2880] and down [32*2880][2880] with bf16 N(0,1) activations.
-Metric: decoded weights/s over the whole step (and HBM GB/s of the dominant kernel).
+Headline (the metric): one step = one batch-1 fused decode GEMV, y = W x, on the gate_up matrices
+of all 32 experts of the hidden-2880 MoE layer stacked into one matrix (184320 x 2880, 2-bit
+trellis stream, one UE8M0 scale per 32 weights, seg_len 32; bf16 N(0,1) activations, bf16 out),
+through trellis_gemv (the activation split and the decode-MMA product: two launches). Steps rotate
+over three distinct resident matrices (450 MB, > 3x L2) and eight activation vectors, so no step
+finds its weights in L2. value = decoded weights/s of the whole job; roofline = that call.
+
+Extra rows, each timed on its own with CUDA events on the launching stream after warm-up:
+  * gemv_down: the same GEMV on the down matrices stacked (92160 x 2880);
+  * expand: decode-only expansion of the whole layer into resident MXFP4 (gate_up + down);
+  * moe_t1: routing + fused grouped MoE of the layer at batch 1, top-4 of 32;
+  * moe_sweep: the same at T = 1, 2, 4, 8, 16, 32 with N(0,1) routing, and with every token on the
+    same four experts (forced skew), with the kernel instance each call takes;
+  * gemv_sweep: fused decode GEMV and MXFP4 GEMV of the gate_up stack at T = 1 .. 32;
+  * single_2048: one 2048 x 2048 matrix at batch 1, back to back over 512 distinct matrices
+    (576 MB) in a CUDA graph, and the single-call latency with L2 flushed before each call;
+  * moe_7168: the 256-expert hidden-7168 layer (intermediate 2048, top-8, all 3.17 GB of experts
+    resident) at T = 1, 8, 32;
+  * mxfp4_consumer, encoder, repack_interleaved, gemv_e5m3_gate_up: the further rows.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tcf4|reference]
-With N > 1 it runs under torchrun, one independent replica of the step per GPU (weak scaling).
+With N > 1 it runs under torchrun, one independent replica per GPU (weak scaling).
 """
 import argparse
+import concurrent.futures as cf
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -31,20 +42,22 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-E, H, I, K_TOP, T = 32, 2880, 2880, 4, 1
+E, H, I, K_TOP = 32, 2880, 2880, 4
 SEG = 32
+ROT = 3     # distinct resident gate_up matrices the headline steps rotate over
+NVAR = 8    # activation / logits variants
 METRIC = "fused trellis-decode GEMV: decoded weights/s and HBM GB/s (% of B200 peak)"
 UNIT = "decoded weights/s"
-WORKLOAD = ("32-expert hidden-2880 MoE layer (gate_up 5760x2880 + down 2880x2880 per expert, 2-bit trellis, "
-            "UE8M0/32, seg_len 32): expand all experts to MXFP4 + route and fused-decode grouped MoE at batch 1 "
-            "(top-4) + batch-1 fused decode GEMV over every expert matrix")
+WORKLOAD = ("batch-1 fused trellis-decode GEMV on the gate_up matrices of all 32 experts of the hidden-2880 MoE "
+            "layer stacked (184320 x 2880, 2-bit trellis, UE8M0 per 32, seg_len 32), bf16 N(0,1) x, bf16 y")
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0
 
-# DRAM traffic per launch measured with ncu (dram__bytes_read.sum + dram__bytes_write.sum), per
-# decoded weight, for the kernel as it is now; None when not yet measured for this kernel version.
-# gemv: 153,369,088 bytes over the 530,841,600 weights of the gate_up launch; expand:
-# 375,607,040 bytes over the same weights (profiles/k_mma_gemv_gate_up.md, profiles/k_expand_gate_up.md).
-NCU_TRAFFIC_B_PER_WEIGHT = {"expand": 375607040 / 530841600, "gemv": 153748224 / 530841600}
+# DRAM traffic of one launch of the product kernel on this workload, dram__bytes_read.sum +
+# dram__bytes_write.sum from `ncu --set full --clock-control none -k regex:k_mma -c 1` of
+# `python bench.py --only gemv_gate_up --warmup 2 --steps 1`; None until taken for the kernel as
+# it now is.
+NCU_TRAFFIC_GEMV_GATE_UP = None
 
 
 def measured_hbm_peak():
@@ -82,9 +95,6 @@ class ClockSampler:
             self.proc = None
         self.t_start = time.time()
 
-    def mark(self):
-        return time.time()
-
     def stop(self, t0, t1):
         if self.proc is None:
             return None
@@ -110,14 +120,14 @@ class ClockSampler:
                 pass
         if not rows:
             return {"samples": 0}
-        # nvidia-smi -lms writes one row per period from start; map rows to wall-clock times
-        period = 0.05
+        period = 0.05  # nvidia-smi -lms writes one row per period from its start
         times = [self.t_start + i * period for i in range(len(rows))]
         inside = [r for r, t in zip(rows, times) if t0 - period <= t <= t1 + period]
         window = "timed"
         if not inside:
             inside = rows
             window = "whole run (timed region shorter than the sampling period)"
+
         def num(v):
             try:
                 return float(v)
@@ -132,255 +142,421 @@ class ClockSampler:
                 "power_w_max": max([num(r[3]) for r in inside if num(r[3]) is not None] or [0.0])}
 
 
-# ----------------------------------------------------------------------------- the step
+# ----------------------------------------------------------------------------- helpers
 
-class Step:
-    """Device buffers and the 9 launches of one step (all on the current stream)."""
+def gemv_bytes(rows, cols, T, bytes_per_weight=0.28125):
+    """Algorithmic bytes of one product: weights (stream + scales, or nibbles + scales), x in, y out."""
+    return int(rows * cols * bytes_per_weight) + 2 * cols * T + 2 * rows * T
+
+
+def rate(nbytes, us, peak):
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"avg_us": round(us, 3), "algo_bytes": int(nbytes), "gb_s": round(gbs, 1),
+            "frac_of_measured_hbm": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / SPEC_HBM_GBS, 4)}
+
+
+def time_calls(fn, n, warm=3):
+    """Average CUDA-event time in microseconds of fn(i) over n calls back to back (after warm-up)."""
+    for i in range(warm):
+        fn(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(n):
+        fn(i)
+    e1.record()
+    torch.cuda.synchronize()
+    return 1e3 * e0.elapsed_time(e1) / n
+
+
+def time_graph(fn, n, reps=5):
+    """The n calls fn(0..n-1) captured once in a CUDA graph, replayed reps times: microseconds per
+    call (launch overhead of the host excluded)."""
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(n):
+                fn(i)
+    torch.cuda.current_stream().wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = 1e3 * e0.elapsed_time(e1) / (reps * n)
+    del g
+    return us
+
+
+def flush_l2(buf):
+    buf.add_(1)  # read and write a buffer larger than L2
+
+
+def rand_words(n_words, gen, device):
+    """Uniform random 32-bit words (uniform 2-bit trellis symbols) as int32, on the device."""
+    return torch.randint(-2 ** 31, 2 ** 31, (n_words,), dtype=torch.int64, device=device, generator=gen).to(torch.int32)
+
+
+def rand_scales(n, lo, hi, gen, device):
+    return torch.randint(lo, hi + 1, (n,), dtype=torch.int32, device=device, generator=gen).to(torch.uint8)
+
+
+# ----------------------------------------------------------------------------- the 32-expert layer
+
+class Layer:
+    """The 32-expert hidden-2880 layer: stacked gate_up / down matrices (and per-expert views), plus
+    ROT - 1 further random gate_up stacks for the headline rotation."""
 
     def __init__(self, seed, device):
         import trellis_coded_fp4_b200 as tc
         from trellis_coded_fp4_b200 import synth
-        self.tc = tc
+        self.tc, self.device = tc, device
         self.layer = synth.moe_layer(E, H, I, seed=seed)
         lay = self.layer
         self.G = tc.TrellisMatrix.from_numpy(lay.gu_stream, lay.gu_scales, E * 2 * I, H, SEG, device)
         self.D = tc.TrellisMatrix.from_numpy(lay.dn_stream, lay.dn_scales, E * H, I, SEG, device)
-        # expert views onto the same resident buffers
-        gu = self.G.stream.view(E, -1)
-        gus = self.G.scales.view(E, -1)
-        dn = self.D.stream.view(E, -1)
-        dns = self.D.scales.view(E, -1)
+        gen = torch.Generator(device=device).manual_seed(seed)
+        self.Grot = [self.G] + [tc.TrellisMatrix(rand_words(self.G.stream.numel(), gen, device),
+                                                 rand_scales(self.G.scales.numel(), 120, 126, gen, device),
+                                                 self.G.rows, self.G.cols, SEG) for _ in range(ROT - 1)]
+        gu, gus = self.G.stream.view(E, -1), self.G.scales.view(E, -1)
+        dn, dns = self.D.stream.view(E, -1), self.D.scales.view(E, -1)
         self.M = tc.MoEWeights([tc.TrellisMatrix(gu[e], gus[e], 2 * I, H, SEG) for e in range(E)],
                                [tc.TrellisMatrix(dn[e], dns[e], H, I, SEG) for e in range(E)], H, I)
-        nvar = 8  # rotating activations / logits
-        self.x = [synth.activations(T, H, seed=seed, sub=i).to(device) for i in range(nvar)]
-        self.xd = [synth.activations(T, I, seed=seed, sub=100 + i).to(device) for i in range(nvar)]
-        self.logits = [synth.logits(T, E, seed=seed, sub=i).to(device) for i in range(nvar)]
-        self.nibG = torch.empty((E * 2 * I, H // 2), dtype=torch.uint8, device=device)
-        self.scG = torch.empty((E * 2 * I, H // 32), dtype=torch.uint8, device=device)
-        self.nibD = torch.empty((E * H, I // 2), dtype=torch.uint8, device=device)
-        self.scD = torch.empty((E * H, I // 32), dtype=torch.uint8, device=device)
-        self.yG = torch.empty((T, E * 2 * I), dtype=torch.bfloat16, device=device)
-        self.yD = torch.empty((T, E * H), dtype=torch.bfloat16, device=device)
-        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-        self.ids = torch.empty((T, K_TOP), dtype=torch.int32, device=device)
-        self.wts = torch.empty((T, K_TOP), dtype=torch.float32, device=device)
-        self.ws = torch.empty(self.M.workspace_bytes(T, K_TOP), dtype=torch.uint8, device=device)
-        self.wsG = torch.empty(max(1, tc.gemv_workspace_bytes(self.G, T)), dtype=torch.uint8, device=device)
-        self.wsD = torch.empty(max(1, tc.gemv_workspace_bytes(self.D, T)), dtype=torch.uint8, device=device)
-        # expansion 2, route 1, grouped MoE 3 (the split of x, gate/up whose epilogue also splits h,
-        # down), GEMV 2 x (split + product)
-        self.launches_per_step = 2 + 1 + 3 + 4
-        self.nG, self.nD = E * 2 * I * H, E * H * I
-        self.moe_weights = K_TOP * (2 * I * H + H * I)  # distinct experts at T = 1: exactly k
-        self.weights_per_step = self.nG + self.nD + self.moe_weights + self.nG + self.nD
+        self.x = [synth.activations(1, H, seed=seed, sub=i).to(device) for i in range(NVAR)]
+        self.xd = [synth.activations(1, I, seed=seed, sub=100 + i).to(device) for i in range(NVAR)]
+        self.yG = torch.empty((1, E * 2 * I), dtype=torch.bfloat16, device=device)
+        self.yD = torch.empty((1, E * H), dtype=torch.bfloat16, device=device)
+        self.wsG = torch.empty(max(1, tc.gemv_workspace_bytes(self.G, 1)), dtype=torch.uint8, device=device)
+        self.wsD = torch.empty(max(1, tc.gemv_workspace_bytes(self.D, 1)), dtype=torch.uint8, device=device)
+        self.launches_per_step = 2  # the activation split and the decode-MMA product
 
-    def run(self, i, ev=None, only=None):
-        tc = self.tc
-        v = i % len(self.x)
-        if only is not None:
-            calls = {"expand_gate_up": lambda: tc.decode_to_mxfp4(self.G, self.nibG, self.scG),
-                     "expand_down": lambda: tc.decode_to_mxfp4(self.D, self.nibD, self.scD),
-                     "route": lambda: tc.moe_route(self.logits[v], K_TOP, self.ids, self.wts),
-                     "grouped_moe": lambda: tc.grouped_moe(self.M, self.x[v], self.ids, self.wts, self.out, self.ws),
-                     "gemv_gate_up": lambda: tc.gemv(self.G, self.x[v], self.yG, self.wsG),
-                     "gemv_down": lambda: tc.gemv(self.D, self.xd[v], self.yD, self.wsD)}
-            if only == "grouped_moe":
-                calls["route"]()
-            calls[only]()
-            return
-        def mark(name):
-            if ev is not None:
-                e = torch.cuda.Event(enable_timing=True)
-                e.record()
-                ev.append((name, e))
-        mark("expand_gate_up")
-        tc.decode_to_mxfp4(self.G, self.nibG, self.scG)
-        mark("expand_down")
-        tc.decode_to_mxfp4(self.D, self.nibD, self.scD)
-        mark("route")
-        tc.moe_route(self.logits[v], K_TOP, self.ids, self.wts)
-        mark("grouped_moe")
-        tc.grouped_moe(self.M, self.x[v], self.ids, self.wts, self.out, self.ws)
-        mark("gemv_gate_up")
-        tc.gemv(self.G, self.x[v], self.yG, self.wsG)
-        mark("gemv_down")
-        tc.gemv(self.D, self.xd[v], self.yD, self.wsD)
-        mark("end")
+    def step(self, i):
+        self.tc.gemv(self.Grot[i % ROT], self.x[i % NVAR], self.yG, self.wsG)
 
-    # the next row beyond the step: products read straight from the resident MXFP4 tensors that the
-    # step's expansion calls wrote (HEPH serving mode 2, consumer side)
-    def mx_weights(self):
+    def run_only(self, name, i):
+        """One call of one row (profiling mode)."""
         tc = self.tc
-        if not hasattr(self, "_mxG"):
-            self._mxG = tc.Mxfp4Matrix(self.nibG, self.scG, E * 2 * I, H)
-            self._mxD = tc.Mxfp4Matrix(self.nibD, self.scD, E * H, I)
-            ng, sg, nd, sd = self.nibG.view(E, -1), self.scG.view(E, -1), self.nibD.view(E, -1), self.scD.view(E, -1)
-            self._mxM = tc.Mxfp4MoEWeights([tc.Mxfp4Matrix(ng[e], sg[e], 2 * I, H) for e in range(E)],
-                                           [tc.Mxfp4Matrix(nd[e], sd[e], H, I) for e in range(E)], H, I)
-            self._mxws = torch.empty(max(1, self._mxM.workspace_bytes(T, K_TOP)), dtype=torch.uint8,
-                                     device=self.nibG.device)
-        return self._mxG, self._mxD, self._mxM
-
-    def run_mx(self, name, i):
-        tc = self.tc
-        G, D, M = self.mx_weights()
-        v = i % len(self.x)
-        if name == "mxfp4_gemv_gate_up":
-            tc.mxfp4_gemv(G, self.x[v], self.yG, self.wsG)
-        elif name == "mxfp4_gemv_down":
-            tc.mxfp4_gemv(D, self.xd[v], self.yD, self.wsD)
+        if name == "gemv_gate_up":
+            self.step(i)
+        elif name == "gemv_down":
+            tc.gemv(self.D, self.xd[i % NVAR], self.yD, self.wsD)
+        elif name == "expand_gate_up":
+            self._expanded()
+            tc.decode_to_mxfp4(self.G, self.nibG, self.scG)
+        elif name == "grouped_moe":
+            self.moe_call(1)(i)
         else:
-            tc.moe_route(self.logits[v], K_TOP, self.ids, self.wts)
-            tc.mxfp4_grouped_moe(M, self.x[v], self.ids, self.wts, self.out, self._mxws)
+            raise ValueError(name)
 
-    def mx_algo_bytes(self):
-        def gemv(rows, cols):
-            return rows * cols // 2 + rows * cols // 32 + 2 * cols * T + 2 * rows * T
-        return {"mxfp4_gemv_gate_up": gemv(E * 2 * I, H), "mxfp4_gemv_down": gemv(E * H, I),
-                "mxfp4_grouped_moe": K_TOP * (gemv(2 * I, H) + gemv(H, I))}
+    def _expanded(self):
+        if not hasattr(self, "nibG"):
+            d = self.device
+            self.nibG = torch.empty((E * 2 * I, H // 2), dtype=torch.uint8, device=d)
+            self.scG = torch.empty((E * 2 * I, H // 32), dtype=torch.uint8, device=d)
+            self.nibD = torch.empty((E * H, I // 2), dtype=torch.uint8, device=d)
+            self.scD = torch.empty((E * H, I // 32), dtype=torch.uint8, device=d)
+            self.tc.decode_to_mxfp4(self.G, self.nibG, self.scG)
+            self.tc.decode_to_mxfp4(self.D, self.nibD, self.scD)
 
-    # algorithmic bytes per call (what the method must move)
-    def algo_bytes(self):
-        def expand(rows, cols):
-            return rows * cols // 4 + rows * cols // 2 + 2 * (rows * cols // 32)
-        def gemv(rows, cols):
-            return rows * cols // 4 + rows * cols // 32 + 2 * cols * T + 2 * rows * T
-        moe = K_TOP * (gemv(2 * I, H) + gemv(H, I))
-        return {"expand_gate_up": expand(E * 2 * I, H), "expand_down": expand(E * H, I),
-                "route": 4 * T * E + 8 * T * K_TOP, "grouped_moe": moe,
-                "gemv_gate_up": gemv(E * 2 * I, H), "gemv_down": gemv(E * H, I)}
+    def moe_call(self, T, skew=False, mx=False):
+        """fn(i): routing of T tokens (N(0,1) logits, top-4) + the grouped MoE, on preallocated
+        buffers; skew: every token on experts 0..3 with fixed random weights instead."""
+        from trellis_coded_fp4_b200 import synth
+        tc, d = self.tc, self.device
+        xs = [synth.activations(T, H, seed=900 + T, sub=i).to(d) for i in range(NVAR)]
+        lg = [synth.logits(T, E, seed=900 + T, sub=i).to(d) for i in range(NVAR)]
+        ids = torch.empty((T, K_TOP), dtype=torch.int32, device=d)
+        wts = torch.empty((T, K_TOP), dtype=torch.float32, device=d)
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=d)
+        if mx:
+            self._expanded()
+            ng, sg, nd, sd = self.nibG.view(E, -1), self.scG.view(E, -1), self.nibD.view(E, -1), self.scD.view(E, -1)
+            M = tc.Mxfp4MoEWeights([tc.Mxfp4Matrix(ng[e], sg[e], 2 * I, H) for e in range(E)],
+                                   [tc.Mxfp4Matrix(nd[e], sd[e], H, I) for e in range(E)], H, I)
+            run = tc.mxfp4_grouped_moe
+        else:
+            M, run = self.M, tc.grouped_moe
+        ws = torch.empty(max(1, M.workspace_bytes(T, K_TOP)), dtype=torch.uint8, device=d)
+        if skew:
+            ids.copy_(torch.arange(K_TOP, dtype=torch.int32, device=d).repeat(T, 1))
+            wts.copy_(torch.rand((T, K_TOP), generator=torch.Generator().manual_seed(T)).to(d))
 
-    def weights(self):
-        return {"expand_gate_up": self.nG, "expand_down": self.nD, "route": 0, "grouped_moe": self.moe_weights,
-                "gemv_gate_up": self.nG, "gemv_down": self.nD}
-
-
-def batch_sweep(step, device, n):
-    """Fused decode GEMV and MXFP4 GEMV of the 184320 x 2880 gate_up matrix at T = 1 .. 32: CUDA-event
-    time per call over n calls back to back after warm-up, algorithmic bytes (stream or nibbles, scales,
-    activations and outputs) per second, and the fraction of the measured copy peak."""
-    tc = step.tc
-    peak, _ = measured_hbm_peak()
-    G = step.G
-    Gm = tc.Mxfp4Matrix(step.nibG, step.scG, G.rows, G.cols)
-    tc.decode_to_mxfp4(G, step.nibG, step.scG)
-    out = {"sweep": "gemv gate_up 184320x2880", "calls": n, "peak_gb_s": peak, "rows": []}
-    for T in (1, 2, 4, 8, 16, 32):
-        x = synth_activations(T, G.cols, device)
-        y = torch.empty((T, G.rows), dtype=torch.bfloat16, device=device)
-        row = {"T": T}
-        for name, fn, w, wbytes in (("fused", tc.gemv, G, G.rows * G.cols // 4),
-                                    ("mxfp4", tc.mxfp4_gemv, Gm, G.rows * G.cols // 2)):
-            ws = torch.empty(max(1, tc.gemv_workspace_bytes(G, T)), dtype=torch.uint8, device=device)
-            for _ in range(3):
-                fn(w, x, y, ws)
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(n):
-                fn(w, x, y, ws)
-            e1.record()
-            torch.cuda.synchronize()
-            us = 1e3 * e0.elapsed_time(e1) / n
-            nbytes = wbytes + G.rows * G.cols // 32 + 2 * G.cols * T + 2 * G.rows * T
-            gbs = nbytes / (us * 1e-6) / 1e9
-            row[name] = {"us": round(us, 2), "gb_s": round(gbs, 1), "frac": round(gbs / peak, 3)}
-        out["rows"].append(row)
-    out["timeouts"] = tc.device_timeouts()
-    return out
+        def fn(i):
+            if not skew:
+                tc.moe_route(lg[i % NVAR], K_TOP, ids, wts)
+            run(M, xs[i % NVAR], ids, wts, out, ws)
+        fn.ids_of = lambda i: (ids.clone() if skew else tc.moe_route(lg[i % NVAR], K_TOP)[0]).cpu().numpy()
+        fn.keep = (M, xs, lg, ids, wts, out, ws)
+        return fn
 
 
-def synth_activations(T, cols, device):
+def moe_bytes(distinct, T, H_, I_, bpw=0.28125):
+    return int(distinct * (2 * I_ * H_ + H_ * I_) * bpw) + 2 * T * H_ + 2 * T * H_
+
+
+def moe_paths(ids, T):
+    """The product-kernel instance a call takes and its routing groups (same rule as the library:
+    up to 5 tokens per group on the 32-row B operand, else groups of up to 16 on the 96-row one)."""
+    gmax = 5 if T <= 5 else 16
+    cnt = np.bincount(ids.ravel(), minlength=E)
+    groups = int(sum((c + gmax - 1) // gmax for c in cnt if c > 0))
+    return {"instance": "32-row B, two MMA issuers" if gmax == 5 else "96-row B, 16-block stages",
+            "distinct_experts": int((cnt > 0).sum()), "groups": groups, "max_tokens_per_expert": int(cnt.max())}
+
+
+# ----------------------------------------------------------------------------- extra rows
+
+def row_gemv_down(L, n, peak):
+    us = time_calls(lambda i: L.tc.gemv(L.D, L.xd[i % NVAR], L.yD, L.wsD), n)
+    return {**rate(gemv_bytes(E * H, I, 1), us, peak), "decoded_weights_per_s": E * H * I / (us * 1e-6),
+            "shape": "92160 x 2880, T = 1", "calls": n}
+
+
+def row_expand(L, n, peak):
+    L._expanded()
+    tc = L.tc
+    exb = lambda rows, cols: rows * cols // 4 + rows * cols // 2 + 2 * (rows * cols // 32)  # noqa: E731
+
+    def fn(i):
+        tc.decode_to_mxfp4(L.G, L.nibG, L.scG)
+        tc.decode_to_mxfp4(L.D, L.nibD, L.scD)
+    us = time_calls(fn, n)
+    us_g = time_calls(lambda i: tc.decode_to_mxfp4(L.G, L.nibG, L.scG), n)
+    nb = exb(E * 2 * I, H) + exb(E * H, I)
+    return {**rate(nb, us, peak), "decoded_weights_per_s": (E * 2 * I * H + E * H * I) / (us * 1e-6),
+            "gate_up_only": rate(exb(E * 2 * I, H), us_g, peak),
+            "what": "trellis_decode_to_mxfp4 of gate_up (184320 x 2880) then down (92160 x 2880); bit-exact "
+                    "nibbles and scales (tests)", "calls": n}
+
+
+def row_moe(L, T, n, peak, skew=False, mx=False):
+    fn = L.moe_call(T, skew=skew, mx=mx)
+    us = time_calls(fn, n)
+    ids = [fn.ids_of(i) for i in range(1 if skew else NVAR)]
+    paths = [moe_paths(a, T) for a in ids]
+    distinct = statistics.mean(p["distinct_experts"] for p in paths)
+    nb = moe_bytes(distinct, T, H, I, 0.53125 if mx else 0.28125)
+    return {**rate(nb, us, peak), "T": T, "routing": "forced skew (experts 0-3)" if skew else "N(0,1) logits, top-4",
+            "includes_route": not skew, "path": paths[0] if skew else
+            {"instance": paths[0]["instance"], "distinct_experts_mean": distinct,
+             "groups_mean": statistics.mean(p["groups"] for p in paths),
+             "max_tokens_per_expert": max(p["max_tokens_per_expert"] for p in paths)}, "calls": n}
+
+
+def row_gemv_sweep(L, n, peak):
+    tc, d = L.tc, L.device
+    L._expanded()
+    G = L.G
+    Gm = tc.Mxfp4Matrix(L.nibG, L.scG, G.rows, G.cols)
     from trellis_coded_fp4_b200 import synth
-    return synth.activations(T, cols, seed=synth.SEED_BASE + 90 + T).to(device)
+    out = []
+    for T in (1, 2, 4, 8, 16, 32):
+        x = synth.activations(T, G.cols, seed=synth.SEED_BASE + 90 + T).to(d)
+        y = torch.empty((T, G.rows), dtype=torch.bfloat16, device=d)
+        ws_f = torch.empty(max(1, tc.gemv_workspace_bytes(G, T)), dtype=torch.uint8, device=d)
+        ws_m = torch.empty(max(1, tc.mxfp4_gemv_workspace_bytes(Gm, T)), dtype=torch.uint8, device=d)
+        us_f = time_calls(lambda i: tc.gemv(G, x, y, ws_f), n)
+        us_m = time_calls(lambda i: tc.mxfp4_gemv(Gm, x, y, ws_m), n)
+        out.append({"T": T, "fused": rate(gemv_bytes(G.rows, G.cols, T), us_f, peak),
+                    "mxfp4": rate(gemv_bytes(G.rows, G.cols, T, 0.53125), us_m, peak)})
+    return {"shape": "184320 x 2880", "calls": n, "rows": out}
 
 
-def run_e2e(step, steps, device):
-    """The same step through the public API with HOST buffers: every input (stream words, scales,
-    activations, logits) is copied from pinned host memory and every output (MXFP4 nibbles and
-    scales, GEMV outputs, MoE output) is copied back, inside the timed region."""
-    lay = step.layer
-    h_gu = torch.from_numpy(lay.gu_stream.view("int32").reshape(-1)).pin_memory()
-    h_gus = torch.from_numpy(lay.gu_scales.reshape(-1)).pin_memory()
-    h_dn = torch.from_numpy(lay.dn_stream.view("int32").reshape(-1)).pin_memory()
-    h_dns = torch.from_numpy(lay.dn_scales.reshape(-1)).pin_memory()
-    h_x = [x.cpu().pin_memory() for x in step.x]
-    h_xd = [x.cpu().pin_memory() for x in step.xd]
-    h_lg = [lg.cpu().pin_memory() for lg in step.logits]
-    outs = [step.nibG, step.scG, step.nibD, step.scD, step.yG, step.yD, step.out]
-    h_outs = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
-    h2d = sum(t.numel() * t.element_size() for t in (h_gu, h_gus, h_dn, h_dns, h_x[0], h_xd[0], h_lg[0]))
-    d2h = sum(t.numel() * t.element_size() for t in h_outs)
+def row_single_2048(L, peak, device):
+    """2048 x 2048 at batch 1: 512 distinct matrices (576 MB, > 4x L2) back to back in a CUDA graph;
+    and one call with L2 flushed before it (median of 20)."""
+    tc = L.tc
+    gen = torch.Generator(device=device).manual_seed(0x7CF40000)
+    nmat, n = 512, 2048
+    st = rand_words(nmat * n * (n // 32) * 2, gen, device).view(nmat, -1)
+    sc = rand_scales(nmat * n * (n // 32), 120, 126, gen, device).view(nmat, -1)
+    mats = [tc.TrellisMatrix(st[j], sc[j], n, n, SEG) for j in range(nmat)]
+    from trellis_coded_fp4_b200 import synth
+    x = synth.activations(1, n, seed=synth.SEED_BASE).to(device)
+    y = torch.empty((1, n), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(max(1, tc.gemv_workspace_bytes(mats[0], 1)), dtype=torch.uint8, device=device)
+    call = lambda i: tc.gemv(mats[i % nmat], x, y, ws)  # noqa: E731
+    nb = gemv_bytes(n, n, 1)
+    res = {"shape": "2048 x 2048, T = 1, seg_len 32", "matrices": nmat}
+    try:
+        res["graph"] = {**rate(nb, time_graph(call, nmat), peak), "note": "back to back, CUDA graph of 512 calls"}
+    except Exception as ex:  # capture unavailable: host-launched back to back instead
+        res["graph"] = {"error": str(ex)[:200]}
+    res["stream"] = {**rate(nb, time_calls(call, nmat), peak), "note": "back to back, launched from the host"}
+    flush = torch.empty(256 * 2 ** 20 // 4, dtype=torch.float32, device=device)
+    lat = []
+    for j in range(20):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call(j)
+        e1.record()
+        torch.cuda.synchronize()
+        lat.append(1e3 * e0.elapsed_time(e1))
+    res["cold_latency_us"] = {"median": round(statistics.median(lat), 3), "p10": round(float(np.percentile(lat, 10)), 3),
+                              "p90": round(float(np.percentile(lat, 90)), 3)}
+    del st, sc, mats, flush
+    return res
+
+
+def row_moe_7168(tc, peak, device, n):
+    """256 experts, hidden 7168, intermediate 2048, top-8 of N(0,1) logits, T = 1, 8, 32; random
+    2-bit streams and UE8M0 bytes in [118, 126] generated on the device (3.17 GB resident)."""
+    from trellis_coded_fp4_b200 import synth
+    E4, H4, I4, k4 = 256, 7168, 2048, 8
+    gen = torch.Generator(device=device).manual_seed(0x7CF40004)
+    gu = rand_words(E4 * 2 * I4 * (H4 // 32) * 2, gen, device).view(E4, -1)
+    gus = rand_scales(E4 * 2 * I4 * (H4 // 32), 118, 126, gen, device).view(E4, -1)
+    dn = rand_words(E4 * H4 * (I4 // 32) * 2, gen, device).view(E4, -1)
+    dns = rand_scales(E4 * H4 * (I4 // 32), 118, 126, gen, device).view(E4, -1)
+    M = tc.MoEWeights([tc.TrellisMatrix(gu[e], gus[e], 2 * I4, H4, SEG) for e in range(E4)],
+                      [tc.TrellisMatrix(dn[e], dns[e], H4, I4, SEG) for e in range(E4)], H4, I4)
+    rows = []
+    for T in (1, 8, 32):
+        xs = [synth.activations(T, H4, seed=0x7CF40004 + T, sub=i).to(device) for i in range(NVAR)]
+        lg = [synth.logits(T, E4, seed=0x7CF40004 + T, sub=i).to(device) for i in range(NVAR)]
+        ids = torch.empty((T, k4), dtype=torch.int32, device=device)
+        wts = torch.empty((T, k4), dtype=torch.float32, device=device)
+        out = torch.empty((T, H4), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(max(1, M.workspace_bytes(T, k4)), dtype=torch.uint8, device=device)
+
+        def fn(i):
+            tc.moe_route(lg[i % NVAR], k4, ids, wts)
+            tc.grouped_moe(M, xs[i % NVAR], ids, wts, out, ws)
+        us = time_calls(fn, n)
+        distinct = statistics.mean(len(np.unique(tc.moe_route(lg[i], k4)[0].cpu().numpy())) for i in range(NVAR))
+        nb = moe_bytes(distinct, T, H4, I4)
+        rows.append({**rate(nb, us, peak), "T": T, "distinct_experts_mean": distinct, "includes_route": True,
+                     "decoded_weights_per_s": distinct * 3 * H4 * I4 / (us * 1e-6)})
+    del gu, gus, dn, dns, M
+    return {"layer": "256 experts, hidden 7168, intermediate 2048, top-8, 3.17 GB resident", "calls": n, "rows": rows}
+
+
+def row_mxfp4(L, n, peak):
+    tc, d = L.tc, L.device
+    L._expanded()
+    Gm = tc.Mxfp4Matrix(L.nibG, L.scG, E * 2 * I, H)
+    Dm = tc.Mxfp4Matrix(L.nibD, L.scD, E * H, I)
+    wsg = torch.empty(max(1, tc.mxfp4_gemv_workspace_bytes(Gm, 1)), dtype=torch.uint8, device=d)
+    wsd = torch.empty(max(1, tc.mxfp4_gemv_workspace_bytes(Dm, 1)), dtype=torch.uint8, device=d)
+    ug = time_calls(lambda i: tc.mxfp4_gemv(Gm, L.x[i % NVAR], L.yG, wsg), n)
+    ud = time_calls(lambda i: tc.mxfp4_gemv(Dm, L.xd[i % NVAR], L.yD, wsd), n)
+    return {"mxfp4_gemv_gate_up": rate(gemv_bytes(E * 2 * I, H, 1, 0.53125), ug, peak),
+            "mxfp4_gemv_down": rate(gemv_bytes(E * H, I, 1, 0.53125), ud, peak),
+            "mxfp4_grouped_moe_t1": row_moe(L, 1, n, peak, mx=True), "calls": n}
+
+
+def row_encoder(L, seed, device):
+    tc = L.tc
+    enc_rows, enc_cols = 296, H
+    gen = torch.Generator(device=device).manual_seed(seed)
+    et = torch.randn(enc_rows, enc_cols, dtype=torch.float64, device=device, generator=gen)
+    eD = torch.rand(enc_rows, enc_cols, dtype=torch.float64, device=device, generator=gen) + 0.1
+    esc = L.G.scales[: enc_rows * (enc_cols // 32)]
+    ms = time_calls(lambda i: tc.encode(et, eD, esc, 32), 3, warm=1) / 1e3
+    return {"ms_per_call": round(ms, 3), "weights": enc_rows * enc_cols, "seg_len": 32,
+            "weights_per_s": enc_rows * enc_cols / (ms * 1e-3), "bound": "alu",
+            "note": "2^16 candidate paths per weight, fp64 costs evaluated exactly (no fused operations)"}
+
+
+def row_repack(L, n, peak):
+    tc = L.tc
+    out = torch.empty_like(L.G.stream)
+    us = time_calls(lambda i: tc.repack_interleaved(L.G.stream, L.G.rows, L.G.cols, out=out), n)
+    res = {**rate(16 * L.G.rows * (L.G.cols // 32), us, peak), "calls": n, "bound": "hbm",
+           "note": "8 bytes read + 8 written per 32-weight block"}
+    del out
+    return res
+
+
+def row_e5m3(L, n, peak, seed):
+    tc, d = L.tc, L.device
+    g5 = torch.Generator(device=d).manual_seed(seed + 5)
+    m5 = torch.randint(0, 8, L.G.scales.shape, dtype=torch.int32, device=d, generator=g5)
+    sc5 = (((L.G.scales.to(torch.int32) - 112) << 3) | m5).to(torch.uint8)
+    W5 = tc.TrellisMatrix(L.G.stream, sc5, L.G.rows, L.G.cols, L.G.seg_len)
+    us = time_calls(lambda i: tc.gemv_e5m3(W5, L.x[i % NVAR], out=L.yG), n)
+    return {**rate(gemv_bytes(E * 2 * I, H, 1), us, peak), "decoded_weights_per_s": W5.rows * W5.cols / (us * 1e-6),
+            "calls": n, "note": "E5M3 block scales of the same binades, batch 1"}
+
+
+# ----------------------------------------------------------------------------- end to end
+
+def run_e2e(L, steps):
+    """The headline metric through the public API with HOST buffers: every step copies the gate_up
+    stream, its scales and x from pinned host memory, runs trellis_gemv and copies y back."""
+    lay = L.layer
+    h_st = torch.from_numpy(lay.gu_stream.view("int32").reshape(-1)).pin_memory()
+    h_sc = torch.from_numpy(lay.gu_scales.reshape(-1)).pin_memory()
+    h_x = [x.cpu().pin_memory() for x in L.x]
+    h_y = torch.empty(L.yG.shape, dtype=L.yG.dtype).pin_memory()
+    h2d = h_st.numel() * 4 + h_sc.numel() + h_x[0].numel() * 2
+    d2h = h_y.numel() * 2
 
     def one(i):
-        v = i % len(h_x)
-        step.G.stream.copy_(h_gu, non_blocking=True)
-        step.G.scales.copy_(h_gus, non_blocking=True)
-        step.D.stream.copy_(h_dn, non_blocking=True)
-        step.D.scales.copy_(h_dns, non_blocking=True)
-        step.x[v].copy_(h_x[v], non_blocking=True)
-        step.xd[v].copy_(h_xd[v], non_blocking=True)
-        step.logits[v].copy_(h_lg[v], non_blocking=True)
-        step.run(i)
-        for o, h in zip(outs, h_outs):
-            h.copy_(o, non_blocking=True)
-
-    for i in range(2):
-        one(i)
-    torch.cuda.synchronize()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for i in range(steps):
-        one(i)
-    t1.record()
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / steps
-    return {"value": step.weights_per_step / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+        L.G.stream.copy_(h_st, non_blocking=True)
+        L.G.scales.copy_(h_sc, non_blocking=True)
+        L.x[i % NVAR].copy_(h_x[i % NVAR], non_blocking=True)
+        L.tc.gemv(L.G, L.x[i % NVAR], L.yG, L.wsG)
+        h_y.copy_(L.yG, non_blocking=True)
+    us = time_calls(one, steps, warm=2)
+    return {"value": L.G.rows * L.G.cols / (us * 1e-6), "unit": UNIT, "ms_per_step": us / 1e3,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 
-# ----------------------------------------------------------------------------- CPU oracle sample
+# ----------------------------------------------------------------------------- CPU oracle
 
-def oracle_sample(layer, x_bits, logits, stride):
-    """Run the oracle on every `stride`-th row of each matrix the step touches, doing per row the
-    work the step does (expand; multiply; MoE gate/up then down). Returns decoded weights."""
+def oracle_gemv_sample(layer, x_bits, stride, threads):
+    """The oracle's batch-1 GEMV on every `stride`-th row of the stacked gate_up matrix, the rows
+    split over `threads` threads (each call is one plain C loop; ctypes releases the GIL).
+    Returns the decoded weights."""
     import oracle
-    n = 0
-    gu_all = layer.gu_stream.reshape(E * 2 * I, H // 32, 2)
-    gus_all = layer.gu_scales.reshape(E * 2 * I, H // 32)
-    dn_all = layer.dn_stream.reshape(E * H, I // 32, 2)
-    dns_all = layer.dn_scales.reshape(E * H, I // 32)
-    for st, sc, rows, cols in ((gu_all, gus_all, E * 2 * I, H), (dn_all, dns_all, E * H, I)):
-        sel = np.arange(0, rows, stride)
-        oracle.expand_mxfp4(st[sel], sc[sel], len(sel), cols, SEG)
-        oracle.gemv(st, sc, rows, cols, SEG, x_bits, row_ids=sel)
-        n += 2 * len(sel) * cols
-    ids, w = oracle.route(logits, K_TOP)
-    for j in range(K_TOP):
-        e = int(ids[0, j])
-        ri = np.arange(0, I, stride)
-        y, _ = oracle.gemv(layer.gu_stream[e], layer.gu_scales[e], 2 * I, H, SEG, x_bits,
-                           row_ids=np.concatenate([ri, I + ri]))
-        h = np.zeros((1, I), np.uint16)
-        h[0, ri] = oracle.bf16_round_array(oracle.silu(y[0, :len(ri)]) * y[0, len(ri):])
-        rn = np.arange(0, H, stride)
-        oracle.gemv(layer.dn_stream[e], layer.dn_scales[e], H, I, SEG, h, row_ids=rn)
-        n += 2 * len(ri) * H + len(rn) * I
-    return n
+    st = layer.gu_stream.reshape(E * 2 * I, H // 32, 2)
+    sc = layer.gu_scales.reshape(E * 2 * I, H // 32)
+    sel = np.arange(0, E * 2 * I, stride)
+    parts = np.array_split(sel, threads)
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda r: oracle.gemv(st, sc, E * 2 * I, H, SEG, x_bits, row_ids=r), parts))
+    return len(sel) * H
 
 
-def cpu_baseline(layer, seed, stride=16):
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(layer, seed):
     from trellis_coded_fp4_b200 import synth
-    xb = synth.bf16_bits(synth.activations(T, H, seed=seed))
-    lg = synth.logits(T, E, seed=seed).numpy()
-    t0 = time.perf_counter()
-    n = oracle_sample(layer, xb, lg, stride)
-    dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": UNIT, "cores": 1, "kind": "oracle", "seconds": dt,
-            "sample": (f"every {stride}th row of each matrix the step touches (expansion and batch-1 GEMV of "
-                       f"gate_up and down; MoE gate/up rows and down rows of the 4 routed experts), "
-                       f"{n} decoded weights, single-threaded plain C oracle")}
+    xb = synth.bf16_bits(synth.activations(1, H, seed=seed))
+    ncores = len(os.sched_getaffinity(0))
+    res = {}
+    for name, stride, threads in (("single", 8, 1), ("all", 1, ncores)):
+        t0 = time.perf_counter()
+        n = oracle_gemv_sample(layer, xb, stride, threads)
+        dt = time.perf_counter() - t0
+        res[name] = {"value": n / dt, "cores": threads, "seconds": round(dt, 3), "weights": n, "stride": stride}
+    a, s = res["all"], res["single"]
+    return {"value": a["value"], "unit": UNIT, "cores": a["cores"], "kind": "oracle",
+            "sample": (f"batch-1 GEMV of every {a['stride']}th row of the stacked gate_up matrix ({a['weights']} decoded "
+                       f"weights), rows split over {a['cores']} threads of the plain C oracle"),
+            "single_core": {"value": s["value"], "cores": 1,
+                            "sample": f"every {s['stride']}th row ({s['weights']} weights), one thread"},
+            "cpu_model": cpu_model()}
 
 
 # ----------------------------------------------------------------------------- arms
@@ -399,30 +575,38 @@ def job_value(world: int, weights_per_step: int, steps: int, ms_total: float) ->
 
 
 def reference_arm(args):
+    """The oracle as it stands, on a bounded sample of the headline workload (every stride-th row of
+    the stacked gate_up matrix per step, rows split over the host's cores; the stride is set from a
+    first timed sample so that warm-up and steps together take about a minute); rank 0 only."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from trellis_coded_fp4_b200 import synth
     seed = synth.SEED_BASE + 1
     layer = synth.moe_layer(E, H, I, seed=seed)
-    stride = 256
-    xb = synth.bf16_bits(synth.activations(T, H, seed=seed))
-    lg = synth.logits(T, E, seed=seed).numpy()
+    ncores = len(os.sched_getaffinity(0))
+    xb = synth.bf16_bits(synth.activations(1, H, seed=seed))
+    t0 = time.perf_counter()
+    n0 = oracle_gemv_sample(layer, xb, 1024, ncores)
+    rate0 = n0 / (time.perf_counter() - t0)
+    budget_s = 60.0
+    rows_per_step = rate0 * budget_s / H / max(1, args.steps + args.warmup)
+    stride = int(max(64, min(E * 2 * I, np.ceil(E * 2 * I / max(rows_per_step, 1.0)))))
     for _ in range(args.warmup):
-        oracle_sample(layer, xb, lg, stride)
+        oracle_gemv_sample(layer, xb, stride, ncores)
     t0 = time.perf_counter()
     n = 0
     for _ in range(args.steps):
-        n += oracle_sample(layer, xb, lg, stride)
+        n += oracle_gemv_sample(layer, xb, stride, ncores)
     dt = time.perf_counter() - t0
     value = n / dt
-    sample = (f"every {stride}th row of each matrix the step touches, {n // max(args.steps, 1)} decoded weights "
-              "per step, single-threaded plain C oracle")
+    sample = (f"every {stride}th row of the stacked gate_up matrix, {n // max(args.steps, 1)} decoded weights per "
+              f"step, plain C oracle, rows split over {ncores} threads")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * dt / max(args.steps, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "sample": sample}, "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": ncores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line))
@@ -432,16 +616,15 @@ def reference_arm(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)  # ~0.3 s timed: several clock samples
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=5000)  # ~0.3 s timed: several clock samples
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="tcf4", choices=["tcf4", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="the headline only, without the extra rows")
     ap.add_argument("--only", default=None,
-                    help="run only this call of the step (e.g. gemv_gate_up), for profiling one kernel")
-    ap.add_argument("--sweep", action="store_true",
-                    help="batch sweep instead of the step: fused decode GEMV and MXFP4 GEMV of the gate_up "
-                         "matrix at T = 1, 2, 4, 8, 16, 32 (one JSON line, not a bench line)")
+                    help="run only this call (gemv_gate_up, gemv_down, expand_gate_up, grouped_moe) warmup + "
+                         "steps times, for profiling one kernel; prints no bench line")
     args = ap.parse_args()
     if args.impl == "reference":
         return reference_arm(args)
@@ -460,28 +643,22 @@ def main():
     from trellis_coded_fp4_b200 import build, synth
     build.build()
     seed = synth.SEED_BASE + 1 + rank
-    step = Step(seed, device)
-    if args.sweep:
-        print(json.dumps(batch_sweep(step, device, max(10, args.steps // 10))))
-        return 0
-    if args.only is not None:  # profiling mode: a few launches of one call, no timing line
+    L = Layer(seed, device)
+    if args.only is not None:
         for i in range(args.warmup + args.steps):
-            step.run(i, only=args.only)
+            L.run_only(args.only, i)
         torch.cuda.synchronize()
         print(json.dumps({"only": args.only, "launches": args.warmup + args.steps,
-                          "timeouts": step.tc.device_timeouts()}))
+                          "timeouts": L.tc.device_timeouts()}))
         return 0
 
-    for i in range(max(args.warmup, 3)):
-        step.run(i)
+    warm = max(args.warmup, 3)
+    for i in range(warm):
+        L.step(i)
     torch.cuda.synchronize()
-
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.15)
-    # The step is timed with events at its two ends only: an event between two calls would sit
-    # between their kernels in the stream and keep a call from overlapping its predecessor's tail
-    # (the kernels are dependent launches).
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -489,7 +666,7 @@ def main():
     tw0 = time.time()
     start.record()
     for i in range(args.steps):
-        step.run(i)
+        L.step(i)
     end.record()
     torch.cuda.synchronize()
     tw1 = time.time()
@@ -498,148 +675,52 @@ def main():
     clocks = sampler.stop(tw0, tw1)
     ms_total = max_over_ranks(start.elapsed_time(end), dist, device)
     ms_per_step = ms_total / args.steps
-
-    # per-call durations from a second pass with an event before each call (on the launching
-    # stream); these set the roofline of the dominant call and the shares
-    events = []
-    n_per = max(10, args.steps // 4)
-    for i in range(n_per):
-        step.run(i, events)
-    torch.cuda.synchronize()
-    per = {}
-    for (name, e0), (_, e1) in zip(events[:-1], events[1:]):
-        if name == "end":
-            continue
-        per.setdefault(name, []).append(e0.elapsed_time(e1))
-    avg_us = {k: 1e3 * statistics.mean(v) for k, v in per.items()}
-    algo = step.algo_bytes()
-    wts = step.weights()
+    weights_per_step = L.G.rows * L.G.cols
     peak, peak_kind = measured_hbm_peak()
-    kernels = {}
-    for k, us in avg_us.items():
-        gbs = algo[k] / (us * 1e-6) / 1e9
-        kernels[k] = {"avg_us": round(us, 3), "algo_bytes": algo[k], "gb_s": round(gbs, 1),
-                      "frac_of_measured_hbm": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / 8000.0, 4),
-                      "decoded_weights_per_s": (wts[k] / (us * 1e-6)) if wts[k] else None,
-                      "share": round(us / (1e3 * ms_per_step), 4), "calls": n_per}
-    dom = max(avg_us, key=avg_us.get)
-    dom_gbs = algo[dom] / (avg_us[dom] * 1e-6) / 1e9
-    kind = "expand" if dom.startswith("expand") else ("gemv" if dom.startswith("gemv") else None)
-    tpw = NCU_TRAFFIC_B_PER_WEIGHT.get(kind) if kind else None
-    roofline = {"bound": "hbm", "achieved": round(dom_gbs, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(dom_gbs / peak, 4), "traffic": (tpw * wts[dom]) if tpw else None,
-                "kernel": dom, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
-                else "fallback 6650 GB/s"}
-
-    value = job_value(world, step.weights_per_step, args.steps, ms_total)
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic",
-            "config": {"workload": WORKLOAD, "tokens": T, "top_k": K_TOP, "experts": E, "hidden": H,
-                       "intermediate": I, "seg_len": SEG, "decoded_weights_per_step": step.weights_per_step,
-                       "l2": "inputs larger than L2 (each step streams >900 MB of stream/MXFP4 bytes through L2)",
+    nb = gemv_bytes(L.G.rows, L.G.cols, 1)
+    achieved = nb / (ms_per_step * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC_GEMV_GATE_UP,
+                "kernel": "trellis_gemv: k_bsplit_gemv + k_mma (decode-MMA) on the 184320 x 2880 gate_up stack, T = 1",
+                "algo_bytes_per_launch": nb, "avg_us": round(ms_per_step * 1e3, 3),
+                "frac_of_8tbs": round(achieved / SPEC_HBM_GBS, 4),
+                "peak_source": (f"{peak_kind}: MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured"
+                                else "fallback 6650 GB/s")}
+    value = job_value(world, weights_per_step, args.steps, ms_total)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": warm,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u32 decode, f32 accumulate", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "rows": L.G.rows, "cols": L.G.cols, "tokens": 1, "seg_len": SEG,
+                       "decoded_weights_per_step": weights_per_step,
+                       "l2": f"inputs larger than L2: steps rotate over {ROT} distinct resident matrices "
+                             f"({ROT * nb / 1e6:.0f} MB) and {NVAR} activation vectors",
                        "parallelism": f"replicas x{world}",
-                       "arithmetic": "decode: u32 bit logic; products: block-scaled MXFP4 tensor-core MMA (activations as "
-                                     "six E2M1 terms per 32-block), fp32 accumulation"},
-            "roofline": roofline, "kernels": kernels,
-            "gpu_launches": step.launches_per_step * args.steps, "clocks": clocks}
+                       "arithmetic": "decode: u32 bit logic; products: block-scaled MXFP4 tensor-core MMA "
+                                     "(activations as six E2M1 terms per 32-block), fp32 accumulation, bf16 out"},
+            "roofline": roofline, "gpu_launches": L.launches_per_step * args.steps, "clocks": clocks}
 
-    # the next row (outside the step): products from the resident MXFP4 tensors, each call timed on
-    # its own with CUDA events after warm-up, inputs > L2 (the tensors are 423 MB)
-    mx = {}
-    for name, nbytes in step.mx_algo_bytes().items():
-        for i in range(3):
-            step.run_mx(name, i)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_mx = max(10, args.steps // 4)
-        e0.record()
-        for i in range(n_mx):
-            step.run_mx(name, i)
-        e1.record()
-        torch.cuda.synchronize()
-        us = 1e3 * e0.elapsed_time(e1) / n_mx
-        gbs = nbytes / (us * 1e-6) / 1e9
-        mx[name] = {"avg_us": round(us, 3), "algo_bytes": nbytes, "gb_s": round(gbs, 1),
-                    "frac_of_measured_hbm": round(gbs / peak, 4), "frac_of_8tbs": round(gbs / 8000.0, 4),
-                    "calls": n_mx, "note": "includes route" if name == "mxfp4_grouped_moe" else ""}
-    # the upstream encoder (D-weighted Viterbi): 296 rows of the gate_up matrix re-encoded from their
-    # decoded values with random D, segments of 32 weights; compute-bound, timed over 3 calls
-    enc_rows, enc_cols = 296, H
-    gen = torch.Generator(device=device).manual_seed(seed)
-    et = torch.randn(enc_rows, enc_cols, dtype=torch.float64, device=device, generator=gen)
-    eD = torch.rand(enc_rows, enc_cols, dtype=torch.float64, device=device, generator=gen) + 0.1
-    esc = step.G.scales[: enc_rows * (enc_cols // 32)]
-    step.tc.encode(et, eD, esc, 32)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(3):
-        step.tc.encode(et, eD, esc, 32)
-    e1.record()
-    torch.cuda.synchronize()
-    enc_ms = e0.elapsed_time(e1) / 3
-    encoder = {"ms_per_call": round(enc_ms, 3), "weights": enc_rows * enc_cols, "seg_len": 32,
-               "weights_per_s": enc_rows * enc_cols / (enc_ms * 1e-3), "bound": "alu",
-               "note": "2^16 candidate paths per weight, fp64 costs evaluated exactly (no fused operations)"}
-    # the interleaved-packing repack of the gate_up stream (184320 x 2880: 133 MB read, 133 MB
-    # written per call, more than L2 holds), back to back after warm-up
-    rp_out = torch.empty_like(step.G.stream)
-    rp_rows, rp_cols = step.G.rows, step.G.cols
-    for _ in range(3):
-        step.tc.repack_interleaved(step.G.stream, rp_rows, rp_cols, out=rp_out)
-    torch.cuda.synchronize()
-    n_rp = max(10, args.steps // 4)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(n_rp):
-        step.tc.repack_interleaved(step.G.stream, rp_rows, rp_cols, out=rp_out)
-    e1.record()
-    torch.cuda.synchronize()
-    rp_us = 1e3 * e0.elapsed_time(e1) / n_rp
-    rp_bytes = 16 * rp_rows * (rp_cols // 32)
-    rp_gbs = rp_bytes / (rp_us * 1e-6) / 1e9
-    repack = {"avg_us": round(rp_us, 3), "algo_bytes": rp_bytes, "gb_s": round(rp_gbs, 1),
-              "frac_of_measured_hbm": round(rp_gbs / peak, 4), "frac_of_8tbs": round(rp_gbs / 8000.0, 4),
-              "calls": n_rp, "bound": "hbm", "note": "8 bytes read + 8 written per 32-weight block"}
-    del rp_out
-    # the E5M3 block-scale variant: the gate_up stream (184320 x 2880) with E5M3 scale bytes of the
-    # same binades as its UE8M0 ones and random mantissas, batch 1, on the CUDA-core kernel
-    g5 = torch.Generator(device=device).manual_seed(seed + 5)
-    m5 = torch.randint(0, 8, step.G.scales.shape, dtype=torch.int32, device=device, generator=g5)
-    sc5 = (((step.G.scales.to(torch.int32) - 112) << 3) | m5).to(torch.uint8)
-    W5 = step.tc.TrellisMatrix(step.G.stream, sc5, step.G.rows, step.G.cols, step.G.seg_len)
-    y5 = torch.empty((T, W5.rows), dtype=torch.bfloat16, device=device)
-    for i in range(3):
-        step.tc.gemv_e5m3(W5, step.x[i % len(step.x)], out=y5)
-    torch.cuda.synchronize()
-    n5 = max(10, args.steps // 20)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(n5):
-        step.tc.gemv_e5m3(W5, step.x[i % len(step.x)], out=y5)
-    e1.record()
-    torch.cuda.synchronize()
-    g5_us = 1e3 * e0.elapsed_time(e1) / n5
-    g5_bytes = step.algo_bytes()["gemv_gate_up"]
-    g5_gbs = g5_bytes / (g5_us * 1e-6) / 1e9
-    e5m3 = {"avg_us": round(g5_us, 3), "algo_bytes": g5_bytes, "gb_s": round(g5_gbs, 1),
-            "frac_of_measured_hbm": round(g5_gbs / peak, 4), "frac_of_8tbs": round(g5_gbs / 8000.0, 4),
-            "decoded_weights_per_s": W5.rows * W5.cols / (g5_us * 1e-6), "calls": n5,
-            "note": "CUDA-core kernel (a block-scaled MMA takes power-of-two scales only)"}
-    del W5, sc5, m5, y5
-    line["next_rows"] = {"mxfp4_consumer": mx, "encoder": encoder, "repack_interleaved": repack,
-                         "gemv_e5m3_gate_up": e5m3,
-                         "description": "products read straight from the resident MXFP4 tensors the step's "
-                         "expansion wrote (HEPH serving mode 2), the D-weighted Viterbi encoder, the "
-                         "interleaved-to-planar stream repack and the E5M3 block-scale GEMV; outside the "
-                         "step and its value"}
+    if not args.no_rows:
+        n = 200
+        rows = {}
+        rows["gemv_down"] = row_gemv_down(L, n, peak)
+        rows["expand"] = row_expand(L, 100, peak)
+        rows["moe_t1"] = row_moe(L, 1, n, peak)
+        rows["moe_sweep"] = {"natural": [row_moe(L, T, 100, peak) for T in (1, 2, 4, 8, 16, 32)],
+                             "skew": [row_moe(L, T, 100, peak, skew=True) for T in (1, 8, 16, 32)]}
+        rows["gemv_sweep"] = row_gemv_sweep(L, 50, peak)
+        rows["single_2048"] = row_single_2048(L, peak, device)
+        rows["moe_7168"] = row_moe_7168(L.tc, peak, device, 50)
+        rows["mxfp4_consumer"] = row_mxfp4(L, n, peak)
+        rows["encoder"] = row_encoder(L, seed, device)
+        rows["repack_interleaved"] = row_repack(L, n, peak)
+        rows["gemv_e5m3_gate_up"] = row_e5m3(L, 50, peak, seed)
+        rows["timeouts"] = L.tc.device_timeouts()
+        line["rows"] = rows
 
     if rank == 0:
-        line["e2e"] = run_e2e(step, args.e2e_steps, device)
+        line["e2e"] = run_e2e(L, args.e2e_steps)
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(step.layer, seed)
+            line["cpu_baseline"] = cpu_baseline(L.layer, seed)
         print(json.dumps(line))
     if dist is not None:
         dist.barrier()
