@@ -88,16 +88,50 @@ def _lop3(a, b, c, lut):
     return out & M32
 
 
-def test_delta_swap_select_table():
-    # Each three-input op in delta_swap takes operands (mask, x, y) and must compute mask ? x : y.
+def _luts(fn_name, next_name):
     text = open(HEADER).read()
-    body = text[text.index("void delta_swap"):text.index("void planes_to_nibbles_interleaved")]
-    luts = [int(v, 16) for v in re.findall(r"lop3\.b32 %0, %1, %2, %3, (0x[0-9A-Fa-f]+);", body)]
-    assert len(luts) == 2
+    body = text[text.index("void " + fn_name + "("):text.index(next_name)]
+    return [int(v, 16) for v in re.findall(r"lop3\.b32 %0, %1, %2, %3, (0x[0-9A-Fa-f]+);", body)]
+
+
+def test_delta_swap_select_table():
+    # Each three-input op in delta_swap takes operands (x, y, mask) and must compute mask ? x : y;
+    # delta_swap_inv_b reads its second word inverted: mask ? x : ~y, then mask ? ~x : y.
     rng = np.random.default_rng(7)
-    m, x, y = (rng.integers(0, 1 << 32, 64, dtype=np.uint64) for _ in range(3))
+    x, y, m = (rng.integers(0, 1 << 32, 64, dtype=np.uint64) for _ in range(3))
+    sel = lambda m, x, y: ((m & x) | (~m & y)) & M32  # noqa: E731
+    luts = _luts("delta_swap", "delta_swap_inv_b")
+    assert len(luts) == 2
     for lut in luts:
-        assert (_lop3(m, x, y, lut) == ((m & x) | (~m & y & M32))).all(), hex(lut)
+        assert (_lop3(x, y, m, lut) == sel(m, x, y)).all(), hex(lut)
+    inv = _luts("delta_swap_inv_b", "void planes_to_nibbles_interleaved")
+    assert len(inv) == 2
+    assert (_lop3(x, y, m, inv[0]) == sel(m, x, ~y & M32)).all(), hex(inv[0])
+    assert (_lop3(x, y, m, inv[1]) == sel(m, ~x & M32, y)).all(), hex(inv[1])
+
+
+def test_transpose_absorbing_the_inversion():
+    # planes_to_nibbles_interleaved_i3 (n3 given inverted, swaps emulated with the header's LUTs)
+    # equals the plain transpose of the true planes
+    luts, inv = _luts("delta_swap", "delta_swap_inv_b"), _luts("delta_swap_inv_b", "void planes_to_nibbles_interleaved")
+    rng = np.random.default_rng(10)
+    n = [rng.integers(0, 1 << 32, 256, dtype=np.uint64) for _ in range(4)]
+
+    def swap(a, b, s, mask, l0, l1):
+        ms = np.uint64(mask)
+        nb = _lop3(a >> np.uint64(s), b, ms, l0)
+        na = _lop3((b << np.uint64(s)) & M32, a, (ms << np.uint64(s)) & M32, l1)
+        return na, nb
+    a, b = swap(n[0], n[1], 1, 0x55555555, *luts)
+    c, d = swap(n[2], ~n[3] & M32, 1, 0x55555555, *inv)
+    a, c = swap(a, c, 2, 0x33333333, *luts)
+    b, d = swap(b, d, 2, 0x33333333, *luts)
+    ra, rb = _delta_swap(n[0], n[1], 1, 0x55555555)
+    rc, rd = _delta_swap(n[2], n[3], 1, 0x55555555)
+    ra, rc = _delta_swap(ra, rc, 2, 0x33333333)
+    rb, rd = _delta_swap(rb, rd, 2, 0x33333333)
+    for got, ref in zip((a, b, c, d), (ra, rb, rc, rd)):
+        assert (got == ref).all()
 
 
 def _delta_swap(a, b, s, mask):

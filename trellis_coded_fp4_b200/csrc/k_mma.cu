@@ -79,7 +79,10 @@ struct Cfg {
   static constexpr uint32_t kWStage = 1024u * kKB;             // 128 rows x 8 KB bytes of words
   static constexpr uint32_t kSbo = 128u * kKB;                 // B: 8 rows x KB chunks x 16 bytes
   static constexpr uint32_t kBStage = NMAX * 16u * kKB;        // NMAX rows x 32 KB E2M1
-  static constexpr uint32_t kSfbStage = (kKB / 4) * kC * 128u;  // [group][column][lane] u32
+  // B scale factors of a stage: per 4-block group a 32 x 16-byte tile, row r = the group's UE8M0
+  // words of B rows r, 32 + r, 64 + r (and one spare word), the source of one tcgen05.cp
+  static constexpr uint32_t kSfbStage = (kKB / 4) * 512u;
+  static constexpr uint32_t kBSlot = kBStage + kSfbStage;       // one stage of terms + scales
   // MMA issuers: one per half stage, each into its own accumulator, where TMEM has room for the
   // two accumulator pairs (one issuing thread sustains about one MMA per 60 cycles; two of them in
   // different warps run concurrently).
@@ -194,12 +197,14 @@ __device__ __forceinline__ float pow2f(int e) {
   return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
-// Per group of token slots, the activation terms of each stage: Bg [S][kBStage] (one K-major B
-// stage each) and Bsf [S][kSfbStage]: word (g, c, lane) of a stage holds the UE8M0 bytes of B row
-// 32c+lane for the stage's blocks 4g..4g+3 (byte i = block 4g+i).
+// Per group of token slots, the activation terms of each stage, stage after stage ([S][kBSlot]):
+// the K-major E2M1 B operand (kBStage bytes), then its scale factors: for each 4-block group g a
+// 512-byte tile whose 16-byte row r holds, at word c, the UE8M0 bytes of B row 32c + r for the
+// stage's blocks 4g..4g+3 (byte i = block 4g+i). One tcgen05.cp (32x128b, copied to all four lane
+// quarters) moves a group's tile to TMEM, where B row 32c + r reads column c of the group.
 template <int NMAX>
 __host__ __device__ inline size_t terms_bytes(int S) {
-  return (size_t)S * (Cfg<NMAX>::kBStage + Cfg<NMAX>::kSfbStage);
+  return (size_t)S * Cfg<NMAX>::kBSlot;
 }
 
 // One 32-element block kb of NT activation rows (lane = element; v[i] is slot t0 + i) -> kTerms
@@ -217,8 +222,9 @@ __device__ __forceinline__ void split_terms_n(const float *v, int t0, int nvalid
   using C = Cfg<NMAX>;
   const int lane = threadIdx.x & 31;
   const int s = kb / C::kKB, c = kb - s * C::kKB, h = c >> 2;
-  uint8_t *bst = terms + (size_t)s * C::kBStage;
-  uint8_t *sfs = terms + (size_t)S_total * C::kBStage + (size_t)s * C::kSfbStage;
+  (void)S_total;
+  uint8_t *bst = terms + (size_t)s * C::kBSlot;
+  uint8_t *sfs = bst + C::kBStage;
   const int kp = NAT ? lane : kpos_of_weight(lane);
   float r[NT];
 #pragma unroll
@@ -247,7 +253,7 @@ __device__ __forceinline__ void split_terms_n(const float *v, int t0, int nvalid
       if (t0 + i < nvalid && n < NMAX) {
         if ((kp & 1) == 0)
           bst[chunk_off<NMAX>((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code[i] | (partner << 4));
-        if (lane == 0) sfs[((h * C::kC + (n >> 5)) * 32 + (n & 31)) * 4 + (c & 3)] = (uint8_t)(S[i] + 127);
+        if (lane == 0) sfs[(h * 32 + (n & 31)) * 16 + (n >> 5) * 4 + (c & 3)] = (uint8_t)(S[i] + 127);
       }
     }
   }
@@ -323,7 +329,7 @@ __host__ __device__ inline MmaGeom mma_geom(int mode, bool mx = false) {
   MmaGeom g;
   g.off_W = 1024u;
   g.off_B = g.off_W + (mx ? C::kNWX * C::kWStageX : C::kNW * C::kWStage);
-  g.off_U = g.off_B + C::kNB * C::kBStage;
+  g.off_U = g.off_B + C::kNB * C::kBSlot;
   g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)C::kTok * 4u : 0u);
   g.smem = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
   return g;
@@ -467,6 +473,12 @@ __device__ __forceinline__ void mma_mxf4_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], [%1], %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
+}
+
+// One thread: copy a 32-row x 16-byte shared-memory tile (descriptor desc) into TMEM columns
+// taddr..taddr+3 of every lane quarter: row r to lane 32q + r of each quarter q.
+__device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 
 // The same MMA with A from shared memory (descriptor a_desc).
@@ -697,48 +709,41 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
 
   if (MX && warp < C::kDecWarps) {
     // ---------------------------------------------------------------- scale-factor warps (MX)
-    // Warp w < 4 writes, for every stage, the scale factors of tile rows 32w..32w+31 (its lane
-    // quarter): each row's KB UE8M0 bytes (A) and this lane's B scale words (every quarter holds a
-    // copy). The next stage's bytes are loaded while the current stage's are stored.
+    // Warp w < 4 writes, for every stage, the UE8M0 bytes of tile rows 32w..32w+31 (its lane
+    // quarter): each row's KB bytes, four per group column. The next stage's bytes are loaded while
+    // the current stage's are stored. (The activation terms' scale factors reach TMEM by
+    // tcgen05.cp from the MMA issuers.)
     if (warp < 4) {
       constexpr int kG = kKB / 4;  // scale groups per stage
       const int m = 32 * warp + lane;
       const uint32_t tq = tbase + ((uint32_t)(32 * warp) << 16);
-      uint32_t pa[kKB / 2], pb[kG][C::kC];
+      uint32_t pa[kKB / 2];
       int qp = 0, jl_p = 0, s_p = 0;
       const unsigned short *srow = nullptr;
-      const uint32_t *sfb_src = nullptr;
-      auto load_sf = [&](uint32_t(&da)[kKB / 2], uint32_t(&db)[kG][C::kC]) {
+      auto load_sf = [&](uint32_t(&da)[kKB / 2]) {
         if (qp >= nq) return;
         if (s_p == 0) {
           const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_p));
           const int row = tile_row(jr, m);
-          srow = row >= 0 ? reinterpret_cast<const unsigned short *>(jr.sc + (size_t)row * nbr) : nullptr;
-          sfb_src = reinterpret_cast<const uint32_t *>(a.terms + (size_t)jr.group * tbytes + (size_t)S * C::kBStage) + lane;
+          srow = reinterpret_cast<const unsigned short *>(jr.sc + (size_t)(row >= 0 ? row : jr.y0) * nbr);
         }
-        const int lim = nbr - kKB * s_p;  // blocks of the stage inside the row
+        const int lim = nbr - kKB * s_p;  // blocks of the stage inside the row (even)
+        const unsigned short *p = srow + (kKB / 2) * s_p;
 #pragma unroll
-        for (int i = 0; i < kKB / 2; i++)
-          da[i] = srow != nullptr && 2 * i < lim ? (uint32_t)__ldg(srow + (kKB / 2) * s_p + i) : 0u;
-#pragma unroll
-        for (int g = 0; g < kG; g++)
-#pragma unroll
-          for (int c = 0; c < C::kC; c++)
-            db[g][c] = __ldg(sfb_src + (size_t)s_p * (C::kSfbStage / 4) + (g * C::kC + c) * 32);
+        for (int i = 0; i < kKB / 2; i++) da[i] = 2 * i < lim ? (uint32_t)__ldg(p + i) : 0u;
         qp++;
         if (++s_p == S) {
           s_p = 0;
           jl_p++;
         }
       };
-      grid_dep_wait();  // the activation terms (B scales) come from the preceding kernel (a split, or gate/up)
-      load_sf(pa, pb);
+      load_sf(pa);
       uint32_t b = 0;
       bool ok = true;
 #pragma unroll 1
       for (int q = 0; q < nq; q++) {
-        uint32_t na[kKB / 2], nb[kG][C::kC];
-        load_sf(na, nb);
+        uint32_t na[kKB / 2];
+        load_sf(na);
         if (q >= kNA) {
           const uint32_t ph = (uint32_t)((q - kNA) / kNA) & 1u;
           if (!(ok = warp_wait(&a_empty[2 * b], ph, tmo, abort_flag) && warp_wait(&a_empty[2 * b + 1], ph, tmo, abort_flag)))
@@ -746,11 +751,8 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
           tc_fence_after();
         }
 #pragma unroll
-        for (int g = 0; g < kG; g++) {
+        for (int g = 0; g < kG; g++)
           tmem_st_x1(tq + kSfaCol + kKB * b + 4u * (uint32_t)g + (uint32_t)warp, pa[2 * g] | (pa[2 * g + 1] << 16));
-#pragma unroll
-          for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + kSfbCol + kKB * b + 4u * (uint32_t)g + (uint32_t)c, pb[g][c]);
-        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -758,10 +760,6 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         mbar_arrive_one(&a_full[2 * b + 1]);
 #pragma unroll
         for (int i = 0; i < kKB / 2; i++) pa[i] = na[i];
-#pragma unroll
-        for (int g = 0; g < kG; g++)
-#pragma unroll
-          for (int c = 0; c < C::kC; c++) pb[g][c] = nb[g][c];
         b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
       }
       if (!ok) *abort_flag = 1;
@@ -782,38 +780,35 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
     for (int i = 0; i < 4; i++) wlo[i] = ((uint32_t)i ^ (sw & 3u)) * 16u;
     const uint32_t tq = tbase + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lane quarter
 
-    // Scale factors of this thread's kNG groups of four blocks, loaded one stage ahead of their use:
-    // its row's bytes (16-bit loads of block pairs) and the words of the B rows 32c + lane, c < kC.
-    uint32_t pa[kNBT / 2], pb[kNG][C::kC];
+    // The UE8M0 bytes of this thread's kNG groups of four blocks (16-bit loads of block pairs),
+    // loaded one stage ahead of their use. Rows outside the tile read the job's first row instead
+    // (their products are never stored). Only the weights' scales: the activation terms' scale
+    // factors reach TMEM by tcgen05.cp from the MMA issuers, so nothing here waits for the
+    // preceding kernel.
+    uint32_t pa[kNBT / 2];
     int qp = 0, jl_p = 0, s_p = 0;
     const unsigned short *srow = nullptr;  // row m's scales of the front job, from block kNBT h on
-    const uint32_t *sfb_src = nullptr;     // the front job's B scale words of this lane
-    auto load_sf = [&](uint32_t(&da)[kNBT / 2], uint32_t(&db)[kNG][C::kC]) {
+    auto load_sf = [&](uint32_t(&da)[kNBT / 2]) {
       if (qp >= nq) return;
       if (s_p == 0) {
         const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_p));
         const int row = tile_row(jr, m);
-        srow = row >= 0 ? reinterpret_cast<const unsigned short *>(jr.sc + (size_t)row * nbr + kNBT * h) : nullptr;
-        sfb_src = reinterpret_cast<const uint32_t *>(a.terms + (size_t)jr.group * tbytes + (size_t)S * C::kBStage) +
-                  (size_t)(h * kNG * C::kC) * 32 + lane;
+        srow = reinterpret_cast<const unsigned short *>(jr.sc + (size_t)(row >= 0 ? row : jr.y0) * nbr + kNBT * h);
       }
-      const int lim = nbr - kKB * s_p - kNBT * h;  // blocks of this thread's range inside the row
+      // blocks of this thread's range inside the row (even, so no 16-bit load crosses the row end).
+      // Predicated loads, no branch: a branch around them would make the compiler wait for the
+      // loads where the paths join, exposing their latency at the start of every stage.
+      const int lim = nbr - kKB * s_p - kNBT * h;
+      const unsigned short *p = srow + (kKB / 2) * s_p;
 #pragma unroll
-      for (int i = 0; i < kNBT / 2; i++)
-        da[i] = srow != nullptr && 2 * i < lim ? (uint32_t)__ldg(srow + (kKB / 2) * s_p + i) : 0u;
-#pragma unroll
-      for (int g = 0; g < kNG; g++)
-#pragma unroll
-        for (int c = 0; c < C::kC; c++)
-          db[g][c] = __ldg(sfb_src + (size_t)s_p * (C::kSfbStage / 4) + (g * C::kC + c) * 32);
+      for (int i = 0; i < kNBT / 2; i++) da[i] = 2 * i < lim ? (uint32_t)__ldg(p + i) : 0u;
       qp++;
       if (++s_p == S) {
         s_p = 0;
         jl_p++;
       }
     };
-    grid_dep_wait();  // the activation terms (B scales) come from the preceding kernel (a split, or gate/up)
-    load_sf(pa, pb);
+    load_sf(pa);
 
     // Barrier latencies are hidden: the release of this stage's A slot and the arrival of the next
     // stage's words are tested (non-blocking) before a chunk's decode and their results read after
@@ -851,8 +846,8 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
           }
         }
       }
-      uint32_t na[kNBT / 2], nb[kNG][C::kC];
-      load_sf(na, nb);  // the next stage's scale factors; their latency hides behind this stage
+      uint32_t na[kNBT / 2];
+      load_sf(na);  // the next stage's scale bytes; their latency hides behind this stage
       const uint32_t wa = wrow + ws * kWStage;
       const uint32_t ws1 = ws + 1 == (uint32_t)kNW ? 0u : ws + 1;
       uint32_t ae = 1u, wf = 0u;
@@ -878,10 +873,10 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         } else {
 #pragma unroll
           for (int i = 0; i < 4; i++) {
-            planes_to_nibbles_interleaved(decode_block0(cw[i].x, cw[i].y), W[2 * i][0], W[2 * i][1], W[2 * i][2],
-                                          W[2 * i][3]);
-            planes_to_nibbles_interleaved(decode_block0(cw[i].z, cw[i].w), W[2 * i + 1][0], W[2 * i + 1][1],
-                                          W[2 * i + 1][2], W[2 * i + 1][3]);
+            planes_to_nibbles_interleaved_i3(decode_block0_i3(cw[i].x, cw[i].y), W[2 * i][0], W[2 * i][1],
+                                             W[2 * i][2], W[2 * i][3]);
+            planes_to_nibbles_interleaved_i3(decode_block0_i3(cw[i].z, cw[i].w), W[2 * i + 1][0], W[2 * i + 1][1],
+                                             W[2 * i + 1][2], W[2 * i + 1][3]);
           }
         }
         if (ch == C::kNCh - 1) {  // every word of the stage has been read (and used): free the slot
@@ -901,14 +896,11 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       if (!ok) break;
       wf_ready = __all_sync(0xffffffffu, wf != 0u);
       ws = ws1;
-      // the scale factors of this row (its own quarter, column 4g + quarter of group g) and of B
-      // rows 32c + lane (every quarter holds a copy)
+      // the scale factors of this row: its own quarter, column 4g + quarter of group g
 #pragma unroll
       for (int g = 0; g < kNG; g++) {
         const uint32_t gg = (uint32_t)(kNG * h + g);
         tmem_st_x1(tq + kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[2 * g] | (pa[2 * g + 1] << 16));
-#pragma unroll
-        for (int c = 0; c < C::kC; c++) tmem_st_x1(tq + kSfbCol + kKB * b + 4u * gg + (uint32_t)c, pb[g][c]);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -916,10 +908,6 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       mbar_arrive_one(&a_full[2 * b + hf]);
 #pragma unroll
       for (int i = 0; i < kNBT / 2; i++) pa[i] = na[i];
-#pragma unroll
-      for (int g = 0; g < kNG; g++)
-#pragma unroll
-        for (int c = 0; c < C::kC; c++) pb[g][c] = nb[g][c];
       b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
       if constexpr (CARRY) {
         r_c += seg_inc;
@@ -1021,8 +1009,8 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         if (q >= C::kNB && !(ok = mbar_wait_sleep(&b_empty[bb], (uint32_t)((q - C::kNB) / C::kNB) & 1u, tmo,
                                                   kLoaderSleepNs)))
           break;
-        mbar_arrive_expect_tx(&b_full[bb], C::kBStage);
-        bulk_g2s(smem + geo.off_B + (uint32_t)bb * C::kBStage, src + (size_t)s * C::kBStage, C::kBStage, &b_full[bb]);
+        mbar_arrive_expect_tx(&b_full[bb], C::kBSlot);
+        bulk_g2s(smem + geo.off_B + (uint32_t)bb * C::kBSlot, src + (size_t)s * C::kBSlot, C::kBSlot, &b_full[bb]);
         issued++;
         if (++s == S) {
           s = 0;
@@ -1171,7 +1159,8 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         ok = mbar_wait_sleep(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo, kMmaSleepNs);
       const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
       const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
-      const uint64_t bd = smem_desc(b0 + (uint32_t)bb * C::kBStage, 128u, C::kSbo);
+      const uint64_t bd = smem_desc(b0 + (uint32_t)bb * C::kBSlot, 128u, C::kSbo);
+      const uint32_t bsf0 = b0 + (uint32_t)bb * C::kBSlot + C::kBStage;  // the stage's B scale tiles
       const uint32_t sfa = tbase + kSfaCol + kKB * (uint32_t)b, sfb = tbase + kSfbCol + kKB * (uint32_t)b;
       const int wsx = q % kNW;  // MX: the stage's word slot
       const uint64_t ad0 = MX ? desc_sw128(smem_u32(smem + geo.off_W) + (uint32_t)wsx * kWStage) : 0ull;
@@ -1186,6 +1175,11 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         const int jfirst = C::kNI == 2 ? hh * kKB / 4 : 0;  // this issuer's first MMA of a job
         const uint32_t d_t = tbase + (uint32_t)(((jl & 1) * C::kNI + (C::kNI == 2 ? hh : 0)) * NMAX);
         if (leader) {
+          // the B scale factors of this half's groups (4 blocks each), ahead of the MMAs that read
+          // them: tcgen05 operations of one thread run in issue order
+#pragma unroll
+          for (int g = hh * kKB / 8; g < (hh + 1) * kKB / 8; g++)
+            if (2 * g < nmma) tmem_cp_sf(sfb + 4u * (uint32_t)g, smem_desc(bsf0 + 512u * (uint32_t)g, 128u, 128u));
 #pragma unroll
           for (int j = hh * kKB / 4; j < (hh + 1) * kKB / 4; j++) {
             if (j < nmma) {

@@ -59,27 +59,47 @@ __device__ __forceinline__ Planes decode_block(uint32_t L, uint32_t H, uint32_t 
 //   L2 ^ L4 = F << 2,  L3 ^ L5 = F << 3,  L1 ^ L7 = U << 1,  H4 ^ H6 = G << 4,  H3 ^ H5 = G << 3,
 // and X = H ^ F2 ^ L7 is shared by q1 (X ^ H1) and n1 (H1 cancels): 11 shifts and 9 XOR terms
 // instead of 14 and 10.
-__device__ __forceinline__ Planes decode_block0(uint32_t L, uint32_t H) {
+// decode_block0 with n3 returned inverted (n3 = ~H ^ q1, returned as H ^ q1), for the transpose
+// that absorbs the inversion.
+__device__ __forceinline__ Planes decode_block0_i3(uint32_t L, uint32_t H) {
   const uint32_t F = L ^ (L << 2), U = L ^ (L << 6), H2 = H << 2, G = H ^ H2;
   const uint32_t X = H ^ (F << 2) ^ (L << 7);
   const uint32_t q1h = X ^ (H << 1);  // H ^ q1
   Planes r;
-  r.n3 = ~q1h;
+  r.n3 = q1h;
   r.n0 = ~(q1h ^ (U << 1) ^ (G << 4));
   r.n1 = ~(X ^ (F << 3) ^ (H << 7));
   r.n2 = ~(q1h ^ U ^ (G << 3) ^ H2);
   return r;
 }
 
+__device__ __forceinline__ Planes decode_block0(uint32_t L, uint32_t H) {
+  Planes r = decode_block0_i3(L, H);
+  r.n3 = ~r.n3;
+  return r;
+}
+
 // Exchange the bits of a selected by (M << S) with the bits of b selected by M, as two bit selects
-// (two shifts and two three-input logic ops; with operands (mask, x, y), lop3 LUT 0xCA is
-// "mask ? x : y").
+// (two shifts and two three-input logic ops; with operands (x, y, mask), lop3 LUT 0xE4 is
+// "mask ? x : y"; the masks are immediates).
 template <int S, uint32_t M>
 __device__ __forceinline__ void delta_swap(uint32_t &a, uint32_t &b) {
   uint32_t na, nb;
   const uint32_t a_sh = a >> S, b_sh = b << S;
-  asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(nb) : "r"(M), "r"(a_sh), "r"(b));
-  asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(na) : "r"(M << S), "r"(b_sh), "r"(a));
+  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(nb) : "r"(a_sh), "r"(b), "n"(M));
+  asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(na) : "r"(b_sh), "r"(a), "n"(M << S));
+  a = na;
+  b = nb;
+}
+
+// The same exchange for b given inverted (bi = ~b): the selects read ~bi (LUTs 0xB1 for
+// "mask ? x : ~y" and 0x4E for "mask ? ~x : y"), so the inversion costs no instruction.
+template <int S, uint32_t M>
+__device__ __forceinline__ void delta_swap_inv_b(uint32_t &a, uint32_t &b, uint32_t bi) {
+  uint32_t na, nb;
+  const uint32_t a_sh = a >> S, bi_sh = bi << S;
+  asm("lop3.b32 %0, %1, %2, %3, 0xB1;" : "=r"(nb) : "r"(a_sh), "r"(bi), "n"(M));
+  asm("lop3.b32 %0, %1, %2, %3, 0x4E;" : "=r"(na) : "r"(bi_sh), "r"(a), "n"(M << S));
   a = na;
   b = nb;
 }
@@ -93,6 +113,21 @@ __device__ __forceinline__ void planes_to_nibbles_interleaved(const Planes &p, u
   delta_swap<1, 0x55555555u>(c, d);  // c: (n2,n3) of even weights; d: of odd weights
   delta_swap<2, 0x33333333u>(a, c);  // a: nibbles of weights 4v; c: of 4v+2
   delta_swap<2, 0x33333333u>(b, d);  // b: nibbles of weights 4v+1; d: of 4v+3
+  w0 = a;
+  w1 = b;
+  w2 = c;
+  w3 = d;
+}
+
+// The same from planes whose n3 is given inverted (n3i = ~n3, as the segment-start decoder
+// produces it).
+__device__ __forceinline__ void planes_to_nibbles_interleaved_i3(const Planes &p, uint32_t &w0, uint32_t &w1,
+                                                                 uint32_t &w2, uint32_t &w3) {
+  uint32_t a = p.n0, b = p.n1, c = p.n2, d;
+  delta_swap<1, 0x55555555u>(a, b);
+  delta_swap_inv_b<1, 0x55555555u>(c, d, p.n3);
+  delta_swap<2, 0x33333333u>(a, c);
+  delta_swap<2, 0x33333333u>(b, d);
   w0 = a;
   w1 = b;
   w2 = c;
