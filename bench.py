@@ -4,12 +4,16 @@
 Headline (the metric): one step = one batch-1 fused decode GEMV, y = W x, on the gate_up matrices
 of all 32 experts of the hidden-2880 MoE layer stacked into one matrix (184320 x 2880, 2-bit
 trellis stream, one UE8M0 scale per 32 weights, seg_len 32; bf16 N(0,1) activations, bf16 out),
-through trellis_gemv (the activation split and the decode-MMA product: two launches). Steps rotate
-over three distinct resident matrices (450 MB, > 3x L2) and eight activation vectors, so no step
-finds its weights in L2. value = decoded weights/s of the whole job; roofline = that call.
+through trellis_gemv_tiled (the activation split and the decode-MMA product: two launches), the
+weights' UE8M0 scales held as scale tiles (the same bytes, rearranged once at load time by
+trellis_make_scale_tiles, outside the timed region). Steps rotate over three distinct resident
+matrices (450 MB, > 3x L2) and eight activation vectors, so no step finds its weights in L2.
+value = decoded weights/s of the whole job; roofline = that call.
 
 Extra rows, each timed on its own with CUDA events on the launching stream after warm-up:
-  * gemv_down: the same GEMV on the down matrices stacked (92160 x 2880);
+  * gemv_gate_up_raw_scales: the headline call through trellis_gemv, scales in their [rows][cols/32]
+    layout;
+  * gemv_down: the same GEMV on the down matrices stacked (92160 x 2880), scale tiles;
   * expand: decode-only expansion of the whole layer into resident MXFP4 (gate_up + down);
   * moe_t1: routing + fused grouped MoE of the layer at batch 1, top-4 of 32;
   * moe_sweep: the same at T = 1, 2, 4, 8, 16, 32 with N(0,1) routing, and with every token on the
@@ -227,6 +231,8 @@ class Layer:
         self.Grot = [self.G] + [tc.TrellisMatrix(rand_words(self.G.stream.numel(), gen, device),
                                                  rand_scales(self.G.scales.numel(), 120, 126, gen, device),
                                                  self.G.rows, self.G.cols, SEG) for _ in range(ROT - 1)]
+        # the scale tiles of every rotated matrix and of down, made once (load time)
+        self.Trot = [tc.scale_tiles(g) for g in self.Grot]
         gu, gus = self.G.stream.view(E, -1), self.G.scales.view(E, -1)
         dn, dns = self.D.stream.view(E, -1), self.D.scales.view(E, -1)
         self.M = tc.MoEWeights([tc.TrellisMatrix(gu[e], gus[e], 2 * I, H, SEG) for e in range(E)],
@@ -237,9 +243,13 @@ class Layer:
         self.yD = torch.empty((1, E * H), dtype=torch.bfloat16, device=device)
         self.wsG = torch.empty(max(1, tc.gemv_workspace_bytes(self.G, 1)), dtype=torch.uint8, device=device)
         self.wsD = torch.empty(max(1, tc.gemv_workspace_bytes(self.D, 1)), dtype=torch.uint8, device=device)
+        self.TD = tc.scale_tiles(self.D)
         self.launches_per_step = 2  # the activation split and the decode-MMA product
 
     def step(self, i):
+        self.tc.gemv_tiled(self.Grot[i % ROT], self.Trot[i % ROT], self.x[i % NVAR], self.yG, self.wsG)
+
+    def step_raw(self, i):
         self.tc.gemv(self.Grot[i % ROT], self.x[i % NVAR], self.yG, self.wsG)
 
     def run_only(self, name, i):
@@ -247,8 +257,10 @@ class Layer:
         tc = self.tc
         if name == "gemv_gate_up":
             self.step(i)
+        elif name == "gemv_gate_up_raw":
+            self.step_raw(i)
         elif name == "gemv_down":
-            tc.gemv(self.D, self.xd[i % NVAR], self.yD, self.wsD)
+            tc.gemv_tiled(self.D, self.TD, self.xd[i % NVAR], self.yD, self.wsD)
         elif name == "expand_gate_up":
             self._expanded()
             tc.decode_to_mxfp4(self.G, self.nibG, self.scG)
@@ -316,9 +328,18 @@ def moe_paths(ids, T):
 # ----------------------------------------------------------------------------- extra rows
 
 def row_gemv_down(L, n, peak):
-    us = time_calls(lambda i: L.tc.gemv(L.D, L.xd[i % NVAR], L.yD, L.wsD), n)
+    us = time_calls(lambda i: L.tc.gemv_tiled(L.D, L.TD, L.xd[i % NVAR], L.yD, L.wsD), n)
+    us_raw = time_calls(lambda i: L.tc.gemv(L.D, L.xd[i % NVAR], L.yD, L.wsD), n)
     return {**rate(gemv_bytes(E * H, I, 1), us, peak), "decoded_weights_per_s": E * H * I / (us * 1e-6),
-            "shape": "92160 x 2880, T = 1", "calls": n}
+            "shape": "92160 x 2880, T = 1, scale tiles", "raw_scales": rate(gemv_bytes(E * H, I, 1), us_raw, peak),
+            "calls": n}
+
+
+def row_gemv_raw(L, n, peak):
+    us = time_calls(L.step_raw, n)
+    return {**rate(gemv_bytes(L.G.rows, L.G.cols, 1), us, peak),
+            "decoded_weights_per_s": L.G.rows * L.G.cols / (us * 1e-6),
+            "what": "the headline call through trellis_gemv (scales in their [rows][cols/32] layout)", "calls": n}
 
 
 def row_expand(L, n, peak):
@@ -364,9 +385,11 @@ def row_gemv_sweep(L, n, peak):
         y = torch.empty((T, G.rows), dtype=torch.bfloat16, device=d)
         ws_f = torch.empty(max(1, tc.gemv_workspace_bytes(G, T)), dtype=torch.uint8, device=d)
         ws_m = torch.empty(max(1, tc.mxfp4_gemv_workspace_bytes(Gm, T)), dtype=torch.uint8, device=d)
-        us_f = time_calls(lambda i: tc.gemv(G, x, y, ws_f), n)
+        us_f = time_calls(lambda i: tc.gemv_tiled(G, L.Trot[0], x, y, ws_f), n)
+        us_r = time_calls(lambda i: tc.gemv(G, x, y, ws_f), n)
         us_m = time_calls(lambda i: tc.mxfp4_gemv(Gm, x, y, ws_m), n)
         out.append({"T": T, "fused": rate(gemv_bytes(G.rows, G.cols, T), us_f, peak),
+                    "fused_raw_scales": rate(gemv_bytes(G.rows, G.cols, T), us_r, peak),
                     "mxfp4": rate(gemv_bytes(G.rows, G.cols, T, 0.53125), us_m, peak)})
     return {"shape": "184320 x 2880", "calls": n, "rows": out}
 
@@ -493,10 +516,10 @@ def row_e5m3(L, n, peak, seed):
 
 def run_e2e(L, steps):
     """The headline metric through the public API with HOST buffers: every step copies the gate_up
-    stream, its scales and x from pinned host memory, runs trellis_gemv and copies y back."""
+    stream, its scale tiles and x from pinned host memory, runs trellis_gemv_tiled and copies y back."""
     lay = L.layer
     h_st = torch.from_numpy(lay.gu_stream.view("int32").reshape(-1)).pin_memory()
-    h_sc = torch.from_numpy(lay.gu_scales.reshape(-1)).pin_memory()
+    h_sc = L.Trot[0].cpu().pin_memory()  # the scale tiles, as stored
     h_x = [x.cpu().pin_memory() for x in L.x]
     h_y = torch.empty(L.yG.shape, dtype=L.yG.dtype).pin_memory()
     h2d = h_st.numel() * 4 + h_sc.numel() + h_x[0].numel() * 2
@@ -504,9 +527,9 @@ def run_e2e(L, steps):
 
     def one(i):
         L.G.stream.copy_(h_st, non_blocking=True)
-        L.G.scales.copy_(h_sc, non_blocking=True)
+        L.Trot[0].copy_(h_sc, non_blocking=True)
         L.x[i % NVAR].copy_(h_x[i % NVAR], non_blocking=True)
-        L.tc.gemv(L.G, L.x[i % NVAR], L.yG, L.wsG)
+        L.tc.gemv_tiled(L.G, L.Trot[0], L.x[i % NVAR], L.yG, L.wsG)
         h_y.copy_(L.yG, non_blocking=True)
     us = time_calls(one, steps, warm=2)
     return {"value": L.G.rows * L.G.cols / (us * 1e-6), "unit": UNIT, "ms_per_step": us / 1e3,
@@ -681,7 +704,8 @@ def main():
     achieved = nb / (ms_per_step * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": NCU_TRAFFIC_GEMV_GATE_UP,
-                "kernel": "trellis_gemv: k_bsplit_gemv + k_mma (decode-MMA) on the 184320 x 2880 gate_up stack, T = 1",
+                "kernel": "trellis_gemv_tiled: k_bsplit_gemv + k_mma (decode-MMA, scale tiles) on the 184320 x 2880 "
+                          "gate_up stack, T = 1",
                 "algo_bytes_per_launch": nb, "avg_us": round(ms_per_step * 1e3, 3),
                 "frac_of_8tbs": round(achieved / SPEC_HBM_GBS, 4),
                 "peak_source": (f"{peak_kind}: MEASURED_PEAKS.json hbm_gbs" if peak_kind == "measured"
@@ -692,6 +716,7 @@ def main():
             "dtype": "u32 decode, f32 accumulate", "data": "synthetic",
             "config": {"workload": WORKLOAD, "rows": L.G.rows, "cols": L.G.cols, "tokens": 1, "seg_len": SEG,
                        "decoded_weights_per_step": weights_per_step,
+                       "scales": "UE8M0 scale tiles (the same bytes as [rows][cols/32], rearranged once at load time)",
                        "l2": f"inputs larger than L2: steps rotate over {ROT} distinct resident matrices "
                              f"({ROT * nb / 1e6:.0f} MB) and {NVAR} activation vectors",
                        "parallelism": f"replicas x{world}",
@@ -702,6 +727,7 @@ def main():
     if not args.no_rows:
         n = 200
         rows = {}
+        rows["gemv_gate_up_raw_scales"] = row_gemv_raw(L, 1000, peak)
         rows["gemv_down"] = row_gemv_down(L, n, peak)
         rows["expand"] = row_expand(L, 100, peak)
         rows["moe_t1"] = row_moe(L, 1, n, peak)

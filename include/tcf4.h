@@ -106,6 +106,25 @@ TCF4_API size_t trellis_gemv_workspace(tcf4_matrix w, int32_t T);
 TCF4_API tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *workspace,
                                   size_t ws_bytes, void *stream);
 
+/* Scale tiles: the weights' UE8M0 scales rearranged once, at load time, into the layout the tensor
+ * cores' scale-factor copies read (HEPH abstract, first serving mode: the grid-aligned scale of each
+ * 32-weight block; the bytes are the same, only their order changes). For 128-row tile t and
+ * 4-block group g (g < 8 * ceil(cols / 1024), a whole number of 32-block stages per tile) a
+ * 512-byte tile at byte offset (t * groups + g) * 512 whose byte 16 r + 4 q + i is the scale of
+ * row 128 t + 32 q + r, block 4 g + i, or 0 past the matrix.
+ *   trellis_scale_tiles_bytes: the size (0 for an invalid or empty matrix).
+ *   trellis_make_scale_tiles: writes them from w.scales; tiles 16-byte aligned, caller-owned. */
+TCF4_API size_t trellis_scale_tiles_bytes(tcf4_matrix w);
+TCF4_API tcf4_status trellis_make_scale_tiles(tcf4_matrix w, uint8_t *tiles, void *stream);
+
+/* trellis_gemv with the weights' scales read from scale tiles (w.scales is not read and may be
+ * NULL). Same result, accuracy, workspace (trellis_gemv_workspace) and limits as trellis_gemv, on
+ * the tensor-core path only: cols a multiple of 64 and tiles 16-byte aligned, else
+ * TCF4_ERR_UNSUPPORTED. The decode then does no scale work: the scale tiles of each stage are
+ * bulk-copied beside its stream words and moved to the tensor memory by the MMA issuers. */
+TCF4_API tcf4_status trellis_gemv_tiled(tcf4_matrix w, const uint8_t *tiles, const uint16_t *x, int32_t T,
+                                        uint16_t *y, void *workspace, size_t ws_bytes, void *stream);
+
 /* The XOR-Trellis news page's grouping format: E2M1 elements with E5M3 block scales (its paragraph
  * on the format; no encoding given). w.scales holds one E5M3 byte per 32-weight block, read as: no
  * sign bit, exponent bits 7..3 with bias 15, mantissa bits 2..0, exponent 0 subnormal (2^-14 m/8),

@@ -144,3 +144,28 @@ def test_encode_argument_checks(lib):
     assert e(p8, p8, p16, 2, 64, 32, p8, s0, ctypes.c_void_p(256 * 64 + 128), 1 << 20, s0) == 2
     assert e(p8, p8, p16, 1 << 20, 1 << 12, 32, p8, s0, ws, 1 << 20, s0) == 3   # 2^32 weights
     assert e(p8, p8, p16, 0, 64, 32, p8, s0, s0, 0, s0) == 0
+
+
+def test_scale_tile_sizes_and_checks(lib):
+    # 128-row tiles x 8 groups per started 1024 columns x 512 bytes; host checks before any launch
+    assert lib.trellis_scale_tiles_bytes(_mat(rows=1, cols=64)) == 1 * 8 * 512
+    assert lib.trellis_scale_tiles_bytes(_mat(rows=128, cols=1024)) == 1 * 8 * 512
+    assert lib.trellis_scale_tiles_bytes(_mat(rows=129, cols=1056)) == 2 * 16 * 512
+    assert lib.trellis_scale_tiles_bytes(_mat(rows=184320, cols=2880)) == 1440 * 24 * 512
+    assert lib.trellis_scale_tiles_bytes(_mat(rows=0)) == 0
+    assert lib.trellis_scale_tiles_bytes(_mat(cols=48)) == 0
+    s0 = ctypes.c_void_p(0)
+    assert lib.trellis_make_scale_tiles(_mat(), ctypes.c_void_p(0), s0) == 1       # null tiles
+    assert lib.trellis_make_scale_tiles(_mat(), ctypes.c_void_p(4104), s0) == 2    # misaligned tiles
+    assert lib.trellis_make_scale_tiles(_mat(cols=48), ctypes.c_void_p(4096), s0) == 1
+    assert lib.trellis_make_scale_tiles(_mat(rows=0), ctypes.c_void_p(0), s0) == 0  # empty: nothing to do
+    ok_x, ok_y, ok_t = ctypes.c_void_p(4096), ctypes.c_void_p(8192), ctypes.c_void_p(16384)
+
+    def gemv_tiled(w, t, x, T, y):
+        return lib.trellis_gemv_tiled(w, t, x, T, y, ctypes.c_void_p(0), 0, s0)
+
+    assert gemv_tiled(_mat(scales=0), ctypes.c_void_p(0), ok_x, 1, ok_y) == 1   # null tiles
+    assert gemv_tiled(_mat(scales=0), ctypes.c_void_p(16392), ok_x, 1, ok_y) == 2
+    assert gemv_tiled(_mat(), ok_t, ok_x, 33, ok_y) == 3                         # T > 32
+    assert gemv_tiled(_mat(cols=48), ok_t, ok_x, 1, ok_y) == 1
+    assert gemv_tiled(_mat(), ok_t, ok_x, 0, ok_y) == 0                          # T == 0: no-op

@@ -16,7 +16,8 @@ import torch
 
 from . import _abi
 
-__all__ = ["TrellisMatrix", "MoEWeights", "decode_to_mxfp4", "gemv", "gemv_workspace_bytes", "moe_route",
+__all__ = ["TrellisMatrix", "MoEWeights", "decode_to_mxfp4", "gemv", "gemv_workspace_bytes", "scale_tiles",
+           "gemv_tiled", "moe_route",
            "grouped_moe",
            "moe_workspace_bytes", "moe_hidden_offset", "device_timeouts", "Tcf4Error"]
 
@@ -88,6 +89,29 @@ def gemv(w: TrellisMatrix, x: torch.Tensor, out=None, workspace=None):
     nbytes = workspace.numel() if workspace is not None else 0
     _abi.check(_abi.load().trellis_gemv(w.abi(), _ptr(x), T, _ptr(out), _ptr(workspace), nbytes, _stream_handle()),
                "trellis_gemv")
+    return out
+
+
+def scale_tiles(w: TrellisMatrix, out=None):
+    """The weights' UE8M0 scales rearranged once into scale tiles (uint8, trellis_scale_tiles_bytes
+    long), the layout trellis_gemv_tiled reads."""
+    n = int(_abi.load().trellis_scale_tiles_bytes(w.abi()))
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=w.stream.device)
+    _abi.check(_abi.load().trellis_make_scale_tiles(w.abi(), _ptr(out), _stream_handle()), "trellis_make_scale_tiles")
+    return out
+
+
+def gemv_tiled(w: TrellisMatrix, tiles: torch.Tensor, x: torch.Tensor, out=None, workspace=None):
+    """gemv with the weights' scales read from scale tiles (see scale_tiles): bf16 [T][rows]."""
+    x = x if x.dim() == 2 else x.view(1, -1)
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, w.rows), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(gemv_workspace_bytes(w, T), 1), dtype=torch.uint8, device=x.device)
+    _abi.check(_abi.load().trellis_gemv_tiled(w.abi(), _ptr(tiles), _ptr(x), T, _ptr(out), _ptr(workspace),
+                                              workspace.numel(), _stream_handle()), "trellis_gemv_tiled")
     return out
 
 

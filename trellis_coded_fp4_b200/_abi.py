@@ -15,6 +15,7 @@ EXPORTED = ("trellis_decode_to_mxfp4", "trellis_gemv_workspace", "trellis_gemv",
             "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "mxfp4_gemv_workspace", "mxfp4_gemv",
             "mxfp4_grouped_moe_workspace", "mxfp4_grouped_moe_hidden_offset", "mxfp4_grouped_moe",
             "trellis_encode_workspace", "trellis_encode", "trellis_repack_interleaved", "trellis_gemv_e5m3",
+            "trellis_scale_tiles_bytes", "trellis_make_scale_tiles", "trellis_gemv_tiled",
             "tcf4_device_timeouts", "tcf4_status_string")
 
 
@@ -65,6 +66,12 @@ def load(path: str = LIB_PATH):
     L.trellis_gemv_workspace.restype = sz
     L.trellis_gemv.argtypes = [Matrix, vp, i32, vp, vp, sz, vp]
     L.trellis_gemv.restype = ctypes.c_int
+    L.trellis_scale_tiles_bytes.argtypes = [Matrix]
+    L.trellis_scale_tiles_bytes.restype = sz
+    L.trellis_make_scale_tiles.argtypes = [Matrix, vp, vp]
+    L.trellis_make_scale_tiles.restype = ctypes.c_int
+    L.trellis_gemv_tiled.argtypes = [Matrix, vp, vp, i32, vp, vp, sz, vp]
+    L.trellis_gemv_tiled.restype = ctypes.c_int
     L.trellis_gemv_noalloc.argtypes = [Matrix, vp, i32, vp, vp]
     L.trellis_gemv_noalloc.restype = ctypes.c_int
     L.trellis_moe_route.argtypes = [vp, i32, i32, i32, vp, vp, vp]

@@ -83,6 +83,9 @@ struct Cfg {
   // words of B rows r, 32 + r, 64 + r (and one spare word), the source of one tcgen05.cp
   static constexpr uint32_t kSfbStage = (kKB / 4) * 512u;
   static constexpr uint32_t kBSlot = kBStage + kSfbStage;       // one stage of terms + scales
+  // Weights' scales as scale tiles (trellis_gemv_tiled): per 4-block group a 512-byte tile, row r
+  // = the group's UE8M0 words of tile rows r, 32 + r, 64 + r, 96 + r; KB/4 tiles per stage.
+  static constexpr uint32_t kSfaTile = (kKB / 4) * 512u;
   // MMA issuers: one per half stage, each into its own accumulator, where TMEM has room for the
   // two accumulator pairs (one issuing thread sustains about one MMA per 60 cycles; two of them in
   // different warps run concurrently).
@@ -318,18 +321,20 @@ __global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ 
 
 // ------------------------------------------------------------------------------- geometry
 
-// Shared memory: barriers + tensor-map copy | word ring | B ring | gate/up exchange | group plan.
+// Shared memory: barriers + tensor-map copy | word ring | B ring (with the weights' scale tiles
+// when tiled) | gate/up exchange | group plan.
 struct MmaGeom {
-  uint32_t off_W, off_B, off_U, off_P, smem;
+  uint32_t off_W, off_B, bslot, off_U, off_P, smem;
 };
 
 template <int NMAX>
-__host__ __device__ inline MmaGeom mma_geom(int mode, bool mx = false) {
+__host__ __device__ inline MmaGeom mma_geom(int mode, bool mx = false, bool tiled = false) {
   using C = Cfg<NMAX>;
   MmaGeom g;
   g.off_W = 1024u;
   g.off_B = g.off_W + (mx ? C::kNWX * C::kWStageX : C::kNW * C::kWStage);
-  g.off_U = g.off_B + C::kNB * C::kBSlot;
+  g.bslot = C::kBSlot + (tiled ? C::kSfaTile : 0u);
+  g.off_U = g.off_B + C::kNB * g.bslot;
   g.off_P = g.off_U + (mode == kModeGateUp ? 2u * 64u * (uint32_t)C::kTok * 4u : 0u);
   g.smem = g.off_P + (mode == kModeGemv ? 0u : round_up((uint32_t)sizeof(GroupPlan), 128u));
   return g;
@@ -543,6 +548,8 @@ struct MmaArgs {
   int *counters;          // 4 per 128-row chunk of H
   uint16_t *out;          // [T][H] bf16
   unsigned char *maps;    // MoE: per-CTA tensor-map slots [gridDim][kMapSlots][128]
+  const uint8_t *sf_tiles;  // tiled GEMV: the weights' scale tiles, sf_groups 512-byte tiles per 128-row tile
+  int sf_groups;
 };
 
 // A job is one 128-row tile: tile rows [0, 64) are matrix rows y0.., tile rows [64, 128) matrix
@@ -622,7 +629,12 @@ __device__ __forceinline__ int tile_row(const JobRows &j, int m) {
 // eight other warps give theirs down to 48 (16 x 32 x 96 + 8 x 32 x 48 = 61440). Launched only after
 // the host has checked that the compiled kernel's registers cover that sum, since a larger request
 // than the launch holds would never be granted.
-template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS = false>
+// TILED (plain GEMV only): the weights' scales come as scale tiles; the B loader bulk-copies each
+// stage's tiles into its B slot (after the activation terms) and the MMA issuers move them to TMEM
+// with tcgen05.cp, so the decode warps handle no scale factors at all. (In the B ring they are
+// released with the stage's MMAs; a ring of their own beside the word ring held back the word
+// loads, whose slots free up earlier.)
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS = false, bool TILED = false>
 __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
                                                      const __grid_constant__ MoeTable<MAXE> tab,
                                                      const __grid_constant__ CUtensorMap wmap) {
@@ -634,7 +646,8 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = a.nbr, S = (nbr + kKB - 1) / kKB;
-  const MmaGeom geo = mma_geom<NMAX>(MODE, MX);
+  static_assert(!TILED || (MODE == kModeGemv && !MX), "scale tiles: plain decode GEMV only");
+  const MmaGeom geo = mma_geom<NMAX>(MODE, MX, TILED);
   static_assert((MX ? 2 * kNW : kNW) <= 8 && kNA <= 4 && C::kNB <= 4,
                 "barrier block: 8 word slots, 4 A and 4 B slots");
   // 49 barriers in bytes [0, 392). The A operand of a stage is filled and released in two halves
@@ -789,7 +802,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
     int qp = 0, jl_p = 0, s_p = 0;
     const unsigned short *srow = nullptr;  // row m's scales of the front job, from block kNBT h on
     auto load_sf = [&](uint32_t(&da)[kNBT / 2]) {
-      if (qp >= nq) return;
+      if (TILED || qp >= nq) return;
       if (s_p == 0) {
         const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_p));
         const int row = tile_row(jr, m);
@@ -897,10 +910,12 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       wf_ready = __all_sync(0xffffffffu, wf != 0u);
       ws = ws1;
       // the scale factors of this row: its own quarter, column 4g + quarter of group g
+      if constexpr (!TILED) {
 #pragma unroll
-      for (int g = 0; g < kNG; g++) {
-        const uint32_t gg = (uint32_t)(kNG * h + g);
-        tmem_st_x1(tq + kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[2 * g] | (pa[2 * g + 1] << 16));
+        for (int g = 0; g < kNG; g++) {
+          const uint32_t gg = (uint32_t)(kNG * h + g);
+          tmem_st_x1(tq + kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[2 * g] | (pa[2 * g + 1] << 16));
+        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -1004,13 +1019,22 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       for (int q = 0; q < nq; q++) {
         if (*abort_flag) break;
         const int bb = q % C::kNB;
-        if (s == 0) src = a.terms + (size_t)job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl)).group * tbytes;
+        int job_chunk = 0;
+        if (s == 0) {
+          const JobRows jq = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl));
+          src = a.terms + (size_t)jq.group * tbytes;
+        }
+        if (TILED) job_chunk = job_of(jl);  // plain GEMV: the job is the 128-row tile
         // up to kNB stages ahead of the MMAs: the slot is free once its last use was released
         if (q >= C::kNB && !(ok = mbar_wait_sleep(&b_empty[bb], (uint32_t)((q - C::kNB) / C::kNB) & 1u, tmo,
                                                   kLoaderSleepNs)))
           break;
-        mbar_arrive_expect_tx(&b_full[bb], C::kBSlot);
-        bulk_g2s(smem + geo.off_B + (uint32_t)bb * C::kBSlot, src + (size_t)s * C::kBSlot, C::kBSlot, &b_full[bb]);
+        mbar_arrive_expect_tx(&b_full[bb], geo.bslot);
+        bulk_g2s(smem + geo.off_B + (uint32_t)bb * geo.bslot, src + (size_t)s * C::kBSlot, C::kBSlot, &b_full[bb]);
+        if (TILED)
+          bulk_g2s(smem + geo.off_B + (uint32_t)bb * geo.bslot + C::kBSlot,
+                   a.sf_tiles + ((size_t)job_chunk * a.sf_groups + (size_t)s * (kKB / 4)) * 512u, C::kSfaTile,
+                   &b_full[bb]);
         issued++;
         if (++s == S) {
           s = 0;
@@ -1159,8 +1183,8 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         ok = mbar_wait_sleep(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo, kMmaSleepNs);
       const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
       const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
-      const uint64_t bd = smem_desc(b0 + (uint32_t)bb * C::kBSlot, 128u, C::kSbo);
-      const uint32_t bsf0 = b0 + (uint32_t)bb * C::kBSlot + C::kBStage;  // the stage's B scale tiles
+      const uint64_t bd = smem_desc(b0 + (uint32_t)bb * geo.bslot, 128u, C::kSbo);
+      const uint32_t bsf0 = b0 + (uint32_t)bb * geo.bslot + C::kBStage;  // the stage's B scale tiles
       const uint32_t sfa = tbase + kSfaCol + kKB * (uint32_t)b, sfb = tbase + kSfbCol + kKB * (uint32_t)b;
       const int wsx = q % kNW;  // MX: the stage's word slot
       const uint64_t ad0 = MX ? desc_sw128(smem_u32(smem + geo.off_W) + (uint32_t)wsx * kWStage) : 0ull;
@@ -1180,6 +1204,12 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
 #pragma unroll
           for (int g = hh * kKB / 8; g < (hh + 1) * kKB / 8; g++)
             if (2 * g < nmma) tmem_cp_sf(sfb + 4u * (uint32_t)g, smem_desc(bsf0 + 512u * (uint32_t)g, 128u, 128u));
+          if constexpr (TILED) {  // the weights' scale factors: tile row r to lanes r, 32 + r, 64 + r, 96 + r
+            const uint32_t asf0 = b0 + (uint32_t)bb * geo.bslot + C::kBSlot;  // the weights' scale tiles
+#pragma unroll
+            for (int g = hh * kKB / 8; g < (hh + 1) * kKB / 8; g++)
+              if (2 * g < nmma) tmem_cp_sf(sfa + 4u * (uint32_t)g, smem_desc(asf0 + 512u * (uint32_t)g, 128u, 128u));
+          }
 #pragma unroll
           for (int j = hh * kKB / 4; j < (hh + 1) * kKB / 4; j++) {
             if (j < nmma) {
@@ -1270,11 +1300,11 @@ static bool make_word_map(CUtensorMap *map, const void *stream, int rows, int nb
 constexpr int kGemvTok = Cfg<96>::kTok;
 static int nmax_for(int tokens_per_group) { return tokens_per_group <= Cfg<32>::kTok ? 32 : 96; }
 
-static bool mma_fits(int NMAX, int mode, bool mx = false) {
+static bool mma_fits(int NMAX, int mode, bool mx = false, bool tiled = false) {
   int dev = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
-  const uint32_t need = NMAX == 32 ? mma_geom<32>(mode, mx).smem : mma_geom<96>(mode, mx).smem;
+  const uint32_t need = NMAX == 32 ? mma_geom<32>(mode, mx, tiled).smem : mma_geom<96>(mode, mx, tiled).smem;
   return need <= (uint32_t)optin;
 }
 
@@ -1300,10 +1330,51 @@ bool mx_gemv_supported(const MatView &w, int T) {
          mma_fits(nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv, true);
 }
 
+// The tiled GEMV: the tensor-core path with the scale-tile ring (the tiles' pointer 16-byte aligned).
+bool gemv_tiled_supported(const MatView &w, const uint8_t *tiles, int T) {
+  return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.stream) & 15u) == 0 &&
+         (reinterpret_cast<uintptr_t>(tiles) & 15u) == 0 && tensor_map_encoder() != nullptr &&
+         mma_fits(nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv, false, true);
+}
+
+static int sm_count_impl();
+static int sm_count() { return sm_count_impl(); }
+
+// Scale tiles of a [rows][nbr] matrix: 128-row tiles, each with sf_groups = 8 * ceil(nbr / 32)
+// tiles of 512 bytes (a whole number of 32-block stages); byte 16 r + 4 q + i of group g of tile t
+// is the scale of row 128 t + 32 q + r, block 4 g + i (0 past the matrix).
+static int scale_tile_groups(int nbr) { return 8 * ((nbr + 31) / 32); }
+size_t scale_tiles_bytes(const MatView &w) { return (size_t)((w.rows + 127) / 128) * scale_tile_groups(w.nbr) * 512u; }
+
+__global__ void __launch_bounds__(256) k_scale_tiles(const uint8_t *__restrict__ sc, int rows, int nbr, int groups,
+                                                     uint32_t *__restrict__ tiles, size_t nwords) {
+  grid_dep_wait();
+  grid_dep_release();
+  for (size_t w = (size_t)blockIdx.x * blockDim.x + threadIdx.x; w < nwords; w += (size_t)gridDim.x * blockDim.x) {
+    const size_t t = w / ((size_t)groups * 128u);
+    const uint32_t rem = (uint32_t)(w - t * groups * 128u), g = rem >> 7, r = (rem >> 2) & 31u, q = rem & 3u;
+    const int row = (int)(128u * t + 32u * q + r);
+    uint32_t v = 0;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const int blk = (int)(4u * g) + i;
+      if (row < rows && blk < nbr) v |= (uint32_t)sc[(size_t)row * nbr + blk] << (8 * i);
+    }
+    tiles[w] = v;
+  }
+}
+
+cudaError_t launch_scale_tiles(const MatView &w, uint8_t *tiles, cudaStream_t s) {
+  const size_t nwords = scale_tiles_bytes(w) / 4;
+  const int grid = (int)((nwords + 255) / 256 < (size_t)(8 * sm_count()) ? (nwords + 255) / 256 : 8 * sm_count());
+  return launch_dependent(k_scale_tiles, dim3(grid), dim3(256), 0, s, w.scales, w.rows, w.nbr,
+                          scale_tile_groups(w.nbr), reinterpret_cast<uint32_t *>(tiles), nwords);
+}
+
 // Tokens beyond kGemvTok run as further passes, each with its own split of x.
 size_t gemv_mma_workspace(const MatView &w, int T) { return terms_for(w.nbr, nmax_for(T < kGemvTok ? T : kGemvTok)); }
 
-static int sm_count() {
+static int sm_count_impl() {
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
@@ -1311,44 +1382,50 @@ static int sm_count() {
 }
 
 // One launch of a product kernel instance (dynamic shared memory attribute set once per instance).
-template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS>
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS, bool TILED = false>
 static cudaError_t launch_product_rs(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
                                      cudaStream_t s) {
   static unsigned long long attr = 0;
-  cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS>, attr);
+  cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS, TILED>, attr);
   if (e != cudaSuccess) return e;
-  return launch_dependent(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS>, dim3(grid), dim3(Cfg<NMAX>::kThreads),
-                          mma_geom<NMAX>(MODE, MX).smem, s, args, tab, map);
+  return launch_dependent(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS, TILED>, dim3(grid), dim3(Cfg<NMAX>::kThreads),
+                          mma_geom<NMAX>(MODE, MX, TILED).smem, s, args, tab, map);
 }
 
 // True when the register-split instance was compiled with at least kRsLaunchRegs registers per
 // thread, so that its split can be granted (checked once per instance).
-template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY>
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool TILED>
 static bool register_split_ok() {
   static int ok = -1;
   if (ok < 0) {
     cudaFuncAttributes fa;
-    ok = cudaFuncGetAttributes(&fa, k_mma<MAXE, MODE, NMAX, MX, CARRY, true>) == cudaSuccess &&
+    ok = cudaFuncGetAttributes(&fa, k_mma<MAXE, MODE, NMAX, MX, CARRY, true, TILED>) == cudaSuccess &&
          fa.numRegs >= kRsLaunchRegs;
   }
   return ok == 1;
 }
 
 // The decode GEMV at NMAX = 32 takes the register split when its compiled registers allow it.
-template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY>
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool TILED = false>
 static cudaError_t launch_product(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
                                   cudaStream_t s) {
   if constexpr (MODE == kModeGemv && NMAX == 32 && !MX) {
-    if (register_split_ok<MAXE, MODE, NMAX, MX, CARRY>())
-      return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, true>(grid, args, tab, map, s);
+    if (register_split_ok<MAXE, MODE, NMAX, MX, CARRY, TILED>())
+      return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, true, TILED>(grid, args, tab, map, s);
   }
-  return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, false>(grid, args, tab, map, s);
+  return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, false, TILED>(grid, args, tab, map, s);
 }
 template <int MAXE, int MODE, int NMAX, bool MX>
 static cudaError_t launch_product_seg(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
                                       cudaStream_t s) {
   if constexpr (MX) {
     return launch_product<MAXE, MODE, NMAX, true, false>(grid, args, tab, map, s);
+  } else if constexpr (MODE == kModeGemv) {
+    if (args.sf_tiles != nullptr)
+      return args.seg_blocks > 1 ? launch_product<MAXE, MODE, NMAX, false, true, true>(grid, args, tab, map, s)
+                                 : launch_product<MAXE, MODE, NMAX, false, false, true>(grid, args, tab, map, s);
+    return args.seg_blocks > 1 ? launch_product<MAXE, MODE, NMAX, false, true>(grid, args, tab, map, s)
+                               : launch_product<MAXE, MODE, NMAX, false, false>(grid, args, tab, map, s);
   } else {
     return args.seg_blocks > 1 ? launch_product<MAXE, MODE, NMAX, false, true>(grid, args, tab, map, s)
                                : launch_product<MAXE, MODE, NMAX, false, false>(grid, args, tab, map, s);
@@ -1357,7 +1434,7 @@ static cudaError_t launch_product_seg(int grid, const MmaArgs &args, const MoeTa
 
 template <int NMAX, bool MX>
 static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, const uint16_t *x, int T, uint16_t *y,
-                                    void *ws, cudaStream_t s) {
+                                    void *ws, cudaStream_t s, const uint8_t *tiles) {
   uint8_t *terms = static_cast<uint8_t *>(ws);
   const int warps = T * w.nbr;
   cudaError_t e =
@@ -1373,12 +1450,15 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
   args.terms = terms;
   args.T = T;
   args.y = y;
+  args.sf_tiles = tiles;
+  args.sf_groups = scale_tile_groups(w.nbr);
   MoeTable<32> none{};
   return launch_product_seg<32, kModeGemv, NMAX, MX>(ntiles < nsm ? ntiles : nsm, args, none, map, s);
 }
 
 template <bool MX>
-static cudaError_t launch_gemv_t(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
+static cudaError_t launch_gemv_t(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s,
+                                 const uint8_t *tiles = nullptr) {
   CUtensorMap map;
   if (!make_word_map(&map, w.stream, w.rows, w.nbr, MX ? 16 : 8)) return cudaErrorInvalidValue;
   const bool n32 = nmax_for(T < kGemvTok ? T : kGemvTok) == 32;
@@ -1387,7 +1467,8 @@ static cudaError_t launch_gemv_t(const MatView &w, const uint16_t *x, int T, uin
     const uint16_t *xp = x + (size_t)t0 * w.nbr * 32;
     uint16_t *yp = y + (size_t)t0 * w.rows;
     cudaError_t e =
-        n32 ? launch_gemv_pass<32, MX>(w, map, xp, n, yp, ws, s) : launch_gemv_pass<96, MX>(w, map, xp, n, yp, ws, s);
+        n32 ? launch_gemv_pass<32, MX>(w, map, xp, n, yp, ws, s, tiles)
+            : launch_gemv_pass<96, MX>(w, map, xp, n, yp, ws, s, tiles);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -1398,6 +1479,10 @@ cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t
 }
 cudaError_t launch_mx_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
   return launch_gemv_t<true>(w, x, T, y, ws, s);
+}
+cudaError_t launch_gemv_tiled(const MatView &w, const uint8_t *tiles, const uint16_t *x, int T, uint16_t *y, void *ws,
+                              cudaStream_t s) {
+  return launch_gemv_t<false>(w, x, T, y, ws, s, tiles);
 }
 
 // ----------------------------------------------------------------------------- MoE on the tensor cores

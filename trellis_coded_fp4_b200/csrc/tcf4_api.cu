@@ -154,6 +154,39 @@ tcf4_status trellis_gemv(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *
   return from_cuda(launch_gemv(v, x, T, y, static_cast<cudaStream_t>(stream)));
 }
 
+size_t trellis_scale_tiles_bytes(tcf4_matrix w) {
+  if (check_matrix(w) != TCF4_OK || w.rows == 0 || w.cols == 0) return 0;
+  return scale_tiles_bytes(view(w));
+}
+
+tcf4_status trellis_make_scale_tiles(tcf4_matrix w, uint8_t *tiles, void *stream) {
+  tcf4_status st = check_matrix(w);
+  if (st != TCF4_OK) return st;
+  if (w.rows == 0 || w.cols == 0) return TCF4_OK;
+  if (tiles == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(tiles)) return TCF4_ERR_MISALIGNED;
+  if (scale_tiles_bytes(view(w)) / 4 >= ((size_t)1 << 31)) return TCF4_ERR_UNSUPPORTED;
+  clear_pending_error();
+  return from_cuda(launch_scale_tiles(view(w), tiles, static_cast<cudaStream_t>(stream)));
+}
+
+tcf4_status trellis_gemv_tiled(tcf4_matrix w, const uint8_t *tiles, const uint16_t *x, int32_t T, uint16_t *y,
+                               void *workspace, size_t ws_bytes, void *stream) {
+  tcf4_matrix wc = w;
+  if (wc.scales == nullptr) wc.scales = tiles;  // the raw scales are not read here
+  tcf4_status st = check_gemv(wc, T);
+  if (st != TCF4_OK) return st;
+  if (T == 0 || w.rows == 0) return TCF4_OK;
+  if (x == nullptr || y == nullptr || tiles == nullptr) return TCF4_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(tiles)) return TCF4_ERR_MISALIGNED;
+  const MatView v = view(wc);
+  if (!gemv_tiled_supported(v, tiles, T)) return TCF4_ERR_UNSUPPORTED;
+  if (workspace == nullptr || ws_bytes < gemv_mma_workspace(v, T)) return TCF4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
+  clear_pending_error();
+  return from_cuda(launch_gemv_tiled(v, tiles, x, T, y, workspace, static_cast<cudaStream_t>(stream)));
+}
+
 tcf4_status trellis_gemv_e5m3(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream) {
   tcf4_status st = check_gemv(w, T);
   if (st != TCF4_OK) return st;

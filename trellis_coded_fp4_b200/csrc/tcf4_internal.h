@@ -96,6 +96,13 @@ cudaError_t launch_moe(const tcf4_moe &m, int gu_seg, int dn_seg, const uint16_t
 bool gemv_mma_supported(const MatView &w, int T);
 size_t gemv_mma_workspace(const MatView &w, int T);
 cudaError_t launch_gemv_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s);
+// The same with the weights' scales as scale tiles (k_mma.cu): their size, the rearranging kernel,
+// whether the tiled path applies, its launch (workspace as for launch_gemv_mma).
+size_t scale_tiles_bytes(const MatView &w);
+cudaError_t launch_scale_tiles(const MatView &w, uint8_t *tiles, cudaStream_t s);
+bool gemv_tiled_supported(const MatView &w, const uint8_t *tiles, int T);
+cudaError_t launch_gemv_tiled(const MatView &w, const uint8_t *tiles, const uint16_t *x, int T, uint16_t *y, void *ws,
+                              cudaStream_t s);
 
 // Tensor-core grouped MoE (k_mma.cu): workspace regions (bytes, 256-aligned): the down kernel's
 // counters (4 per 128-row chunk of H), h (bf16 [T*k][I]), y (fp32 [T*k][H]), the activation terms
