@@ -136,8 +136,12 @@ struct GroupPlan {
   int n_groups;
 };
 
-// All threads of the CTA. Pairs whose expert id is outside [0, E) are dropped. Deterministic.
+// All threads of the CTA. Pairs whose expert id is outside [0, E) are dropped. Deterministic: groups
+// in expert order, the pairs of an expert in p order. The offsets come from one warp's prefix sum
+// over the experts (eight per lane), not a serial walk, so the plan costs little more than the load
+// of the routing ids.
 __device__ void build_groups(GroupPlan &pl, const int32_t *__restrict__ ids, int P, int E, int gmax) {
+  static_assert(kMaxExperts == 8 * 32, "eight experts per lane of the planning warp");
   const int tid = threadIdx.x;
   for (int e = tid; e < E; e += blockDim.x) pl.cnt[e] = 0;
   for (int p = tid; p < P; p += blockDim.x) pl.ids[p] = ids[p];
@@ -147,19 +151,39 @@ __device__ void build_groups(GroupPlan &pl, const int32_t *__restrict__ ids, int
     if (e >= 0 && e < E) atomicAdd(&pl.cnt[e], 1);
   }
   __syncthreads();
-  if (tid == 0) {
-    int o = 0, ng = 0;
-    for (int e = 0; e < E; e++) {
-      pl.off[e] = o;
-      for (int f = 0; f < pl.cnt[e]; f += gmax) {
+  if (tid < 32) {
+    int c[8], cs = 0, gs = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const int e = 8 * tid + i;
+      c[i] = e < E ? pl.cnt[e] : 0;
+      cs += c[i];
+      gs += (c[i] + gmax - 1) / gmax;
+    }
+    // exclusive prefix sums over the lanes
+    int ci = cs, gi = gs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int cu = __shfl_up_sync(0xffffffffu, ci, o), gu = __shfl_up_sync(0xffffffffu, gi, o);
+      if (tid >= o) {
+        ci += cu;
+        gi += gu;
+      }
+    }
+    int o = ci - cs, ng = gi - gs;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const int e = 8 * tid + i;
+      if (e < E) pl.off[e] = o;
+      for (int f = 0; f < c[i]; f += gmax) {
         pl.g_e[ng] = e;
         pl.g_first[ng] = o + f;
-        pl.g_cnt[ng] = pl.cnt[e] - f < gmax ? pl.cnt[e] - f : gmax;
+        pl.g_cnt[ng] = c[i] - f < gmax ? c[i] - f : gmax;
         ng++;
       }
-      o += pl.cnt[e];
+      o += c[i];
     }
-    pl.n_groups = ng;
+    if (tid == 31) pl.n_groups = ng;
   }
   __syncthreads();
   for (int p = tid; p < P; p += blockDim.x) {
@@ -1124,9 +1148,13 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
           if (jr.row0 + 32 * eq < a.I) {  // warp-uniform
             const int S_dn = (a.I / 32 + kKB - 1) / kKB, kb_dn = jr.row0 / 32 + eq;
             uint8_t *tg = a.terms_dn + (size_t)jr.group * terms_bytes<NMAX>(S_dn);
+            if (jr.cnt == 1) {  // one token in the group (batch 1 and most small batches): split it alone
+              split_terms_n<NMAX, MX, 1>(hv, 0, 1, kb_dn, S_dn, tg);
+            } else {
 #pragma unroll
-            for (int t0 = 0; t0 < kTokPad; t0 += NT)
-              if (t0 < jr.cnt) split_terms_n<NMAX, MX, NT>(hv + t0, t0, jr.cnt, kb_dn, S_dn, tg);
+              for (int t0 = 0; t0 < kTokPad; t0 += NT)
+                if (t0 < jr.cnt) split_terms_n<NMAX, MX, NT>(hv + t0, t0, jr.cnt, kb_dn, S_dn, tg);
+            }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&u_empty[buf]);
@@ -1149,12 +1177,21 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
           const int n = jr.row0 + mrow;
           if (n < a.H)
             for (int t = 0; t < a.Tm; t++) {
-              float acc = 0.f;
-              for (int jj = 0; jj < a.k; jj++) {
-                const int p = t * a.k + jj, ee = pl->ids[p];
-                if (ee < 0 || ee >= a.E) continue;
-                acc = fmaf(__ldg(a.wts + p), __ldcg(a.yws + (size_t)p * a.H + n), acc);
+              // every load of the token's pairs first (their latencies overlap), then the sum in j order
+              float yv[kMaxTopK], wv[kMaxTopK];
+              bool use[kMaxTopK];
+#pragma unroll
+              for (int jj = 0; jj < kMaxTopK; jj++) {
+                const int p = t * a.k + jj;
+                const int ee = jj < a.k ? pl->ids[p] : -1;
+                use[jj] = ee >= 0 && ee < a.E;
+                yv[jj] = use[jj] ? __ldcg(a.yws + (size_t)p * a.H + n) : 0.f;
+                wv[jj] = use[jj] ? __ldg(a.wts + p) : 0.f;
               }
+              float acc = 0.f;
+#pragma unroll
+              for (int jj = 0; jj < kMaxTopK; jj++)
+                if (use[jj]) acc = fmaf(wv[jj], yv[jj], acc);
               a.out[(size_t)t * a.H + n] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
             }
         }
