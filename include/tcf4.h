@@ -138,14 +138,14 @@ TCF4_API tcf4_status trellis_gemv_e5m3(tcf4_matrix w, const uint16_t *x, int32_t
  * For callers that cannot hand over device scratch memory: a host program that holds only the
  * device pointers it was given and has no device allocator of its own, or a serving loop that must
  * not allocate while it runs because its memory was reserved up front.
- * The scratch is one 1 MiB array per device, inside this library. Every call looks up that array's
+ * The scratch is one 2 MiB array per device, inside this library. Every call looks up that array's
  * address on the current device through the CUDA runtime (nothing is cached, so the address stays
  * right after a cudaDeviceReset). The first lookup on a device may load the library's module there,
  * so make the first call on each device before beginning any stream capture. All calls on a device
  * share the array and leave in it whatever they last wrote; nothing in it has to start at zero, as
  * each call writes the scratch it reads. Calls that overlap in time on one device (other streams or
  * host threads) race on the array: the caller must serialize them.
- * Returns TCF4_ERR_WORKSPACE when the call would need more than 1 MiB of scratch (not reached
+ * Returns TCF4_ERR_WORKSPACE when the call would need more than 2 MiB of scratch (not reached
  * within the limits of trellis_gemv), TCF4_ERR_CUDA when the address lookup fails. */
 TCF4_API tcf4_status trellis_gemv_noalloc(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream);
 

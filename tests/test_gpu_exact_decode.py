@@ -11,7 +11,7 @@ decoder bullet; HEPH's grid-aligned scales), not in a separate decoder.
 Instances covered (each is its own template instance of the product kernel):
   * up to five tokens per call: the 32-row B operand with two MMA issuers and the register split;
   * 6-16 tokens: the 96-row B operand, 16-block stages;
-  * 32 tokens: two passes of 16;
+  * 17-32 tokens: the 192-row B operand with one accumulator;
   * each of the above for 32-weight segments and for one segment per row (state carried across
     blocks and stages);
   * the resident-MXFP4 source mode (products from the expanded tensor);

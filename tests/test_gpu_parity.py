@@ -135,8 +135,8 @@ def test_gemv_2048_square_batch1(seg):
 def test_gemv_full_moe_layer_sampled(T):
     # Every expert matrix of the 32-expert hidden-2880 layer stacked (gate_up 184320 x 2880, down
     # 92160 x 2880): the shapes and launch configuration the bench times at T = 1 (register-split
-    # instance), and T = 32 (the largest batch, two passes of the 16-token instance). 64 sampled
-    # rows per matrix against the oracle, plus every output finite.
+    # instance), and T = 32 (the largest batch, one pass of the 192-row B operand). 64 sampled rows
+    # per matrix against the oracle, plus every output finite.
     E, H, I = 32, 2880, 2880
     layer = synth.moe_layer(E, H, I, seed=synth.SEED_BASE + 1)
     r = np.random.default_rng(6 + T)

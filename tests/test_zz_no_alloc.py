@@ -18,7 +18,7 @@ from gpu_common import assert_products_close, bf16_to_f64, xnorms
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("rows,cols,T", [(1000, 2880, 1), (300, 7168, 5), (129, 1024, 16)])
+@pytest.mark.parametrize("rows,cols,T", [(1000, 2880, 1), (300, 7168, 5), (129, 1024, 16), (130, 16384, 32)])
 def test_noalloc_matches_workspace_entry_point(rows, cols, T):
     st = synth.stream(rows, cols, seed=7000 + T)
     sc = synth.scales(rows, cols, seed=7000 + T)

@@ -58,11 +58,13 @@ constexpr int kRsLaunchRegs = 80, kRsDecRegs = 96, kRsOtherRegs = 48;
 
 template <int NMAX>
 struct Cfg {
-  static_assert(NMAX <= 128, "B scale factors of a 4-block group fit one 4-column TMEM slot");
+  static_assert(NMAX <= 256, "B rows of one MMA");
   static constexpr int kTok = NMAX / kTerms;                   // tokens per group
   static constexpr int kSlots = (NMAX + kTerms - 1) / kTerms;  // token slots the split writes
   static constexpr int kSplitNT = kTok <= 6 ? kTok : 4;        // slots split side by side
   static constexpr int kC = (NMAX + 31) / 32;                  // B scale columns per 4-block group
+  static constexpr int kNTile = (kC + 3) / 4;                  // 32 x 16-byte B scale tiles per group
+  static constexpr uint32_t kSfbGCols = 4u * kNTile;           // TMEM columns of a group's B scales
   static constexpr int kKB = NMAX <= 32 ? 32 : 16;             // 32-blocks per row per stage
   // Warps: kDecWarps decode warps (four per group of 8 blocks of a stage), then the word loader, two
   // MMA issuer slots, the B loader and four epilogue warps.
@@ -72,16 +74,17 @@ struct Cfg {
   static constexpr int kNBT = 8;                               // blocks per decode thread per stage
   static constexpr int kNCh = kNBT / 8;                        // decoded in chunks of 8 blocks
   static constexpr int kNG = kNBT / 4;                         // scale groups per decode thread
-  static constexpr int kNW = kKB == 32 ? 3 : 6;                // word stages in flight
-  static constexpr int kNA = NMAX <= 32 ? 2 : 3;               // A / scale-factor stages (TMEM)
-  static constexpr int kNB = 4;                                // B stages (shared memory)
+  static constexpr int kNW = kKB == 32 ? 3 : (NMAX > 96 ? 5 : 6);  // word stages in flight
+  static constexpr int kNA = NMAX <= 32 ? 2 : (NMAX > 96 ? 2 : 3);  // A / scale-factor stages (TMEM)
+  static constexpr int kNB = NMAX > 96 ? 2 : 4;                // B stages (shared memory)
   static constexpr int kBoxCols = kKB / 16;                    // 128-byte TMA boxes per 64 rows
   static constexpr uint32_t kWStage = 1024u * kKB;             // 128 rows x 8 KB bytes of words
   static constexpr uint32_t kSbo = 128u * kKB;                 // B: 8 rows x KB chunks x 16 bytes
   static constexpr uint32_t kBStage = NMAX * 16u * kKB;        // NMAX rows x 32 KB E2M1
-  // B scale factors of a stage: per 4-block group a 32 x 16-byte tile, row r = the group's UE8M0
-  // words of B rows r, 32 + r, 64 + r (and one spare word), the source of one tcgen05.cp
-  static constexpr uint32_t kSfbStage = (kKB / 4) * 512u;
+  // B scale factors of a stage: per 4-block group kNTile tiles of 32 x 16 bytes, row r of tile i =
+  // the group's UE8M0 words of B rows 128 i + r, 128 i + 32 + r, ... (spare words past NMAX), the
+  // sources of kNTile tcgen05.cp
+  static constexpr uint32_t kSfbStage = (kKB / 4) * 512u * kNTile;
   static constexpr uint32_t kBSlot = kBStage + kSfbStage;       // one stage of terms + scales
   // Weights' scales as scale tiles (trellis_gemv_tiled): per 4-block group a 512-byte tile, row r
   // = the group's UE8M0 words of tile rows r, 32 + r, 64 + r, 96 + r; KB/4 tiles per stage.
@@ -90,11 +93,14 @@ struct Cfg {
   // two accumulator pairs (one issuing thread sustains about one MMA per 60 cycles; two of them in
   // different warps run concurrently).
   static constexpr int kNI = NMAX <= 32 ? 2 : 1;
+  // accumulators per issuer: two (a job's epilogue overlaps the next job's MMAs) where TMEM has room
+  static constexpr int kNAcc = NMAX > 96 ? 1 : 2;
   static constexpr uint32_t kACols = 4u * kKB;                 // TMEM columns of a stage's A
-  static constexpr uint32_t kACol = 2u * kNI * NMAX;           // TMEM: accumulators first, then
+  static constexpr uint32_t kSfbCols = (kKB / 4) * kSfbGCols;  // TMEM columns of a stage's B scales
+  static constexpr uint32_t kACol = kNAcc * kNI * NMAX;        // TMEM: accumulators first, then
   static constexpr uint32_t kSfaCol = kACol + kACols * kNA;    // A stages, A scales (KB columns per
-  static constexpr uint32_t kSfbCol = kSfaCol + kKB * kNA;     // stage), B scales (KB per stage)
-  static constexpr uint32_t kUsed = kSfbCol + kKB * kNA;
+  static constexpr uint32_t kSfbCol = kSfaCol + kKB * kNA;     // stage), B scales (kSfbCols per stage)
+  static constexpr uint32_t kUsed = kSfbCol + kSfbCols * kNA;
   static constexpr uint32_t kTmemCols = kUsed <= 128 ? 128 : (kUsed <= 256 ? 256 : 512);
   static_assert(kUsed <= 512, "TMEM budget");
   // Resident-MXFP4 source (the expanded tensor): the A operand is a shared-memory tile of nibbles
@@ -102,9 +108,9 @@ struct Cfg {
   // the scale factors.
   static constexpr int kNWX = NMAX <= 32 ? 2 : 3;              // A-tile stages in flight
   static constexpr uint32_t kWStageX = 2048u * kKB;
-  static constexpr uint32_t kSfaColX = 2u * kNI * NMAX;
+  static constexpr uint32_t kSfaColX = kNAcc * kNI * NMAX;
   static constexpr uint32_t kSfbColX = kSfaColX + kKB * kNA;
-  static constexpr uint32_t kUsedX = kSfbColX + kKB * kNA;
+  static constexpr uint32_t kUsedX = kSfbColX + kSfbCols * kNA;
   static constexpr uint32_t kTmemColsX = kUsedX <= 128 ? 128 : (kUsedX <= 256 ? 256 : 512);
   static_assert(kUsedX <= 512, "TMEM budget");
 };
@@ -280,7 +286,8 @@ __device__ __forceinline__ void split_terms_n(const float *v, int t0, int nvalid
       if (t0 + i < nvalid && n < NMAX) {
         if ((kp & 1) == 0)
           bst[chunk_off<NMAX>((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code[i] | (partner << 4));
-        if (lane == 0) sfs[(h * 32 + (n & 31)) * 16 + (n >> 5) * 4 + (c & 3)] = (uint8_t)(S[i] + 127);
+        if (lane == 0)
+          sfs[((h * C::kNTile + (n >> 7)) * 32 + (n & 31)) * 16 + ((n >> 5) & 3) * 4 + (c & 3)] = (uint8_t)(S[i] + 127);
       }
     }
   }
@@ -1076,10 +1083,11 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
     const int eq = warp & 3;
     auto epilogue = [&](int jl_e) {
       const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
-      const int buf = jl_e & 1;
+      const int buf = jl_e & 1;                   // the gate/up exchange buffer
+      const int abuf = jl_e % C::kNAcc;           // the accumulator
       // one warp polls; the others wait at a named barrier (no issue slots taken meanwhile)
       if (warp == C::kEpiWarp0) {
-        if (!mbar_wait_sleep(&acc_full[buf], (uint32_t)(jl_e >> 1) & 1u, tmo, kEpiSleepNs)) *abort_flag = 1;
+        if (!mbar_wait_sleep(&acc_full[abuf], (uint32_t)(jl_e / C::kNAcc) & 1u, tmo, kEpiSleepNs)) *abort_flag = 1;
       }
       named_bar(1, 128);
       if (*abort_flag) return;
@@ -1094,7 +1102,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
 #pragma unroll
         for (int c0 = 0; c0 < C::kTok * kTerms; c0 += 16) {
           uint32_t r[16];
-          tmem_ld_x16(tbase + ((uint32_t)(32 * eq) << 16) + (uint32_t)((buf * C::kNI + ia) * NMAX + c0), r);
+          tmem_ld_x16(tbase + ((uint32_t)(32 * eq) << 16) + (uint32_t)((abuf * C::kNI + ia) * NMAX + c0), r);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; i++)
@@ -1103,7 +1111,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (lane == 0) mbar_arrive(&acc_empty[abuf]);
       const int mrow = 32 * eq + lane;
       if (MODE == kModeGemv) {
         const int row = tile_row(jr, mrow);
@@ -1216,13 +1224,13 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       const uint32_t ph = (uint32_t)(q / kNA) & 1u;
       const int bb = q % C::kNB;
       ok = mbar_wait_sleep(&b_full[bb], (uint32_t)(q / C::kNB) & 1u, tmo, kMmaSleepNs);
-      if (ok && s == 0 && jl >= 2)
-        ok = mbar_wait_sleep(&acc_empty[jl & 1], (uint32_t)((jl >> 1) - 1) & 1u, tmo, kMmaSleepNs);
+      if (ok && s == 0 && jl >= C::kNAcc)  // the job's accumulator was read out by its last user
+        ok = mbar_wait_sleep(&acc_empty[jl % C::kNAcc], (uint32_t)(jl / C::kNAcc - 1) & 1u, tmo, kMmaSleepNs);
       const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
       const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
       const uint64_t bd = smem_desc(b0 + (uint32_t)bb * geo.bslot, 128u, C::kSbo);
       const uint32_t bsf0 = b0 + (uint32_t)bb * geo.bslot + C::kBStage;  // the stage's B scale tiles
-      const uint32_t sfa = tbase + kSfaCol + kKB * (uint32_t)b, sfb = tbase + kSfbCol + kKB * (uint32_t)b;
+      const uint32_t sfa = tbase + kSfaCol + kKB * (uint32_t)b, sfb = tbase + kSfbCol + C::kSfbCols * (uint32_t)b;
       const int wsx = q % kNW;  // MX: the stage's word slot
       const uint64_t ad0 = MX ? desc_sw128(smem_u32(smem + geo.off_W) + (uint32_t)wsx * kWStage) : 0ull;
 #pragma unroll
@@ -1234,13 +1242,17 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
         if (!ok) break;
         tc_fence_after();
         const int jfirst = C::kNI == 2 ? hh * kKB / 4 : 0;  // this issuer's first MMA of a job
-        const uint32_t d_t = tbase + (uint32_t)(((jl & 1) * C::kNI + (C::kNI == 2 ? hh : 0)) * NMAX);
+        const uint32_t d_t = tbase + (uint32_t)(((jl % C::kNAcc) * C::kNI + (C::kNI == 2 ? hh : 0)) * NMAX);
         if (leader) {
           // the B scale factors of this half's groups (4 blocks each), ahead of the MMAs that read
           // them: tcgen05 operations of one thread run in issue order
 #pragma unroll
           for (int g = hh * kKB / 8; g < (hh + 1) * kKB / 8; g++)
-            if (2 * g < nmma) tmem_cp_sf(sfb + 4u * (uint32_t)g, smem_desc(bsf0 + 512u * (uint32_t)g, 128u, 128u));
+#pragma unroll
+            for (int ti = 0; ti < C::kNTile; ti++)
+              if (2 * g < nmma)
+                tmem_cp_sf(sfb + C::kSfbGCols * (uint32_t)g + 4u * ti,
+                           smem_desc(bsf0 + 512u * (uint32_t)(C::kNTile * g + ti), 128u, 128u));
           if constexpr (TILED) {  // the weights' scale factors: tile row r to lanes r, 32 + r, 64 + r, 96 + r
             const uint32_t asf0 = b0 + (uint32_t)bb * geo.bslot + C::kBSlot;  // the weights' scale tiles
 #pragma unroll
@@ -1255,18 +1267,18 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
               if constexpr (MX)  // A: column box j / 4 (16 KB apart), 32 bytes per MMA inside it
                 mma_mxf4_ss(d_t, ad0 + (uint64_t)((j >> 2) * 1024 + 2 * (j & 3)), bd + 16u * (uint64_t)j,
                             (j & 1) ? idesc2 : idesc0, (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30),
-                            (sfb + 4u * (uint32_t)(j >> 1)) | (sf << 30), !(s == 0 && j == jfirst));
+                            (sfb + C::kSfbGCols * (uint32_t)(j >> 1)) | (sf << 30), !(s == 0 && j == jfirst));
               else
                 mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
-                            (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30), (sfb + 4u * (uint32_t)(j >> 1)) | (sf << 30),
-                            !(s == 0 && j == jfirst));
+                            (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30),
+                            (sfb + C::kSfbGCols * (uint32_t)(j >> 1)) | (sf << 30), !(s == 0 && j == jfirst));
             }
           }
           tc_commit(&a_empty[2 * b + hh]);
           if (MX) tc_commit(&w_empty[2 * wsx + hh]);
           if (hh == h_hi - 1) {
             tc_commit(&b_empty[bb]);
-            if (s == S - 1) tc_commit(&acc_full[jl & 1]);
+            if (s == S - 1) tc_commit(&acc_full[jl % C::kNAcc]);
           }
         }
       }
@@ -1333,15 +1345,27 @@ static bool make_word_map(CUtensorMap *map, const void *stream, int rows, int nb
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// GEMV tokens per pass; B width (template NMAX) for a pass or group of T tokens.
-constexpr int kGemvTok = Cfg<96>::kTok;
-static int nmax_for(int tokens_per_group) { return tokens_per_group <= Cfg<32>::kTok ? 32 : 96; }
+// GEMV tokens per pass; B width (template NMAX) for a pass or group of T tokens: up to 5 tokens on
+// the 32-row B operand, up to 16 on the 96-row one, up to 32 on the 192-row one.
+constexpr int kGemvTok = Cfg<192>::kTok;
+static int nmax_for(int tokens_per_group) {
+  return tokens_per_group <= Cfg<32>::kTok ? 32 : (tokens_per_group <= Cfg<96>::kTok ? 96 : 192);
+}
+// The grouped MoE keeps groups of at most 16 tokens: with routed tokens spread over the experts a
+// wider B operand would mostly multiply empty slots.
+static int moe_nmax_for(int T) { return nmax_for(T) == 32 ? 32 : 96; }
+template <int NMAX>
+static uint32_t geom_smem(int mode, bool mx, bool tiled) { return mma_geom<NMAX>(mode, mx, tiled).smem; }
+static uint32_t geom_smem_for(int NMAX, int mode, bool mx, bool tiled) {
+  return NMAX == 32 ? geom_smem<32>(mode, mx, tiled)
+                    : (NMAX == 96 ? geom_smem<96>(mode, mx, tiled) : geom_smem<192>(mode, mx, tiled));
+}
 
 static bool mma_fits(int NMAX, int mode, bool mx = false, bool tiled = false) {
   int dev = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
-  const uint32_t need = NMAX == 32 ? mma_geom<32>(mode, mx, tiled).smem : mma_geom<96>(mode, mx, tiled).smem;
+  const uint32_t need = geom_smem_for(NMAX, mode, mx, tiled);
   return need <= (uint32_t)optin;
 }
 
@@ -1351,7 +1375,8 @@ static bool k_ok(int nbr) { return nbr >= 2 && nbr % 2 == 0; }
 
 static size_t terms_for(int nbr, int NMAX) {
   return NMAX == 32 ? terms_bytes<32>((nbr + Cfg<32>::kKB - 1) / Cfg<32>::kKB)
-                    : terms_bytes<96>((nbr + Cfg<96>::kKB - 1) / Cfg<96>::kKB);
+                    : (NMAX == 96 ? terms_bytes<96>((nbr + Cfg<96>::kKB - 1) / Cfg<96>::kKB)
+                                  : terms_bytes<192>((nbr + Cfg<192>::kKB - 1) / Cfg<192>::kKB));
 }
 
 // The scale-factor threads read a row's scale bytes in pairs (16-bit loads): the scales must be
@@ -1498,14 +1523,14 @@ static cudaError_t launch_gemv_t(const MatView &w, const uint16_t *x, int T, uin
                                  const uint8_t *tiles = nullptr) {
   CUtensorMap map;
   if (!make_word_map(&map, w.stream, w.rows, w.nbr, MX ? 16 : 8)) return cudaErrorInvalidValue;
-  const bool n32 = nmax_for(T < kGemvTok ? T : kGemvTok) == 32;
+  const int nm = nmax_for(T < kGemvTok ? T : kGemvTok);
   for (int t0 = 0; t0 < T; t0 += kGemvTok) {
     const int n = T - t0 < kGemvTok ? T - t0 : kGemvTok;
     const uint16_t *xp = x + (size_t)t0 * w.nbr * 32;
     uint16_t *yp = y + (size_t)t0 * w.rows;
-    cudaError_t e =
-        n32 ? launch_gemv_pass<32, MX>(w, map, xp, n, yp, ws, s, tiles)
-            : launch_gemv_pass<96, MX>(w, map, xp, n, yp, ws, s, tiles);
+    cudaError_t e = nm == 32   ? launch_gemv_pass<32, MX>(w, map, xp, n, yp, ws, s, tiles)
+                    : nm == 96 ? launch_gemv_pass<96, MX>(w, map, xp, n, yp, ws, s, tiles)
+                               : launch_gemv_pass<192, MX>(w, map, xp, n, yp, ws, s, tiles);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -1534,7 +1559,7 @@ bool moe_mma_supported(const tcf4_moe &m, int gu_seg, int dn_seg, int T) {
     if (((reinterpret_cast<uintptr_t>(m.gate_up[e].stream) | reinterpret_cast<uintptr_t>(m.down[e].stream)) & 15u) ||
         ((reinterpret_cast<uintptr_t>(m.gate_up[e].scales) | reinterpret_cast<uintptr_t>(m.down[e].scales)) & 1u))
       return false;
-  const int NMAX = nmax_for(T);
+  const int NMAX = moe_nmax_for(T);
   return mma_fits(NMAX, kModeGateUp) && mma_fits(NMAX, kModeDown);
 }
 // The same layer as resident MXFP4 (stream fields point at the nibble matrices).
@@ -1544,14 +1569,14 @@ bool moe_mx_supported(const tcf4_moe &m, int T) {
     if (((reinterpret_cast<uintptr_t>(m.gate_up[e].stream) | reinterpret_cast<uintptr_t>(m.down[e].stream)) & 15u) ||
         ((reinterpret_cast<uintptr_t>(m.gate_up[e].scales) | reinterpret_cast<uintptr_t>(m.down[e].scales)) & 1u))
       return false;
-  const int NMAX = nmax_for(T);
+  const int NMAX = moe_nmax_for(T);
   return mma_fits(NMAX, kModeGateUp, true) && mma_fits(NMAX, kModeDown, true);
 }
 
 MoeMmaWorkspace moe_mma_workspace_layout(const tcf4_moe &m, int T, int k) {
   auto a256 = [](size_t v) { return (v + 255) & ~(size_t)255; };
-  const int P = T * k, NMAX = nmax_for(T);
-  const int G = moe_groups_max(m.E, P, NMAX == 32 ? Cfg<32>::kTok : Cfg<96>::kTok);
+  const int P = T * k, NMAX = moe_nmax_for(T);
+  const int G = moe_groups_max(m.E, P, NMAX == 32 ? Cfg<32>::kTok : (NMAX == 96 ? Cfg<96>::kTok : Cfg<192>::kTok));
   MoeMmaWorkspace L;
   size_t off = 0;
   L.counters = off; off = a256(off + sizeof(int) * 4 * ((m.H + 127) / 128));
@@ -1636,7 +1661,7 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
 template <bool MX>
 static cudaError_t launch_moe_t(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts,
                                 int k, uint16_t *out, void *ws, cudaStream_t s) {
-  const bool n32 = nmax_for(T) == 32;
+  const bool n32 = moe_nmax_for(T) == 32;
   if (m.E <= 32)
     return n32 ? launch_moe_mma_t<32, 32, MX>(m, x, T, ids, wts, k, out, ws, s)
                : launch_moe_mma_t<32, 96, MX>(m, x, T, ids, wts, k, out, ws, s);

@@ -12,7 +12,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = size_t(1) << 20;  // 1 MiB: the largest GEMV workspace for cols <= 16384
+constexpr size_t kScratchBytes = size_t(2) << 20;  // 2 MiB: the largest GEMV workspace for cols <= 16384 is 1.63 MiB
 
 static __device__ __align__(256) unsigned char g_gemv_scratch[kScratchBytes];
 
