@@ -10,7 +10,8 @@ decoder bullet; HEPH's grid-aligned scales), not in a separate decoder.
 
 Instances covered (each is its own template instance of the product kernel):
   * up to five tokens per call: the 32-row B operand with two MMA issuers and the register split;
-  * 6-16 tokens: the 96-row B operand, 16-block stages;
+  * 6-10 tokens: the 64-row B operand, 32-block stages, one issuer;
+  * 11-16 tokens: the 96-row B operand, 16-block stages;
   * 17-32 tokens: the 192-row B operand with one accumulator;
   * each of the above for 32-weight segments and for one segment per row (state carried across
     blocks and stages);
@@ -57,7 +58,7 @@ def _assert_columns(got, w, what):
 
 
 @pytest.mark.parametrize("seg", [32, COLS])
-@pytest.mark.parametrize("T", [5, 16, 32])
+@pytest.mark.parametrize("T", [5, 8, 16, 32])
 def test_fused_gemv_returns_every_decoded_column(T, seg):
     st, sc, W = upload_matrix(ROWS, COLS, seed=5100 + T + seg, seg_len=seg)
     assert tc.gemv_workspace_bytes(W, T) > 0  # the tensor-core path

@@ -70,7 +70,7 @@ def test_gemv_tiled_full_size_sampled():
 
 
 @pytest.mark.parametrize("seg", [32, 2880])
-@pytest.mark.parametrize("T", [5, 16, 32])
+@pytest.mark.parametrize("T", [5, 8, 16, 32])
 def test_gemv_tiled_returns_every_decoded_column(T, seg):
     rows, cols = 300, 2880
     st, sc, W = upload_matrix(rows, cols, seed=8200 + T + seg, seg_len=seg)

@@ -65,7 +65,7 @@ struct Cfg {
   static constexpr int kC = (NMAX + 31) / 32;                  // B scale columns per 4-block group
   static constexpr int kNTile = (kC + 3) / 4;                  // 32 x 16-byte B scale tiles per group
   static constexpr uint32_t kSfbGCols = 4u * kNTile;           // TMEM columns of a group's B scales
-  static constexpr int kKB = NMAX <= 32 ? 32 : 16;             // 32-blocks per row per stage
+  static constexpr int kKB = NMAX <= 64 ? 32 : 16;             // 32-blocks per row per stage
   // Warps: kDecWarps decode warps (four per group of 8 blocks of a stage), then the word loader, two
   // MMA issuer slots, the B loader and four epilogue warps.
   static constexpr int kDecWarps = kKB / 2;
@@ -75,8 +75,8 @@ struct Cfg {
   static constexpr int kNCh = kNBT / 8;                        // decoded in chunks of 8 blocks
   static constexpr int kNG = kNBT / 4;                         // scale groups per decode thread
   static constexpr int kNW = kKB == 32 ? 3 : (NMAX > 96 ? 5 : 6);  // word stages in flight
-  static constexpr int kNA = NMAX <= 32 ? 2 : (NMAX > 96 ? 2 : 3);  // A / scale-factor stages (TMEM)
-  static constexpr int kNB = NMAX > 96 ? 2 : 4;                // B stages (shared memory)
+  static constexpr int kNA = NMAX <= 64 ? 2 : (NMAX > 96 ? 2 : 3);  // A / scale-factor stages (TMEM)
+  static constexpr int kNB = NMAX > 96 ? 2 : (NMAX > 32 && NMAX <= 64 ? 3 : 4);  // B stages (shared memory)
   static constexpr int kBoxCols = kKB / 16;                    // 128-byte TMA boxes per 64 rows
   static constexpr uint32_t kWStage = 1024u * kKB;             // 128 rows x 8 KB bytes of words
   static constexpr uint32_t kSbo = 128u * kKB;                 // B: 8 rows x KB chunks x 16 bytes
@@ -1348,17 +1348,29 @@ static bool make_word_map(CUtensorMap *map, const void *stream, int rows, int nb
 // GEMV tokens per pass; B width (template NMAX) for a pass or group of T tokens: up to 5 tokens on
 // the 32-row B operand, up to 16 on the 96-row one, up to 32 on the 192-row one.
 constexpr int kGemvTok = Cfg<192>::kTok;
+// (6 to 10 tokens on the 64-row one, which keeps the 32-block stages and their 16 decode warps).
 static int nmax_for(int tokens_per_group) {
-  return tokens_per_group <= Cfg<32>::kTok ? 32 : (tokens_per_group <= Cfg<96>::kTok ? 96 : 192);
+  return tokens_per_group <= Cfg<32>::kTok   ? 32
+         : tokens_per_group <= Cfg<64>::kTok ? 64
+         : tokens_per_group <= Cfg<96>::kTok ? 96
+                                             : 192;
+}
+// The resident-MXFP4 source has no 64-row configuration (its 32-block A tiles leave no room).
+static int mx_nmax_for(int tokens_per_group) {
+  const int n = nmax_for(tokens_per_group);
+  return n == 64 ? 96 : n;
 }
 // The grouped MoE keeps groups of at most 16 tokens: with routed tokens spread over the experts a
 // wider B operand would mostly multiply empty slots.
 static int moe_nmax_for(int T) { return nmax_for(T) == 32 ? 32 : 96; }
+static uint32_t geom_smem_for(int NMAX, int mode, bool mx, bool tiled);
 template <int NMAX>
 static uint32_t geom_smem(int mode, bool mx, bool tiled) { return mma_geom<NMAX>(mode, mx, tiled).smem; }
 static uint32_t geom_smem_for(int NMAX, int mode, bool mx, bool tiled) {
-  return NMAX == 32 ? geom_smem<32>(mode, mx, tiled)
-                    : (NMAX == 96 ? geom_smem<96>(mode, mx, tiled) : geom_smem<192>(mode, mx, tiled));
+  return NMAX == 32   ? geom_smem<32>(mode, mx, tiled)
+         : NMAX == 64 ? geom_smem<64>(mode, mx, tiled)
+         : NMAX == 96 ? geom_smem<96>(mode, mx, tiled)
+                      : geom_smem<192>(mode, mx, tiled);
 }
 
 static bool mma_fits(int NMAX, int mode, bool mx = false, bool tiled = false) {
@@ -1374,9 +1386,10 @@ static bool mma_fits(int NMAX, int mode, bool mx = false, bool tiled = false) {
 static bool k_ok(int nbr) { return nbr >= 2 && nbr % 2 == 0; }
 
 static size_t terms_for(int nbr, int NMAX) {
-  return NMAX == 32 ? terms_bytes<32>((nbr + Cfg<32>::kKB - 1) / Cfg<32>::kKB)
-                    : (NMAX == 96 ? terms_bytes<96>((nbr + Cfg<96>::kKB - 1) / Cfg<96>::kKB)
-                                  : terms_bytes<192>((nbr + Cfg<192>::kKB - 1) / Cfg<192>::kKB));
+  return NMAX == 32   ? terms_bytes<32>((nbr + Cfg<32>::kKB - 1) / Cfg<32>::kKB)
+         : NMAX == 64 ? terms_bytes<64>((nbr + Cfg<64>::kKB - 1) / Cfg<64>::kKB)
+         : NMAX == 96 ? terms_bytes<96>((nbr + Cfg<96>::kKB - 1) / Cfg<96>::kKB)
+                      : terms_bytes<192>((nbr + Cfg<192>::kKB - 1) / Cfg<192>::kKB);
 }
 
 // The scale-factor threads read a row's scale bytes in pairs (16-bit loads): the scales must be
@@ -1389,7 +1402,7 @@ bool gemv_mma_supported(const MatView &w, int T) {
 bool mx_gemv_supported(const MatView &w, int T) {
   return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.stream) & 15u) == 0 &&
          (reinterpret_cast<uintptr_t>(w.scales) & 1u) == 0 && tensor_map_encoder() != nullptr &&
-         mma_fits(nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv, true);
+         mma_fits(mx_nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv, true);
 }
 
 // The tiled GEMV: the tensor-core path with the scale-tile ring (the tiles' pointer 16-byte aligned).
@@ -1435,6 +1448,7 @@ cudaError_t launch_scale_tiles(const MatView &w, uint8_t *tiles, cudaStream_t s)
 
 // Tokens beyond kGemvTok run as further passes, each with its own split of x.
 size_t gemv_mma_workspace(const MatView &w, int T) { return terms_for(w.nbr, nmax_for(T < kGemvTok ? T : kGemvTok)); }
+size_t mx_gemv_workspace(const MatView &w, int T) { return terms_for(w.nbr, mx_nmax_for(T < kGemvTok ? T : kGemvTok)); }
 
 static int sm_count_impl() {
   int dev = 0, nsm = 148;
@@ -1523,14 +1537,22 @@ static cudaError_t launch_gemv_t(const MatView &w, const uint16_t *x, int T, uin
                                  const uint8_t *tiles = nullptr) {
   CUtensorMap map;
   if (!make_word_map(&map, w.stream, w.rows, w.nbr, MX ? 16 : 8)) return cudaErrorInvalidValue;
-  const int nm = nmax_for(T < kGemvTok ? T : kGemvTok);
+  const int nm = MX ? mx_nmax_for(T < kGemvTok ? T : kGemvTok) : nmax_for(T < kGemvTok ? T : kGemvTok);
   for (int t0 = 0; t0 < T; t0 += kGemvTok) {
     const int n = T - t0 < kGemvTok ? T - t0 : kGemvTok;
     const uint16_t *xp = x + (size_t)t0 * w.nbr * 32;
     uint16_t *yp = y + (size_t)t0 * w.rows;
-    cudaError_t e = nm == 32   ? launch_gemv_pass<32, MX>(w, map, xp, n, yp, ws, s, tiles)
-                    : nm == 96 ? launch_gemv_pass<96, MX>(w, map, xp, n, yp, ws, s, tiles)
-                               : launch_gemv_pass<192, MX>(w, map, xp, n, yp, ws, s, tiles);
+    cudaError_t e;
+    if (nm == 32)
+      e = launch_gemv_pass<32, MX>(w, map, xp, n, yp, ws, s, tiles);
+    else if (nm == 96)
+      e = launch_gemv_pass<96, MX>(w, map, xp, n, yp, ws, s, tiles);
+    else if (nm == 192)
+      e = launch_gemv_pass<192, MX>(w, map, xp, n, yp, ws, s, tiles);
+    else if constexpr (!MX)
+      e = launch_gemv_pass<64, false>(w, map, xp, n, yp, ws, s, tiles);
+    else
+      e = cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

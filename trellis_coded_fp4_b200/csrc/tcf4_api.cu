@@ -269,7 +269,7 @@ tcf4_status trellis_grouped_moe(const tcf4_moe *m, const uint16_t *x, int32_t T,
 
 size_t mxfp4_gemv_workspace(tcf4_mxfp4 w, int32_t T) {
   if (check_mx(w) != TCF4_OK || T <= 0 || T > kMaxTokens || w.rows == 0 || w.cols == 0) return 0;
-  return gemv_mma_workspace(mx_view(w), T);
+  return mx_gemv_workspace(mx_view(w), T);
 }
 
 tcf4_status mxfp4_gemv(tcf4_mxfp4 w, const uint16_t *x, int32_t T, uint16_t *y, void *workspace, size_t ws_bytes,
@@ -284,7 +284,7 @@ tcf4_status mxfp4_gemv(tcf4_mxfp4 w, const uint16_t *x, int32_t T, uint16_t *y, 
   if (!aligned16(x) || !aligned16(y)) return TCF4_ERR_MISALIGNED;
   const MatView v = mx_view(w);
   if (!mx_gemv_supported(v, T)) return TCF4_ERR_UNSUPPORTED;
-  if (workspace == nullptr || ws_bytes < gemv_mma_workspace(v, T)) return TCF4_ERR_WORKSPACE;
+  if (workspace == nullptr || ws_bytes < mx_gemv_workspace(v, T)) return TCF4_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
   clear_pending_error();
   return from_cuda(launch_mx_gemv(v, x, T, y, workspace, static_cast<cudaStream_t>(stream)));

@@ -120,6 +120,7 @@ cudaError_t launch_encode(const double *target, const double *D, const uint8_t *
 // Resident MXFP4 consumers (the tensor-core kernel reading nibble tiles): the views' stream fields
 // point at the nibble matrices [rows][cols/2]. Workspaces are the same as the trellis paths'.
 bool mx_gemv_supported(const MatView &w, int T);
+size_t mx_gemv_workspace(const MatView &w, int T);
 cudaError_t launch_mx_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s);
 bool moe_mx_supported(const tcf4_moe &m, int T);
 cudaError_t launch_moe_mx(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts, int k,
