@@ -508,9 +508,11 @@ def row_e5m3(L, n, peak, seed):
     m5 = torch.randint(0, 8, L.G.scales.shape, dtype=torch.int32, device=d, generator=g5)
     sc5 = (((L.G.scales.to(torch.int32) - 112) << 3) | m5).to(torch.uint8)
     W5 = tc.TrellisMatrix(L.G.stream, sc5, L.G.rows, L.G.cols, L.G.seg_len)
-    us = time_calls(lambda i: tc.gemv_e5m3(W5, L.x[i % NVAR], out=L.yG), n)
+    ws5 = torch.empty(max(1, tc.gemv_e5m3_workspace_bytes(W5, 1)), dtype=torch.uint8, device=d)
+    us = time_calls(lambda i: tc.gemv_e5m3(W5, L.x[i % NVAR], out=L.yG, workspace=ws5), n)
     return {**rate(gemv_bytes(E * 2 * I, H, 1), us, peak), "decoded_weights_per_s": W5.rows * W5.cols / (us * 1e-6),
-            "calls": n, "note": "E5M3 block scales of the same binades, batch 1"}
+            "calls": n, "note": "E5M3 block scales of the same binades, batch 1; tensor cores, four block-scaled "
+                                "MMAs per K-step (one per power of two of the scale)"}
 
 
 # ----------------------------------------------------------------------------- end to end

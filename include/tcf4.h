@@ -129,9 +129,15 @@ TCF4_API tcf4_status trellis_gemv_tiled(tcf4_matrix w, const uint8_t *tiles, con
  * on the format; no encoding given). w.scales holds one E5M3 byte per 32-weight block, read as: no
  * sign bit, exponent bits 7..3 with bias 15, mantissa bits 2..0, exponent 0 subnormal (2^-14 m/8),
  * exponent 31 NaN. Otherwise as trellis_gemv: y[t][n] = bf16( sum_k w[n][k] * x[t][k] ), same
- * shapes, alignment and limits, same accuracy bound. CUDA cores only (a block-scaled MMA takes
- * power-of-two scales), so no workspace; each block's partial sum is scaled once in fp32. */
-TCF4_API tcf4_status trellis_gemv_e5m3(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream);
+ * shapes, alignment, limits and accuracy bound, and the same two paths. On the tensor cores (cols a
+ * multiple of 64) each E5M3 scale is written as the sum of at most four powers of two (the implicit
+ * bit and each set significand bit), so a block's product is four block-scaled MMAs of the same
+ * decoded weights, one per power; an absent power adds the block's product times 2^-127. That path
+ * needs trellis_gemv_e5m3_workspace(w, T) bytes of workspace (256-byte aligned, caller-owned);
+ * otherwise the CUDA-core kernel scales each block's partial sum once and needs none (0 bytes). */
+TCF4_API size_t trellis_gemv_e5m3_workspace(tcf4_matrix w, int32_t T);
+TCF4_API tcf4_status trellis_gemv_e5m3(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *workspace,
+                                       size_t ws_bytes, void *stream);
 
 /* trellis_gemv without a caller-provided workspace (the source pages have no counterpart; this is
  * a convenience of this library). Same arguments, result and accuracy as trellis_gemv.

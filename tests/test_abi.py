@@ -119,7 +119,11 @@ def test_repack_argument_checks(lib):
 def test_e5m3_gemv_argument_checks(lib):
     s0 = ctypes.c_void_p(0)
     ok_x, ok_y = ctypes.c_void_p(4096), ctypes.c_void_p(8192)
-    g = lib.trellis_gemv_e5m3
+    ws0 = ctypes.c_void_p(0)
+
+    def g(w, x, T, y, s):  # these checks never reach a launch, so no workspace is involved
+        return lib.trellis_gemv_e5m3(w, x, T, y, ws0, 0, s)
+
     assert g(_mat(cols=48), ok_x, 1, ok_y, s0) == 1
     assert g(_mat(seg=96), ok_x, 1, ok_y, s0) == 1
     assert g(_mat(stream=8), ok_x, 1, ok_y, s0) == 2
@@ -129,6 +133,26 @@ def test_e5m3_gemv_argument_checks(lib):
     assert g(_mat(), ok_x, -1, ok_y, s0) == 1
     assert g(_mat(), ctypes.c_void_p(0), 1, ok_y, s0) == 1
     assert g(_mat(), ok_x, 0, ok_y, s0) == 0 and g(_mat(rows=0), ok_x, 1, ok_y, s0) == 0
+    assert lib.trellis_gemv_e5m3_workspace(_mat(cols=48), 1) == 0
+
+
+def test_e5m3_scale_sets_sum_to_the_e5m3_value():
+    # The tensor-core path writes each E5M3 scale as four powers of two (UE8M0 bytes, byte 0 read as
+    # 2^-127 and standing for an absent power): restated here, their sum must be the oracle's E5M3
+    # value for every byte, up to the 2^-127 stand-ins; byte 0xF8.. (NaN) gives a NaN byte.
+    import oracle
+    for b in range(256):
+        e, m = b >> 3, b & 7
+        nz, nan, ee = int(e >= 1), int(e == 31), max(e, 1)
+        st = [((e + 112) if nz else 0) | (0xFF if nan else 0),
+              (ee + 111) if (m >> 2) & 1 else 0, (ee + 110) if (m >> 1) & 1 else 0, (ee + 109) if m & 1 else 0]
+        if nan:
+            assert st[0] == 0xFF
+            continue
+        total = sum(2.0 ** (v - 127) for v in st if v != 0)
+        tiny = sum(1 for v in st if v == 0) * 2.0 ** -127
+        assert total == oracle.e5m3_value(b), b
+        assert all(0 <= v < 255 for v in st) and tiny <= 4 * 2.0 ** -127
 
 
 def test_encode_argument_checks(lib):

@@ -115,13 +115,23 @@ def gemv_tiled(w: TrellisMatrix, tiles: torch.Tensor, x: torch.Tensor, out=None,
     return out
 
 
-def gemv_e5m3(w: TrellisMatrix, x: torch.Tensor, out=None):
-    """y = bf16(W x) with w.scales read as E5M3 block scales (CUDA-core kernel): bf16 [T][rows]."""
+def gemv_e5m3_workspace_bytes(w: TrellisMatrix, T: int) -> int:
+    """Scratch bytes trellis_gemv_e5m3 needs for T tokens (0: the call needs none)."""
+    return int(_abi.load().trellis_gemv_e5m3_workspace(w.abi(), T))
+
+
+def gemv_e5m3(w: TrellisMatrix, x: torch.Tensor, out=None, workspace=None):
+    """y = bf16(W x) with w.scales read as E5M3 block scales: bf16 [T][rows]."""
     x = x if x.dim() == 2 else x.view(1, -1)
     T = x.shape[0]
     if out is None:
         out = torch.empty((T, w.rows), dtype=torch.bfloat16, device=x.device)
-    _abi.check(_abi.load().trellis_gemv_e5m3(w.abi(), _ptr(x), T, _ptr(out), _stream_handle()), "trellis_gemv_e5m3")
+    need = gemv_e5m3_workspace_bytes(w, T)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    nbytes = workspace.numel() if workspace is not None else 0
+    _abi.check(_abi.load().trellis_gemv_e5m3(w.abi(), _ptr(x), T, _ptr(out), _ptr(workspace), nbytes,
+                                             _stream_handle()), "trellis_gemv_e5m3")
     return out
 
 

@@ -15,6 +15,7 @@ EXPORTED = ("trellis_decode_to_mxfp4", "trellis_gemv_workspace", "trellis_gemv",
             "trellis_grouped_moe", "trellis_grouped_moe_hidden_offset", "mxfp4_gemv_workspace", "mxfp4_gemv",
             "mxfp4_grouped_moe_workspace", "mxfp4_grouped_moe_hidden_offset", "mxfp4_grouped_moe",
             "trellis_encode_workspace", "trellis_encode", "trellis_repack_interleaved", "trellis_gemv_e5m3",
+            "trellis_gemv_e5m3_workspace",
             "trellis_scale_tiles_bytes", "trellis_make_scale_tiles", "trellis_gemv_tiled",
             "tcf4_device_timeouts", "tcf4_status_string")
 
@@ -59,7 +60,9 @@ def load(path: str = LIB_PATH):
     L.trellis_decode_to_mxfp4.argtypes = [Matrix, vp, vp, vp]
     L.trellis_decode_to_mxfp4.restype = ctypes.c_int
     L.trellis_repack_interleaved.argtypes = [vp, ctypes.c_int64, ctypes.c_int64, vp, vp]
-    L.trellis_gemv_e5m3.argtypes = [Matrix, vp, ctypes.c_int32, vp, vp]
+    L.trellis_gemv_e5m3_workspace.argtypes = [Matrix, ctypes.c_int32]
+    L.trellis_gemv_e5m3_workspace.restype = ctypes.c_size_t
+    L.trellis_gemv_e5m3.argtypes = [Matrix, vp, ctypes.c_int32, vp, vp, ctypes.c_size_t, vp]
     L.trellis_gemv_e5m3.restype = ctypes.c_int
     L.trellis_repack_interleaved.restype = ctypes.c_int
     L.trellis_gemv_workspace.argtypes = [Matrix, i32]

@@ -56,16 +56,19 @@ enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
 // decode warps and of the other warps after the split.
 constexpr int kRsLaunchRegs = 80, kRsDecRegs = 96, kRsOtherRegs = 48;
 
-template <int NMAX>
+// SETS: sets of UE8M0 scale factors of the weights per block (1; 4 for E5M3 block scales, whose
+// significand bits each get a power-of-two set, see k_mma). Four sets need the 16-block stages.
+template <int NMAX, int SETS = 1>
 struct Cfg {
   static_assert(NMAX <= 256, "B rows of one MMA");
+  static_assert(SETS == 1 || SETS == 4, "one or four scale sets");
   static constexpr int kTok = NMAX / kTerms;                   // tokens per group
   static constexpr int kSlots = (NMAX + kTerms - 1) / kTerms;  // token slots the split writes
   static constexpr int kSplitNT = kTok <= 6 ? kTok : 4;        // slots split side by side
   static constexpr int kC = (NMAX + 31) / 32;                  // B scale columns per 4-block group
   static constexpr int kNTile = (kC + 3) / 4;                  // 32 x 16-byte B scale tiles per group
   static constexpr uint32_t kSfbGCols = 4u * kNTile;           // TMEM columns of a group's B scales
-  static constexpr int kKB = NMAX <= 64 ? 32 : 16;             // 32-blocks per row per stage
+  static constexpr int kKB = NMAX <= 64 && SETS == 1 ? 32 : 16;  // 32-blocks per row per stage
   // Warps: kDecWarps decode warps (four per group of 8 blocks of a stage), then the word loader, two
   // MMA issuer slots, the B loader and four epilogue warps.
   static constexpr int kDecWarps = kKB / 2;
@@ -75,7 +78,7 @@ struct Cfg {
   static constexpr int kNCh = kNBT / 8;                        // decoded in chunks of 8 blocks
   static constexpr int kNG = kNBT / 4;                         // scale groups per decode thread
   static constexpr int kNW = kKB == 32 ? 3 : (NMAX > 96 ? 5 : 6);  // word stages in flight
-  static constexpr int kNA = NMAX <= 64 ? 2 : (NMAX > 96 ? 2 : 3);  // A / scale-factor stages (TMEM)
+  static constexpr int kNA = NMAX <= 64 || SETS > 1 ? 2 : (NMAX > 96 ? 2 : 3);  // A / scale-factor stages (TMEM)
   static constexpr int kNB = NMAX > 96 ? 2 : (NMAX > 32 && NMAX <= 64 ? 3 : 4);  // B stages (shared memory)
   static constexpr int kBoxCols = kKB / 16;                    // 128-byte TMA boxes per 64 rows
   static constexpr uint32_t kWStage = 1024u * kKB;             // 128 rows x 8 KB bytes of words
@@ -99,8 +102,8 @@ struct Cfg {
   static constexpr uint32_t kSfbCols = (kKB / 4) * kSfbGCols;  // TMEM columns of a stage's B scales
   static constexpr uint32_t kACol = kNAcc * kNI * NMAX;        // TMEM: accumulators first, then
   static constexpr uint32_t kSfaCol = kACol + kACols * kNA;    // A stages, A scales (KB columns per
-  static constexpr uint32_t kSfbCol = kSfaCol + kKB * kNA;     // stage), B scales (kSfbCols per stage)
-  static constexpr uint32_t kUsed = kSfbCol + kSfbCols * kNA;
+  static constexpr uint32_t kSfbCol = kSfaCol + SETS * kKB * kNA;  // stage and set), B scales
+  static constexpr uint32_t kUsed = kSfbCol + kSfbCols * kNA;     // (kSfbCols per stage)
   static constexpr uint32_t kTmemCols = kUsed <= 128 ? 128 : (kUsed <= 256 ? 256 : 512);
   static_assert(kUsed <= 512, "TMEM budget");
   // Resident-MXFP4 source (the expanded tensor): the A operand is a shared-memory tile of nibbles
@@ -124,9 +127,9 @@ __host__ __device__ constexpr int kpos_of_weight(int i) { return 8 * (i & 3) + (
 // rows x 16 bytes, LBO = 128 (adjacent chunks), SBO = 128 KB (adjacent 8-row groups). In TMEM the A
 // operand holds the same 16-byte chunks, four 32-bit columns each (element e of a column in bits
 // 4e..4e+3).
-template <int NMAX>
+template <int NMAX, int SETS = 1>
 __host__ __device__ constexpr uint32_t chunk_off(uint32_t n, uint32_t c) {
-  return (n >> 3) * Cfg<NMAX>::kSbo + c * 128u + (n & 7u) * 16u;
+  return (n >> 3) * Cfg<NMAX, SETS>::kSbo + c * 128u + (n & 7u) * 16u;
 }
 
 // ------------------------------------------------------------------------------- routing groups
@@ -235,9 +238,9 @@ __device__ __forceinline__ float pow2f(int e) {
 // 512-byte tile whose 16-byte row r holds, at word c, the UE8M0 bytes of B row 32c + r for the
 // stage's blocks 4g..4g+3 (byte i = block 4g+i). One tcgen05.cp (32x128b, copied to all four lane
 // quarters) moves a group's tile to TMEM, where B row 32c + r reads column c of the group.
-template <int NMAX>
+template <int NMAX, int SETS = 1>
 __host__ __device__ inline size_t terms_bytes(int S) {
-  return (size_t)S * Cfg<NMAX>::kBSlot;
+  return (size_t)S * Cfg<NMAX, SETS>::kBSlot;
 }
 
 // One 32-element block kb of NT activation rows (lane = element; v[i] is slot t0 + i) -> kTerms
@@ -249,10 +252,10 @@ __host__ __device__ inline size_t terms_bytes(int S) {
 // The NT slots are split side by side (their dependent chains overlap); slots at or past `nvalid`
 // are computed but not stored.
 // NAT: natural K order within a block (the MXFP4 tensor's), else the decoder's interleaved order.
-template <int NMAX, bool NAT, int NT>
+template <int NMAX, bool NAT, int NT, int SETS = 1>
 __device__ __forceinline__ void split_terms_n(const float *v, int t0, int nvalid, int kb, int S_total,
                                               uint8_t *terms) {
-  using C = Cfg<NMAX>;
+  using C = Cfg<NMAX, SETS>;
   const int lane = threadIdx.x & 31;
   const int s = kb / C::kKB, c = kb - s * C::kKB, h = c >> 2;
   (void)S_total;
@@ -285,7 +288,7 @@ __device__ __forceinline__ void split_terms_n(const float *v, int t0, int nvalid
       const int n = kTerms * (t0 + i) + j;
       if (t0 + i < nvalid && n < NMAX) {
         if ((kp & 1) == 0)
-          bst[chunk_off<NMAX>((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code[i] | (partner << 4));
+          bst[chunk_off<NMAX, SETS>((uint32_t)n, (uint32_t)c) + (kp >> 1)] = (uint8_t)(code[i] | (partner << 4));
         if (lane == 0)
           sfs[((h * C::kNTile + (n >> 7)) * 32 + (n & 31)) * 16 + ((n >> 5) & 3) * 4 + (c & 3)] = (uint8_t)(S[i] + 127);
       }
@@ -293,9 +296,9 @@ __device__ __forceinline__ void split_terms_n(const float *v, int t0, int nvalid
   }
 }
 
-template <int NMAX, bool NAT = false>
+template <int NMAX, bool NAT = false, int SETS = 1>
 __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total, uint8_t *terms) {
-  split_terms_n<NMAX, NAT, 1>(&v, t, t + 1, kb, S_total, terms);
+  split_terms_n<NMAX, NAT, 1, SETS>(&v, t, t + 1, kb, S_total, terms);
 }
 
 // Plain GEMV: one group, token slots 0..T-1. The B rows of the other slots are not written: an MMA
@@ -303,16 +306,17 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
 // The GEMV's product kernel is launched as a programmatic dependent of this split: it starts its
 // TMEM setup and its first weight tiles (which do not depend on the split) at once and waits for
 // the split's completion only before it reads the activation terms.
-template <int NMAX, bool NAT>
+template <int NMAX, bool NAT, int SETS = 1>
 __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
                                                      uint8_t *__restrict__ terms) {
   grid_dep_wait();     // x may come from, and terms may still be read by, the preceding kernel
   grid_dep_release();  // the product kernel may start; it waits for this grid before reading terms
-  const int nb = K >> 5, S = (nb + Cfg<NMAX>::kKB - 1) / Cfg<NMAX>::kKB, lane = threadIdx.x & 31;
+  const int nb = K >> 5, S = (nb + Cfg<NMAX, SETS>::kKB - 1) / Cfg<NMAX, SETS>::kKB, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < T * nb; wi += nwarps) {
     const int t = wi / nb, kb = wi - t * nb;
-    split_terms<NMAX, NAT>(__uint_as_float((uint32_t)x[(size_t)t * K + kb * 32 + lane] << 16), t, kb, S, terms);
+    split_terms<NMAX, NAT, SETS>(__uint_as_float((uint32_t)x[(size_t)t * K + kb * 32 + lane] << 16), t, kb, S,
+                                 terms);
   }
 }
 
@@ -358,9 +362,9 @@ struct MmaGeom {
   uint32_t off_W, off_B, bslot, off_U, off_P, smem;
 };
 
-template <int NMAX>
+template <int NMAX, int SETS = 1>
 __host__ __device__ inline MmaGeom mma_geom(int mode, bool mx = false, bool tiled = false) {
-  using C = Cfg<NMAX>;
+  using C = Cfg<NMAX, SETS>;
   MmaGeom g;
   g.off_W = 1024u;
   g.off_B = g.off_W + (mx ? C::kNWX * C::kWStageX : C::kNW * C::kWStage);
@@ -559,6 +563,22 @@ __device__ __forceinline__ void tmap_acquire(const void *gmap) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(gmap) : "memory");
 }
 
+// The UE8M0 scale sets of four E5M3 block-scale bytes (one per byte of w, each byte on its own, no
+// carries between bytes): for exponent field e and significand bits m2 m1 m0, set 0 holds
+// 2^(e-15) (e + 112; 0, i.e. 2^-127, when e = 0; 0xFF, NaN, when e = 31) and set k = 1, 2, 3 holds
+// 2^(max(e,1) - 15 - k) when significand bit 3 - k is set, else 0 (2^-127). The sum over the sets
+// is the E5M3 value 2^(e-15) (1 + m/8), or m 2^-17 when e = 0.
+__device__ __forceinline__ void e5m3_scale_sets(uint32_t w, uint32_t (&st)[4]) {
+  const uint32_t e = (w >> 3) & 0x1F1F1F1Fu, m = w & 0x07070707u;
+  const uint32_t nz = ((e + 0x7F7F7F7Fu) & 0x80808080u) >> 7;   // 1 in the bytes with e >= 1
+  const uint32_t nan = ((e + 0x61616161u) & 0x80808080u) >> 7;  // 1 in the bytes with e == 31
+  const uint32_t ee = e | (nz ^ 0x01010101u);                   // max(e, 1)
+  st[0] = ((e + 0x70707070u) & (nz * 0xFFu)) | (nan * 0xFFu);
+  st[1] = (ee + 0x6F6F6F6Fu) & (((m >> 2) & 0x01010101u) * 0xFFu);
+  st[2] = (ee + 0x6E6E6E6Eu) & (((m >> 1) & 0x01010101u) * 0xFFu);
+  st[3] = (ee + 0x6D6D6D6Du) & ((m & 0x01010101u) * 0xFFu);
+}
+
 // ------------------------------------------------------------------------------- kernel arguments
 
 struct MmaArgs {
@@ -665,11 +685,17 @@ __device__ __forceinline__ int tile_row(const JobRows &j, int m) {
 // with tcgen05.cp, so the decode warps handle no scale factors at all. (In the B ring they are
 // released with the stage's MMAs; a ring of their own beside the word ring held back the word
 // loads, whose slots free up earlier.)
-template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS = false, bool TILED = false>
-__global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
-                                                     const __grid_constant__ MoeTable<MAXE> tab,
-                                                     const __grid_constant__ CUtensorMap wmap) {
-  using C = Cfg<NMAX>;
+// SETS = 4: the weights' scale bytes are E5M3 block scales ("XOR-Trellis" news page, its grouping
+// format), read as s = 2^(e-15) (1 + m/8) (subnormal below e = 1). Such a scale is the sum of at
+// most four powers of two, 2^(e-15) for the implicit bit and 2^(e-16), 2^(e-17), 2^(e-18) for the
+// significand bits that are set, so the product of a block is four block-scaled MMAs of the same A
+// and B, one per power, summed in the accumulator; an absent power takes the smallest UE8M0 scale
+// 2^-127 (its contribution is below 2^-124 of |x| per weight) and a NaN scale (e = 31) gives NaN.
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS = false, bool TILED = false, int SETS = 1>
+__global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __grid_constant__ MmaArgs a,
+                                                           const __grid_constant__ MoeTable<MAXE> tab,
+                                                           const __grid_constant__ CUtensorMap wmap) {
+  using C = Cfg<NMAX, SETS>;
   constexpr int kNW = MX ? C::kNWX : C::kNW, kNA = C::kNA, kKB = C::kKB, kNBT = C::kNBT, kNG = C::kNG;
   constexpr uint32_t kWStage = MX ? C::kWStageX : C::kWStage;
   constexpr uint32_t kSfaCol = MX ? C::kSfaColX : C::kSfaCol, kSfbCol = MX ? C::kSfbColX : C::kSfbCol;
@@ -678,7 +704,8 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbr = a.nbr, S = (nbr + kKB - 1) / kKB;
   static_assert(!TILED || (MODE == kModeGemv && !MX), "scale tiles: plain decode GEMV only");
-  const MmaGeom geo = mma_geom<NMAX>(MODE, MX, TILED);
+  static_assert(SETS == 1 || (MODE == kModeGemv && !MX && !TILED), "E5M3 scale sets: plain decode GEMV only");
+  const MmaGeom geo = mma_geom<NMAX, SETS>(MODE, MX, TILED);
   static_assert((MX ? 2 * kNW : kNW) <= 8 && kNA <= 4 && C::kNB <= 4,
                 "barrier block: 8 word slots, 4 A and 4 B slots");
   // 49 barriers in bytes [0, 392). The A operand of a stage is filled and released in two halves
@@ -693,7 +720,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
   unsigned char *smap = smem + 512;  // shared-memory copy of the tensor map (grouped MoE)
   unsigned int *tmo = &g_tcf4_timeouts_mma;
   GroupPlan *pl = reinterpret_cast<GroupPlan *>(smem + geo.off_P);
-  const size_t tbytes = terms_bytes<NMAX>(S);
+  const size_t tbytes = terms_bytes<NMAX, SETS>(S);
 
   if (tid == 0) {
     for (int i = 0; i < (MX ? 2 * kNW : kNW); i++) {
@@ -944,8 +971,16 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       if constexpr (!TILED) {
 #pragma unroll
         for (int g = 0; g < kNG; g++) {
-          const uint32_t gg = (uint32_t)(kNG * h + g);
-          tmem_st_x1(tq + kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, pa[2 * g] | (pa[2 * g + 1] << 16));
+          const uint32_t gg = (uint32_t)(kNG * h + g), wg = pa[2 * g] | (pa[2 * g + 1] << 16);
+          if constexpr (SETS == 1) {
+            tmem_st_x1(tq + kSfaCol + kKB * b + 4u * gg + (uint32_t)sp, wg);
+          } else {  // the four powers of two of each E5M3 scale, set i at column i KB of the stage
+            uint32_t st4[4];
+            e5m3_scale_sets(wg, st4);
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+              tmem_st_x1(tq + kSfaCol + SETS * kKB * b + (uint32_t)i * kKB + 4u * gg + (uint32_t)sp, st4[i]);
+          }
         }
       }
       tmem_wait_st();
@@ -1230,7 +1265,7 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
       const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
       const uint64_t bd = smem_desc(b0 + (uint32_t)bb * geo.bslot, 128u, C::kSbo);
       const uint32_t bsf0 = b0 + (uint32_t)bb * geo.bslot + C::kBStage;  // the stage's B scale tiles
-      const uint32_t sfa = tbase + kSfaCol + kKB * (uint32_t)b, sfb = tbase + kSfbCol + C::kSfbCols * (uint32_t)b;
+      const uint32_t sfa = tbase + kSfaCol + SETS * kKB * (uint32_t)b, sfb = tbase + kSfbCol + C::kSfbCols * (uint32_t)b;
       const int wsx = q % kNW;  // MX: the stage's word slot
       const uint64_t ad0 = MX ? desc_sw128(smem_u32(smem + geo.off_W) + (uint32_t)wsx * kWStage) : 0ull;
 #pragma unroll
@@ -1269,9 +1304,12 @@ __global__ void __launch_bounds__(Cfg<NMAX>::kThreads, 1) k_mma(const __grid_con
                             (j & 1) ? idesc2 : idesc0, (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30),
                             (sfb + C::kSfbGCols * (uint32_t)(j >> 1)) | (sf << 30), !(s == 0 && j == jfirst));
               else
-                mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
-                            (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30),
-                            (sfb + C::kSfbGCols * (uint32_t)(j >> 1)) | (sf << 30), !(s == 0 && j == jfirst));
+#pragma unroll
+                for (int st = 0; st < SETS; st++)  // one MMA per scale set (SETS = 4: E5M3)
+                  mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
+                              (sfa + (uint32_t)st * kKB + 4u * (uint32_t)(j >> 1)) | (sf << 30),
+                              (sfb + C::kSfbGCols * (uint32_t)(j >> 1)) | (sf << 30),
+                              !(s == 0 && j == jfirst && st == 0));
             }
           }
           tc_commit(&a_empty[2 * b + hh]);
@@ -1364,20 +1402,25 @@ static int mx_nmax_for(int tokens_per_group) {
 // wider B operand would mostly multiply empty slots.
 static int moe_nmax_for(int T) { return nmax_for(T) == 32 ? 32 : 96; }
 static uint32_t geom_smem_for(int NMAX, int mode, bool mx, bool tiled);
-template <int NMAX>
-static uint32_t geom_smem(int mode, bool mx, bool tiled) { return mma_geom<NMAX>(mode, mx, tiled).smem; }
-static uint32_t geom_smem_for(int NMAX, int mode, bool mx, bool tiled) {
+// E5M3 scales (four scale sets) have no 64-row configuration either.
+static int e5_nmax_for(int tokens_per_group) { return mx_nmax_for(tokens_per_group); }
+template <int NMAX, int SETS = 1>
+static uint32_t geom_smem(int mode, bool mx, bool tiled) { return mma_geom<NMAX, SETS>(mode, mx, tiled).smem; }
+static uint32_t geom_smem_for(int NMAX, int mode, bool mx, bool tiled, int sets = 1) {
+  if (sets == 4)
+    return NMAX == 32 ? geom_smem<32, 4>(mode, mx, tiled)
+                      : (NMAX == 96 ? geom_smem<96, 4>(mode, mx, tiled) : geom_smem<192, 4>(mode, mx, tiled));
   return NMAX == 32   ? geom_smem<32>(mode, mx, tiled)
          : NMAX == 64 ? geom_smem<64>(mode, mx, tiled)
          : NMAX == 96 ? geom_smem<96>(mode, mx, tiled)
                       : geom_smem<192>(mode, mx, tiled);
 }
 
-static bool mma_fits(int NMAX, int mode, bool mx = false, bool tiled = false) {
+static bool mma_fits(int NMAX, int mode, bool mx = false, bool tiled = false, int sets = 1) {
   int dev = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return false;
   if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
-  const uint32_t need = geom_smem_for(NMAX, mode, mx, tiled);
+  const uint32_t need = geom_smem_for(NMAX, mode, mx, tiled, sets);
   return need <= (uint32_t)optin;
 }
 
@@ -1385,7 +1428,11 @@ static bool mma_fits(int NMAX, int mode, bool mx = false, bool tiled = false) {
 // pitch that is a multiple of 16 bytes for the tensor map) and a 16-byte aligned stream.
 static bool k_ok(int nbr) { return nbr >= 2 && nbr % 2 == 0; }
 
-static size_t terms_for(int nbr, int NMAX) {
+static size_t terms_for(int nbr, int NMAX, int sets = 1) {
+  if (sets == 4)
+    return NMAX == 32   ? terms_bytes<32, 4>((nbr + Cfg<32, 4>::kKB - 1) / Cfg<32, 4>::kKB)
+           : NMAX == 96 ? terms_bytes<96, 4>((nbr + Cfg<96, 4>::kKB - 1) / Cfg<96, 4>::kKB)
+                        : terms_bytes<192, 4>((nbr + Cfg<192, 4>::kKB - 1) / Cfg<192, 4>::kKB);
   return NMAX == 32   ? terms_bytes<32>((nbr + Cfg<32>::kKB - 1) / Cfg<32>::kKB)
          : NMAX == 64 ? terms_bytes<64>((nbr + Cfg<64>::kKB - 1) / Cfg<64>::kKB)
          : NMAX == 96 ? terms_bytes<96>((nbr + Cfg<96>::kKB - 1) / Cfg<96>::kKB)
@@ -1449,6 +1496,15 @@ cudaError_t launch_scale_tiles(const MatView &w, uint8_t *tiles, cudaStream_t s)
 // Tokens beyond kGemvTok run as further passes, each with its own split of x.
 size_t gemv_mma_workspace(const MatView &w, int T) { return terms_for(w.nbr, nmax_for(T < kGemvTok ? T : kGemvTok)); }
 size_t mx_gemv_workspace(const MatView &w, int T) { return terms_for(w.nbr, mx_nmax_for(T < kGemvTok ? T : kGemvTok)); }
+// E5M3 scales on the tensor cores: the trellis conditions, with the four-set configurations.
+bool gemv_e5m3_mma_supported(const MatView &w, int T) {
+  return k_ok(w.nbr) && (reinterpret_cast<uintptr_t>(w.stream) & 15u) == 0 &&
+         (reinterpret_cast<uintptr_t>(w.scales) & 1u) == 0 && tensor_map_encoder() != nullptr &&
+         mma_fits(e5_nmax_for(T < kGemvTok ? T : kGemvTok), kModeGemv, false, false, 4);
+}
+size_t gemv_e5m3_mma_workspace(const MatView &w, int T) {
+  return terms_for(w.nbr, e5_nmax_for(T < kGemvTok ? T : kGemvTok), 4);
+}
 
 static int sm_count_impl() {
   int dev = 0, nsm = 148;
@@ -1458,14 +1514,15 @@ static int sm_count_impl() {
 }
 
 // One launch of a product kernel instance (dynamic shared memory attribute set once per instance).
-template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS, bool TILED = false>
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool RS, bool TILED = false, int SETS = 1>
 static cudaError_t launch_product_rs(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
                                      cudaStream_t s) {
   static unsigned long long attr = 0;
-  cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS, TILED>, attr);
+  cudaError_t e = ensure_max_dynamic_smem(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS, TILED, SETS>, attr);
   if (e != cudaSuccess) return e;
-  return launch_dependent(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS, TILED>, dim3(grid), dim3(Cfg<NMAX>::kThreads),
-                          mma_geom<NMAX>(MODE, MX, TILED).smem, s, args, tab, map);
+  return launch_dependent(k_mma<MAXE, MODE, NMAX, MX, CARRY, RS, TILED, SETS>, dim3(grid),
+                          dim3(Cfg<NMAX, SETS>::kThreads), mma_geom<NMAX, SETS>(MODE, MX, TILED).smem, s, args, tab,
+                          map);
 }
 
 // True when the register-split instance was compiled with at least kRsLaunchRegs registers per
@@ -1482,19 +1539,22 @@ static bool register_split_ok() {
 }
 
 // The decode GEMV at NMAX = 32 takes the register split when its compiled registers allow it.
-template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool TILED = false>
+template <int MAXE, int MODE, int NMAX, bool MX, bool CARRY, bool TILED = false, int SETS = 1>
 static cudaError_t launch_product(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
                                   cudaStream_t s) {
-  if constexpr (MODE == kModeGemv && NMAX == 32 && !MX) {
+  if constexpr (MODE == kModeGemv && NMAX == 32 && !MX && SETS == 1) {
     if (register_split_ok<MAXE, MODE, NMAX, MX, CARRY, TILED>())
       return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, true, TILED>(grid, args, tab, map, s);
   }
-  return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, false, TILED>(grid, args, tab, map, s);
+  return launch_product_rs<MAXE, MODE, NMAX, MX, CARRY, false, TILED, SETS>(grid, args, tab, map, s);
 }
-template <int MAXE, int MODE, int NMAX, bool MX>
+template <int MAXE, int MODE, int NMAX, bool MX, int SETS = 1>
 static cudaError_t launch_product_seg(int grid, const MmaArgs &args, const MoeTable<MAXE> &tab, const CUtensorMap &map,
                                       cudaStream_t s) {
-  if constexpr (MX) {
+  if constexpr (SETS > 1) {
+    return args.seg_blocks > 1 ? launch_product<MAXE, MODE, NMAX, false, true, false, SETS>(grid, args, tab, map, s)
+                               : launch_product<MAXE, MODE, NMAX, false, false, false, SETS>(grid, args, tab, map, s);
+  } else if constexpr (MX) {
     return launch_product<MAXE, MODE, NMAX, true, false>(grid, args, tab, map, s);
   } else if constexpr (MODE == kModeGemv) {
     if (args.sf_tiles != nullptr)
@@ -1508,13 +1568,13 @@ static cudaError_t launch_product_seg(int grid, const MmaArgs &args, const MoeTa
   }
 }
 
-template <int NMAX, bool MX>
+template <int NMAX, bool MX, int SETS = 1>
 static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, const uint16_t *x, int T, uint16_t *y,
                                     void *ws, cudaStream_t s, const uint8_t *tiles) {
   uint8_t *terms = static_cast<uint8_t *>(ws);
   const int warps = T * w.nbr;
-  cudaError_t e =
-      launch_dependent(k_bsplit_gemv<NMAX, MX>, dim3((warps + 7) / 8), dim3(256), 0, s, x, T, w.nbr * 32, terms);
+  cudaError_t e = launch_dependent(k_bsplit_gemv<NMAX, MX, SETS>, dim3((warps + 7) / 8), dim3(256), 0, s, x, T,
+                                   w.nbr * 32, terms);
   if (e != cudaSuccess) return e;
   const int ntiles = (w.rows + 127) / 128, nsm = sm_count();
   MmaArgs args{};
@@ -1529,7 +1589,7 @@ static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, co
   args.sf_tiles = tiles;
   args.sf_groups = scale_tile_groups(w.nbr);
   MoeTable<32> none{};
-  return launch_product_seg<32, kModeGemv, NMAX, MX>(ntiles < nsm ? ntiles : nsm, args, none, map, s);
+  return launch_product_seg<32, kModeGemv, NMAX, MX, SETS>(ntiles < nsm ? ntiles : nsm, args, none, map, s);
 }
 
 template <bool MX>
@@ -1567,6 +1627,21 @@ cudaError_t launch_mx_gemv(const MatView &w, const uint16_t *x, int T, uint16_t 
 cudaError_t launch_gemv_tiled(const MatView &w, const uint8_t *tiles, const uint16_t *x, int T, uint16_t *y, void *ws,
                               cudaStream_t s) {
   return launch_gemv_t<false>(w, x, T, y, ws, s, tiles);
+}
+cudaError_t launch_gemv_e5m3_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s) {
+  CUtensorMap map;
+  if (!make_word_map(&map, w.stream, w.rows, w.nbr, 8)) return cudaErrorInvalidValue;
+  const int nm = e5_nmax_for(T < kGemvTok ? T : kGemvTok);
+  for (int t0 = 0; t0 < T; t0 += kGemvTok) {
+    const int n = T - t0 < kGemvTok ? T - t0 : kGemvTok;
+    const uint16_t *xp = x + (size_t)t0 * w.nbr * 32;
+    uint16_t *yp = y + (size_t)t0 * w.rows;
+    const cudaError_t e = nm == 32   ? launch_gemv_pass<32, false, 4>(w, map, xp, n, yp, ws, s, nullptr)
+                          : nm == 96 ? launch_gemv_pass<96, false, 4>(w, map, xp, n, yp, ws, s, nullptr)
+                                     : launch_gemv_pass<192, false, 4>(w, map, xp, n, yp, ws, s, nullptr);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // ----------------------------------------------------------------------------- MoE on the tensor cores

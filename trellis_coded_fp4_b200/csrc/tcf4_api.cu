@@ -187,14 +187,31 @@ tcf4_status trellis_gemv_tiled(tcf4_matrix w, const uint8_t *tiles, const uint16
   return from_cuda(launch_gemv_tiled(v, tiles, x, T, y, workspace, static_cast<cudaStream_t>(stream)));
 }
 
-tcf4_status trellis_gemv_e5m3(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *stream) {
+static bool gemv_e5m3_uses_mma(const tcf4_matrix &w, int32_t T) {
+  return w.rows > 0 && T > 0 && gemv_e5m3_mma_supported(view(w), T);
+}
+
+size_t trellis_gemv_e5m3_workspace(tcf4_matrix w, int32_t T) {
+  if (check_gemv(w, T) != TCF4_OK || T == 0 || w.rows == 0) return 0;
+  return gemv_e5m3_uses_mma(w, T) ? gemv_e5m3_mma_workspace(view(w), T) : 0;
+}
+
+tcf4_status trellis_gemv_e5m3(tcf4_matrix w, const uint16_t *x, int32_t T, uint16_t *y, void *workspace,
+                              size_t ws_bytes, void *stream) {
   tcf4_status st = check_gemv(w, T);
   if (st != TCF4_OK) return st;
   if (T == 0 || w.rows == 0) return TCF4_OK;
   if (x == nullptr || y == nullptr) return TCF4_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(y)) return TCF4_ERR_MISALIGNED;
+  const MatView v = view(w);
+  if (gemv_e5m3_uses_mma(w, T)) {
+    if (workspace == nullptr || ws_bytes < gemv_e5m3_mma_workspace(v, T)) return TCF4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TCF4_ERR_MISALIGNED;
+    clear_pending_error();
+    return from_cuda(launch_gemv_e5m3_mma(v, x, T, y, workspace, static_cast<cudaStream_t>(stream)));
+  }
   clear_pending_error();
-  return from_cuda(launch_gemv(view(w), x, T, y, static_cast<cudaStream_t>(stream), true));
+  return from_cuda(launch_gemv(v, x, T, y, static_cast<cudaStream_t>(stream), true));
 }
 
 tcf4_status trellis_moe_route(const float *logits, int32_t T, int32_t E, int32_t k, int32_t *topk_ids,

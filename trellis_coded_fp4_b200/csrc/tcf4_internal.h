@@ -121,6 +121,10 @@ cudaError_t launch_encode(const double *target, const double *D, const uint8_t *
 // point at the nibble matrices [rows][cols/2]. Workspaces are the same as the trellis paths'.
 bool mx_gemv_supported(const MatView &w, int T);
 size_t mx_gemv_workspace(const MatView &w, int T);
+// E5M3 block scales on the tensor cores (k_mma.cu, four UE8M0 scale sets per block).
+bool gemv_e5m3_mma_supported(const MatView &w, int T);
+size_t gemv_e5m3_mma_workspace(const MatView &w, int T);
+cudaError_t launch_gemv_e5m3_mma(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s);
 cudaError_t launch_mx_gemv(const MatView &w, const uint16_t *x, int T, uint16_t *y, void *ws, cudaStream_t s);
 bool moe_mx_supported(const tcf4_moe &m, int T);
 cudaError_t launch_moe_mx(const tcf4_moe &m, const uint16_t *x, int T, const int32_t *ids, const float *wts, int k,
