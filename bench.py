@@ -266,7 +266,25 @@ class Layer:
             self._expanded()
             tc.decode_to_mxfp4(self.G, self.nibG, self.scG)
         elif name == "grouped_moe":
-            self.moe_call(1)(i)
+            if not hasattr(self, "_moe1"):
+                self._moe1 = self.moe_call(1)
+            self._moe1(i)
+        elif name == "gemv_gate_up_t32":
+            if not hasattr(self, "_x32"):
+                from trellis_coded_fp4_b200 import synth
+                self._x32 = synth.activations(32, H, seed=synth.SEED_BASE + 122).to(self.device)
+                self._y32 = torch.empty((32, self.G.rows), dtype=torch.bfloat16, device=self.device)
+                self._ws32 = torch.empty(tc.gemv_workspace_bytes(self.G, 32), dtype=torch.uint8, device=self.device)
+            tc.gemv_tiled(self.G, self.Trot[0], self._x32, self._y32, self._ws32)
+        elif name == "gemv_e5m3":
+            if not hasattr(self, "_W5"):
+                g5 = torch.Generator(device=self.device).manual_seed(5)
+                m5 = torch.randint(0, 8, self.G.scales.shape, dtype=torch.int32, device=self.device, generator=g5)
+                sc5 = (((self.G.scales.to(torch.int32) - 112) << 3) | m5).to(torch.uint8)
+                self._W5 = tc.TrellisMatrix(self.G.stream, sc5, self.G.rows, self.G.cols, SEG)
+                self._ws5 = torch.empty(tc.gemv_e5m3_workspace_bytes(self._W5, 1), dtype=torch.uint8,
+                                        device=self.device)
+            tc.gemv_e5m3(self._W5, self.x[i % NVAR], out=self.yG, workspace=self._ws5)
         else:
             raise ValueError(name)
 
@@ -649,7 +667,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="the headline only, without the extra rows")
     ap.add_argument("--only", default=None,
-                    help="run only this call (gemv_gate_up, gemv_down, expand_gate_up, grouped_moe) warmup + "
+                    help="run only this call (gemv_gate_up, gemv_gate_up_raw, gemv_gate_up_t32, gemv_down, gemv_e5m3, "
+                         "expand_gate_up, grouped_moe) warmup + "
                          "steps times, for profiling one kernel; prints no bench line")
     args = ap.parse_args()
     if args.impl == "reference":
