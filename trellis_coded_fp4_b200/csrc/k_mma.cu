@@ -515,6 +515,9 @@ __device__ __forceinline__ void mma_mxf4_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// A 64-bit descriptor from its two words (a register pair, no instruction).
+__device__ __forceinline__ uint64_t desc_of(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
+
 // One thread: copy a 32-row x 16-byte shared-memory tile (descriptor desc) into TMEM columns
 // taddr..taddr+3 of every lane quarter: row r to lane 32q + r of each quarter q.
 __device__ __forceinline__ void tmem_cp_sf(uint32_t taddr, uint64_t desc) {
@@ -1263,53 +1266,72 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
         ok = mbar_wait_sleep(&acc_empty[jl % C::kNAcc], (uint32_t)(jl / C::kNAcc - 1) & 1u, tmo, kMmaSleepNs);
       const int nmma = (nbr - kKB * s < kKB ? nbr - kKB * s : kKB) >> 1;
       const uint32_t at = tbase + C::kACol + C::kACols * (uint32_t)b;
+      // Descriptors of this stage's B slot: the low words of a start address advance by immediates
+      // (16-byte units, inside the 14-bit field), the high words stay.
       const uint64_t bd = smem_desc(b0 + (uint32_t)bb * geo.bslot, 128u, C::kSbo);
-      const uint32_t bsf0 = b0 + (uint32_t)bb * geo.bslot + C::kBStage;  // the stage's B scale tiles
+      const uint32_t bd_lo = (uint32_t)bd, bd_hi = (uint32_t)(bd >> 32);
+      // the stage's B scale tiles, then (TILED) the weights' scale tiles: 512 bytes = 32 units each
+      const uint64_t sd = smem_desc(b0 + (uint32_t)bb * geo.bslot + C::kBStage, 128u, 128u);
+      const uint32_t sd_lo = (uint32_t)sd, sd_hi = (uint32_t)(sd >> 32);
       const uint32_t sfa = tbase + kSfaCol + SETS * kKB * (uint32_t)b, sfb = tbase + kSfbCol + C::kSfbCols * (uint32_t)b;
       const int wsx = q % kNW;  // MX: the stage's word slot
       const uint64_t ad0 = MX ? desc_sw128(smem_u32(smem + geo.off_W) + (uint32_t)wsx * kWStage) : 0ull;
+      // This issuer's halves of the stage, in order: half h_lo only with two issuers, both with one.
+      // Inside a half every operand is a per-half base plus a compile-time offset (kKB / 4 MMAs of
+      // K = 64, kKB / 8 groups of four blocks; kKB / 4 is even, so MMA j0 + jj takes scale id
+      // 2 (jj & 1) of group g0 + jj / 2).
 #pragma unroll
-      for (int hh = h_lo; hh < h_hi; hh++) {  // this issuer's halves of the stage, in order
+      for (int hi = 0; hi < 3 - C::kNI; hi++) {
+        const int hh = C::kNI == 2 ? h_lo : hi;
         ok = __all_sync(0xffffffffu, ok && mbar_wait_sleep(&a_full[2 * b + hh], ph, tmo, kMmaSleepNs));
         if (MX && ok)
           ok = __all_sync(0xffffffffu,
                           mbar_wait_sleep(&w_full[2 * wsx + hh], (uint32_t)(q / kNW) & 1u, tmo, kMmaSleepNs));
         if (!ok) break;
         tc_fence_after();
-        const int jfirst = C::kNI == 2 ? hh * kKB / 4 : 0;  // this issuer's first MMA of a job
+        const int j0 = hh * (kKB / 4), g0 = hh * (kKB / 8);
+        const int lim = nmma - j0;  // MMAs of this half inside the row (fewer in a row's last stage)
+        // the first MMA of a job into this issuer's accumulator starts it (each issuer has its own)
+        const bool first = s == 0 && (C::kNI == 2 || hh == 0);
         const uint32_t d_t = tbase + (uint32_t)(((jl % C::kNAcc) * C::kNI + (C::kNI == 2 ? hh : 0)) * NMAX);
         if (leader) {
-          // the B scale factors of this half's groups (4 blocks each), ahead of the MMAs that read
-          // them: tcgen05 operations of one thread run in issue order
+          // the B scale factors of this half's groups, ahead of the MMAs that read them (tcgen05
+          // operations of one thread run in issue order)
+          const uint32_t sdb = sd_lo + 32u * (uint32_t)(C::kNTile * g0), sfb_h = sfb + C::kSfbGCols * (uint32_t)g0;
 #pragma unroll
-          for (int g = hh * kKB / 8; g < (hh + 1) * kKB / 8; g++)
+          for (int gg = 0; gg < kKB / 8; gg++)
+            if (2 * gg < lim)
 #pragma unroll
-            for (int ti = 0; ti < C::kNTile; ti++)
-              if (2 * g < nmma)
-                tmem_cp_sf(sfb + C::kSfbGCols * (uint32_t)g + 4u * ti,
-                           smem_desc(bsf0 + 512u * (uint32_t)(C::kNTile * g + ti), 128u, 128u));
+              for (int ti = 0; ti < C::kNTile; ti++)
+                tmem_cp_sf(sfb_h + C::kSfbGCols * (uint32_t)gg + 4u * ti,
+                           desc_of(sdb + 32u * (uint32_t)(C::kNTile * gg + ti), sd_hi));
+          const uint32_t sfa_h = sfa + 4u * (uint32_t)g0;
           if constexpr (TILED) {  // the weights' scale factors: tile row r to lanes r, 32 + r, 64 + r, 96 + r
-            const uint32_t asf0 = b0 + (uint32_t)bb * geo.bslot + C::kBSlot;  // the weights' scale tiles
+            const uint32_t sda = sd_lo + (C::kSfbStage >> 4) + 32u * (uint32_t)g0;
 #pragma unroll
-            for (int g = hh * kKB / 8; g < (hh + 1) * kKB / 8; g++)
-              if (2 * g < nmma) tmem_cp_sf(sfa + 4u * (uint32_t)g, smem_desc(asf0 + 512u * (uint32_t)g, 128u, 128u));
+            for (int gg = 0; gg < kKB / 8; gg++)
+              if (2 * gg < lim) tmem_cp_sf(sfa_h + 4u * (uint32_t)gg, desc_of(sda + 32u * (uint32_t)gg, sd_hi));
           }
+          const uint32_t at_h = at + 8u * (uint32_t)j0, bd_h = bd_lo + 16u * (uint32_t)j0;
 #pragma unroll
-          for (int j = hh * kKB / 4; j < (hh + 1) * kKB / 4; j++) {
-            if (j < nmma) {
-              const uint32_t sf = (uint32_t)(j & 1) * 2u;
-              // +256 bytes of B per MMA: the descriptor's start address counts 16-byte units
+          for (int jj = 0; jj < kKB / 4; jj++) {
+            if (jj < lim) {
+              // +256 bytes of B per MMA: the descriptor's start address counts 16-byte units; the
+              // scale id sits in bits 30-31 of the scale-factor address (zero lane bits here)
+              const uint32_t sfo = 4u * (uint32_t)(jj >> 1) + ((uint32_t)(jj & 1) << 31);
+              const uint32_t id = (jj & 1) ? idesc2 : idesc0;
               if constexpr (MX)  // A: column box j / 4 (16 KB apart), 32 bytes per MMA inside it
-                mma_mxf4_ss(d_t, ad0 + (uint64_t)((j >> 2) * 1024 + 2 * (j & 3)), bd + 16u * (uint64_t)j,
-                            (j & 1) ? idesc2 : idesc0, (sfa + 4u * (uint32_t)(j >> 1)) | (sf << 30),
-                            (sfb + C::kSfbGCols * (uint32_t)(j >> 1)) | (sf << 30), !(s == 0 && j == jfirst));
+                mma_mxf4_ss(d_t, ad0 + (uint64_t)(((j0 + jj) >> 2) * 1024 + 2 * (jj & 3)),
+                            desc_of(bd_h + 16u * (uint32_t)jj, bd_hi), id, sfa_h + sfo,
+                            sfb_h + C::kSfbGCols * (uint32_t)(jj >> 1) + ((uint32_t)(jj & 1) << 31),
+                            !(first && jj == 0));
               else
 #pragma unroll
                 for (int st = 0; st < SETS; st++)  // one MMA per scale set (SETS = 4: E5M3)
-                  mma_mxf4_ts(d_t, at + 8u * (uint32_t)j, bd + 16u * (uint64_t)j, (j & 1) ? idesc2 : idesc0,
-                              (sfa + (uint32_t)st * kKB + 4u * (uint32_t)(j >> 1)) | (sf << 30),
-                              (sfb + C::kSfbGCols * (uint32_t)(j >> 1)) | (sf << 30),
-                              !(s == 0 && j == jfirst && st == 0));
+                  mma_mxf4_ts(d_t, at_h + 8u * (uint32_t)jj, desc_of(bd_h + 16u * (uint32_t)jj, bd_hi), id,
+                              sfa_h + (uint32_t)st * kKB + sfo,
+                              sfb_h + C::kSfbGCols * (uint32_t)(jj >> 1) + ((uint32_t)(jj & 1) << 31),
+                              !(first && jj == 0 && st == 0));
             }
           }
           tc_commit(&a_empty[2 * b + hh]);
