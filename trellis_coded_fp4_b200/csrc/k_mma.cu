@@ -48,6 +48,7 @@ constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped 
 
 // Sleep between barrier tests of the idle roles. The loaders run stages ahead and the MMA issuers
 // have about two stages (~3 us) of slack, so these only bound how soon a completed phase is seen.
+constexpr int kSplitThreads = 128;  // activation-split CTAs (see k_bsplit_gemv)
 constexpr uint32_t kLoaderSleepNs = 200u, kMmaSleepNs = 100u, kEpiSleepNs = 200u;
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
@@ -305,9 +306,12 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
 // column depends only on its own B row (and its scale), and no output reads those columns.
 // The GEMV's product kernel is launched as a programmatic dependent of this split: it starts its
 // TMEM setup and its first weight tiles (which do not depend on the split) at once and waits for
-// the split's completion only before it reads the activation terms.
+// the split's completion only before it reads the activation terms. CTAs of 128 threads with at most
+// 32 registers each (4096) fit beside a resident product CTA (768 threads x 80 registers = 61440 of
+// the SM's 65536): the split of the next call can wait on its grid dependency on any SM while the
+// current product kernel runs, and it never keeps a product CTA from starting.
 template <int NMAX, bool NAT, int SETS = 1>
-__global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
+__global__ void __launch_bounds__(kSplitThreads, 65536 / (32 * kSplitThreads)) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
                                                      uint8_t *__restrict__ terms) {
   grid_dep_wait();     // x may come from, and terms may still be read by, the preceding kernel
   grid_dep_release();  // the product kernel may start; it waits for this grid before reading terms
@@ -324,9 +328,10 @@ __global__ void __launch_bounds__(256) k_bsplit_gemv(const uint16_t *__restrict_
 // (rows of tokens: div = k, as for x before gate/up; rows of pairs: div = 1). Only the slots that
 // hold a pair are split (the B rows of empty slots feed MMA columns nothing reads). The down
 // product's terms do not come from here: the gate/up epilogue writes them. Block 0 also clears the
-// down kernel's counters when `counters` is given.
+// down kernel's counters when `counters` is given. CTAs of 128 threads with at most 32 registers, so
+// that they fit beside a resident product CTA (as k_bsplit_gemv's).
 template <int NMAX, bool NAT>
-__global__ void __launch_bounds__(256) k_bsplit_moe(const int32_t *__restrict__ ids, int P, int E, int div,
+__global__ void __launch_bounds__(kSplitThreads, 65536 / (32 * kSplitThreads)) k_bsplit_moe(const int32_t *__restrict__ ids, int P, int E, int div,
                                                     const uint16_t *__restrict__ src, int K, uint8_t *__restrict__ terms,
                                                     int *__restrict__ counters, int n_counters) {
   __shared__ GroupPlan pl;
@@ -1594,9 +1599,9 @@ template <int NMAX, bool MX, int SETS = 1>
 static cudaError_t launch_gemv_pass(const MatView &w, const CUtensorMap &map, const uint16_t *x, int T, uint16_t *y,
                                     void *ws, cudaStream_t s, const uint8_t *tiles) {
   uint8_t *terms = static_cast<uint8_t *>(ws);
-  const int warps = T * w.nbr;
-  cudaError_t e = launch_dependent(k_bsplit_gemv<NMAX, MX, SETS>, dim3((warps + 7) / 8), dim3(256), 0, s, x, T,
-                                   w.nbr * 32, terms);
+  const int warps = T * w.nbr, wpc = kSplitThreads / 32;
+  cudaError_t e = launch_dependent(k_bsplit_gemv<NMAX, MX, SETS>, dim3((warps + wpc - 1) / wpc), dim3(kSplitThreads),
+                                   0, s, x, T, w.nbr * 32, terms);
   if (e != cudaSuccess) return e;
   const int ntiles = (w.rows + 127) / 128, nsm = sm_count();
   MmaArgs args{};
@@ -1748,10 +1753,10 @@ static cudaError_t launch_moe_mma_t(const tcf4_moe &m, const uint16_t *x, int T,
   {
     uint8_t *terms = reinterpret_cast<uint8_t *>(base + L.bg_gu);
     const int nbr = m.H / 32;
-    const int warps = P * nbr;  // one warp per routed pair and 32-block
-    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX, MX>, dim3((warps + 7) / 8 < 4 * nsm ? (warps + 7) / 8 : 4 * nsm),
-                                     dim3(256), 0, s, ids, P, m.E, k, x, m.H, terms, args.counters,
-                                     4 * ((m.H + 127) / 128));
+    const int warps = P * nbr, wpc = kSplitThreads / 32;  // one warp per routed pair and 32-block
+    const int sgrid = (warps + wpc - 1) / wpc < 8 * nsm ? (warps + wpc - 1) / wpc : 8 * nsm;
+    cudaError_t e = launch_dependent(k_bsplit_moe<NMAX, MX>, dim3(sgrid), dim3(kSplitThreads), 0, s, ids, P, m.E, k, x,
+                                     m.H, terms, args.counters, 4 * ((m.H + 127) / 128));
     if (e != cudaSuccess) return e;
     args.nbr = nbr;
     args.terms = terms;
