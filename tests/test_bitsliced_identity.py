@@ -175,3 +175,42 @@ def test_factored_segment_start_form():
            (~(q1h ^ U ^ s(G, 3) ^ H2)) & M32, (~q1h) & M32)
     for a, b in zip(got, ref):
         assert (a == b).all()
+
+
+def _decoder_luts(fn_name, next_name):
+    """The lop3<...> truth tables of a decoder in the header, in source order."""
+    text = open(HEADER).read()
+    body = text[text.index("Planes " + fn_name + "("):text.index(next_name)]
+    return [int(v, 16) for v in re.findall(r"lop3<(0x[0-9A-Fa-f]+)>\(", body)]
+
+
+def test_decoder_truth_tables_match_the_identity():
+    # The decoders write their XOR sums as three-input ops with immediate truth tables. Applied in
+    # the header's source order to the same operands, those tables must give the planes of the
+    # identity above (checked against the oracle for every state), with and without a carry.
+    rng = np.random.default_rng(11)
+    L, H, pL, pH = (rng.integers(0, 1 << 32, 512, dtype=np.uint64) for _ in range(4))
+    t = _decoder_luts("decode_block", "// Segment-start form")
+    assert len(t) == 9
+    Ld = {d: _dly(L, pL, d) for d in range(1, 8)}
+    Hd = {d: _dly(H, pH, d) for d in range(1, 8)}
+    neg = _lop3(H, _lop3(Ld[7], Ld[4], Ld[2], t[1]), Hd[1], t[0])
+    n0 = _lop3(neg, _lop3(Ld[7], Hd[6], Hd[4], t[3]), Ld[1], t[2])
+    n1 = _lop3(neg, _lop3(Hd[7], Ld[5], Ld[3], t[5]), Hd[1], t[4])
+    n2 = _lop3(_lop3(neg, L, Ld[6], t[7]), _lop3(Hd[5], Hd[3], np.zeros_like(L), t[8]), Hd[2], t[6])
+    for got, ref in zip((n0, n1, n2, neg), _planes(L, H, pL, pH)):
+        assert (got == ref).all()
+    # segment-start form, n3 returned inverted
+    t = _decoder_luts("decode_block0_i3", "__device__ __forceinline__ Planes decode_block0(")
+    assert len(t) == 9
+    z = np.zeros_like(L)
+    sh = lambda x, d: (x << np.uint64(d)) & M32  # noqa: E731
+    F, U, H2 = _lop3(L, sh(L, 2), z, t[0]), _lop3(L, sh(L, 6), z, t[1]), sh(H, 2)
+    G = _lop3(H, H2, z, t[2])
+    X = _lop3(H, sh(F, 2), sh(L, 7), t[3])
+    q1h = _lop3(X, sh(H, 1), z, t[4])
+    n0 = _lop3(q1h, sh(U, 1), sh(G, 4), t[5])
+    n1 = _lop3(X, sh(F, 3), sh(H, 7), t[6])
+    n2 = _lop3(_lop3(q1h, U, sh(G, 3), t[8]), H2, z, t[7])
+    for got, ref in zip((n0, n1, n2, ~q1h & M32), _planes(L, H, z, z)):
+        assert (got == ref).all()

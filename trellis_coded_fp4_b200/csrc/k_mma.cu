@@ -1064,6 +1064,10 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
           }
         }
       }
+      // At the start the first stage is let land before the third is requested: with every CTA's
+      // stages requested at once, the first lands only near the end of the whole burst, and the
+      // decode warps wait for it.
+      if (!MX && qi == 1 && lane == 0 && ok) ok = mbar_wait_sleep(&w_full[0], 0u, tmo, 32u);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       wi = wi + 1 == (uint32_t)kNW ? 0u : wi + 1;

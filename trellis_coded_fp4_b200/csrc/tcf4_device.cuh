@@ -19,7 +19,7 @@
 //   neg = ~(H ^ q1)            (entries 0 and 1 of every palette are the negative ones)
 //   n0  = p0 ^ neg,  n1 = p1 ^ neg,  n2 = L ^ q0 ^ neg,  n3 = neg.
 //
-// So a whole 32-weight block decodes with ~14 shifts and ~9 three-input XORs, independent of
+// So a whole 32-weight block decodes with 11 to 14 shifts and 9 three-input XORs, independent of
 // any table. The identity is checked bit-exactly against the oracle by the GPU parity tests and
 // over all 65,536 states by a CPU test.
 #pragma once
@@ -38,18 +38,29 @@ __device__ __forceinline__ uint32_t dly(uint32_t x, uint32_t px) {
   return __funnelshift_l(px, x, D);
 }
 
+// Three-input logic op with an immediate truth table over (a, b, c) = (0xF0, 0xCC, 0xAA). The XOR
+// sums below are written with it: left to the compiler, not every three-input XOR became one
+// instruction (2.4 M of 31 M instructions of the gate_up GEMV). Tables used: a ^ b = 0x3C,
+// ~(a ^ b) = 0xC3, a ^ b ^ c = 0x96, ~(a ^ b ^ c) = 0x69.
+template <uint32_t LUT>
+__device__ __forceinline__ uint32_t lop3(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, %4;" : "=r"(d) : "r"(a), "r"(b), "r"(c), "n"(LUT));
+  return d;
+}
+
 // Decode one block. (L, H) are its planes; (pL, pH) the previous block's planes in the same
-// segment (zero at a segment start).
+// segment (zero at a segment start). 14 funnel shifts and 9 three-input XORs.
 __device__ __forceinline__ Planes decode_block(uint32_t L, uint32_t H, uint32_t pL, uint32_t pH) {
   const uint32_t L1 = dly<1>(L, pL), L2 = dly<2>(L, pL), L3 = dly<3>(L, pL), L4 = dly<4>(L, pL);
   const uint32_t L5 = dly<5>(L, pL), L6 = dly<6>(L, pL), L7 = dly<7>(L, pL);
   const uint32_t H1 = dly<1>(H, pH), H2 = dly<2>(H, pH), H3 = dly<3>(H, pH), H4 = dly<4>(H, pH);
   const uint32_t H5 = dly<5>(H, pH), H6 = dly<6>(H, pH), H7 = dly<7>(H, pH);
-  const uint32_t neg = ~(H ^ L7 ^ L4 ^ L2 ^ H1);  // ~(H ^ q1)
+  const uint32_t neg = lop3<0x69>(H, lop3<0x96>(L7, L4, L2), H1);  // ~(H ^ q1)
   Planes r;
-  r.n0 = neg ^ L7 ^ H6 ^ H4 ^ L1;                  // p0 ^ neg
-  r.n1 = neg ^ H7 ^ L5 ^ L3 ^ H1;                  // p1 ^ neg
-  r.n2 = neg ^ L ^ L6 ^ H5 ^ H3 ^ H2;              // e0 ^ neg, e0 = L ^ q0
+  r.n0 = lop3<0x96>(neg, lop3<0x96>(L7, H6, H4), L1);              // p0 ^ neg
+  r.n1 = lop3<0x96>(neg, lop3<0x96>(H7, L5, L3), H1);              // p1 ^ neg
+  r.n2 = lop3<0x96>(lop3<0x96>(neg, L, L6), lop3<0x3C>(H5, H3, 0u), H2);  // e0 ^ neg, e0 = L ^ q0
   r.n3 = neg;
   return r;
 }
@@ -57,19 +68,20 @@ __device__ __forceinline__ Planes decode_block(uint32_t L, uint32_t H, uint32_t 
 // Segment-start form (no carry from a previous block). Delays are then plain shifts, which
 // distribute over XOR, so shared sums are shifted once: with F = L ^ L2, U = L ^ L6, G = H ^ H2,
 //   L2 ^ L4 = F << 2,  L3 ^ L5 = F << 3,  L1 ^ L7 = U << 1,  H4 ^ H6 = G << 4,  H3 ^ H5 = G << 3,
-// and X = H ^ F2 ^ L7 is shared by q1 (X ^ H1) and n1 (H1 cancels): 11 shifts and 9 XOR terms
+// and X = H ^ F2 ^ L7 is shared by q1 (X ^ H1) and n1 (H1 cancels): 11 shifts and 9 XORs
 // instead of 14 and 10.
 // decode_block0 with n3 returned inverted (n3 = ~H ^ q1, returned as H ^ q1), for the transpose
 // that absorbs the inversion.
 __device__ __forceinline__ Planes decode_block0_i3(uint32_t L, uint32_t H) {
-  const uint32_t F = L ^ (L << 2), U = L ^ (L << 6), H2 = H << 2, G = H ^ H2;
-  const uint32_t X = H ^ (F << 2) ^ (L << 7);
-  const uint32_t q1h = X ^ (H << 1);  // H ^ q1
+  const uint32_t F = lop3<0x3C>(L, L << 2, 0u), U = lop3<0x3C>(L, L << 6, 0u), H2 = H << 2;
+  const uint32_t G = lop3<0x3C>(H, H2, 0u);
+  const uint32_t X = lop3<0x96>(H, F << 2, L << 7);
+  const uint32_t q1h = lop3<0x3C>(X, H << 1, 0u);  // H ^ q1
   Planes r;
   r.n3 = q1h;
-  r.n0 = ~(q1h ^ (U << 1) ^ (G << 4));
-  r.n1 = ~(X ^ (F << 3) ^ (H << 7));
-  r.n2 = ~(q1h ^ U ^ (G << 3) ^ H2);
+  r.n0 = lop3<0x69>(q1h, U << 1, G << 4);
+  r.n1 = lop3<0x69>(X, F << 3, H << 7);
+  r.n2 = lop3<0xC3>(lop3<0x96>(q1h, U, G << 3), H2, 0u);
   return r;
 }
 
