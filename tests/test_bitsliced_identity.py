@@ -206,11 +206,11 @@ def test_decoder_truth_tables_match_the_identity():
     z = np.zeros_like(L)
     sh = lambda x, d: (x << np.uint64(d)) & M32  # noqa: E731
     F, U, H2 = _lop3(L, sh(L, 2), z, t[0]), _lop3(L, sh(L, 6), z, t[1]), sh(H, 2)
-    G = _lop3(H, H2, z, t[2])
-    X = _lop3(H, sh(F, 2), sh(L, 7), t[3])
-    q1h = _lop3(X, sh(H, 1), z, t[4])
-    n0 = _lop3(q1h, sh(U, 1), sh(G, 4), t[5])
-    n1 = _lop3(X, sh(F, 3), sh(H, 7), t[6])
-    n2 = _lop3(_lop3(q1h, U, sh(G, 3), t[8]), H2, z, t[7])
+    tt = _lop3(U, sh(_lop3(H, H2, z, t[3]), 3), z, t[2])
+    X = _lop3(H, sh(F, 2), sh(L, 7), t[4])
+    q1h = _lop3(X, sh(H, 1), z, t[5])
+    n0 = _lop3(q1h, sh(tt, 1), z, t[6])
+    n1 = _lop3(X, sh(F, 3), sh(H, 7), t[7])
+    n2 = _lop3(q1h, tt, H2, t[8])
     for got, ref in zip((n0, n1, n2, ~q1h & M32), _planes(L, H, z, z)):
         assert (got == ref).all()

@@ -892,7 +892,9 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
     // Barrier latencies are hidden: the release of this stage's A slot and the arrival of the next
     // stage's words are tested (non-blocking) before a chunk's decode and their results read after
     // it; only a barrier found incomplete costs a blocking wait.
-    uint32_t ws = 0, b = 0;
+    // ring positions with their barrier phases, advanced as the slots wrap: word slot ws (phase
+    // wph of its next fill), A slot b (bph = parity of the uses of slot b so far)
+    uint32_t ws = 0, b = 0, wph = 0, bph = 0;
     bool ok = true, wf_ready = false;
     // carry path: this thread's first block of the stage is block kKB s_c + kNBT h of its row, at
     // position r_c of its segment (r_c = 0: a segment starts there); srow_w = the row's words
@@ -901,7 +903,7 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
     const uint2 *srow_w = nullptr;
 #pragma unroll 1
     for (int q = 0; q < nq; q++) {
-      if (!wf_ready && !(ok = warp_wait(&w_full[ws], (uint32_t)(q / kNW) & 1u, tmo, abort_flag))) break;
+      if (!wf_ready && !(ok = warp_wait(&w_full[ws], wph, tmo, abort_flag))) break;
       uint32_t cL = 0u, cH = 0u, smask = 0xFFu;  // carry into the first block; blocks that start a segment
       if constexpr (CARRY) {
         if (s_c == 0) {
@@ -928,7 +930,7 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
       uint32_t na[kNBT / 2];
       load_sf(na);  // the next stage's scale bytes; their latency hides behind this stage
       const uint32_t wa = wrow + ws * kWStage;
-      const uint32_t ws1 = ws + 1 == (uint32_t)kNW ? 0u : ws + 1;
+      const uint32_t ws1 = ws + 1 == (uint32_t)kNW ? 0u : ws + 1, wph1 = ws1 == 0u ? wph ^ 1u : wph;
       uint32_t ae = 1u, wf = 0u;
 #pragma unroll 1
       for (int ch = 0; ch < C::kNCh; ch++) {
@@ -937,8 +939,8 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
         uint4 cw[4];
 #pragma unroll
         for (int i = 0; i < 4; i++) cw[i] = lds_u4(wc + wlo[i]);
-        if (ch == 0 && q >= kNA) ae = mbar_test(&a_empty[2 * b + hf], (uint32_t)((q - kNA) / kNA) & 1u);
-        if (ch == C::kNCh - 1 && q + 1 < nq) wf = mbar_test(&w_full[ws1], (uint32_t)((q + 1) / kNW) & 1u);
+        if (ch == 0 && q >= kNA) ae = mbar_test(&a_empty[2 * b + hf], bph ^ 1u);
+        if (ch == C::kNCh - 1 && q + 1 < nq) wf = mbar_test(&w_full[ws1], wph1);
         uint32_t W[8][4];
         if constexpr (CARRY) {
 #pragma unroll
@@ -963,8 +965,7 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
           mbar_arrive_one(&w_empty[ws]);
         }
         if (ch == 0 && q >= kNA) {
-          if (!__all_sync(0xffffffffu, ae != 0u) &&
-              !(ok = warp_wait(&a_empty[2 * b + hf], (uint32_t)((q - kNA) / kNA) & 1u, tmo, abort_flag)))
+          if (!__all_sync(0xffffffffu, ae != 0u) && !(ok = warp_wait(&a_empty[2 * b + hf], bph ^ 1u, tmo, abort_flag)))
             break;
           tc_fence_after();
         }
@@ -975,6 +976,7 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
       if (!ok) break;
       wf_ready = __all_sync(0xffffffffu, wf != 0u);
       ws = ws1;
+      wph = wph1;
       // the scale factors of this row: its own quarter, column 4g + quarter of group g
       if constexpr (!TILED) {
 #pragma unroll
@@ -997,7 +999,10 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
       mbar_arrive_one(&a_full[2 * b + hf]);
 #pragma unroll
       for (int i = 0; i < kNBT / 2; i++) pa[i] = na[i];
-      b = b + 1 == (uint32_t)kNA ? 0u : b + 1;
+      if (++b == (uint32_t)kNA) {
+        b = 0;
+        bph ^= 1u;
+      }
       if constexpr (CARRY) {
         r_c += seg_inc;
         if (r_c >= segb) r_c -= segb;
