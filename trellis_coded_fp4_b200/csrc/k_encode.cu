@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(kEncThreads, 1)
   double *red_c = reinterpret_cast<double *>(codes_s + 4 * kEncThreads);  // 32 warp minima
   int *red_w = reinterpret_cast<int *>(red_c + 32);
   grid_dep_wait();  // the inputs may come from, and the outputs still be read by, preceding kernels
-  grid_dep_release();
+  // No early release: this kernel writes weights, which a following product kernel may read before
+  // its own grid-dependency wait; its dependents start once it has exited.
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int segs_per_row = cols / seg, nseg = rows * segs_per_row, nbr = cols / 32;
   uint32_t *my_back = back + (size_t)blockIdx.x * seg * kEncThreads;

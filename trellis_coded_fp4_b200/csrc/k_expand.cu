@@ -53,7 +53,8 @@ __global__ void __launch_bounds__(256) k_expand(const uint2 *__restrict__ stream
                                                 uint4 *__restrict__ out, const uint8_t *__restrict__ scales,
                                                 uint8_t *__restrict__ out_scales, int scales_aligned16) {
   grid_dep_wait();  // out may still be read by the preceding kernel
-  grid_dep_release();
+  // No early release: this kernel writes weights, which a following product kernel may read before
+  // its own grid-dependency wait; its dependents start once it has exited.
   const uint32_t npairs = (nblocks + 1u) >> 1;
   const uint32_t base = blockIdx.x * (256u * PT) + threadIdx.x;
   uint4 v[PT];
@@ -139,7 +140,8 @@ __global__ void __launch_bounds__(256) k_expand_q(const uint2 *__restrict__ stre
                                                   uint4 *__restrict__ out, const uint8_t *__restrict__ scales,
                                                   uint8_t *__restrict__ out_scales, int scales_aligned16) {
   grid_dep_wait();  // out may still be read by the preceding kernel
-  grid_dep_release();
+  // No early release: this kernel writes weights, which a following product kernel may read before
+  // its own grid-dependency wait; its dependents start once it has exited.
   const uint32_t g0 = 4u * (blockIdx.x * 256u + threadIdx.x);
   if (g0 + 3u < nblocks) {
     uint4 a, b, o0, o1;

@@ -304,17 +304,20 @@ __device__ __forceinline__ void split_terms(float v, int t, int kb, int S_total,
 
 // Plain GEMV: one group, token slots 0..T-1. The B rows of the other slots are not written: an MMA
 // column depends only on its own B row (and its scale), and no output reads those columns.
-// The GEMV's product kernel is launched as a programmatic dependent of this split: it starts its
-// TMEM setup and its first weight tiles (which do not depend on the split) at once and waits for
-// the split's completion only before it reads the activation terms. CTAs of 128 threads with at most
+// The GEMV's product kernel is launched as a programmatic dependent of this split, released before
+// the split's own grid-dependency wait: it starts its TMEM setup, weight tiles and first decodes
+// (none of which depend on the split or on the kernels before it) while the preceding kernel still
+// runs, and waits for the split's completion only before it reads the activation terms. (The
+// library's kernels that write weights release no dependents early, so a product kernel launched
+// after one of them finds its weights complete.) CTAs of 128 threads with at most
 // 32 registers each (4096) fit beside a resident product CTA (768 threads x 80 registers = 61440 of
 // the SM's 65536): the split of the next call can wait on its grid dependency on any SM while the
 // current product kernel runs, and it never keeps a product CTA from starting.
 template <int NMAX, bool NAT, int SETS = 1>
 __global__ void __launch_bounds__(kSplitThreads, 65536 / (32 * kSplitThreads)) k_bsplit_gemv(const uint16_t *__restrict__ x, int T, int K,
                                                      uint8_t *__restrict__ terms) {
-  grid_dep_wait();     // x may come from, and terms may still be read by, the preceding kernel
   grid_dep_release();  // the product kernel may start; it waits for this grid before reading terms
+  grid_dep_wait();     // x may come from, and terms may still be read by, the preceding kernel
   const int nb = K >> 5, S = (nb + Cfg<NMAX, SETS>::kKB - 1) / Cfg<NMAX, SETS>::kKB, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   for (int wi = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; wi < T * nb; wi += nwarps) {
@@ -1507,7 +1510,8 @@ size_t scale_tiles_bytes(const MatView &w) { return (size_t)((w.rows + 127) / 12
 __global__ void __launch_bounds__(256) k_scale_tiles(const uint8_t *__restrict__ sc, int rows, int nbr, int groups,
                                                      uint32_t *__restrict__ tiles, size_t nwords) {
   grid_dep_wait();
-  grid_dep_release();
+  // No early release: this kernel writes weights, which a following product kernel may read before
+  // its own grid-dependency wait; its dependents start once it has exited.
   for (size_t w = (size_t)blockIdx.x * blockDim.x + threadIdx.x; w < nwords; w += (size_t)gridDim.x * blockDim.x) {
     const size_t t = w / ((size_t)groups * 128u);
     const uint32_t rem = (uint32_t)(w - t * groups * 128u), g = rem >> 7, r = (rem >> 2) & 31u, q = rem & 3u;

@@ -73,7 +73,8 @@ constexpr int kRepackThreads = 256, kRepackUnits = 2;
 template <int BPU>
 __global__ void __launch_bounds__(kRepackThreads) k_repack(const uint2 *in, uint2 *out, uint32_t nblocks) {
   grid_dep_wait();  // the input may come from, and the output still be read by, preceding kernels
-  grid_dep_release();
+  // No early release: this kernel writes weights, which a following product kernel may read before
+  // its own grid-dependency wait; its dependents start once it has exited.
   const uint32_t nunits = nblocks / BPU;
   const uint32_t u0 = blockIdx.x * (kRepackThreads * kRepackUnits) + threadIdx.x;
   uint2 v[kRepackUnits][BPU];
