@@ -76,7 +76,6 @@ struct Cfg {
   static constexpr int kWLoadWarp = kDecWarps, kMmaWarp = kDecWarps + 1, kBLoadWarp = kDecWarps + 3;
   static constexpr int kEpiWarp0 = kDecWarps + 4, kThreads = 32 * (kDecWarps + 8);
   static constexpr int kNBT = 8;                               // blocks per decode thread per stage
-  static constexpr int kNCh = kNBT / 8;                        // decoded in chunks of 8 blocks
   static constexpr int kNG = kNBT / 4;                         // scale groups per decode thread
   static constexpr int kNW = kKB == 32 ? 3 : (NMAX > 96 ? 5 : 6);  // word stages in flight
   static constexpr int kNA = NMAX <= 64 || SETS > 1 ? 2 : (NMAX > 96 ? 2 : 3);  // A / scale-factor stages (TMEM)
@@ -857,10 +856,16 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
     // c0 + i (c0 = 0 or 4) of one box row: at (c0 ^ (sw & 4)) | (i ^ (sw & 3)).
     const uint32_t rb = (uint32_t)(m & 63), sw = rb & 7u;
     const uint32_t wrow = smem_u32(smem + geo.off_W) + (uint32_t)(m >> 6) * C::kBoxCols * 8192u + rb * 128u;
-    uint32_t wlo[4];
+    static_assert(kNBT == 8, "one 8-block chunk (64 bytes of words) per decode thread and stage");
+    // this thread's blocks are bytes 64 h .. 64 h + 63 of its stage row: the four reads of a stage
+    // at wrd[i] + (slot offset)
+    const uint32_t byte0 = (uint32_t)(kNBT * h) * 8u;
+    const uint32_t wc0 = wrow + (byte0 >> 7) * 8192u + ((((byte0 >> 4) & 7u) ^ (sw & 4u)) * 16u);
+    uint32_t wrd[4];
 #pragma unroll
-    for (int i = 0; i < 4; i++) wlo[i] = ((uint32_t)i ^ (sw & 3u)) * 16u;
+    for (int i = 0; i < 4; i++) wrd[i] = wc0 + ((uint32_t)i ^ (sw & 3u)) * 16u;
     const uint32_t tq = tbase + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lane quarter
+    const uint32_t acol = tq + C::kACol + 4u * (uint32_t)(kNBT * h);  // its A columns in stage 0
 
     // The UE8M0 bytes of this thread's kNG groups of four blocks (16-bit loads of block pairs),
     // loaded one stage ahead of their use. Rows outside the tile read the job's first row instead
@@ -932,50 +937,43 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
       }
       uint32_t na[kNBT / 2];
       load_sf(na);  // the next stage's scale bytes; their latency hides behind this stage
-      const uint32_t wa = wrow + ws * kWStage;
+      const uint32_t wa = ws * kWStage;
       const uint32_t ws1 = ws + 1 == (uint32_t)kNW ? 0u : ws + 1, wph1 = ws1 == 0u ? wph ^ 1u : wph;
+      uint4 cw[4];
+#pragma unroll
+      for (int i = 0; i < 4; i++) cw[i] = lds_u4(wrd[i] + wa);
       uint32_t ae = 1u, wf = 0u;
-#pragma unroll 1
-      for (int ch = 0; ch < C::kNCh; ch++) {
-        const uint32_t byte0 = (uint32_t)(kNBT * h + 8 * ch) * 8u;  // the chunk's offset in the stage row
-        const uint32_t wc = wa + (byte0 >> 7) * 8192u + ((((byte0 >> 4) & 7u) ^ (sw & 4u)) * 16u);
-        uint4 cw[4];
+      if (q >= kNA) ae = mbar_test(&a_empty[2 * b + hf], bph ^ 1u);
+      if (q + 1 < nq) wf = mbar_test(&w_full[ws1], wph1);
+      uint32_t W[8][4];
+      if constexpr (CARRY) {
 #pragma unroll
-        for (int i = 0; i < 4; i++) cw[i] = lds_u4(wc + wlo[i]);
-        if (ch == 0 && q >= kNA) ae = mbar_test(&a_empty[2 * b + hf], bph ^ 1u);
-        if (ch == C::kNCh - 1 && q + 1 < nq) wf = mbar_test(&w_full[ws1], wph1);
-        uint32_t W[8][4];
-        if constexpr (CARRY) {
+        for (int i = 0; i < 8; i++) {
+          const uint32_t L = (i & 1) ? cw[i >> 1].z : cw[i >> 1].x, Hh = (i & 1) ? cw[i >> 1].w : cw[i >> 1].y;
+          if ((smask >> i) & 1u) cL = cH = 0u;
+          planes_to_nibbles_interleaved(decode_block(L, Hh, cL, cH), W[i][0], W[i][1], W[i][2], W[i][3]);
+          cL = L;
+          cH = Hh;
+        }
+      } else {
 #pragma unroll
-          for (int i = 0; i < 8; i++) {
-            const uint32_t L = (i & 1) ? cw[i >> 1].z : cw[i >> 1].x, Hh = (i & 1) ? cw[i >> 1].w : cw[i >> 1].y;
-            if ((smask >> i) & 1u) cL = cH = 0u;
-            planes_to_nibbles_interleaved(decode_block(L, Hh, cL, cH), W[i][0], W[i][1], W[i][2], W[i][3]);
-            cL = L;
-            cH = Hh;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 4; i++) {
-            planes_to_nibbles_interleaved_i3(decode_block0_i3(cw[i].x, cw[i].y), W[2 * i][0], W[2 * i][1],
-                                             W[2 * i][2], W[2 * i][3]);
-            planes_to_nibbles_interleaved_i3(decode_block0_i3(cw[i].z, cw[i].w), W[2 * i + 1][0], W[2 * i + 1][1],
-                                             W[2 * i + 1][2], W[2 * i + 1][3]);
-          }
+        for (int i = 0; i < 4; i++) {
+          planes_to_nibbles_interleaved_i3(decode_block0_i3(cw[i].x, cw[i].y), W[2 * i][0], W[2 * i][1],
+                                           W[2 * i][2], W[2 * i][3]);
+          planes_to_nibbles_interleaved_i3(decode_block0_i3(cw[i].z, cw[i].w), W[2 * i + 1][0], W[2 * i + 1][1],
+                                           W[2 * i + 1][2], W[2 * i + 1][3]);
         }
-        if (ch == C::kNCh - 1) {  // every word of the stage has been read (and used): free the slot
-          __syncwarp();
-          mbar_arrive_one(&w_empty[ws]);
-        }
-        if (ch == 0 && q >= kNA) {
-          if (!__all_sync(0xffffffffu, ae != 0u) && !(ok = warp_wait(&a_empty[2 * b + hf], bph ^ 1u, tmo, abort_flag)))
-            break;
-          tc_fence_after();
-        }
-        // the chunk's codes: columns 4 (kNBT h + 8 ch).. of the stage's A. Columns of blocks beyond
-        // the row's end hold the decode of the zero fill; no MMA reads them.
-        tmem_st_codes<8>(tq + C::kACol + C::kACols * b + 4u * (uint32_t)(kNBT * h + 8 * ch), W);
       }
+      __syncwarp();  // every word of the stage has been read (and used): free the slot
+      mbar_arrive_one(&w_empty[ws]);
+      if (q >= kNA) {
+        if (!__all_sync(0xffffffffu, ae != 0u) && !(ok = warp_wait(&a_empty[2 * b + hf], bph ^ 1u, tmo, abort_flag)))
+          break;
+        tc_fence_after();
+      }
+      // the codes: columns 4 kNBT h.. of the stage's A. Columns of blocks beyond the row's end hold
+      // the decode of the zero fill; no MMA reads them.
+      tmem_st_codes<8>(acol + C::kACols * b, W);
       if (!ok) break;
       wf_ready = __all_sync(0xffffffffu, wf != 0u);
       ws = ws1;
