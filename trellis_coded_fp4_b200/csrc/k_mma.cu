@@ -1138,8 +1138,10 @@ __global__ void __launch_bounds__(Cfg<NMAX, SETS>::kThreads, 1) k_mma(const __gr
       const JobRows jr = job_rows<MAXE, MODE, NMAX>(a, tab, pl, job_of(jl_e));
       const int buf = jl_e & 1;                   // the gate/up exchange buffer
       const int abuf = jl_e % C::kNAcc;           // the accumulator
-      // one warp polls; the others wait at a named barrier (no issue slots taken meanwhile)
-      if (warp == C::kEpiWarp0) {
+      // one warp polls; the others wait at a named barrier (no issue slots taken meanwhile). The
+      // poller is the epilogue warp on the sub-partition of the B loader (warp % 4 == 3): the word
+      // loader's and the MMA issuers' sub-partitions carry more besides their four decode warps.
+      if (warp == C::kEpiWarp0 + 3) {
         if (!mbar_wait_sleep(&acc_full[abuf], (uint32_t)(jl_e / C::kNAcc) & 1u, tmo, kEpiSleepNs)) *abort_flag = 1;
       }
       named_bar(1, 128);
