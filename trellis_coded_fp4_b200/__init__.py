@@ -92,10 +92,15 @@ def gemv(w: TrellisMatrix, x: torch.Tensor, out=None, workspace=None):
     return out
 
 
+def scale_tiles_bytes(w: TrellisMatrix) -> int:
+    """Bytes of w's scale tiles (trellis_scale_tiles_bytes)."""
+    return int(_abi.load().trellis_scale_tiles_bytes(w.abi()))
+
+
 def scale_tiles(w: TrellisMatrix, out=None):
     """The weights' UE8M0 scales rearranged once into scale tiles (uint8, trellis_scale_tiles_bytes
     long), the layout trellis_gemv_tiled reads."""
-    n = int(_abi.load().trellis_scale_tiles_bytes(w.abi()))
+    n = scale_tiles_bytes(w)
     if out is None:
         out = torch.empty(n, dtype=torch.uint8, device=w.stream.device)
     _abi.check(_abi.load().trellis_make_scale_tiles(w.abi(), _ptr(out), _stream_handle()), "trellis_make_scale_tiles")
