@@ -92,13 +92,13 @@ struct Cfg {
   // Weights' scales as scale tiles (trellis_gemv_tiled): per 4-block group a 512-byte tile, row r
   // = the group's UE8M0 words of tile rows r, 32 + r, 64 + r, 96 + r; KB/4 tiles per stage.
   static constexpr uint32_t kSfaTile = (kKB / 4) * 512u;
-  // MMA issuers: one per half stage, each into its own accumulator, up to 64 B rows (one issuing
+  // MMA issuers: one per half stage, each into its own accumulator, up to 96 B rows (one issuing
   // thread sustains about one MMA per 60 cycles, two in different warps run concurrently, and a
   // single issuer's instructions slow the decode warps of its sub-partition).
-  static constexpr int kNI = NMAX <= 64 ? 2 : 1;
-  // accumulators per issuer: two (a job's epilogue overlaps the next job's MMAs) where TMEM has room;
-  // at 64 B rows one each, so that both issuers fit (2 x 64 + 256 A + 64 + 64 scale columns = 512)
-  static constexpr int kNAcc = NMAX > 96 || NMAX == 64 ? 1 : 2;
+  static constexpr int kNI = NMAX <= 96 ? 2 : 1;
+  // accumulators per issuer: two (a job's epilogue overlaps the next job's MMAs) at 32 B rows; one
+  // each above, so that both issuers fit (at 64 rows: 2 x 64 + 256 A + 64 + 64 scale columns = 512)
+  static constexpr int kNAcc = NMAX > 32 ? 1 : 2;
   static constexpr uint32_t kACols = 4u * kKB;                 // TMEM columns of a stage's A
   static constexpr uint32_t kSfbCols = (kKB / 4) * kSfbGCols;  // TMEM columns of a stage's B scales
   static constexpr uint32_t kACol = kNAcc * kNI * NMAX;        // TMEM: accumulators first, then
