@@ -32,6 +32,15 @@
  *   calls (cudaGetLastError), so that it is not mistaken for its own; a failed launch then returns
  *   TCF4_ERR_CUDA with the CUDA error left set for the caller to read. Empty problems (rows == 0,
  *   T == 0) return TCF4_OK and launch nothing.
+ * Stream order. Kernels are launched as programmatic dependents of the preceding work on the
+ *   stream: each waits for its predecessor before it reads what that predecessor may write (x,
+ *   routing, workspace) or writes what it may still read (y, workspace). The product kernels read
+ *   their weights (stream words, scales, scale tiles, MXFP4 nibbles) before that wait, while the
+ *   preceding kernel may still run; the weights must therefore be complete when the call is
+ *   enqueued, or be written by work that has completed by then in stream order without releasing
+ *   its dependents early. The library's own weight-writing calls (trellis_repack_interleaved,
+ *   trellis_make_scale_tiles, trellis_decode_to_mxfp4, trellis_encode) release no dependents
+ *   early, so a product call right after one of them reads the finished weights.
  * Threads. Calls are reentrant. The only process state the library writes is a one-time
  *   per-device kernel attribute (the dynamic shared-memory limit of its kernels).
  */
