@@ -9,25 +9,27 @@
 // y[t] = sum_j D[:, kTerms*t + j] in fp32.
 //
 // One persistent CTA per SM, over 128-row tiles ("jobs") of K stages of KB blocks of 32 (KB = 32 for
-// up to five tokens per group, else 16):
+// up to ten tokens per group, else 16):
 //  * word loader warp: lane 0 streams each stage's trellis words (128 rows x 8 KB bytes) into a ring
-//    of shared-memory slots with 2-D TMA tile loads (128-byte swizzle).
+//    of shared-memory slots with 2-D TMA tile loads (128-byte swizzle, no multicast).
 //  * KB/2 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and the 8 K-blocks 8(w/4)..
-//    of a stage (two scale-factor groups). It reads its 64 bytes of trellis words, decodes them in
-//    registers (bit-sliced) and stores the blocks' E2M1 codes, packed eight per 32-bit column, into
-//    the stage's A operand in TMEM, together with the groups' scale factors of its row (A) and of
-//    the B rows its lane stands for (tcgen05.st into its own lane quarter; the scale bytes are
-//    loaded one stage ahead). The decoded weights never touch shared memory. A stage's A operand
-//    is handed over in two halves (the first and last KB/2 blocks), each with its own barriers.
-//  * B loader warp: lane 0 bulk-copies each stage's activation terms into a 4-slot B ring, up to four
-//    stages ahead of the MMAs.
-//  * MMA warp(s): with up to five tokens per group two issuer warps, one per half stage, each into
-//    its own accumulator of a double-buffered pair (a single issuing thread sustains about one MMA
-//    per 60 cycles; two in different warps run concurrently); otherwise one warp issues both
-//    halves. A half's MMAs (A from TMEM, B from shared memory) are released with one commit.
+//    of a stage. It reads its 64 bytes of trellis words, decodes them in registers (bit-sliced) and
+//    stores the blocks' E2M1 codes, packed eight per 32-bit column, into the stage's A operand in
+//    TMEM (tcgen05.st into its own lane quarter); with the weights' scales in their stored layout it
+//    also stores its row's scale bytes (loaded one stage ahead). The decoded weights never touch
+//    shared memory. A stage's A operand is handed over in two halves (the first and last KB/2
+//    blocks), each with its own barriers.
+//  * B loader warp: lane 0 bulk-copies each stage's activation terms and their scale-factor tiles
+//    (and, with scale tiles, the weights' tiles of the stage) into a ring of B slots, ahead of the
+//    MMAs; it alone waits for the preceding kernel (the split that wrote the terms).
+//  * MMA warp(s): up to 96 B rows two issuer warps, one per half stage, each into its own
+//    accumulator (a double-buffered pair at 32 rows, one each at 64 and 96, as TMEM allows); at 192
+//    rows one warp issues both halves. An issuer moves the stage's scale-factor tiles into TMEM with
+//    tcgen05.cp, then issues its MMAs (A from TMEM, B from shared memory), released with one commit.
 //  * 4 epilogue warps (one per TMEM lane quarter): the epilogue of each job (tcgen05.ld, then the
-//    GEMV output, the SwiGLU of gate/up rows, or the MoE down rows and their combine), overlapping
-//    the next job's stages.
+//    GEMV output, the SwiGLU of gate/up rows and its split into the down product's terms, or the MoE
+//    down rows and their combine), overlapping the next job's stages where the accumulators are
+//    double-buffered.
 // Every wait is bounded; a wait that gives up raises a shared abort flag that the other roles see,
 // and each role drains its own asynchronous copies and MMAs before the CTA frees its TMEM.
 #include <cuda.h>
@@ -46,9 +48,10 @@ __device__ unsigned int g_tcf4_timeouts_mma = 0;
 constexpr int kTerms = 6;            // E2M1 terms per activation block
 constexpr int kMapSlots = 8;         // per-CTA tensor-map slots of the grouped MoE (> jobs in flight)
 
+constexpr int kSplitThreads = 128;  // activation-split CTAs (see k_bsplit_gemv)
+
 // Sleep between barrier tests of the idle roles. The loaders run stages ahead and the MMA issuers
 // have about two stages (~3 us) of slack, so these only bound how soon a completed phase is seen.
-constexpr int kSplitThreads = 128;  // activation-split CTAs (see k_bsplit_gemv)
 constexpr uint32_t kLoaderSleepNs = 200u, kMmaSleepNs = 100u, kEpiSleepNs = 200u;
 
 enum MmaMode { kModeGemv = 0, kModeGateUp = 1, kModeDown = 2 };
