@@ -9,7 +9,7 @@
 // y[t] = sum_j D[:, kTerms*t + j] in fp32.
 //
 // One persistent CTA per SM, over 128-row tiles ("jobs") of K stages of KB blocks of 32 (KB = 32 for
-// up to ten tokens per group, else 16):
+// up to ten tokens per group with one scale set, else 16):
 //  * word loader warp: lane 0 streams each stage's trellis words (128 rows x 8 KB bytes) into a ring
 //    of shared-memory slots with 2-D TMA tile loads (128-byte swizzle, no multicast).
 //  * KB/2 decode warps: thread (warp w, lane l) owns tile row 32(w%4)+l and the 8 K-blocks 8(w/4)..
