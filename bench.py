@@ -271,13 +271,15 @@ class Layer:
             if not hasattr(self, "_moe1"):
                 self._moe1 = self.moe_call(1)
             self._moe1(i)
-        elif name == "gemv_gate_up_t32":
-            if not hasattr(self, "_x32"):
+        elif name.startswith("gemv_gate_up_t"):  # gemv_gate_up_t<T>: the tiled call at T tokens
+            T = int(name[len("gemv_gate_up_t"):])
+            if getattr(self, "_tT", None) != T:
                 from trellis_coded_fp4_b200 import synth
-                self._x32 = synth.activations(32, H, seed=synth.SEED_BASE + 122).to(self.device)
-                self._y32 = torch.empty((32, self.G.rows), dtype=torch.bfloat16, device=self.device)
-                self._ws32 = torch.empty(tc.gemv_workspace_bytes(self.G, 32), dtype=torch.uint8, device=self.device)
-            tc.gemv_tiled(self.G, self.Trot[0], self._x32, self._y32, self._ws32)
+                self._tT = T
+                self._xT = synth.activations(T, H, seed=synth.SEED_BASE + 90 + T).to(self.device)
+                self._yT = torch.empty((T, self.G.rows), dtype=torch.bfloat16, device=self.device)
+                self._wsT = torch.empty(tc.gemv_workspace_bytes(self.G, T), dtype=torch.uint8, device=self.device)
+            tc.gemv_tiled(self.G, self.Trot[0], self._xT, self._yT, self._wsT)
         elif name == "encoder":
             if not hasattr(self, "_enc"):
                 g = torch.Generator(device=self.device).manual_seed(7)
@@ -682,7 +684,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="the headline only, without the extra rows")
     ap.add_argument("--only", default=None,
-                    help="run only this call (gemv_gate_up, gemv_gate_up_raw, gemv_gate_up_t32, gemv_down, gemv_e5m3, "
+                    help="run only this call (gemv_gate_up, gemv_gate_up_raw, gemv_gate_up_t<T>, gemv_down, gemv_e5m3, "
                          "expand_gate_up, grouped_moe, encoder) warmup + "
                          "steps times, for profiling one kernel; prints no bench line")
     args = ap.parse_args()
